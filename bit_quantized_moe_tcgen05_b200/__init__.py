@@ -1,0 +1,207 @@
+"""W4A4 quantized linear layer for NVIDIA B200 (sm_100a): Python binding over libqlinear.
+
+Argument marshalling only.  Every step of the forward path runs in the CUDA kernels of
+``libqlinear.so`` (built in-tree by ``bit_quantized_moe_tcgen05_b200.build``); torch supplies
+device memory and the current stream.  Importing this package fails if the library is missing:
+there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = [
+    "lib", "LIB_PATH", "QLError", "WeightDesc", "QLinear", "quantize_act", "prepare_prquant",
+    "check", "QL_W_MXFP4_E8M0_B32", "QL_A_MXFP4_E8M0_B32", "EXPORTED_SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlinear.so")
+
+QL_OK = 0
+QL_W_MXFP4_E8M0_B32, QL_W_NVFP4_E4M3_B16, QL_W_VQ_PRESCALE_E4M3_B16 = 1, 2, 3
+QL_W_CLUSTER4_ROW16_BF16, QL_W_INT4_G128_BSR = 4, 5
+QL_A_MXFP4_E8M0_B32, QL_A_FP4_E4M3_B16_TS, QL_A_INT4_TOK_G128 = 1, 2, 3
+
+_STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED", 3: "QL_ERR_CUDA",
+           4: "QL_ERR_OOM", 5: "QL_ERR_TIMEOUT", 6: "QL_ERR_WORKSPACE"}
+
+# Every entry point declared in include/qlinear.h.
+EXPORTED_SYMBOLS = (
+    "ql_version", "ql_last_error", "qlinear_create", "qlinear_destroy", "qlinear_workspace_bytes",
+    "qlinear_forward", "quantize_act", "ql_check", "qlinear_prepare_prquant",
+    "qlinear_quantize_input", "qlinear_gemm",
+)
+
+
+class QLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = lib.ql_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class WeightDesc(ctypes.Structure):
+    _fields_ = [
+        ("wfmt", ctypes.c_int), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+        ("k_tail", ctypes.c_int32), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+        ("w_tensor_scale", ctypes.c_float), ("indices", ctypes.c_void_p),
+        ("codebooks", ctypes.c_void_p), ("qblock_n", ctypes.c_int32), ("qblock_k", ctypes.c_int32),
+        ("bsr_rowptr", ctypes.c_void_p), ("bsr_col", ctypes.c_void_p),
+        ("bsr_codes", ctypes.c_void_p), ("bsr_scales", ctypes.c_void_p),
+        ("bsr_block_n", ctypes.c_int32), ("bsr_block_k", ctypes.c_int32),
+        ("bsr_nnzb", ctypes.c_int32),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "`python -m bit_quantized_moe_tcgen05_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    L.ql_version.restype = ctypes.c_char_p
+    L.ql_last_error.restype = ctypes.c_char_p
+    sig = {
+        "qlinear_create": [ctypes.POINTER(WeightDesc), vp, ctypes.POINTER(vp)],
+        "qlinear_destroy": [vp],
+        "qlinear_workspace_bytes": [vp, i64, ctypes.POINTER(sz)],
+        "qlinear_forward": [vp, vp, i64, vp, vp, vp, sz, vp],
+        "qlinear_quantize_input": [vp, vp, i64, vp, sz, vp],
+        "qlinear_gemm": [vp, i64, vp, vp, vp, sz, vp],
+        "quantize_act": [ctypes.c_int, vp, i64, i64, vp, vp, vp, vp],
+        "ql_check": [vp],
+        "qlinear_prepare_prquant": [vp, i64, i64, i32, vp, vp, vp],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def _ok(status: int, where: str) -> None:
+    if status != QL_OK:
+        raise QLError(status, where)
+
+
+def _stream(stream=None) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def check(stream=None) -> None:
+    """Synchronise and raise if any kernel recorded a device-side timeout."""
+    _ok(lib.ql_check(_stream(stream)), "ql_check")
+
+
+def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None):
+    """Quantize bf16 activations [M, K] on the GPU.  Returns (codes uint8 [M, K/2],
+    scales uint8 [M, K/32]) for MXFP4 E8M0-B32."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    M, K = x.shape
+    if fmt != QL_A_MXFP4_E8M0_B32:
+        raise ValueError("only QL_A_MXFP4_E8M0_B32 is exposed here")
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
+    _ok(lib.quantize_act(fmt, x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), None,
+                         _stream(stream)), "quantize_act")
+    return codes, scales
+
+
+class QLinear:
+    """A quantized linear layer y = x W^T whose weight lives in library-owned device memory.
+
+    MXFP4 (E8M0-B32) weights: ``codes`` uint8 [N, K/2] (low nibble = even k) and ``scales``
+    uint8 [N, K/32] E8M0 bytes, host numpy arrays.  ``k_tail`` > 0 makes it a PRQuant
+    augmented weight whose last ``k_tail`` columns are the tail residual; the activation then
+    has K - k_tail channels.
+    """
+
+    def __init__(self, codes: np.ndarray, scales: np.ndarray, k_tail: int = 0,
+                 wfmt: int = QL_W_MXFP4_E8M0_B32, stream=None):
+        codes = np.ascontiguousarray(codes, dtype=np.uint8)
+        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        N, half_k = codes.shape
+        self.N, self.K, self.k_tail = N, 2 * half_k, int(k_tail)
+        self.C = self.K - self.k_tail
+        d = WeightDesc(wfmt=wfmt, N=N, K=self.K, k_tail=self.k_tail,
+                       codes=codes.ctypes.data, scales=scales.ctypes.data)
+        h = ctypes.c_void_p()
+        _ok(lib.qlinear_create(ctypes.byref(d), _stream(stream), ctypes.byref(h)), "qlinear_create")
+        self._h = h
+        self._ws = None
+
+    def workspace_bytes(self, M: int) -> int:
+        n = ctypes.c_size_t()
+        _ok(lib.qlinear_workspace_bytes(self._h, M, ctypes.byref(n)), "qlinear_workspace_bytes")
+        return n.value
+
+    def _workspace(self, M: int, device):
+        import torch
+        need = self.workspace_bytes(M)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=device)
+        return self._ws
+
+    def forward(self, x, out=None, out_f32=None, ws=None, stream=None):
+        """x: bf16 [M, K - k_tail] on the GPU.  Returns y bf16 [M, N] (and fills out_f32)."""
+        import torch
+        assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+        M, C = x.shape
+        if C != self.C:
+            raise ValueError(f"x has {C} channels, layer expects {self.C}")
+        if out is None:
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device)
+        if ws is None:
+            ws = self._workspace(M, x.device)
+        _ok(lib.qlinear_forward(self._h, x.data_ptr(), M, out.data_ptr(), _ptr(out_f32),
+                                ws.data_ptr(), ws.numel(), _stream(stream)), "qlinear_forward")
+        return out
+
+    __call__ = forward
+
+    def quantize_input(self, x, ws, stream=None) -> None:
+        """First half of forward: quantize x into the workspace ``ws``."""
+        M = x.shape[0]
+        _ok(lib.qlinear_quantize_input(self._h, x.data_ptr(), M, ws.data_ptr(), ws.numel(),
+                                       _stream(stream)), "qlinear_quantize_input")
+
+    def gemm(self, M: int, out, ws, out_f32=None, stream=None) -> None:
+        """Second half of forward: the FP4 GEMM from the quantized input in ``ws``."""
+        _ok(lib.qlinear_gemm(self._h, M, out.data_ptr(), _ptr(out_f32), ws.data_ptr(), ws.numel(),
+                             _stream(stream)), "qlinear_gemm")
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib.qlinear_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def prepare_prquant(w_bf16_bits: np.ndarray, k: int):
+    """Offline PRQuant preparation on the host (library C++ code, not the oracle).
+    Returns (perm int32 [C], codes uint8 [N, (C+k)/2], scales uint8 [N, (C+k)/32])."""
+    w = np.ascontiguousarray(w_bf16_bits, dtype=np.uint16)
+    N, C = w.shape
+    perm = np.empty(C, np.int32)
+    codes = np.empty((N, (C + k) // 2), np.uint8)
+    scales = np.empty((N, (C + k) // 32), np.uint8)
+    _ok(lib.qlinear_prepare_prquant(w.ctypes.data, N, C, k, perm.ctypes.data, codes.ctypes.data,
+                                    scales.ctypes.data), "qlinear_prepare_prquant")
+    return perm, codes, scales

@@ -1,0 +1,256 @@
+// Block-scaled FP4 GEMM on tcgen05 tensor cores (sm_100a), with the PRQuant K-extension.
+//
+//   y[m, n] = alpha * sum_k x_q[m, k] * w_q[n, k]
+//
+// over packed E2M1 operands with per-32 E8M0 scales (kind::mxf4) or per-16 UE4M3 scales
+// (kind::mxf4nvf4, alpha = product of the two FP32 tensor scales).  The weight is the MMA's
+// 128-row "A" operand and the tokens are the "B" operand of width BN (8..256), so one kernel
+// serves decode (M = 1..16, with split-K over CTAs) and prefill (M up to thousands).
+//
+// PRQuant ("Kernel design for efficient inference"): the weight is W_aug = Q([W~, R_W]) with
+// reduction width C + k; the activation is quantized once over its C channels and its last k
+// channels are read a second time for the tail stages (activation coordinate C - k + j while
+// the weight coordinate is C + j).  No tail copy is materialised.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + single-thread
+// MMA issuer, warps 2..5 = epilogue (TMEM -> registers -> global).  A STAGES-deep ring of
+// shared-memory stages, each 256 K-elements deep, is guarded by full/empty mbarriers; MMA
+// completion is signalled by tcgen05.commit.  Every wait is bounded (see ptx.cuh).
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace ql {
+
+struct Fp4GemmArgs {
+  int M, N;                 // tokens, output features
+  int C, k_tail;            // activation width; tail width (weight width K' = C + k_tail)
+  int n_base_stages;        // ceil(C / 256)
+  int n_stages_total;       // n_base_stages + ceil(k_tail / 256)
+  int stages_per_split;     // K stages handled by one CTA (gridDim.z = splits)
+  const uint8_t* sfa;       // weight scales, tiled atoms
+  int sfa_atoms;            // atoms per 128-row group of the weight
+  const uint8_t* sfb;       // activation scales, tiled atoms
+  int sfb_atoms;            // atoms per 128-row group of the activation
+  const float* alpha_dev;   // optional device scalar multiplied into alpha (tensor scale of x)
+  float alpha;              // host scalar (tensor scale of w, or 1)
+  __nv_bfloat16* y;         // [M, ldy] bf16 output
+  float* y32;               // optional [M, ldy] fp32 output
+  int ldy;
+  float* partial;           // split-K partials [splits][M][N] (splits > 1)
+  int* counters;            // split-K tickets, one per (n-tile, m-tile); zero on entry
+};
+
+template <int BN, bool E8M0>
+struct Fp4Cfg {
+  static constexpr int kAtomK = E8M0 ? 128 : 64;      // K elements covered by one SF atom
+  static constexpr int kAtoms = 256 / kAtomK;         // SF atoms per stage per 128 rows
+  static constexpr int kG = (BN + 127) / 128;          // 128-row groups of the B operand
+  static constexpr int kABytes = 128 * 128;            // 128 rows x 256 fp4
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kSfaBytes = kAtoms * 512;
+  static constexpr int kSfbBytes = kAtoms * kG * 512;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : (kStagesRaw < 2 ? 2 : kStagesRaw);
+  static constexpr int kSfaCols = kAtoms * 4;          // TMEM columns per stage
+  static constexpr int kSfbCols = kAtoms * 4 * kG;
+  static constexpr int kColsNeeded = BN + kStages * (kSfaCols + kSfbCols);
+  static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
+                                 : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
+  static_assert(kColsNeeded <= 512, "TMEM budget");
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+template <int BN, bool E8M0>
+__global__ void __launch_bounds__(192, 1)
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_x, const Fp4GemmArgs a) {
+  using Cfg = Fp4Cfg<BN, E8M0>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * Cfg::kABytes;
+  uint8_t* sSfa = sB + S * Cfg::kBBytes;
+  uint8_t* sSfb = sSfa + S * Cfg::kSfaBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSfb + S * Cfg::kSfbBytes);
+  uint64_t* empty = full + S;
+  uint64_t* accf = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  int* flag_slot = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN;
+  const int s_begin = blockIdx.z * a.stages_per_split;
+  const int s_end = min(a.n_stages_total, s_begin + a.stages_per_split);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sfa_col0 = BN, sfb_col0 = BN + S * Cfg::kSfaCols;
+
+  // K stage i -> (weight element offset, activation element offset, valid elements)
+  auto stage_coords = [&](int i, int& kw, int& kx, int& valid) {
+    if (i < a.n_base_stages) {
+      kw = i * 256;
+      kx = kw;
+      valid = min(256, a.C - kw);
+    } else {
+      const int j = (i - a.n_base_stages) * 256;
+      kw = a.C + j;
+      kx = a.C - a.k_tail + j;
+      valid = min(256, a.k_tail - j);
+    }
+  };
+
+  bool ok = true;
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = s_begin, it = 0; i < s_end && ok; ++i, ++it) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait(&empty[st], ph ^ 1, 1)) { ok = false; break; }
+        int kw, kx, valid;
+        stage_coords(i, kw, kx, valid);
+        const int nat = valid / Cfg::kAtomK;
+        const uint32_t bytes = Cfg::kABytes + Cfg::kBBytes + nat * 512 * (1 + Cfg::kG);
+        mbar_arrive_expect_tx(&full[st], bytes);
+        tma_load_2d(sA + st * Cfg::kABytes, &tm_w, &full[st], kw >> 1, n0);
+        tma_load_2d(sB + st * Cfg::kBBytes, &tm_x, &full[st], kx >> 1, m0);
+        bulk_load(sSfa + st * Cfg::kSfaBytes,
+                  a.sfa + (static_cast<size_t>(n0 >> 7) * a.sfa_atoms + kw / Cfg::kAtomK) * 512,
+                  nat * 512, &full[st]);
+#pragma unroll
+        for (int g = 0; g < Cfg::kG; ++g)
+          bulk_load(sSfb + st * Cfg::kSfbBytes + g * Cfg::kAtoms * 512,
+                    a.sfb + (static_cast<size_t>((m0 >> 7) + g) * a.sfb_atoms + kx / Cfg::kAtomK) * 512,
+                    nat * 512, &full[st]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc0 = idesc_fp4_block(BN, E8M0);
+      bool first = true;
+      for (int i = s_begin, it = 0; i < s_end && ok; ++i, ++it) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait(&full[st], ph, 2)) { ok = false; break; }
+        tc_fence_after();
+        int kw, kx, valid;
+        stage_coords(i, kw, kx, valid);
+        const int nat = valid / Cfg::kAtomK;
+        const uint32_t ta = tmem + sfa_col0 + st * Cfg::kSfaCols;
+        const uint32_t tb = tmem + sfb_col0 + st * Cfg::kSfbCols;
+        for (int at = 0; at < nat; ++at) {
+          tc_cp_32x128b_warpx4(ta + at * 4,
+                               make_sdesc(smem_u32(sSfa + st * Cfg::kSfaBytes + at * 512), 0, 128, kLayoutNone));
+#pragma unroll
+          for (int g = 0; g < Cfg::kG; ++g)
+            tc_cp_32x128b_warpx4(tb + at * 4 * Cfg::kG + g * 4,
+                                 make_sdesc(smem_u32(sSfb + st * Cfg::kSfbBytes + g * Cfg::kAtoms * 512 + at * 512),
+                                            0, 128, kLayoutNone));
+        }
+        const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
+        const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
+        const int nk = valid / 64;
+        for (int kk = 0; kk < nk; ++kk) {
+          const int at = (kk * 64) / Cfg::kAtomK;
+          const uint32_t byte = E8M0 ? static_cast<uint32_t>((kk & 1) * 2) : 0u;
+          const uint64_t adesc = make_sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128);
+          const uint64_t bdesc = make_sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128);
+          const uint32_t idesc = idesc0 | (byte << 29) | (byte << 4);
+          const uint32_t sfa_t = (ta + at * 4) | (byte << 30);
+          const uint32_t sfb_t = (tb + at * 4 * Cfg::kG) | (byte << 30);
+          if (E8M0)
+            mma_mxf4_block32(tmem, adesc, bdesc, idesc, sfa_t, sfb_t, first ? 0u : 1u);
+          else
+            mma_nvf4_block16(tmem, adesc, bdesc, idesc, sfa_t, sfb_t, first ? 0u : 1u);
+          first = false;
+        }
+        tc_commit(&empty[st]);
+      }
+      tc_commit(accf);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+    const int q = warp & 3;
+    const int n = n0 + q * 32 + lane;
+    const int splits = gridDim.z;
+    const bool have_acc = (s_end > s_begin);
+    float alpha = a.alpha;
+    if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
+    if (have_acc) ok = mbar_wait(accf, 0, 3);
+    tc_fence_after();
+    const int mcount = min(BN, a.M - m0);
+    if (ok) {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 8) {
+        uint32_t r[8];
+        tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int mm = c + j;
+          if (mm >= mcount || n >= a.N) continue;
+          const float v = have_acc ? __uint_as_float(r[j]) : 0.f;
+          const size_t o = static_cast<size_t>(m0 + mm) * a.ldy + n;
+          if (splits == 1) {
+            a.y[o] = __float2bfloat16_rn(v * alpha);
+            if (a.y32 != nullptr) a.y32[o] = v * alpha;
+          } else {
+            a.partial[(static_cast<size_t>(blockIdx.z) * a.M + m0 + mm) * a.N + n] = v;
+          }
+        }
+      }
+    }
+    if (splits > 1) {
+      // Deterministic split-K: the last CTA to finish a tile sums the partials in split order.
+      __threadfence();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 64) {
+        const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+        const int old = atomicAdd(&a.counters[tile], 1);
+        *flag_slot = (old == splits - 1);
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*flag_slot) {
+        __threadfence();
+        if (n < a.N) {
+          for (int mm = 0; mm < mcount; ++mm) {
+            float acc = 0.f;
+            for (int s = 0; s < splits; ++s)
+              acc += __ldcg(&a.partial[(static_cast<size_t>(s) * a.M + m0 + mm) * a.N + n]);
+            const size_t o = static_cast<size_t>(m0 + mm) * a.ldy + n;
+            a.y[o] = __float2bfloat16_rn(acc * alpha);
+            if (a.y32 != nullptr) a.y32[o] = acc * alpha;
+          }
+        }
+        if (threadIdx.x == 64) a.counters[blockIdx.y * gridDim.x + blockIdx.x] = 0;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+}  // namespace ql

@@ -1,0 +1,366 @@
+// libqlinear: C ABI over the sm_100a kernels (see include/qlinear.h for the contract).
+// One translation unit holds every kernel so that they share the device error word.
+#include "qlinear.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "ptx.cuh"
+#include "quant_act.cuh"
+#include "gemm_fp4.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ql_status fail(ql_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define QL_CUDA(call)                                                                  \
+  do {                                                                                 \
+    cudaError_t e_ = (call);                                                           \
+    if (e_ != cudaSuccess)                                                             \
+      return fail(QL_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));        \
+  } while (0)
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ----------------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [rows, inner_bytes] with a 128-byte swizzled box of [box_rows, 128 bytes].
+ql_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows,
+                       uint64_t row_stride, uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner_bytes, rows};
+  cuuint64_t strides[1] = {row_stride};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return QL_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// ----------------------------------------------------------------------- GEMM launch
+template <int BN, bool E8M0>
+ql_status launch_fp4_bn(const CUtensorMap& tw, const CUtensorMap& tx, const ql::Fp4GemmArgs& a,
+                        dim3 grid, cudaStream_t s) {
+  using Cfg = ql::Fp4Cfg<BN, E8M0>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    QL_CUDA(cudaFuncSetAttribute(ql::fp4_gemm_kernel<BN, E8M0>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+    attr_done[dev] = true;
+  }
+  ql::fp4_gemm_kernel<BN, E8M0><<<grid, 192, Cfg::kSmemBytes, s>>>(tw, tx, a);
+  QL_CUDA(cudaGetLastError());
+  return QL_OK;
+}
+
+template <bool E8M0>
+ql_status launch_fp4(int BN, const CUtensorMap& tw, const CUtensorMap& tx,
+                     const ql::Fp4GemmArgs& a, dim3 grid, cudaStream_t s) {
+  switch (BN) {
+    case 16: return launch_fp4_bn<16, E8M0>(tw, tx, a, grid, s);
+    case 32: return launch_fp4_bn<32, E8M0>(tw, tx, a, grid, s);
+    case 64: return launch_fp4_bn<64, E8M0>(tw, tx, a, grid, s);
+    case 128: return launch_fp4_bn<128, E8M0>(tw, tx, a, grid, s);
+    case 256: return launch_fp4_bn<256, E8M0>(tw, tx, a, grid, s);
+  }
+  return fail(QL_ERR_UNSUPPORTED, "no GEMM tile for BN=%d", BN);
+}
+
+int pick_bn(int64_t M) {
+  for (int bn : {16, 32, 64, 128})
+    if (M <= bn) return bn;
+  return 256;
+}
+
+}  // namespace
+
+// ========================================================================= handles
+struct ql_linear {
+  ql_wformat wfmt;
+  int64_t N, K, C;
+  int32_t k_tail;
+  uint8_t* d_codes = nullptr;  // [N, K/2]
+  uint8_t* d_sf = nullptr;     // tiled scale atoms
+  int sf_atoms = 0;            // atoms per 128-row group of the weight
+  float w_ts = 1.f;
+  CUtensorMap tm_w;
+  int n_base_stages = 0, n_stages_total = 0;
+};
+
+namespace {
+
+struct FwdPlan {
+  int BN, splits, spp, tiles_n, tiles_m;
+  int sfb_atoms;
+  size_t codes_off, sf_off, cnt_off, part_off, total;
+};
+
+FwdPlan plan_forward(const ql_linear* L, int64_t M) {
+  FwdPlan p{};
+  p.BN = pick_bn(M);
+  p.tiles_n = static_cast<int>(cdiv(L->N, 128));
+  p.tiles_m = static_cast<int>(cdiv(std::max<int64_t>(M, 1), p.BN));
+  const int tiles = p.tiles_n * p.tiles_m;
+  const int total = L->n_stages_total;
+  int splits = 1;
+  const int sms = sm_count();
+  if (tiles < sms) splits = std::max(1, std::min(total, sms / tiles));
+  p.spp = static_cast<int>(cdiv(total, splits));
+  p.splits = static_cast<int>(cdiv(total, p.spp));
+  const int atomK = 128;  // E8M0-B32: one 512-byte atom covers 128 K elements
+  p.sfb_atoms = static_cast<int>(cdiv(L->C, atomK));
+  const int64_t rows_pad = cdiv(std::max<int64_t>(M, 1), 256) * 256;
+  size_t off = 0;
+  p.codes_off = off;
+  off = align_up(off + static_cast<size_t>(M) * (L->C / 2), 256);
+  p.sf_off = off;
+  off = align_up(off + static_cast<size_t>(rows_pad / 128) * p.sfb_atoms * 512, 256);
+  p.cnt_off = off;
+  off = align_up(off + static_cast<size_t>(tiles) * sizeof(int), 256);
+  p.part_off = off;
+  if (p.splits > 1) off = align_up(off + static_cast<size_t>(p.splits) * M * L->N * 4, 256);
+  p.total = std::max<size_t>(off, 256);
+  return p;
+}
+
+void repack_sf_tiled(const uint8_t* plain, int64_t rows, int64_t cols, int atoms_per_row,
+                     std::vector<uint8_t>& out) {
+  const int64_t groups = cdiv(rows, 128);
+  out.assign(static_cast<size_t>(groups) * atoms_per_row * 512, 0);
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t j = 0; j < cols; ++j)
+      out[ql::sf_tiled_offset(static_cast<int>(r), static_cast<int>(j), atoms_per_row)] =
+          plain[r * cols + j];
+}
+
+ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
+                          uint8_t* st, int st_atoms, int* zero_words, int nzero,
+                          cudaStream_t s) {
+  const long total = static_cast<long>(M) * (K / 8);
+  const long threads = std::max<long>(total, nzero);
+  if (threads == 0) return QL_OK;
+  const int block = 256;
+  const long grid = (threads + block - 1) / block;
+  ql::quant_mx_e8m0_b32_kernel<<<static_cast<unsigned>(grid), block, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K),
+      static_cast<int>(K), codes, static_cast<int>(K / 2), sp, static_cast<int>(K / 32), st,
+      st_atoms, zero_words, nzero);
+  QL_CUDA(cudaGetLastError());
+  return QL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ql_version(void) { return "qlinear-b200 0.1 (sm_100a)"; }
+const char* ql_last_error(void) { return g_last_error.c_str(); }
+
+ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear** out) {
+  if (d == nullptr || out == nullptr) return fail(QL_ERR_INVALID_ARG, "null descriptor/out");
+  *out = nullptr;
+  if (d->wfmt != QL_W_MXFP4_E8M0_B32)
+    return fail(QL_ERR_UNSUPPORTED, "weight format %d not supported by qlinear_create",
+                int(d->wfmt));
+  if (d->codes == nullptr || d->scales == nullptr)
+    return fail(QL_ERR_INVALID_ARG, "codes/scales must be non-null host pointers");
+  if (d->N <= 0 || d->K <= 0 || d->k_tail < 0 || d->k_tail >= d->K)
+    return fail(QL_ERR_INVALID_ARG, "bad sizes N=%lld K=%lld k_tail=%d", (long long)d->N,
+                (long long)d->K, d->k_tail);
+  if (d->N % 16 != 0 || d->K % 128 != 0 || d->k_tail % 128 != 0)
+    return fail(QL_ERR_UNSUPPORTED, "MXFP4 layer needs N%%16==0, K%%128==0, k_tail%%128==0");
+  if (d->N > (1 << 24) || d->K > (1 << 24))
+    return fail(QL_ERR_UNSUPPORTED, "N/K too large");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto* L = new ql_linear();
+  L->wfmt = d->wfmt;
+  L->N = d->N;
+  L->K = d->K;
+  L->k_tail = d->k_tail;
+  L->C = d->K - d->k_tail;
+  L->sf_atoms = static_cast<int>(cdiv(d->K, 128));
+  L->n_base_stages = static_cast<int>(cdiv(L->C, 256));
+  L->n_stages_total = L->n_base_stages + static_cast<int>(cdiv(L->k_tail, 256));
+  std::vector<uint8_t> sf;
+  repack_sf_tiled(static_cast<const uint8_t*>(d->scales), d->N, d->K / 32, L->sf_atoms, sf);
+  const size_t code_bytes = static_cast<size_t>(d->N) * (d->K / 2);
+  auto cleanup = [&](ql_status st) {
+    if (L->d_codes) cudaFree(L->d_codes);
+    if (L->d_sf) cudaFree(L->d_sf);
+    delete L;
+    return st;
+  };
+  if (cudaMalloc(&L->d_codes, code_bytes) != cudaSuccess ||
+      cudaMalloc(&L->d_sf, sf.size()) != cudaSuccess)
+    return cleanup(fail(QL_ERR_OOM, "cudaMalloc of %zu weight bytes failed", code_bytes + sf.size()));
+  if (cudaMemcpyAsync(L->d_codes, d->codes, code_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(L->d_sf, sf.data(), sf.size(), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return cleanup(fail(QL_ERR_CUDA, "weight upload failed"));
+  ql_status st = make_tmap_u8(&L->tm_w, L->d_codes, d->K / 2, d->N, d->K / 2, 128, 128);
+  if (st != QL_OK) return cleanup(st);
+  *out = L;
+  return QL_OK;
+}
+
+ql_status qlinear_destroy(ql_linear* L) {
+  if (L == nullptr) return QL_OK;
+  if (L->d_codes) cudaFree(L->d_codes);
+  if (L->d_sf) cudaFree(L->d_sf);
+  delete L;
+  return QL_OK;
+}
+
+ql_status qlinear_workspace_bytes(const ql_linear* L, int64_t M, size_t* bytes) {
+  if (L == nullptr || bytes == nullptr || M < 0) return fail(QL_ERR_INVALID_ARG, "bad args");
+  *bytes = plan_forward(L, M).total;
+  return QL_OK;
+}
+
+static ql_status check_ws(const ql_linear* L, int64_t M, void* ws, size_t ws_bytes, FwdPlan* p) {
+  if (L == nullptr || M < 0) return fail(QL_ERR_INVALID_ARG, "null layer or negative M");
+  if (M > (1 << 20)) return fail(QL_ERR_UNSUPPORTED, "M too large");
+  *p = plan_forward(L, M);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0 || ws_bytes < p->total)
+    return fail(QL_ERR_WORKSPACE, "workspace needs %zu bytes, 256-aligned", p->total);
+  return QL_OK;
+}
+
+ql_status qlinear_quantize_input(const ql_linear* L, const void* x, int64_t M, void* ws,
+                                 size_t ws_bytes, ql_stream_t stream) {
+  if (L != nullptr && M == 0) return QL_OK;
+  FwdPlan p;
+  ql_status st = check_ws(L, M, ws, ws_bytes, &p);
+  if (st != QL_OK) return st;
+  if (x == nullptr) return fail(QL_ERR_INVALID_ARG, "null x");
+  if ((reinterpret_cast<uintptr_t>(x) & 15) != 0)
+    return fail(QL_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  return launch_quant_mx(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
+                         reinterpret_cast<int*>(w8 + p.cnt_off), p.tiles_n * p.tiles_m,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void* ws,
+                       size_t ws_bytes, ql_stream_t stream) {
+  if (L != nullptr && M == 0) return QL_OK;
+  FwdPlan p;
+  ql_status st = check_ws(L, M, ws, ws_bytes, &p);
+  if (st != QL_OK) return st;
+  if (y == nullptr) return fail(QL_ERR_INVALID_ARG, "null y");
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  CUtensorMap tm_x;
+  st = make_tmap_u8(&tm_x, w8 + p.codes_off, L->C / 2, M, L->C / 2, 128, p.BN);
+  if (st != QL_OK) return st;
+  ql::Fp4GemmArgs a{};
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(L->N);
+  a.C = static_cast<int>(L->C);
+  a.k_tail = L->k_tail;
+  a.n_base_stages = L->n_base_stages;
+  a.n_stages_total = L->n_stages_total;
+  a.stages_per_split = p.spp;
+  a.sfa = L->d_sf;
+  a.sfa_atoms = L->sf_atoms;
+  a.sfb = w8 + p.sf_off;
+  a.sfb_atoms = p.sfb_atoms;
+  a.alpha_dev = nullptr;
+  a.alpha = 1.f;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.y32 = y32;
+  a.ldy = static_cast<int>(L->N);
+  a.partial = reinterpret_cast<float*>(w8 + p.part_off);
+  a.counters = reinterpret_cast<int*>(w8 + p.cnt_off);
+  dim3 grid(p.tiles_n, p.tiles_m, p.splits);
+  return launch_fp4<true>(p.BN, L->tm_w, tm_x, a, grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ql_status qlinear_forward(const ql_linear* L, const void* x, int64_t M, void* y, float* y32,
+                          void* ws, size_t ws_bytes, ql_stream_t stream) {
+  if (L == nullptr || M < 0) return fail(QL_ERR_INVALID_ARG, "null layer or negative M");
+  if (M == 0) return QL_OK;
+  if (x == nullptr || y == nullptr) return fail(QL_ERR_INVALID_ARG, "null x/y");
+  ql_status st = qlinear_quantize_input(L, x, M, ws, ws_bytes, stream);
+  if (st != QL_OK) return st;
+  return qlinear_gemm(L, M, y, y32, ws, ws_bytes, stream);
+}
+
+ql_status quantize_act(ql_aformat fmt, const void* x, int64_t M, int64_t K, void* codes,
+                       void* scales, float* tensor_scale, ql_stream_t stream) {
+  (void)tensor_scale;
+  if (M < 0 || K < 0) return fail(QL_ERR_INVALID_ARG, "negative size");
+  if (M == 0 || K == 0) return QL_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr)
+    return fail(QL_ERR_INVALID_ARG, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(x) & 15) != 0 || (reinterpret_cast<uintptr_t>(codes) & 3) != 0)
+    return fail(QL_ERR_INVALID_ARG, "x must be 16-byte and codes 4-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (fmt) {
+    case QL_A_MXFP4_E8M0_B32:
+      if (K % 32 != 0) return fail(QL_ERR_UNSUPPORTED, "MXFP4 needs K %% 32 == 0");
+      return launch_quant_mx(x, M, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                             nullptr, 0, nullptr, 0, s);
+    default:
+      return fail(QL_ERR_UNSUPPORTED, "activation format %d not supported", int(fmt));
+  }
+}
+
+ql_status ql_check(ql_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  QL_CUDA(cudaStreamSynchronize(s));
+  int err = 0, site = 0, zero = 0;
+  QL_CUDA(cudaMemcpyFromSymbol(&err, ql::g_dev_error, sizeof(int)));
+  QL_CUDA(cudaMemcpyFromSymbol(&site, ql::g_dev_error_site, sizeof(int)));
+  if (err != 0) {
+    QL_CUDA(cudaMemcpyToSymbol(ql::g_dev_error, &zero, sizeof(int)));
+    return fail(QL_ERR_TIMEOUT, "device wait expired (code %d, site %d)", err, site);
+  }
+  return QL_OK;
+}
+
+}  // extern "C"

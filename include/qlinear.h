@@ -1,0 +1,152 @@
+/*
+ * qlinear.h -- C ABI of libqlinear: a W4A4 quantized linear layer y = X W^T for NVIDIA B200
+ * (sm_100a), with block-scaled FP4 weights (E8M0-B32 or E4M3-B16 scales), PRQuant tail-block
+ * residuals, MXCode VQ codebook weights, CodeQuant-style cluster-codebook MoE experts and
+ * MosaicQuant-style INT4 dense + block-sparse weights.
+ *
+ * Sources of the operations (page title, section / table):
+ *   - MXCode (MX-Native Codebook Quantization), Table 1: the block-scaled FP4 formats
+ *     (E2M1 elements; E8M0 scales per 32, or E4M3 scales per 16 plus an FP32 tensor scale).
+ *   - PRQuant: Permutation Residual Quantization, §4 Method, "Kernel design for efficient
+ *     inference": one MXFP4 GEMM whose reduction is extended from C to C + k by an offline
+ *     weight residual on the permuted tail channels; the activation is quantized once and its
+ *     quantized tail reused.
+ *   - MXCode abstract: reconstruct MX-native W4A4 operands from VQ indices and FP4 codebooks
+ *     without materialising high-precision weights.
+ *   - CodeQuant, Figure 4: per-tile lookup table kept in SM shared memory.
+ *   - MosaicQuant, "ZipperEngine": dense INT4 base and sparse INT4 residual fused into one GEMM.
+ *
+ * Conventions
+ *   - All matrices are row-major.  Activations are bf16 [M, K] (token-major); outputs are bf16
+ *     [M, N] (optionally also fp32).  "Device" pointers must be CUDA device memory of the
+ *     current device; "host" pointers are ordinary CPU memory.
+ *   - FP4 codes are packed two per byte, element 2j in the low nibble of byte j; bit 3 of a
+ *     code is its sign.  E8M0 scale bytes hold exponent + 127.  E4M3 scales are OCP FP8 E4M3.
+ *   - Calls that take a cudaStream_t are asynchronous and never synchronise the stream; the
+ *     caller keeps every device buffer alive until the stream has run the work.
+ *   - Every call returns a ql_status.  Argument and shape checks happen before any launch and
+ *     leave device memory untouched.  ql_last_error() gives a thread-local message for the
+ *     last non-OK status.  Kernels whose bounded waits expire set a device error word that
+ *     ql_check() reports (QL_ERR_TIMEOUT); they never trap.  No call falls back to the CPU.
+ */
+#ifndef QLINEAR_H_
+#define QLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ql_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent descriptor */
+  QL_ERR_UNSUPPORTED = 2, /* shape outside what the kernels implement (see each call) */
+  QL_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  QL_ERR_OOM = 4,         /* device allocation failed (create calls only) */
+  QL_ERR_TIMEOUT = 5,     /* a kernel's bounded wait expired (reported by ql_check) */
+  QL_ERR_WORKSPACE = 6    /* workspace pointer null/misaligned or smaller than required */
+} ql_status;
+
+typedef enum {
+  QL_W_MXFP4_E8M0_B32 = 1,       /* codes [N,K/2] + E8M0 bytes [N,K/32]; optional PRQuant tail */
+  QL_W_NVFP4_E4M3_B16 = 2,       /* codes [N,K/2] + E4M3 bytes [N,K/16] + fp32 tensor scale */
+  QL_W_VQ_PRESCALE_E4M3_B16 = 3, /* MXCode PreScale: uint8 indices [N,K/4] into per-QBlock
+                                    codebooks of 256 x 4 E2M1 codes, E4M3 bytes [N,K/16],
+                                    fp32 tensor scale */
+  QL_W_CLUSTER4_ROW16_BF16 = 4,  /* CodeQuant-style: 4-bit indices [N,K/2] into 16 bf16
+                                    centroids per output row */
+  QL_W_INT4_G128_BSR = 5         /* INT4 codes [N,K/2] + fp16 scale per (row,128-group), plus a
+                                    block-sparse INT4 residual on 16x128 blocks (BSR) */
+} ql_wformat;
+
+typedef enum {
+  QL_A_MXFP4_E8M0_B32 = 1,  /* codes [M,K/2] + E8M0 bytes [M,K/32] */
+  QL_A_FP4_E4M3_B16_TS = 2, /* codes [M,K/2] + E4M3 bytes [M,K/16] + fp32 tensor scale */
+  QL_A_INT4_TOK_G128 = 3    /* int4 codes [M,K/2] + fp32 scale per (token,128-group) */
+} ql_aformat;
+
+/* Weight description.  Every array pointer is HOST memory; *_create copies and repacks it. */
+typedef struct ql_weight_desc {
+  ql_wformat wfmt;
+  int64_t N;          /* output features */
+  int64_t K;          /* reduction width of the weight (includes k_tail) */
+  int32_t k_tail;     /* PRQuant: width of the residual K-extension (0 = none); the activation
+                         has K - k_tail channels and its last k_tail channels are reused */
+  const void* codes;  /* packed 4-bit codes (FP4 or INT4) [N, K/2]; cluster indices for fmt 4 */
+  const void* scales; /* E8M0 [N,K/32] | E4M3 [N,K/16] | fp16 [N,K/128] (INT4) */
+  float w_tensor_scale;       /* E4M3-B16 formats: FP32 tensor scale of W (else ignored) */
+  const uint8_t* indices;     /* VQ: [N, K/4] */
+  const void* codebooks;      /* VQ: uint8 [N/qn][K/qk][256][2] (4 packed E2M1 per entry);
+                                 cluster: bf16 [N][16] */
+  int32_t qblock_n, qblock_k; /* VQ QBlock shape (64 x 64) */
+  const int32_t* bsr_rowptr;  /* INT4 residual: [N/bsr_block_n + 1] */
+  const int16_t* bsr_col;     /* [nnzb] 128-group index of each block */
+  const void* bsr_codes;      /* [nnzb][bsr_block_n][bsr_block_k/2] int4 */
+  const void* bsr_scales;     /* [nnzb][bsr_block_n] fp16 */
+  int32_t bsr_block_n, bsr_block_k, bsr_nnzb;
+} ql_weight_desc;
+
+typedef struct ql_linear ql_linear;
+typedef struct ql_moe ql_moe;
+
+/* Version and device queries. */
+const char* ql_version(void);
+const char* ql_last_error(void);
+
+/* Create a linear layer: validates the descriptor, copies the weights to device memory owned
+ * by the returned handle and repacks scales into the tiled layout the MMA consumes.
+ * Supported: QL_W_MXFP4_E8M0_B32 with N % 16 == 0, K % 128 == 0, k_tail % 128 == 0,
+ * 0 <= k_tail < K.  Synchronous with respect to `stream` (uses it for the uploads). */
+ql_status qlinear_create(const ql_weight_desc* desc, ql_stream_t stream, ql_linear** out);
+ql_status qlinear_destroy(ql_linear* layer);
+
+/* Bytes of device workspace that qlinear_forward needs for M tokens. */
+ql_status qlinear_workspace_bytes(const ql_linear* layer, int64_t M, size_t* bytes);
+
+/* y[M,N] = X[M, K-k_tail] (quantized online) times the layer's weight.  x_bf16, y_bf16 and
+ * the workspace are device pointers; y_f32 (device, [M,N]) may be NULL.  ws must be 256-byte
+ * aligned and at least qlinear_workspace_bytes(M) long; its contents on entry do not matter.
+ * Rows of x are contiguous (row stride K - k_tail elements).  M may be 0 (no-op). */
+ql_status qlinear_forward(const ql_linear* layer, const void* x_bf16, int64_t M, void* y_bf16,
+                          float* y_f32, void* ws, size_t ws_bytes, ql_stream_t stream);
+
+/* The two halves of qlinear_forward.  qlinear_quantize_input quantizes x into the workspace
+ * (MXFP4 codes and tiled scales; it also clears the GEMM's split-K tickets); qlinear_gemm runs
+ * the tcgen05 GEMM from that workspace.  Called in this order on one stream with the same M and
+ * workspace they equal qlinear_forward.  A caller whose several layers share one input (gate and
+ * up projections, say) can quantize once; the split also lets a profiler time the GEMM alone. */
+ql_status qlinear_quantize_input(const ql_linear* layer, const void* x_bf16, int64_t M, void* ws,
+                                 size_t ws_bytes, ql_stream_t stream);
+ql_status qlinear_gemm(const ql_linear* layer, int64_t M, void* y_bf16, float* y_f32, void* ws,
+                       size_t ws_bytes, ql_stream_t stream);
+
+/* Online activation quantization (device pointers).
+ * QL_A_MXFP4_E8M0_B32: K % 32 == 0; codes [M,K/2], scales E8M0 [M,K/32]; tensor_scale unused.
+ * Rule (OCP MX, as the PRQuant page applies it): per 32 elements e = floor(log2 amax) - 2
+ * clamped to [-127,127], byte e+127 (0 for an all-zero block), code = E2M1 RNE of x/2^e with
+ * saturation at +-6 and the sign of x. */
+ql_status quantize_act(ql_aformat fmt, const void* x_bf16, int64_t M, int64_t K, void* codes,
+                       void* scales, float* tensor_scale, ql_stream_t stream);
+
+/* Synchronise `stream` and report (then clear) the device error word. */
+ql_status ql_check(ql_stream_t stream);
+
+/* ---- Offline weight preparation (host memory, CPU; not on the forward path) ----------------
+ * PRQuant, §4 "Offline scaling and channel reordering" / "Offline residual augmentation", with
+ * the AWQ scaling taken as identity: MXFP4-quantize W (bf16 [N,C]) along C; per input channel
+ * sum over rows of the squared quantization error; the k largest (ties to the lower index)
+ * become the tail; perm lists the kept channels then the tail channels, each ascending;
+ * W~ = W[:, perm] is re-quantized; R = W~[:, C-k:] - deq(Q(W~))[:, C-k:] is quantized; the
+ * outputs are perm [C] (int32), codes [N,(C+k)/2] and E8M0 bytes [N,(C+k)/32] of Q([W~, R]).
+ * Requires C % 128 == 0, k % 128 == 0, 0 < k <= C. */
+ql_status qlinear_prepare_prquant(const uint16_t* w_bf16, int64_t N, int64_t C, int32_t k,
+                                  int32_t* perm_out, uint8_t* codes_out, uint8_t* scales_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLINEAR_H_ */

@@ -29,15 +29,19 @@ def e2m1_encode(v: np.ndarray) -> np.ndarray:
     zero (and -0.0) give code 0x8.  Input must be finite.
     """
     v = np.asarray(v, dtype=np.float64)
-    a = np.minimum(np.abs(v), 6.0)                         # saturate at the largest magnitude
-    d = np.abs(a[..., None] - E2M1_MAGNITUDES)            # distance to each magnitude
-    best = d.min(axis=-1, keepdims=True)
-    tied = d == best
-    # among the nearest magnitudes prefer an even code; codes ascend with magnitude
-    even = tied & ((np.arange(8) & 1) == 0)
-    code = np.where(even.any(-1), even.argmax(-1), tied.argmax(-1)).astype(np.uint8)
-    sign = np.signbit(v).astype(np.uint8) << 3
-    return (code | sign).astype(np.uint8)
+    out = np.empty(v.shape, dtype=np.uint8)
+    flat, res = v.reshape(-1), out.reshape(-1)
+    step = 1 << 20                                         # bounded temporaries
+    for i in range(0, flat.size, step):
+        c = flat[i:i + step]
+        a = np.minimum(np.abs(c), 6.0)                     # saturate at the largest magnitude
+        d = np.abs(a[:, None] - E2M1_MAGNITUDES)           # distance to each magnitude
+        tied = d == d.min(axis=-1, keepdims=True)
+        # among the nearest magnitudes prefer an even code; codes ascend with magnitude
+        even = tied & ((np.arange(8) & 1) == 0)
+        code = np.where(even.any(-1), even.argmax(-1), tied.argmax(-1)).astype(np.uint8)
+        res[i:i + step] = code | (np.signbit(c).astype(np.uint8) << 3)
+    return out
 
 
 def pack_nibbles(codes: np.ndarray) -> np.ndarray:

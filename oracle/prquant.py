@@ -19,10 +19,14 @@ from . import mx
 
 
 def column_errors(w: np.ndarray) -> np.ndarray:
-    """Per input channel: sum over output rows of (w - deq Q(w))^2, float64."""
+    """Per input channel: sum over output rows of (w - deq Q(w))^2, float64, accumulated in row
+    order n = 0, 1, ... (a fixed order, so the top-k choice is reproducible to the last bit)."""
     codes, sb = mx.quantize_e8m0_b32(w)
     d = w - mx.dequant_e8m0_b32(codes, sb)
-    return (d * d).sum(axis=0)
+    acc = np.zeros(w.shape[1])
+    for n in range(w.shape[0]):
+        acc += d[n] * d[n]
+    return acc
 
 
 def select_tail(err: np.ndarray, k: int) -> np.ndarray:

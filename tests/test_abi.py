@@ -1,0 +1,60 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry point that
+include/qlinear.h declares, rejects bad arguments before touching the device, and its host-side
+offline preparation matches the oracle bit for bit (CPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from tests.conftest import ROOT
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "qlinear.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "defined")))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    import bit_quantized_moe_tcgen05_b200 as ql
+    declared = _declared_functions()
+    assert len(declared) >= 9
+    for name in declared:
+        assert hasattr(ql.lib, name), f"{name} declared in qlinear.h but not exported"
+    assert set(declared) == set(ql.EXPORTED_SYMBOLS)
+    assert b"sm_100a" in ql.lib.ql_version()
+
+
+def test_bad_arguments_rejected_without_device():
+    import bit_quantized_moe_tcgen05_b200 as ql
+    h = ctypes.c_void_p()
+    assert ql.lib.qlinear_create(None, None, ctypes.byref(h)) == 1
+    codes = np.zeros((16, 64), np.uint8)
+    scales = np.zeros((16, 4), np.uint8)
+    d = ql.WeightDesc(wfmt=1, N=16, K=100, k_tail=0, codes=codes.ctypes.data, scales=scales.ctypes.data)
+    assert ql.lib.qlinear_create(ctypes.byref(d), None, ctypes.byref(h)) == 2      # K % 128
+    d = ql.WeightDesc(wfmt=1, N=16, K=128, k_tail=128, codes=codes.ctypes.data, scales=scales.ctypes.data)
+    assert ql.lib.qlinear_create(ctypes.byref(d), None, ctypes.byref(h)) == 1      # k_tail >= K
+    d = ql.WeightDesc(wfmt=1, N=16, K=128, k_tail=0, codes=None, scales=None)
+    assert ql.lib.qlinear_create(ctypes.byref(d), None, ctypes.byref(h)) == 1
+    assert b"codes" in ql.lib.ql_last_error()
+    assert ql.lib.quantize_act(1, None, 4, 32, None, None, None, None) == 1
+    assert ql.lib.quantize_act(1, None, 0, 32, None, None, None, None) == 0        # empty is a no-op
+
+
+@pytest.mark.parametrize("N,C,k", [(32, 512, 128), (64, 1024, 256)])
+def test_prquant_host_preparation_matches_oracle(N, C, k):
+    import bit_quantized_moe_tcgen05_b200 as ql
+    from oracle import formats as F, prquant
+    wb = synth.to_bf16_bits(synth.student_t(11 + N, (N, C), 3.0))
+    perm, codes, scales = ql.prepare_prquant(wb, k)
+    ref = prquant.prepare(synth.bf16_bits_to_f64(wb), k)
+    assert np.array_equal(perm, ref["perm"])
+    assert np.array_equal(codes, F.pack_nibbles(ref["w_codes"]))
+    assert np.array_equal(scales, ref["w_sb"])
