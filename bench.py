@@ -194,7 +194,6 @@ def run_case(w, steps: int, warmup: int, device, flush, e2e: bool = False):
 def cpu_baseline(w, budget_s: float = 15.0) -> dict:
     """The oracle as it stands (numpy, fp64) on a bounded sample of the same workload: the first
     m_s tokens through quantize + augmented GEMM against the full weight."""
-    import threading
     from oracle import formats as F, mx, gemm as G
     import synth
     N, C, k = w["N"], w["C"], w["k"]
@@ -220,7 +219,7 @@ def cpu_baseline(w, budget_s: float = 15.0) -> dict:
     cores = len(os.sched_getaffinity(0))
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{m_s} of {w['M']} tokens of {w['name']} (quantize + fp64 GEMM incl. weight "
-                      f"dequant), {dt:.2f} s, numpy/BLAS threads={threading.active_count()}"}
+                      f"dequant), {dt:.2f} s; numpy BLAS may use every core"}
 
 
 def main():
@@ -231,6 +230,9 @@ def main():
     ap.add_argument("--impl", default="qlinear", choices=["qlinear", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cases", default="all", choices=["all", "headline"])
+    ap.add_argument("--workload", default="prquant_m2048",
+                    choices=["prquant_m2048", "prquant_m512", "prquant_m16", "mxfp4_m16"],
+                    help="headline workload (default: the PRQuant prefill case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -239,7 +241,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    head = prquant_workload(2048)
+    head = {"prquant_m2048": lambda: prquant_workload(2048),
+            "prquant_m512": lambda: prquant_workload(512),
+            "prquant_m16": lambda: prquant_workload(16),
+            "mxfp4_m16": lambda: mxfp4_workload(16)}[args.workload]()
     wk = work_of(head)
 
     if args.impl == "reference":
@@ -250,8 +255,9 @@ def main():
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": wk["flops"] / (cb["value"] * 1e12) * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": head["name"], "M": 2048, "N": 2560,
-                                                "K_aug": 9856, "parallelism": "replicas"},
+                "data": "synthetic", "config": {"workload": head["name"], "M": head["M"],
+                                                "N": head["N"], "K_aug": head["C"] + head["k"],
+                                                "parallelism": "replicas"},
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -296,7 +302,7 @@ def main():
     gemm_tflops = wk["flops"] / (res["gemm_ms"] * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": gemm_tflops / fp4_peak, "traffic": None,
-                "kernel": "fp4_gemm_kernel<256,E8M0> (tcgen05.mma kind::mxf4 block32)",
+                "kernel": "fp4_gemm_kernel (tcgen05.mma kind::mxf4 block32)",
                 "peak_source": f"{peaks['src']} bf16 burst {peaks['bf16']} x {NOMINAL_FP4_OVER_BF16}"
                                " (nominal FP4/bf16 dense ratio)"}
 
@@ -324,8 +330,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp4-e2m1/e8m0 (fp32 accumulate, bf16 out)",
         "data": "synthetic",
-        "config": {"workload": head["name"], "M": 2048, "N": 2560, "K": 9728, "k_tail": 128,
-                   "K_aug": 9856, "parallelism": "replicas" if world > 1 else "single",
+        "config": {"workload": head["name"], "M": head["M"], "N": head["N"], "K": head["C"],
+                   "k_tail": head["k"], "K_aug": head["C"] + head["k"],
+                   "parallelism": "replicas" if world > 1 else "single",
                    "l2": "flushed between steps (256 MiB write)"},
         "roofline": roofline,
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": res["h2d"],
