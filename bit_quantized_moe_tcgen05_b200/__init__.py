@@ -31,7 +31,7 @@ _STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED", 3: "QL_
 EXPORTED_SYMBOLS = (
     "ql_version", "ql_last_error", "qlinear_create", "qlinear_destroy", "qlinear_workspace_bytes",
     "qlinear_forward", "quantize_act", "ql_check", "qlinear_prepare_prquant",
-    "qlinear_quantize_input", "qlinear_gemm",
+    "qlinear_quantize_input", "qlinear_gemm", "qlinear_forward_fixed_scratch",
 )
 
 
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "qlinear_forward": [vp, vp, i64, vp, vp, vp, sz, vp],
         "qlinear_quantize_input": [vp, vp, i64, vp, sz, vp],
         "qlinear_gemm": [vp, i64, vp, vp, vp, sz, vp],
+        "qlinear_forward_fixed_scratch": [vp, vp, i64, vp, vp, vp],
         "quantize_act": [ctypes.c_int, vp, i64, i64, vp, vp, vp, vp],
         "ql_check": [vp],
         "qlinear_prepare_prquant": [vp, i64, i64, i32, vp, vp, vp],
@@ -170,6 +171,22 @@ class QLinear:
         return out
 
     __call__ = forward
+
+    def forward_fixed_scratch(self, x, out=None, out_f32=None, stream=None):
+        """forward() without a workspace: the library's own fixed 8 MiB scratch is used, so
+        nothing is allocated on the device (for callers that may not allocate).  Calls that can
+        overlap on the GPU share that scratch and must be serialised by the caller."""
+        import torch
+        assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+        M, C = x.shape
+        if C != self.C:
+            raise ValueError(f"x has {C} channels, layer expects {self.C}")
+        if out is None:
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device)
+        _ok(lib.qlinear_forward_fixed_scratch(self._h, x.data_ptr(), M, out.data_ptr(),
+                                              _ptr(out_f32), _stream(stream)),
+            "qlinear_forward_fixed_scratch")
+        return out
 
     def quantize_input(self, x, ws, stream=None) -> None:
         """First half of forward: quantize x into the workspace ``ws``."""

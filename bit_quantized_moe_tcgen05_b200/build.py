@@ -10,7 +10,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqlinear.so")
-SOURCES = [os.path.join(CSRC, "qlinear.cu"), os.path.join(CSRC, "prep.cpp")]
+SOURCES = [os.path.join(CSRC, "qlinear.cu"), os.path.join(CSRC, "noalloc.cu"),
+           os.path.join(CSRC, "prep.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, "qlinear.h")]
 

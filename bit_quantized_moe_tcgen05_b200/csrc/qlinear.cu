@@ -364,3 +364,9 @@ ql_status ql_check(ql_stream_t stream) {
 }
 
 }  // extern "C"
+
+// Sets the message that ql_last_error() returns on this thread and passes the status through
+// (used by entry points that live in other source files of the library).
+ql_status ql_set_error(ql_status status, const char* message) {
+  return fail(status, "%s", message);
+}

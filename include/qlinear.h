@@ -124,6 +124,22 @@ ql_status qlinear_quantize_input(const ql_linear* layer, const void* x_bf16, int
 ql_status qlinear_gemm(const ql_linear* layer, int64_t M, void* y_bf16, float* y_f32, void* ws,
                        size_t ws_bytes, ql_stream_t stream);
 
+/* qlinear_forward without a caller-supplied workspace, for callers that cannot allocate device
+ * memory (an engine that plans all device memory ahead and forbids allocation during a forward,
+ * a plugin whose host exposes no allocator, a latency-critical loop that must not enter the
+ * allocator).  The paper has no counterpart to this call; it is a packaging convenience.
+ * The workspace is a fixed 8 MiB array inside the library (each GPU that loads the library keeps
+ * it until the process exits); M whose qlinear_workspace_bytes exceeds 8 MiB is rejected with
+ * QL_ERR_WORKSPACE.  Nothing is allocated: no cudaMalloc/cudaFree, no library allocator.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress with that
+ * device current); make that first call before any stream capture.  All calls share the one
+ * array, which keeps whatever the last call left in it (the parts that must start at zero are
+ * cleared by each call): calls that may overlap on the GPU (different streams, or different host
+ * threads) race on it and must be serialised by the caller.  x, y and y_f32 are device pointers
+ * as for qlinear_forward. */
+ql_status qlinear_forward_fixed_scratch(const ql_linear* layer, const void* x_bf16, int64_t M,
+                                        void* y_bf16, float* y_f32, ql_stream_t stream);
+
 /* Online activation quantization (device pointers).
  * QL_A_MXFP4_E8M0_B32: K % 32 == 0; codes [M,K/2], scales E8M0 [M,K/32]; tensor_scale unused.
  * Rule (OCP MX, as the PRQuant page applies it): per 32 elements e = floor(log2 amax) - 2
