@@ -2,7 +2,8 @@
 """Benchmark of the W4A4 quantized linear layer on B200.
 
 One step = one pass of the layer's hot path over one batch: online MXFP4 quantization of the
-activation, then the tcgen05 block-scaled FP4 GEMM with the PRQuant tail K-extension, on the
+activation, then the tcgen05 block-scaled FP4 GEMM with the PRQuant tail K-extension (the two
+launches replayed from a CUDA graph, as a serving loop would issue them), on the
 PRQuant tail-residual workload (W [2560, 9728] -> K' = 9856, M = 2048 tokens, the prefill case).
 `value` is whole-job TFLOP/s (2*M*N*K' per step over all ranks), timed with CUDA events on the
 device with inputs resident; `e2e` is the same through the C ABI from pinned host buffers.
@@ -133,8 +134,25 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------ GPU arm
+def _time_graph(graph, steps: int, flush, stream) -> float:
+    """Mean device time (ms) of `steps` replays of a captured graph, L2 flushed before each."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        flush()
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
 def run_case(w, steps: int, warmup: int, device, flush, e2e: bool = False):
-    """Times `steps` forwards.  Returns per-step and per-kernel device times (ms)."""
+    """Times `steps` forwards (quantize + GEMM) replayed from CUDA graphs, so the numbers are
+    device time without host launch gaps.  Also times each kernel alone the same way, and (e2e)
+    the public forward call from pinned host memory with the copies inside the timed region."""
     import torch
     import bit_quantized_moe_tcgen05_b200 as ql
     lin = ql.QLinear(w["codes"], w["scales"], k_tail=w["k"])
@@ -142,27 +160,28 @@ def run_case(w, steps: int, warmup: int, device, flush, e2e: bool = False):
     x = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).to(device)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
     ws = torch.empty(lin.workspace_bytes(M), dtype=torch.uint8, device=device)
+    for _ in range(warmup):                       # eager warm-up (also sets kernel attributes)
+        lin.quantize_input(x, ws)
+        lin.gemm(M, y, ws)
+    ql.check()
+    g_step, g_q, g_g = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        lin.quantize_input(x, ws)
+        lin.gemm(M, y, ws)
+    with torch.cuda.graph(g_q):
+        lin.quantize_input(x, ws)
+    with torch.cuda.graph(g_g):
+        lin.gemm(M, y, ws)
     stream = torch.cuda.current_stream(device)
-    for _ in range(warmup):
-        lin.quantize_input(x, ws)
-        lin.gemm(M, y, ws)
+    for g in (g_step, g_q, g_g):
+        for _ in range(warmup):
+            g.replay()
     ql.check()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    torch.cuda.synchronize(device)
-    for i in range(steps):
-        flush()
-        ev[i][0].record(stream)
-        lin.quantize_input(x, ws)
-        ev[i][1].record(stream)
-        lin.gemm(M, y, ws)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize(device)
+    step_ms = _time_graph(g_step, steps, flush, stream)
+    q_ms = _time_graph(g_q, steps, flush, stream)
+    g_ms = _time_graph(g_g, steps, flush, stream)
     ql.check()
-    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(steps)]
-    q_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)]
-    g_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(steps)]
-    out = dict(step_ms=float(np.mean(step_ms)), quant_ms=float(np.mean(q_ms)),
-               gemm_ms=float(np.mean(g_ms)), launches=2 * steps)
+    out = dict(step_ms=step_ms, quant_ms=q_ms, gemm_ms=g_ms, launches=2 * steps)
     if e2e:
         xh = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
         yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
@@ -187,6 +206,7 @@ def run_case(w, steps: int, warmup: int, device, flush, e2e: bool = False):
         out["h2d"] = M * w["C"] * 2
         out["d2h"] = M * N * 2
         out["launches"] += 2 * steps
+    del g_step, g_q, g_g
     lin.close()
     return out
 

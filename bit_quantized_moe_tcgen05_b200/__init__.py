@@ -32,6 +32,7 @@ EXPORTED_SYMBOLS = (
     "ql_version", "ql_last_error", "qlinear_create", "qlinear_destroy", "qlinear_workspace_bytes",
     "qlinear_forward", "quantize_act", "ql_check", "qlinear_prepare_prquant",
     "qlinear_quantize_input", "qlinear_gemm", "qlinear_forward_fixed_scratch",
+    "qlinear_prepare_vq_prescale",
 )
 
 
@@ -74,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "quantize_act": [ctypes.c_int, vp, i64, i64, vp, vp, vp, vp],
         "ql_check": [vp],
         "qlinear_prepare_prquant": [vp, i64, i64, i32, vp, vp, vp],
+        "qlinear_prepare_vq_prescale": [vp, i64, i64, vp, i32, i32, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -106,18 +108,25 @@ def check(stream=None) -> None:
 
 
 def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None):
-    """Quantize bf16 activations [M, K] on the GPU.  Returns (codes uint8 [M, K/2],
-    scales uint8 [M, K/32]) for MXFP4 E8M0-B32."""
+    """Quantize bf16 activations [M, K] on the GPU.
+    MXFP4 E8M0-B32 -> (codes uint8 [M, K/2], E8M0 scales uint8 [M, K/32]);
+    E4M3-B16 + tensor scale -> (codes, E4M3 scales uint8 [M, K/16], ts float32 [1])."""
     import torch
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
     M, K = x.shape
-    if fmt != QL_A_MXFP4_E8M0_B32:
-        raise ValueError("only QL_A_MXFP4_E8M0_B32 is exposed here")
     codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
-    scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
-    _ok(lib.quantize_act(fmt, x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), None,
-                         _stream(stream)), "quantize_act")
-    return codes, scales
+    if fmt == QL_A_MXFP4_E8M0_B32:
+        scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
+        _ok(lib.quantize_act(fmt, x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), None,
+                             _stream(stream)), "quantize_act")
+        return codes, scales
+    if fmt == QL_A_FP4_E4M3_B16_TS:
+        scales = torch.empty((M, K // 16), dtype=torch.uint8, device=x.device)
+        ts = torch.empty(1, dtype=torch.float32, device=x.device)
+        _ok(lib.quantize_act(fmt, x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(),
+                             ts.data_ptr(), _stream(stream)), "quantize_act")
+        return codes, scales, ts
+    raise ValueError(f"activation format {fmt} not exposed")
 
 
 class QLinear:
@@ -129,15 +138,32 @@ class QLinear:
     has K - k_tail channels.
     """
 
-    def __init__(self, codes: np.ndarray, scales: np.ndarray, k_tail: int = 0,
-                 wfmt: int = QL_W_MXFP4_E8M0_B32, stream=None):
-        codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    def __init__(self, codes: np.ndarray | None, scales: np.ndarray, k_tail: int = 0,
+                 wfmt: int = QL_W_MXFP4_E8M0_B32, w_tensor_scale: float = 1.0,
+                 indices: np.ndarray | None = None, codebooks: np.ndarray | None = None,
+                 stream=None):
+        """MXFP4: codes [N, K/2] + E8M0 scales [N, K/32] (+ k_tail).  NVFP4 (E4M3-B16): codes +
+        E4M3 scales [N, K/16] + w_tensor_scale.  VQ PreScale: indices [N, K/4] + packed codebooks
+        [N/64, K/64, 256, 2] + E4M3 scales [N, K/16] + w_tensor_scale (codes = None)."""
         scales = np.ascontiguousarray(scales, dtype=np.uint8)
-        N, half_k = codes.shape
-        self.N, self.K, self.k_tail = N, 2 * half_k, int(k_tail)
+        keep = [scales]
+        if wfmt == QL_W_VQ_PRESCALE_E4M3_B16:
+            indices = np.ascontiguousarray(indices, dtype=np.uint8)
+            codebooks = np.ascontiguousarray(codebooks, dtype=np.uint8)
+            N, K = indices.shape[0], 4 * indices.shape[1]
+            keep += [indices, codebooks]
+            cptr, iptr, cbptr = None, indices.ctypes.data, codebooks.ctypes.data
+        else:
+            codes = np.ascontiguousarray(codes, dtype=np.uint8)
+            N, K = codes.shape[0], 2 * codes.shape[1]
+            keep.append(codes)
+            cptr, iptr, cbptr = codes.ctypes.data, None, None
+        self.N, self.K, self.k_tail = N, K, int(k_tail)
         self.C = self.K - self.k_tail
-        d = WeightDesc(wfmt=wfmt, N=N, K=self.K, k_tail=self.k_tail,
-                       codes=codes.ctypes.data, scales=scales.ctypes.data)
+        self.wfmt = wfmt
+        d = WeightDesc(wfmt=wfmt, N=N, K=self.K, k_tail=self.k_tail, codes=cptr,
+                       scales=scales.ctypes.data, w_tensor_scale=float(w_tensor_scale),
+                       indices=iptr, codebooks=cbptr, qblock_n=64, qblock_k=64)
         h = ctypes.c_void_p()
         _ok(lib.qlinear_create(ctypes.byref(d), _stream(stream), ctypes.byref(h)), "qlinear_create")
         self._h = h
@@ -222,3 +248,19 @@ def prepare_prquant(w_bf16_bits: np.ndarray, k: int):
     _ok(lib.qlinear_prepare_prquant(w.ctypes.data, N, C, k, perm.ctypes.data, codes.ctypes.data,
                                     scales.ctypes.data), "qlinear_prepare_prquant")
     return perm, codes, scales
+
+
+def prepare_vq_prescale(w_bf16_bits: np.ndarray, codebooks_packed: np.ndarray, qn: int = 64,
+                        qk: int = 64):
+    """Offline MXCode PreScale preparation on the host (library C++ code).  codebooks_packed:
+    uint8 [N/qn, K/qk, 256, 2].  Returns (ts float, E4M3 scales uint8 [N, K/16], idx uint8 [N, K/4])."""
+    w = np.ascontiguousarray(w_bf16_bits, dtype=np.uint16)
+    cb = np.ascontiguousarray(codebooks_packed, dtype=np.uint8)
+    N, K = w.shape
+    ts = np.zeros(1, np.float32)
+    scales = np.empty((N, K // 16), np.uint8)
+    idx = np.empty((N, K // 4), np.uint8)
+    _ok(lib.qlinear_prepare_vq_prescale(w.ctypes.data, N, K, cb.ctypes.data, qn, qk, ts.ctypes.data,
+                                        scales.ctypes.data, idx.ctypes.data),
+        "qlinear_prepare_vq_prescale")
+    return np.float32(ts[0]), scales, idx

@@ -13,7 +13,11 @@
 // the weight coordinate is C + j).  No tail copy is materialised.
 //
 // Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + single-thread
-// MMA issuer, warps 2..5 = epilogue (TMEM -> registers -> global).  A STAGES-deep ring of
+// MMA issuer, warps 2..5 = epilogue (TMEM -> registers -> global).  Split-K (decode): the
+// gridDim.z K-splits of one output tile form a thread-block cluster; each CTA parks its fp32
+// partial tile in its own (now idle) operand ring; then each rank sums a share of the token
+// columns over distributed shared memory, adding the ranks in rank order, so the reduction is
+// deterministic and never leaves the chip.  A STAGES-deep ring of
 // shared-memory stages, each 256 K-elements deep, is guarded by full/empty mbarriers; MMA
 // completion is signalled by tcgen05.commit.  Every wait is bounded (see ptx.cuh).
 #pragma once
@@ -21,6 +25,9 @@
 #include "ptx.cuh"
 
 namespace ql {
+
+// Largest cluster of K-splits: bigger clusters co-schedule poorly (few fit on the GPU at once).
+constexpr int kMaxClusterSplits = 4;
 
 struct Fp4GemmArgs {
   int M, N;                 // tokens, output features
@@ -37,11 +44,11 @@ struct Fp4GemmArgs {
   __nv_bfloat16* y;         // [M, ldy] bf16 output
   float* y32;               // optional [M, ldy] fp32 output
   int ldy;
-  float* partial;           // split-K partials [splits][M][N] (splits > 1)
-  int* counters;            // split-K tickets, one per (n-tile, m-tile); zero on entry
+  const uint8_t* lut;       // VQ: packed E2M1 codebooks [N/64][K/64][256][2]
+  int lut_qc;               // VQ: QBlocks along K (K / 64)
 };
 
-template <int BN, bool E8M0>
+template <int BN, bool E8M0, bool VQ = false>
 struct Fp4Cfg {
   static constexpr int kAtomK = E8M0 ? 128 : 64;      // K elements covered by one SF atom
   static constexpr int kAtoms = 256 / kAtomK;         // SF atoms per stage per 128 rows
@@ -50,8 +57,11 @@ struct Fp4Cfg {
   static constexpr int kBBytes = BN * 128;
   static constexpr int kSfaBytes = kAtoms * 512;
   static constexpr int kSfbBytes = kAtoms * kG * 512;
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  static constexpr int kIdxBytes = VQ ? 128 * 64 : 0;   // VQ: 8-bit indices, 128 rows x 64
+  static constexpr int kLutBytes = VQ ? 8 * 512 : 0;    // VQ: 2 x 4 QBlock codebooks of 512 B
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kIdxBytes + kLutBytes;
+  static constexpr int kBudget = (BN <= 64 && !VQ) ? 100 * 1024 : 212 * 1024;
+  static constexpr int kStagesRaw = kBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : (kStagesRaw < 2 ? 2 : kStagesRaw);
   static constexpr int kSfaCols = kAtoms * 4;          // TMEM columns per stage
   static constexpr int kSfbCols = kAtoms * 4 * kG;
@@ -60,13 +70,16 @@ struct Fp4Cfg {
                                  : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
   static_assert(kColsNeeded <= 512, "TMEM budget");
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(BN * 128 * 4 <= kStages * kStageBytes, "split-K partial tile must fit the ring");
 };
 
-template <int BN, bool E8M0>
+// VQ = true (MXCode PreScale weights): tm_w maps the 8-bit index matrix [N, K/4] instead of the
+// weight codes; warps 2..5 decode each stage's operand tile from the shared-memory codebooks.
+template <int BN, bool E8M0, bool VQ = false>
 __global__ void __launch_bounds__(192, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_x, const Fp4GemmArgs a) {
-  using Cfg = Fp4Cfg<BN, E8M0>;
+  using Cfg = Fp4Cfg<BN, E8M0, VQ>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -75,11 +88,13 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sB = sA + S * Cfg::kABytes;
   uint8_t* sSfa = sB + S * Cfg::kBBytes;
   uint8_t* sSfb = sSfa + S * Cfg::kSfaBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSfb + S * Cfg::kSfbBytes);
+  uint8_t* sIdx = sSfb + S * Cfg::kSfbBytes;
+  uint8_t* sLut = sIdx + S * Cfg::kIdxBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sLut + S * Cfg::kLutBytes);
   uint64_t* empty = full + S;
-  uint64_t* accf = empty + S;
+  uint64_t* decd = empty + S;   // VQ: operand tile decoded (count 128)
+  uint64_t* accf = decd + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
-  int* flag_slot = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN;
@@ -90,6 +105,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&decd[s], 128);
     }
     mbar_init(accf, 1);
     fence_mbar_init();
@@ -132,9 +148,19 @@ __global__ void __launch_bounds__(192, 1)
         int kw, kx, valid;
         stage_coords(i, kw, kx, valid);
         const int nat = valid / Cfg::kAtomK;
-        const uint32_t bytes = Cfg::kABytes + Cfg::kBBytes + nat * 512 * (1 + Cfg::kG);
+        const uint32_t wbytes = VQ ? Cfg::kIdxBytes + Cfg::kLutBytes : Cfg::kABytes;
+        const uint32_t bytes = wbytes + Cfg::kBBytes + nat * 512 * (1 + Cfg::kG);
         mbar_arrive_expect_tx(&full[st], bytes);
-        tma_load_2d(sA + st * Cfg::kABytes, &tm_w, &full[st], kw >> 1, n0);
+        if constexpr (VQ) {
+          tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_w, &full[st], kw >> 2, n0);
+#pragma unroll
+          for (int g2 = 0; g2 < 2; ++g2)
+            bulk_load(sLut + st * Cfg::kLutBytes + g2 * 2048,
+                      a.lut + (static_cast<size_t>((n0 >> 6) + g2) * a.lut_qc + (kw >> 6)) * 512,
+                      2048, &full[st]);
+        } else {
+          tma_load_2d(sA + st * Cfg::kABytes, &tm_w, &full[st], kw >> 1, n0);
+        }
         tma_load_2d(sB + st * Cfg::kBBytes, &tm_x, &full[st], kx >> 1, m0);
         bulk_load(sSfa + st * Cfg::kSfaBytes,
                   a.sfa + (static_cast<size_t>(n0 >> 7) * a.sfa_atoms + kw / Cfg::kAtomK) * 512,
@@ -154,6 +180,9 @@ __global__ void __launch_bounds__(192, 1)
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
         if (!mbar_wait(&full[st], ph, 2)) { ok = false; break; }
+        if constexpr (VQ) {
+          if (!mbar_wait(&decd[st], ph, 4)) { ok = false; break; }
+        }
         tc_fence_after();
         int kw, kx, valid;
         stage_coords(i, kw, kx, valid);
@@ -191,10 +220,39 @@ __global__ void __launch_bounds__(192, 1)
       tc_commit(accf);
     }
   } else {
+    if constexpr (VQ) {
+      // ---------------- VQ decode (warps 2..5, 128 threads): for each stage rebuild the
+      // 128 x 256 E2M1 operand tile from 8-bit indices and the QBlock codebooks, in the
+      // 128-byte-swizzled K-major layout the MMA reads (16-byte chunk kc of row r at kc ^ (r%8)).
+      const int t = threadIdx.x - 64;
+      for (int i = s_begin, it = 0; i < s_end && ok; ++i, ++it) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait(&full[st], ph, 5)) { ok = false; break; }
+        const uint8_t* idx_s = sIdx + st * Cfg::kIdxBytes;
+        const uint16_t* lut = reinterpret_cast<const uint16_t*>(sLut + st * Cfg::kLutBytes);
+        uint8_t* a_s = sA + st * Cfg::kABytes;
+#pragma unroll 4
+        for (int j = 0; j < 8; ++j) {
+          const int c = t + 128 * j;             // 16-byte output chunk: row r, chunk kc
+          const int r = c >> 3, kc = c & 7;
+          const uint2 iv = *reinterpret_cast<const uint2*>(idx_s + r * 64 + kc * 8);
+          const uint16_t* L = lut + ((((r >> 6) << 2) + (kc >> 1)) << 8);
+          uint4 o;
+          o.x = L[iv.x & 255u] | (static_cast<uint32_t>(L[(iv.x >> 8) & 255u]) << 16);
+          o.y = L[(iv.x >> 16) & 255u] | (static_cast<uint32_t>(L[iv.x >> 24]) << 16);
+          o.z = L[iv.y & 255u] | (static_cast<uint32_t>(L[(iv.y >> 8) & 255u]) << 16);
+          o.w = L[(iv.y >> 16) & 255u] | (static_cast<uint32_t>(L[iv.y >> 24]) << 16);
+          *reinterpret_cast<uint4*>(a_s + r * 128 + ((kc ^ (r & 7)) << 4)) = o;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&decd[st]);
+      }
+    }
     // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
     const int q = warp & 3;
     const int n = n0 + q * 32 + lane;
-    const int splits = gridDim.z;
+    const int splits = gridDim.z;   // == cluster size along z
     const bool have_acc = (s_end > s_begin);
     float alpha = a.alpha;
     if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
@@ -216,38 +274,58 @@ __global__ void __launch_bounds__(192, 1)
           if (splits == 1) {
             a.y[o] = __float2bfloat16_rn(v * alpha);
             if (a.y32 != nullptr) a.y32[o] = v * alpha;
-          } else {
-            a.partial[(static_cast<size_t>(blockIdx.z) * a.M + m0 + mm) * a.N + n] = v;
           }
+        }
+        if (splits > 1) {
+          float* part = reinterpret_cast<float*>(smem);   // [BN][128] fp32, column = token
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            part[(c + j) * 128 + q * 32 + lane] = have_acc ? __uint_as_float(r[j]) : 0.f;
         }
       }
     }
-    if (splits > 1) {
-      // Deterministic split-K: the last CTA to finish a tile sums the partials in split order.
-      __threadfence();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (threadIdx.x == 64) {
-        const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-        const int old = atomicAdd(&a.counters[tile], 1);
-        *flag_slot = (old == splits - 1);
+  }
+  // ---- split-K reduction across the cluster (all threads take part in the barriers)
+  __syncwarp();
+  cluster_sync_all();
+  if (gridDim.z > 1 && warp >= 2) {
+    // Columns are reduced in chunks of 8 tokens; chunk c belongs to rank c % nsplit, which
+    // loads that chunk from every rank (all loads in flight) and sums them in rank order.
+    const int q = warp & 3;
+    const int n = n0 + q * 32 + lane;
+    const int nsplit = gridDim.z;
+    const int rank = static_cast<int>(cluster_ctarank());
+    float alpha = a.alpha;
+    if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
+    const int mcount = min(BN, a.M - m0);
+    const uint32_t base = smem_u32(smem) + (q * 32 + lane) * 4;
+    for (int c = rank * 8; c < mcount; c += nsplit * 8) {
+      float v[kMaxClusterSplits][8];
+#pragma unroll
+      for (int r = 0; r < kMaxClusterSplits; ++r) {
+        if (r < nsplit) {
+          const uint32_t remote = map_shared_rank(base + c * 512, r);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[r][j] = ld_shared_cluster_f32(remote + j * 512);
+        }
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (*flag_slot) {
-        __threadfence();
-        if (n < a.N) {
-          for (int mm = 0; mm < mcount; ++mm) {
-            float acc = 0.f;
-            for (int s = 0; s < splits; ++s)
-              acc += __ldcg(&a.partial[(static_cast<size_t>(s) * a.M + m0 + mm) * a.N + n]);
-            const size_t o = static_cast<size_t>(m0 + mm) * a.ldy + n;
+      if (n < a.N) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float acc = 0.f;
+#pragma unroll
+          for (int r = 0; r < kMaxClusterSplits; ++r)
+            if (r < nsplit) acc += v[r][j];
+          if (c + j < mcount) {
+            const size_t o = static_cast<size_t>(m0 + c + j) * a.ldy + n;
             a.y[o] = __float2bfloat16_rn(acc * alpha);
             if (a.y32 != nullptr) a.y32[o] = acc * alpha;
           }
         }
-        if (threadIdx.x == 64) a.counters[blockIdx.y * gridDim.x + blockIdx.x] = 0;
       }
     }
   }
+  cluster_sync_all();   // every rank keeps its shared memory until all peers have read it
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);

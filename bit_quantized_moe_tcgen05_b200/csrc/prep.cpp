@@ -117,3 +117,88 @@ extern "C" ql_status qlinear_prepare_prquant(const uint16_t* w_bf16, int64_t N, 
   }
   return QL_OK;
 }
+
+// MXCode PreScale VQ (MXCode abstract; Table 1 row E4M3-B16-FP4): the E4M3 block scales and the
+// FP32 tensor scale are taken from W first; each 4-vector of W / (block scale * tensor scale) is
+// then replaced by the index of the nearest entry of its QBlock's E2M1 codebook.
+namespace {
+
+// Finite non-negative E4M3 values, codes 0x00..0x7E, ascending.
+struct E4m3Table {
+  float v[127];
+  E4m3Table() {
+    for (int b = 0; b < 127; ++b) {
+      const int e = b >> 3, m = b & 7;
+      v[b] = e == 0 ? std::ldexp(static_cast<float>(m), -9)
+                    : std::ldexp(static_cast<float>(8 + m), e - 10);
+    }
+  }
+  // nearest, ties to the even code, saturating at 448
+  uint8_t encode(float r) const {
+    if (!(r > 0.f)) return 0;
+    if (r >= v[126]) return 126;
+    int lo = 0, hi = 126;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) / 2;
+      if (v[mid] <= r) lo = mid; else hi = mid;
+    }
+    const float dlo = r - v[lo], dhi = v[hi] - r;
+    if (dhi < dlo) return static_cast<uint8_t>(hi);
+    if (dlo < dhi) return static_cast<uint8_t>(lo);
+    return static_cast<uint8_t>((lo % 2 == 0) ? lo : hi);
+  }
+};
+
+}  // namespace
+
+extern "C" ql_status qlinear_prepare_vq_prescale(const uint16_t* w_bf16, int64_t N, int64_t K,
+                                                 const uint8_t* codebooks, int32_t qn, int32_t qk,
+                                                 float* ts_out, uint8_t* scales_out,
+                                                 uint8_t* idx_out) {
+  if (w_bf16 == nullptr || codebooks == nullptr || ts_out == nullptr || scales_out == nullptr ||
+      idx_out == nullptr)
+    return QL_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || qn != 64 || qk != 64 || N % qn != 0 || K % qk != 0)
+    return QL_ERR_UNSUPPORTED;
+  static const E4m3Table tab;
+  float amax = 0.f;
+  for (int64_t i = 0; i < N * K; ++i) amax = std::max(amax, std::fabs(bf16_to_f32(w_bf16[i])));
+  const float ts = amax == 0.f ? 1.f : amax / 2688.0f;
+  *ts_out = ts;
+  const int64_t QC = K / qk;
+  // E2M1 values of every codebook entry: [QR][QC][256][4]
+  static const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t n = 0; n < N; ++n) {
+    std::vector<float> v(K);
+    for (int64_t b = 0; b < K / 16; ++b) {
+      float am = 0.f;
+      for (int i = 0; i < 16; ++i) am = std::max(am, std::fabs(bf16_to_f32(w_bf16[n * K + b * 16 + i])));
+      const float t = am / 6.0f;
+      const float r = t / ts;
+      const uint8_t s = tab.encode(r);
+      scales_out[n * (K / 16) + b] = s;
+      const float S = tab.v[s] * ts;
+      for (int i = 0; i < 16; ++i)
+        v[b * 16 + i] = S == 0.f ? 0.f : bf16_to_f32(w_bf16[n * K + b * 16 + i]) / S;
+    }
+    const int64_t qr = n / qn;
+    for (int64_t j = 0; j < K / 4; ++j) {
+      const uint8_t* cb = codebooks + ((qr * QC + (j * 4) / qk) * 256) * 2;
+      int best = 0;
+      double bestd = 0;
+      for (int e = 0; e < 256; ++e) {
+        double d = 0;
+        for (int i = 0; i < 4; ++i) {
+          const uint8_t c = (cb[e * 2 + i / 2] >> (4 * (i & 1))) & 0xF;
+          const double cv = (c & 8) ? -mag[c & 7] : mag[c & 7];
+          const double diff = static_cast<double>(v[j * 4 + i]) - cv;
+          d += diff * diff;
+        }
+        if (e == 0 || d < bestd) { bestd = d; best = e; }
+      }
+      idx_out[n * (K / 4) + j] = static_cast<uint8_t>(best);
+    }
+  }
+  return QL_OK;
+}

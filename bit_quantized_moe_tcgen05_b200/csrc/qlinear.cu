@@ -57,9 +57,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D byte tensor [rows, inner_bytes] with a 128-byte swizzled box of [box_rows, 128 bytes].
+// 2-D byte tensor [rows, inner_bytes], box [box_rows, box_inner bytes], 128-byte swizzle unless
+// `swizzle` is false.
 ql_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows,
-                       uint64_t row_stride, uint32_t box_inner, uint32_t box_rows) {
+                       uint64_t row_stride, uint32_t box_inner, uint32_t box_rows,
+                       bool swizzle = true) {
   auto fn = encode_fn();
   if (fn == nullptr) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {inner_bytes, rows};
@@ -67,7 +69,8 @@ ql_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner_bytes, u
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
   return QL_OK;
@@ -81,32 +84,44 @@ int sm_count() {
 }
 
 // ----------------------------------------------------------------------- GEMM launch
-template <int BN, bool E8M0>
+template <int BN, bool E8M0, bool VQ>
 ql_status launch_fp4_bn(const CUtensorMap& tw, const CUtensorMap& tx, const ql::Fp4GemmArgs& a,
                         dim3 grid, cudaStream_t s) {
-  using Cfg = ql::Fp4Cfg<BN, E8M0>;
+  using Cfg = ql::Fp4Cfg<BN, E8M0, VQ>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    QL_CUDA(cudaFuncSetAttribute(ql::fp4_gemm_kernel<BN, E8M0>,
+    QL_CUDA(cudaFuncSetAttribute(ql::fp4_gemm_kernel<BN, E8M0, VQ>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
     attr_done[dev] = true;
   }
-  ql::fp4_gemm_kernel<BN, E8M0><<<grid, 192, Cfg::kSmemBytes, s>>>(tw, tx, a);
-  QL_CUDA(cudaGetLastError());
+  // K-splits of one output tile form a cluster along z (reduced over DSMEM in the kernel).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = grid.z;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_gemm_kernel<BN, E8M0, VQ>, tw, tx, a));
   return QL_OK;
 }
 
-template <bool E8M0>
+template <bool E8M0, bool VQ>
 ql_status launch_fp4(int BN, const CUtensorMap& tw, const CUtensorMap& tx,
                      const ql::Fp4GemmArgs& a, dim3 grid, cudaStream_t s) {
   switch (BN) {
-    case 16: return launch_fp4_bn<16, E8M0>(tw, tx, a, grid, s);
-    case 32: return launch_fp4_bn<32, E8M0>(tw, tx, a, grid, s);
-    case 64: return launch_fp4_bn<64, E8M0>(tw, tx, a, grid, s);
-    case 128: return launch_fp4_bn<128, E8M0>(tw, tx, a, grid, s);
-    case 256: return launch_fp4_bn<256, E8M0>(tw, tx, a, grid, s);
+    case 16: return launch_fp4_bn<16, E8M0, VQ>(tw, tx, a, grid, s);
+    case 32: return launch_fp4_bn<32, E8M0, VQ>(tw, tx, a, grid, s);
+    case 64: return launch_fp4_bn<64, E8M0, VQ>(tw, tx, a, grid, s);
+    case 128: return launch_fp4_bn<128, E8M0, VQ>(tw, tx, a, grid, s);
+    case 256: return launch_fp4_bn<256, E8M0, VQ>(tw, tx, a, grid, s);
   }
   return fail(QL_ERR_UNSUPPORTED, "no GEMM tile for BN=%d", BN);
 }
@@ -124,9 +139,13 @@ struct ql_linear {
   ql_wformat wfmt;
   int64_t N, K, C;
   int32_t k_tail;
-  uint8_t* d_codes = nullptr;  // [N, K/2]
+  bool e8m0 = true;            // E8M0-B32 scales (else E4M3-B16 + tensor scales)
+  bool vq = false;             // MXCode PreScale VQ weight
+  uint8_t* d_codes = nullptr;  // [N, K/2] codes, or [N, K/4] indices for VQ
+  uint8_t* d_lut = nullptr;    // VQ codebooks [N/64][K/64][256][2]
   uint8_t* d_sf = nullptr;     // tiled scale atoms
   int sf_atoms = 0;            // atoms per 128-row group of the weight
+  int lut_qc = 0;
   float w_ts = 1.f;
   CUtensorMap tm_w;
   int n_base_stages = 0, n_stages_total = 0;
@@ -137,8 +156,10 @@ namespace {
 struct FwdPlan {
   int BN, splits, spp, tiles_n, tiles_m;
   int sfb_atoms;
-  size_t codes_off, sf_off, cnt_off, part_off, total;
+  size_t codes_off, sf_off, scal_off, total;
 };
+
+constexpr int kMaxSplits = ql::kMaxClusterSplits;  // the K-splits of a tile form one cluster
 
 FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   FwdPlan p{};
@@ -147,12 +168,13 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   p.tiles_m = static_cast<int>(cdiv(std::max<int64_t>(M, 1), p.BN));
   const int tiles = p.tiles_n * p.tiles_m;
   const int total = L->n_stages_total;
+  // Narrow token tiles (decode) run two CTAs per SM; split K until the grid fills the GPU.
+  const int target = sm_count() * ((p.BN <= 64 && !L->vq) ? 2 : 1);
   int splits = 1;
-  const int sms = sm_count();
-  if (tiles < sms) splits = std::max(1, std::min(total, sms / tiles));
+  if (tiles < target) splits = std::max(1, std::min({total, target / tiles, kMaxSplits}));
   p.spp = static_cast<int>(cdiv(total, splits));
   p.splits = static_cast<int>(cdiv(total, p.spp));
-  const int atomK = 128;  // E8M0-B32: one 512-byte atom covers 128 K elements
+  const int atomK = L->e8m0 ? 128 : 64;  // K elements covered by one 512-byte scale atom
   p.sfb_atoms = static_cast<int>(cdiv(L->C, atomK));
   const int64_t rows_pad = cdiv(std::max<int64_t>(M, 1), 256) * 256;
   size_t off = 0;
@@ -160,11 +182,9 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   off = align_up(off + static_cast<size_t>(M) * (L->C / 2), 256);
   p.sf_off = off;
   off = align_up(off + static_cast<size_t>(rows_pad / 128) * p.sfb_atoms * 512, 256);
-  p.cnt_off = off;
-  off = align_up(off + static_cast<size_t>(tiles) * sizeof(int), 256);
-  p.part_off = off;
-  if (p.splits > 1) off = align_up(off + static_cast<size_t>(p.splits) * M * L->N * 4, 256);
-  p.total = std::max<size_t>(off, 256);
+  p.scal_off = off;  // E4M3-B16 activations: [0] amax bit pattern, [1] tensor scale
+  off = align_up(off + 2 * sizeof(float), 256);
+  p.total = off;
   return p;
 }
 
@@ -181,7 +201,7 @@ void repack_sf_tiled(const uint8_t* plain, int64_t rows, int64_t cols, int atoms
 ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
                           uint8_t* st, int st_atoms, int* zero_words, int nzero,
                           cudaStream_t s) {
-  const long total = static_cast<long>(M) * (K / 8);
+  const long total = static_cast<long>(M) * (K / 32);
   const long threads = std::max<long>(total, nzero);
   if (threads == 0) return QL_OK;
   const int block = 256;
@@ -190,6 +210,26 @@ ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, u
       static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K),
       static_cast<int>(K), codes, static_cast<int>(K / 2), sp, static_cast<int>(K / 32), st,
       st_atoms, zero_words, nzero);
+  QL_CUDA(cudaGetLastError());
+  return QL_OK;
+}
+
+ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
+                            uint8_t* st, int st_atoms, unsigned* amax_slot, float* ts_out,
+                            cudaStream_t s) {
+  QL_CUDA(cudaMemsetAsync(amax_slot, 0, sizeof(unsigned), s));
+  const long n8 = static_cast<long>(M) * K / 8;
+  const int block = 256;
+  const long want = (n8 + block - 1) / block;
+  const int grid_a = static_cast<int>(std::max<long>(1, std::min<long>(want, 4L * sm_count())));
+  ql::absmax_bf16_kernel<<<grid_a, block, 0, s>>>(static_cast<const __nv_bfloat16*>(x), n8,
+                                                  amax_slot);
+  QL_CUDA(cudaGetLastError());
+  const long total = static_cast<long>(M) * (K / 16);
+  ql::quant_e4m3_b16_kernel<<<static_cast<unsigned>((total + block - 1) / block), block, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K),
+      static_cast<int>(K), amax_slot, ts_out, codes, static_cast<int>(K / 2), sp,
+      static_cast<int>(K / 16), st, st_atoms);
   QL_CUDA(cudaGetLastError());
   return QL_OK;
 }
@@ -204,16 +244,27 @@ const char* ql_last_error(void) { return g_last_error.c_str(); }
 ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear** out) {
   if (d == nullptr || out == nullptr) return fail(QL_ERR_INVALID_ARG, "null descriptor/out");
   *out = nullptr;
-  if (d->wfmt != QL_W_MXFP4_E8M0_B32)
+  const bool mx = d->wfmt == QL_W_MXFP4_E8M0_B32;
+  const bool nv = d->wfmt == QL_W_NVFP4_E4M3_B16;
+  const bool vq = d->wfmt == QL_W_VQ_PRESCALE_E4M3_B16;
+  if (!mx && !nv && !vq)
     return fail(QL_ERR_UNSUPPORTED, "weight format %d not supported by qlinear_create",
                 int(d->wfmt));
-  if (d->codes == nullptr || d->scales == nullptr)
-    return fail(QL_ERR_INVALID_ARG, "codes/scales must be non-null host pointers");
+  if (d->scales == nullptr || (vq ? (d->indices == nullptr || d->codebooks == nullptr)
+                                  : d->codes == nullptr))
+    return fail(QL_ERR_INVALID_ARG, "codes/indices/codebooks/scales must be non-null host pointers");
   if (d->N <= 0 || d->K <= 0 || d->k_tail < 0 || d->k_tail >= d->K)
     return fail(QL_ERR_INVALID_ARG, "bad sizes N=%lld K=%lld k_tail=%d", (long long)d->N,
                 (long long)d->K, d->k_tail);
-  if (d->N % 16 != 0 || d->K % 128 != 0 || d->k_tail % 128 != 0)
+  if (mx && (d->N % 16 != 0 || d->K % 128 != 0 || d->k_tail % 128 != 0))
     return fail(QL_ERR_UNSUPPORTED, "MXFP4 layer needs N%%16==0, K%%128==0, k_tail%%128==0");
+  if (nv && (d->N % 16 != 0 || d->K % 64 != 0 || d->k_tail != 0))
+    return fail(QL_ERR_UNSUPPORTED, "E4M3-B16 layer needs N%%16==0, K%%64==0, no tail");
+  if (vq && (d->N % 128 != 0 || d->K % 256 != 0 || d->k_tail != 0 || d->qblock_n != 64 ||
+             d->qblock_k != 64))
+    return fail(QL_ERR_UNSUPPORTED, "VQ layer needs N%%128==0, K%%256==0, 64x64 QBlocks, no tail");
+  if ((nv || vq) && !(d->w_tensor_scale > 0.f))
+    return fail(QL_ERR_INVALID_ARG, "E4M3-B16 weights need a positive FP32 tensor scale");
   if (d->N > (1 << 24) || d->K > (1 << 24))
     return fail(QL_ERR_UNSUPPORTED, "N/K too large");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -223,26 +274,40 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
   L->K = d->K;
   L->k_tail = d->k_tail;
   L->C = d->K - d->k_tail;
-  L->sf_atoms = static_cast<int>(cdiv(d->K, 128));
+  L->e8m0 = mx;
+  L->vq = vq;
+  L->w_ts = mx ? 1.f : d->w_tensor_scale;
+  const int atomK = mx ? 128 : 64;
+  const int sf_block = mx ? 32 : 16;
+  L->sf_atoms = static_cast<int>(cdiv(d->K, atomK));
   L->n_base_stages = static_cast<int>(cdiv(L->C, 256));
   L->n_stages_total = L->n_base_stages + static_cast<int>(cdiv(L->k_tail, 256));
   std::vector<uint8_t> sf;
-  repack_sf_tiled(static_cast<const uint8_t*>(d->scales), d->N, d->K / 32, L->sf_atoms, sf);
-  const size_t code_bytes = static_cast<size_t>(d->N) * (d->K / 2);
+  repack_sf_tiled(static_cast<const uint8_t*>(d->scales), d->N, d->K / sf_block, L->sf_atoms, sf);
+  const size_t code_bytes = static_cast<size_t>(d->N) * (vq ? d->K / 4 : d->K / 2);
+  const size_t lut_bytes = vq ? static_cast<size_t>(d->N / 64) * (d->K / 64) * 512 : 0;
+  L->lut_qc = vq ? static_cast<int>(d->K / 64) : 0;
   auto cleanup = [&](ql_status st) {
     if (L->d_codes) cudaFree(L->d_codes);
+    if (L->d_lut) cudaFree(L->d_lut);
     if (L->d_sf) cudaFree(L->d_sf);
     delete L;
     return st;
   };
   if (cudaMalloc(&L->d_codes, code_bytes) != cudaSuccess ||
-      cudaMalloc(&L->d_sf, sf.size()) != cudaSuccess)
-    return cleanup(fail(QL_ERR_OOM, "cudaMalloc of %zu weight bytes failed", code_bytes + sf.size()));
-  if (cudaMemcpyAsync(L->d_codes, d->codes, code_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMalloc(&L->d_sf, sf.size()) != cudaSuccess ||
+      (vq && cudaMalloc(&L->d_lut, lut_bytes) != cudaSuccess))
+    return cleanup(fail(QL_ERR_OOM, "cudaMalloc of %zu weight bytes failed",
+                        code_bytes + sf.size() + lut_bytes));
+  const void* src = vq ? static_cast<const void*>(d->indices) : d->codes;
+  if (cudaMemcpyAsync(L->d_codes, src, code_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(L->d_sf, sf.data(), sf.size(), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      (vq && cudaMemcpyAsync(L->d_lut, d->codebooks, lut_bytes, cudaMemcpyHostToDevice, s) !=
+                 cudaSuccess) ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return cleanup(fail(QL_ERR_CUDA, "weight upload failed"));
-  ql_status st = make_tmap_u8(&L->tm_w, L->d_codes, d->K / 2, d->N, d->K / 2, 128, 128);
+  ql_status st = vq ? make_tmap_u8(&L->tm_w, L->d_codes, d->K / 4, d->N, d->K / 4, 64, 128, false)
+                    : make_tmap_u8(&L->tm_w, L->d_codes, d->K / 2, d->N, d->K / 2, 128, 128);
   if (st != QL_OK) return cleanup(st);
   *out = L;
   return QL_OK;
@@ -251,6 +316,7 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
 ql_status qlinear_destroy(ql_linear* L) {
   if (L == nullptr) return QL_OK;
   if (L->d_codes) cudaFree(L->d_codes);
+  if (L->d_lut) cudaFree(L->d_lut);
   if (L->d_sf) cudaFree(L->d_sf);
   delete L;
   return QL_OK;
@@ -281,9 +347,14 @@ ql_status qlinear_quantize_input(const ql_linear* L, const void* x, int64_t M, v
   if ((reinterpret_cast<uintptr_t>(x) & 15) != 0)
     return fail(QL_ERR_INVALID_ARG, "x must be 16-byte aligned");
   uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (!L->e8m0) {
+    unsigned* scal = reinterpret_cast<unsigned*>(w8 + p.scal_off);
+    return launch_quant_e4m3(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
+                             scal, reinterpret_cast<float*>(scal + 1),
+                             reinterpret_cast<cudaStream_t>(stream));
+  }
   return launch_quant_mx(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
-                         reinterpret_cast<int*>(w8 + p.cnt_off), p.tiles_n * p.tiles_m,
-                         reinterpret_cast<cudaStream_t>(stream));
+                         nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void* ws,
@@ -309,15 +380,18 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   a.sfa_atoms = L->sf_atoms;
   a.sfb = w8 + p.sf_off;
   a.sfb_atoms = p.sfb_atoms;
-  a.alpha_dev = nullptr;
-  a.alpha = 1.f;
+  a.alpha_dev = L->e8m0 ? nullptr : reinterpret_cast<const float*>(w8 + p.scal_off) + 1;
+  a.alpha = L->w_ts;
   a.y = static_cast<__nv_bfloat16*>(y);
   a.y32 = y32;
   a.ldy = static_cast<int>(L->N);
-  a.partial = reinterpret_cast<float*>(w8 + p.part_off);
-  a.counters = reinterpret_cast<int*>(w8 + p.cnt_off);
+  a.lut = L->d_lut;
+  a.lut_qc = L->lut_qc;
   dim3 grid(p.tiles_n, p.tiles_m, p.splits);
-  return launch_fp4<true>(p.BN, L->tm_w, tm_x, a, grid, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (L->vq) return launch_fp4<false, true>(p.BN, L->tm_w, tm_x, a, grid, cs);
+  if (!L->e8m0) return launch_fp4<false, false>(p.BN, L->tm_w, tm_x, a, grid, cs);
+  return launch_fp4<true, false>(p.BN, L->tm_w, tm_x, a, grid, cs);
 }
 
 ql_status qlinear_forward(const ql_linear* L, const void* x, int64_t M, void* y, float* y32,
@@ -337,14 +411,26 @@ ql_status quantize_act(ql_aformat fmt, const void* x, int64_t M, int64_t K, void
   if (M == 0 || K == 0) return QL_OK;
   if (x == nullptr || codes == nullptr || scales == nullptr)
     return fail(QL_ERR_INVALID_ARG, "null pointer");
-  if ((reinterpret_cast<uintptr_t>(x) & 15) != 0 || (reinterpret_cast<uintptr_t>(codes) & 3) != 0)
-    return fail(QL_ERR_INVALID_ARG, "x must be 16-byte and codes 4-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(x) & 15) != 0 || (reinterpret_cast<uintptr_t>(codes) & 15) != 0)
+    return fail(QL_ERR_INVALID_ARG, "x and codes must be 16-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (fmt) {
     case QL_A_MXFP4_E8M0_B32:
       if (K % 32 != 0) return fail(QL_ERR_UNSUPPORTED, "MXFP4 needs K %% 32 == 0");
       return launch_quant_mx(x, M, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
                              nullptr, 0, nullptr, 0, s);
+    case QL_A_FP4_E4M3_B16_TS: {
+      if (K % 16 != 0) return fail(QL_ERR_UNSUPPORTED, "E4M3-B16 needs K %% 16 == 0");
+      if (tensor_scale == nullptr)
+        return fail(QL_ERR_INVALID_ARG, "E4M3-B16 needs a device tensor_scale pointer");
+      unsigned* slot = reinterpret_cast<unsigned*>(tensor_scale);
+      ql_status st = launch_quant_e4m3(x, M, K, static_cast<uint8_t*>(codes),
+                                       static_cast<uint8_t*>(scales), nullptr, 0, slot, nullptr, s);
+      if (st != QL_OK) return st;
+      ql::amax_to_tensor_scale_kernel<<<1, 1, 0, s>>>(slot);
+      QL_CUDA(cudaGetLastError());
+      return QL_OK;
+    }
     default:
       return fail(QL_ERR_UNSUPPORTED, "activation format %d not supported", int(fmt));
   }

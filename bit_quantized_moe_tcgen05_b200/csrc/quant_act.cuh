@@ -41,46 +41,173 @@ __host__ __device__ __forceinline__ size_t sf_tiled_offset(int m, int j, int ato
   return atom * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
 }
 
-// One thread per 8 consecutive elements; four threads (one quad of lanes) share a 32-block.
+// Eight E2M1 codes from eight exactly-scaled fp32 values (RNE, satfinite) via the hardware
+// conversion; element 2i lands in the low nibble.  The sign bits are or-ed in from the inputs so
+// that negative values rounding to zero keep code 0x8 whatever the conversion does with zeros.
+__device__ __forceinline__ uint32_t e2m1x8(const float (&f)[8]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7]));
+  return out;
+}
+
+// Sign bits of eight bf16 values packed in four words (element 2i low half of word i) placed at
+// bit 3 of each nibble of the matching code word.
+__device__ __forceinline__ uint32_t bf16x8_sign_nibbles(const uint32_t (&w)[4]) {
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    s |= (((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u)) << (8 * i);
+  return s;
+}
+
+// One thread per 32-element block (4 x 16-byte loads in flight, one 16-byte code store).
 // x: bf16 [M, K] with row stride ldx (elements).  codes: [M, K/2] bytes (row stride ldc),
 // low nibble = even k.  Scales go to the plain [M, K/32] layout and/or the tiled layout.
-// The first `nzero` ints of `zero_words` are cleared (split-K tile tickets of the GEMM that
-// consumes this output).
+// The first `nzero` ints of `zero_words` are cleared (scratch the consumer expects zeroed).
 __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, uint8_t* __restrict__ codes,
     int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
     int sf_atoms_per_row, int* __restrict__ zero_words, int nzero) {
   const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (zero_words != nullptr && gtid < nzero) zero_words[gtid] = 0;
-  const int groups = K >> 3;
-  const long total = static_cast<long>(M) * groups;
-  if (gtid >= total) return;  // total is a multiple of 4: quads stay whole
-  const int m = static_cast<int>(gtid / groups);
-  const int q = static_cast<int>(gtid - static_cast<long>(m) * groups);
-  const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + q);
-  float f[8];
-  bf16x8_to_f32(v, f);
-  float amax = 0.f;
+  const int nblk = K >> 5;
+  if (gtid >= static_cast<long>(M) * nblk) return;
+  const int m = static_cast<int>(gtid / nblk);
+  const int j = static_cast<int>(gtid - static_cast<long>(m) * nblk);
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 4;
+  uint32_t w[16];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-  const unsigned mask = __activemask();
-  amax = fmaxf(amax, __shfl_xor_sync(mask, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(mask, amax, 2));
-  // floor(log2 amax) from the fp32 exponent field; zero and fp32-subnormal amax give an
-  // exponent at or below -127 and clamp to -127.  bf16 cannot exceed 2^128, so e <= 125.
-  const int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF);
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = __ldg(src + i);
+    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+  // amax over 32 bf16 magnitudes as 16-bit unsigned integers (order-preserving for finite values)
+  uint32_t mx = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
+  const uint32_t amax16 = max(mx & 0xFFFFu, mx >> 16);
+  // floor(log2 amax) from the bf16 exponent field; zero or subnormal amax clamps to e = -127.
+  const int E = static_cast<int>(amax16 >> 7);
   const int e = (E == 0) ? -127 : max(E - 129, -127);
   const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, normal
-  uint32_t packed = 0;
+  uint32_t packed[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) packed |= e2m1_rne(f[i] * inv) << (4 * i);
-  *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(m) * ldc + q * 4) = packed;
-  if ((q & 3) == 0) {
-    const uint8_t b = static_cast<uint8_t>(e + 127);
-    const int j = q >> 2;
-    if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = b;
-    if (scales_tiled != nullptr) scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row)] = b;
+  for (int q = 0; q < 4; ++q) {
+    float f[8];
+    const uint32_t ww[4] = {w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(ww[i] << 16) * inv;
+      f[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u) * inv;
+    }
+    packed[q] = e2m1x8(f) | bf16x8_sign_nibbles(ww);
   }
+  *reinterpret_cast<uint4*>(codes + static_cast<size_t>(m) * ldc + j * 16) =
+      make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  const uint8_t b = static_cast<uint8_t>(e + 127);
+  if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = b;
+  if (scales_tiled != nullptr) scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row)] = b;
+}
+
+// ------------------------------------------------------------------ E4M3-B16 + FP32 tensor scale
+// MXCode, Table 1 row E4M3-B16-FP4: per 16 elements an E4M3 block scale and one FP32 tensor
+// scale for the whole tensor.  Steps, each an IEEE fp32 operation in this order:
+//   ts = amax_T / 2688 (1 if amax_T == 0);  s = E4M3_RNE_satfinite((amax_b / 6) / ts);
+//   S = dec(s) * ts;  code = E2M1_RNE_satfinite(x / S)  (zero codes, sign kept, when S == 0).
+
+// Largest |x| of a bf16 tensor as a bf16 bit pattern (16-bit magnitude), max-reduced into
+// *amax16 (which the caller zeroes first).  n8 = number of 8-element (16-byte) groups.
+__global__ void __launch_bounds__(256) absmax_bf16_kernel(const __nv_bfloat16* __restrict__ x,
+                                                           long n8, unsigned* __restrict__ amax16) {
+  uint32_t mx = 0;
+  const uint4* src = reinterpret_cast<const uint4*>(x);
+  for (long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long>(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldg(src + i);
+    mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v.w & 0x7FFF7FFFu);
+  }
+  uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ uint32_t red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) b = max(b, red[w]);
+    atomicMax(amax16, b);
+  }
+}
+
+__device__ __forceinline__ float tensor_scale_from_amax16(uint32_t amax16) {
+  const float amax = __uint_as_float(amax16 << 16);
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, 2688.0f);
+}
+
+// Value of a non-negative E4M3 byte (bias 7; subnormals m * 2^-9).
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  return e == 0 ? static_cast<float>(m) * 0x1p-9f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// One thread per 16-element block.  codes [M, K/2] (row stride ldc), scales plain [M, K/16]
+// and/or tiled (atoms of 64 K).  Thread 0 stores ts to *ts_out when ts_out is not null.
+__global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
+    const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, const unsigned* __restrict__ amax16,
+    float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
+    uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
+    int sf_atoms_per_row) {
+  const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const float ts = tensor_scale_from_amax16(*amax16);
+  if (gtid == 0 && ts_out != nullptr) *ts_out = ts;
+  const int nblk = K >> 4;
+  if (gtid >= static_cast<long>(M) * nblk) return;
+  const int m = static_cast<int>(gtid / nblk);
+  const int j = static_cast<int>(gtid - static_cast<long>(m) * nblk);
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
+  const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  uint32_t mx = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
+  const float amax_b = __uint_as_float(max(mx & 0xFFFFu, mx >> 16) << 16);
+  const float r = __fdiv_rn(__fdiv_rn(amax_b, 6.0f), ts);
+  const uint32_t sb = static_cast<uint32_t>(__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3));
+  const float S = __fmul_rn(e4m3_value(sb), ts);
+  uint32_t packed[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float f[8];
+    const uint32_t ww[4] = {w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __uint_as_float(ww[i] << 16), hi = __uint_as_float(ww[i] & 0xFFFF0000u);
+      f[2 * i] = S == 0.f ? 0.f : __fdiv_rn(lo, S);
+      f[2 * i + 1] = S == 0.f ? 0.f : __fdiv_rn(hi, S);
+    }
+    packed[h] = e2m1x8(f) | bf16x8_sign_nibbles(ww);
+  }
+  *reinterpret_cast<uint2*>(codes + static_cast<size_t>(m) * ldc + j * 8) =
+      make_uint2(packed[0], packed[1]);
+  if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = static_cast<uint8_t>(sb);
+  if (scales_tiled != nullptr)
+    scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row)] = static_cast<uint8_t>(sb);
+}
+
+// Replace the amax bit pattern stored in *slot by the tensor scale it implies (single thread).
+__global__ void amax_to_tensor_scale_kernel(unsigned* slot) {
+  const float ts = tensor_scale_from_amax16(*slot);
+  *reinterpret_cast<float*>(slot) = ts;
 }
 
 }  // namespace ql

@@ -99,8 +99,15 @@ const char* ql_last_error(void);
 
 /* Create a linear layer: validates the descriptor, copies the weights to device memory owned
  * by the returned handle and repacks scales into the tiled layout the MMA consumes.
- * Supported: QL_W_MXFP4_E8M0_B32 with N % 16 == 0, K % 128 == 0, k_tail % 128 == 0,
- * 0 <= k_tail < K.  Synchronous with respect to `stream` (uses it for the uploads). */
+ * Supported:
+ *   QL_W_MXFP4_E8M0_B32        N % 16 == 0, K % 128 == 0, k_tail % 128 == 0, 0 <= k_tail < K;
+ *                              activations quantized to MXFP4 (E8M0-B32).
+ *   QL_W_NVFP4_E4M3_B16        N % 16 == 0, K % 64 == 0, no tail; activations E4M3-B16 + FP32
+ *                              tensor scale; y = (sum) * ts_x * ts_w.
+ *   QL_W_VQ_PRESCALE_E4M3_B16  N % 128 == 0, K % 256 == 0, 64 x 64 QBlocks, no tail; indices,
+ *                              codebooks, E4M3 scales [N,K/16] and w_tensor_scale; the weight
+ *                              operand is rebuilt from the codebooks inside the GEMM.
+ * Synchronous with respect to `stream` (uses it for the uploads). */
 ql_status qlinear_create(const ql_weight_desc* desc, ql_stream_t stream, ql_linear** out);
 ql_status qlinear_destroy(ql_linear* layer);
 
@@ -115,7 +122,7 @@ ql_status qlinear_forward(const ql_linear* layer, const void* x_bf16, int64_t M,
                           float* y_f32, void* ws, size_t ws_bytes, ql_stream_t stream);
 
 /* The two halves of qlinear_forward.  qlinear_quantize_input quantizes x into the workspace
- * (MXFP4 codes and tiled scales; it also clears the GEMM's split-K tickets); qlinear_gemm runs
+ * (MXFP4 codes and tiled scales); qlinear_gemm runs
  * the tcgen05 GEMM from that workspace.  Called in this order on one stream with the same M and
  * workspace they equal qlinear_forward.  A caller whose several layers share one input (gate and
  * up projections, say) can quantize once; the split also lets a profiler time the GEMM alone. */
@@ -144,7 +151,11 @@ ql_status qlinear_forward_fixed_scratch(const ql_linear* layer, const void* x_bf
  * QL_A_MXFP4_E8M0_B32: K % 32 == 0; codes [M,K/2], scales E8M0 [M,K/32]; tensor_scale unused.
  * Rule (OCP MX, as the PRQuant page applies it): per 32 elements e = floor(log2 amax) - 2
  * clamped to [-127,127], byte e+127 (0 for an all-zero block), code = E2M1 RNE of x/2^e with
- * saturation at +-6 and the sign of x. */
+ * saturation at +-6 and the sign of x.
+ * QL_A_FP4_E4M3_B16_TS: K % 16 == 0; codes [M,K/2], E4M3 scales [M,K/16], *tensor_scale (device
+ * float) receives ts = amax(x)/2688 (1 for an all-zero x); per 16 elements
+ * s = E4M3_RNE_satfinite((amax/6)/ts), code = E2M1 RNE of x/(dec(s)*ts) (MXCode Table 1 row
+ * E4M3-B16-FP4), each step an IEEE fp32 operation. */
 ql_status quantize_act(ql_aformat fmt, const void* x_bf16, int64_t M, int64_t K, void* codes,
                        void* scales, float* tensor_scale, ql_stream_t stream);
 
@@ -161,6 +172,17 @@ ql_status ql_check(ql_stream_t stream);
  * Requires C % 128 == 0, k % 128 == 0, 0 < k <= C. */
 ql_status qlinear_prepare_prquant(const uint16_t* w_bf16, int64_t N, int64_t C, int32_t k,
                                   int32_t* perm_out, uint8_t* codes_out, uint8_t* scales_out);
+
+/* MXCode PreScale VQ preparation (MXCode abstract: PreScale extracts the MX scales before the
+ * codebook is learned; Table 1 row E4M3-B16-FP4).  w_bf16 [N,K]; codebooks = packed E2M1 entries
+ * [N/64][K/64][256][2] (entry element 2i in the low nibble of byte i); outputs: the FP32 tensor
+ * scale ts = amax(W)/2688 (1 for an all-zero W), E4M3 block scales [N,K/16]
+ * (s = E4M3_RNE_satfinite((amax16/6)/ts), fp32 steps), and uint8 indices [N,K/4]: the entry of
+ * the row's QBlock nearest (squared distance, exact in double; ties to the lowest index) to
+ * W[n,4j:4j+4] / (dec(s)*ts) (0 in a block whose scale is 0).  qn == qk == 64. Host, CPU. */
+ql_status qlinear_prepare_vq_prescale(const uint16_t* w_bf16, int64_t N, int64_t K,
+                                      const uint8_t* codebooks, int32_t qn, int32_t qk,
+                                      float* ts_out, uint8_t* scales_out, uint8_t* idx_out);
 
 #ifdef __cplusplus
 }

@@ -76,3 +76,46 @@ def uniform_nibble_bytes(seed: int, rows: int, nibbles: int) -> np.ndarray:
 def uniform_bytes(seed: int, shape: tuple[int, ...], lo: int, hi: int) -> np.ndarray:
     """Uniform random bytes in the inclusive range [lo, hi]."""
     return rng(seed).integers(lo, hi + 1, size=shape, dtype=np.uint8)
+
+
+_E2M1_GRID = np.array([-6.0, -4.0, -3.0, -2.0, -1.5, -1.0, -0.5, 0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+_E2M1_CODE = np.array([15, 14, 13, 12, 11, 10, 9, 0, 1, 2, 3, 4, 5, 6, 7], dtype=np.uint8)
+
+
+def vq_codebooks(seed: int, w: np.ndarray, qn: int = 64, qk: int = 64, entries: int = 256,
+                 iters: int = 4, chunk: int = 128) -> np.ndarray:
+    """Synthesize one FP4 codebook per qn x qk QBlock by seeded k-means (data synthesis only).
+
+    Each 4-vector along K is first brought to the E2M1 range by its 16-block's amax / 6 (a
+    generator-side normalisation in float64, not the method's E4M3 scale), then k-means with
+    `entries` centroids (distinct random points as the initial centroids, `iters` Lloyd steps) runs
+    per QBlock, and each centroid coordinate snaps to the closest signed E2M1 grid value.
+    Returns E2M1 codes [N/qn, K/qk, entries, 4] (uint8 nibbles).
+    """
+    g = rng(seed * 31 + 7)
+    N, K = w.shape
+    QR, QC = N // qn, K // qk
+    blk = np.abs(w.reshape(N, K // 16, 16)).max(-1, keepdims=True)
+    v = (w.reshape(N, K // 16, 16) / np.where(blk == 0, 1.0, blk / 6.0)).reshape(N, K)
+    # points per QBlock: [QR*QC, qn*qk/4, 4]
+    pts = v.reshape(QR, qn, QC, qk // 4, 4).transpose(0, 2, 1, 3, 4).reshape(QR * QC, -1, 4)
+    out = np.empty((QR * QC, entries, 4), dtype=np.uint8)
+    P = pts.shape[1]
+    for c0 in range(0, QR * QC, chunk):
+        p = pts[c0:c0 + chunk].astype(np.float32)                      # [B, P, 4]
+        B = p.shape[0]
+        init = np.stack([g.choice(P, entries, replace=False) for _ in range(B)])
+        cent = np.take_along_axis(p, init[:, :, None], axis=1)        # [B, E, 4]
+        for _ in range(iters):
+            d = (p * p).sum(-1)[:, :, None] - 2 * p @ cent.transpose(0, 2, 1) + \
+                (cent * cent).sum(-1)[:, None, :]
+            lab = d.argmin(-1)                                         # [B, P]
+            flat = (lab + np.arange(B)[:, None] * entries).reshape(-1)
+            sums = np.zeros((B * entries, 4), np.float64)
+            np.add.at(sums, flat, p.reshape(-1, 4))
+            cnt = np.bincount(flat, minlength=B * entries).astype(np.float64)
+            newc = (sums / np.maximum(cnt, 1)[:, None]).reshape(B, entries, 4).astype(np.float32)
+            cent = np.where((cnt == 0).reshape(B, entries, 1), cent, newc)
+        snap = np.abs(cent[..., None] - _E2M1_GRID).argmin(-1)
+        out[c0:c0 + B] = _E2M1_CODE[snap]
+    return out.reshape(QR, QC, entries, 4)

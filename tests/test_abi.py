@@ -58,3 +58,17 @@ def test_prquant_host_preparation_matches_oracle(N, C, k):
     assert np.array_equal(perm, ref["perm"])
     assert np.array_equal(codes, F.pack_nibbles(ref["w_codes"]))
     assert np.array_equal(scales, ref["w_sb"])
+
+
+@pytest.mark.parametrize("N,K", [(64, 256), (128, 512)])
+def test_vq_prescale_host_preparation_matches_oracle(N, K):
+    import bit_quantized_moe_tcgen05_b200 as ql
+    from oracle import vq
+    wb = synth.to_bf16_bits(synth.student_t(17 + K, (N, K), 4.0))
+    w = synth.bf16_bits_to_f64(wb)
+    cb = synth.vq_codebooks(17, w)
+    ts, sb, idx = ql.prepare_vq_prescale(wb, vq.pack_codebooks(cb))
+    ref = vq.prepare(w, cb)
+    assert ts == ref["ts"]
+    assert np.array_equal(sb, ref["sb"])
+    assert np.array_equal(idx, ref["idx"])

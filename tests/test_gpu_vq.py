@@ -1,0 +1,127 @@
+"""GPU parity: E4M3-B16 activation quantizer (bit-exact, with its FP32 tensor scale), E4M3-B16
+weights on the kind::mxf4nvf4 MMA, and MXCode PreScale VQ weights decoded inside the GEMM."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import formats as F
+from oracle import gemm as G
+from oracle import mx, vq
+from tests._parity import check_bf16, check_fp32
+
+pytestmark = pytest.mark.gpu
+
+
+def _ql():
+    import bit_quantized_moe_tcgen05_b200 as ql
+    return ql
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _check_quant(xb):
+    ql = _ql()
+    codes, sb, ts = ql.quantize_act(dev_bf16(xb), fmt=ql.QL_A_FP4_E4M3_B16_TS)
+    ql.check()
+    rc, rs, rts = mx.quantize_e4m3_b16(synth.bf16_bits_to_f64(xb).astype(np.float32))
+    assert ts.cpu().numpy()[0] == rts
+    assert np.array_equal(sb.cpu().numpy(), rs)
+    assert np.array_equal(codes.cpu().numpy(), F.pack_nibbles(rc))
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (7, 9728), (64, 512), (300, 160)])
+def test_quant_e4m3_b16_bitexact(M, K):
+    xb, _ = synth.activations_bf16(200 + M, M, K, 0.01, 30.0)
+    _check_quant(xb)
+
+
+def test_quant_e4m3_b16_edge_values():
+    _check_quant(synth.to_bf16_bits(np.zeros((3, 64))))                  # ts = 1, codes 0
+    x = np.zeros((2, 64))
+    x[0, 0] = 1e6
+    x[0, 16:32] = 1e-6                                                    # scale underflows
+    x[1, 32:48] = -1e-30
+    x[1, 48] = -0.0
+    _check_quant(synth.to_bf16_bits(x))
+    g = np.random.default_rng(1)
+    _check_quant(synth.to_bf16_bits(g.standard_normal((4, 256)) * 10.0 ** g.uniform(-30, 30, (4, 1))))
+
+
+def _run(lin, xb):
+    x = dev_bf16(xb)
+    y32 = torch.empty((x.shape[0], lin.N), dtype=torch.float32, device="cuda")
+    y = lin(x, out_f32=y32)
+    _ql().check()
+    return y.float().cpu().numpy(), y32.cpu().numpy()
+
+
+def _x_deq(xb):
+    xc, xs, xts = mx.quantize_e4m3_b16(synth.bf16_bits_to_f64(xb).astype(np.float32))
+    return mx.dequant_e4m3_b16(xc, xs, xts)
+
+
+@pytest.mark.parametrize("N,K,M", [(256, 512, 1), (128, 1024, 64), (272, 320, 100), (512, 9728, 8)])
+def test_nvfp4_weight_linear(N, K, M):
+    """E4M3-B16 weights (random codes, block scales and a tensor scale) on the block16 MMA."""
+    ql = _ql()
+    codes = synth.uniform_nibble_bytes(50 + N, N, K)
+    sb = synth.uniform_bytes(51 + N, (N, K // 16), 0x28, 0x48)
+    ts_w = np.float32(0.0123)
+    lin = ql.QLinear(codes, sb, wfmt=ql.QL_W_NVFP4_E4M3_B16, w_tensor_scale=float(ts_w))
+    xb, _ = synth.activations_bf16(52, M, K, 0.01, 30.0)
+    y, y32 = _run(lin, xb)
+    lin.close()
+    xd = _x_deq(xb)
+    wd = mx.dequant_e4m3_b16(F.unpack_nibbles(codes), sb, ts_w)
+    ref, t = G.gemm_ref(xd, wd), G.abs_scale(xd, wd)
+    check_fp32(y32, ref, t, "nvfp4")
+    check_bf16(y, ref, t, "nvfp4")
+
+
+def _vq_layer(w, cb, prep):
+    ql = _ql()
+    return ql.QLinear(None, prep["sb"], wfmt=ql.QL_W_VQ_PRESCALE_E4M3_B16,
+                      w_tensor_scale=float(prep["ts"]), indices=prep["idx"],
+                      codebooks=vq.pack_codebooks(cb))
+
+
+@pytest.mark.parametrize("N,K,M", [(128, 256, 1), (256, 512, 8), (128, 768, 64), (256, 512, 200)])
+def test_vq_linear_small(N, K, M):
+    w = synth.bf16_bits_to_f64(synth.to_bf16_bits(synth.student_t(60 + K, (N, K), 4.0)))
+    cb = synth.vq_codebooks(60, w)
+    prep = vq.prepare(w, cb)
+    lin = _vq_layer(w, cb, prep)
+    xb, _ = synth.activations_bf16(61, M, K, 0.0, 1.0)
+    y, y32 = _run(lin, xb)
+    lin.close()
+    ref, t = vq.forward(synth.bf16_bits_to_f64(xb), prep, cb)
+    check_fp32(y32, ref, t, f"vq N={N} K={K} M={M}")
+    check_bf16(y, ref, t, f"vq N={N} K={K} M={M}")
+
+
+_C2 = {}
+
+
+def _c2():
+    if not _C2:
+        w = synth.bf16_bits_to_f64(synth.to_bf16_bits(synth.student_t(2, (2560, 9728), 4.0)))
+        cb = synth.vq_codebooks(2, w)
+        _C2.update(w=w, cb=cb, prep=vq.prepare(w, cb))
+    return _C2
+
+
+@pytest.mark.parametrize("M", [1, 8, 64])
+def test_vq_workload_full_size(M):
+    """MXCode-style VQ layer at its full size: W [2560, 9728] Student-t(4), 64 x 64 QBlocks,
+    K = 256 entries of d = 4; X N(0,1); every output compared."""
+    c = _c2()
+    lin = _vq_layer(c["w"], c["cb"], c["prep"])
+    xb, _ = synth.activations_bf16(2, M, 9728, 0.0, 1.0)
+    y, y32 = _run(lin, xb)
+    lin.close()
+    ref, t = vq.forward(synth.bf16_bits_to_f64(xb), c["prep"], c["cb"])
+    check_fp32(y32, ref, t, f"C2 M={M}")
+    check_bf16(y, ref, t, f"C2 M={M}")
