@@ -1,15 +1,18 @@
 #!/usr/bin/env python
 """Benchmark of the W4A4 quantized linear layer on B200.
 
-One step = one pass of the layer's hot path over one batch: online MXFP4 quantization of the
-activation, then the tcgen05 block-scaled FP4 GEMM with the PRQuant tail K-extension (the two
-launches replayed from a CUDA graph, as a serving loop would issue them), on the
-PRQuant tail-residual workload (W [2560, 9728] -> K' = 9856, M = 2048 tokens, the prefill case).
-`value` is whole-job TFLOP/s (2*M*N*K' per step over all ranks), timed with CUDA events on the
-device with inputs resident; `e2e` is the same through the C ABI from pinned host buffers.
-Extra cases (decode M=16, mid M=512, the single MXFP4 linear layer) are reported under "cases".
+Headline workload (the MXCode VQ configuration): W [2560, 9728] stored as 8-bit indices into
+per-64x64-QBlock FP4 codebooks with E4M3-B16 scales and an FP32 tensor scale; activations bf16
+quantized online to E4M3-B16.  One step = the layer's whole hot path (E4M3-B16 activation
+quantization, in-GEMM codebook decode, block16 tcgen05 MMA, epilogue) at each of the decode
+batch sizes M = 1, 8 and 64.  Metric: weight-stream GB/s = weight bytes streamed (3 passes per
+step) / step time, whole job.  Launches are replayed from CUDA graphs; each step uses the next of
+R weight copies whose total exceeds the 126 MB L2, so every pass streams from HBM.
 
-Multi-GPU: the path shards into independent replicas (no collective); each rank runs the same
+Extra cases: the PRQuant tail-residual layer at M = 2048 (prefill, TFLOP/s), 512 and 16, and the
+single MXFP4 layer at M = 16.
+
+Multi-GPU: the layer shards into independent replicas (no collective); each rank runs the same
 workload on its own GPU and `value` sums the ranks' work over the slowest rank's time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qlinear|reference]
@@ -30,6 +33,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "W4A4 linear TFLOP/s (prefill) & weight-stream GB/s (decode) vs B200 roofline"
 NOMINAL_FP4_OVER_BF16 = 4.0      # 9 PFLOP/s dense FP4 / 2.25 PFLOP/s dense bf16
+L2_BYTES = 126 * 1024 * 1024
 
 
 def measured_peaks() -> dict:
@@ -43,47 +47,72 @@ def measured_peaks() -> dict:
 
 
 # ------------------------------------------------------------------------------ workloads
-def prquant_workload(M: int, seed: int = 3):
-    """PRQuant tail-residual layer: W [2560, 9728] bf16 Student-t(3), k = 128 tail channels;
-    X [M, 9728] N(0,1) with 0.5% outlier channels x50, permuted like the weight."""
+def _pack_nibbles(c: np.ndarray) -> np.ndarray:
+    return ((c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def make_vq(Ms=(1, 8, 64), seed: int = 2) -> dict:
+    """MXCode-style VQ layer: W [2560, 9728] Student-t(4) -> PreScale E4M3-B16 scales + FP32
+    tensor scale (library host preparation), seeded k-means FP4 codebooks per 64x64 QBlock
+    (256 entries of d = 4), 8-bit indices; X [M, 9728] N(0,1) for each M."""
+    import synth
+    import bit_quantized_moe_tcgen05_b200 as ql
+    N, K = 2560, 9728
+    wb = synth.to_bf16_bits(synth.student_t(seed, (N, K), 4.0))
+    cb = _pack_nibbles(synth.vq_codebooks(seed, synth.bf16_bits_to_f64(wb)))
+    ts, sb, idx = ql.prepare_vq_prescale(wb, cb)
+    xs = {M: synth.activations_bf16(seed, M, K, 0.0, 1.0)[0] for M in Ms}
+    wbytes = idx.nbytes + cb.nbytes + sb.nbytes
+    return dict(name=f"mxcode_vq_n{N}_k{K}_m{'-'.join(map(str, Ms))}", kind="vq", N=N, K=K, C=K,
+                Ms=list(Ms), xs=xs, weight_bytes=wbytes,
+                make=lambda: ql.QLinear(None, sb, wfmt=ql.QL_W_VQ_PRESCALE_E4M3_B16,
+                                        w_tensor_scale=float(ts), indices=idx, codebooks=cb),
+                oracle=dict(ts=ts, sb=sb, idx=idx, cb=cb))
+
+
+def make_prquant(M: int, seed: int = 3) -> dict:
+    """PRQuant tail-residual layer: W [2560, 9728] bf16 Student-t(3), k = 128 tail channels
+    (library host preparation); X [M, 9728] N(0,1) with 0.5% outlier channels x50, permuted."""
     import synth
     import bit_quantized_moe_tcgen05_b200 as ql
     N, C, k = 2560, 9728, 128
     wb = synth.to_bf16_bits(synth.student_t(seed, (N, C), 3.0))
-    perm, codes, scales = ql.prepare_prquant(wb, k)          # offline, library host code
+    perm, codes, scales = ql.prepare_prquant(wb, k)
     xb, _ = synth.activations_bf16(seed, M, C, 0.005, 50.0)
     xb = np.ascontiguousarray(xb[:, perm])
-    return dict(name=f"prquant_tail_n{N}_c{C}_k{k}_m{M}", N=N, C=C, k=k, M=M, codes=codes,
-                scales=scales, x=xb)
+    return dict(name=f"prquant_tail_n{N}_c{C}_k{k}_m{M}", kind="mx", N=N, K=C + k, C=C, Ms=[M],
+                xs={M: xb}, weight_bytes=codes.nbytes + scales.nbytes,
+                make=lambda: ql.QLinear(codes, scales, k_tail=k))
 
 
-def mxfp4_workload(M: int = 16, seed: int = 1):
+def make_mxfp4(M: int = 16, seed: int = 1) -> dict:
     """Single MXFP4 linear layer: X [16, 2048] N(0,1) with 1% outlier channels x20, W [2048, 2048]
     uniform E2M1 codes with E8M0 exponents uniform in [120, 130]."""
     import synth
+    import bit_quantized_moe_tcgen05_b200 as ql
     N = K = 2048
     codes = synth.uniform_nibble_bytes(seed, N, K)
     scales = synth.uniform_bytes(seed + 1, (N, K // 32), 120, 130)
     xb, _ = synth.activations_bf16(seed, M, K, 0.01, 20.0)
-    return dict(name=f"mxfp4_linear_n{N}_k{K}_m{M}", N=N, C=K, k=0, M=M, codes=codes,
-                scales=scales, x=xb)
+    return dict(name=f"mxfp4_linear_n{N}_k{K}_m{M}", kind="mx", N=N, K=K, C=K, Ms=[M], xs={M: xb},
+                weight_bytes=codes.nbytes + scales.nbytes,
+                make=lambda: ql.QLinear(codes, scales))
 
 
-def work_of(w) -> dict:
-    M, N, C, k = w["M"], w["N"], w["C"], w["k"]
-    Kp = C + k
-    flops = 2.0 * M * N * Kp
-    weight_bytes = N * Kp // 2 + N * Kp // 32
-    bytes_ = weight_bytes + M * C * 2 + M * N * 2          # W codes+scales, X bf16 in, Y bf16 out
-    gemm_bytes = weight_bytes + M * C // 2 + M * C // 32 + M * N * 2
-    return dict(flops=flops, bytes=bytes_, gemm_bytes=gemm_bytes, weight_bytes=weight_bytes)
+def flops_of(w, M) -> float:
+    return 2.0 * M * w["N"] * w["K"]
+
+
+def gemm_bytes_of(w, M) -> float:
+    """Algorithmic bytes of one GEMM launch: weight payload + quantized activation + bf16 y."""
+    sf = 16 if w["kind"] == "vq" else 32
+    return w["weight_bytes"] + M * w["C"] / 2 + M * w["C"] / sf + 2.0 * M * w["N"]
 
 
 # ------------------------------------------------------------------------------ clocks
 class ClockSampler:
     def __init__(self, device_index: int):
         self.p = None
-        self.path = None
         self.dev = device_index
 
     def __enter__(self):
@@ -129,159 +158,180 @@ class ClockSampler:
                 for nm, v in zip(names, parts[5:9]):
                     if v.lower() == "active":
                         reasons.add(nm)
-        med = float(np.median(sm)) if sm else None
-        return {"sm_mhz": med, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
 
 
 # ------------------------------------------------------------------------------ GPU arm
-def _time_graph(graph, steps: int, flush, stream) -> float:
-    """Mean device time (ms) of `steps` replays of a captured graph, L2 flushed before each."""
+def _elapsed(fn, reps: int, stream) -> float:
+    """Device time (ms) of `reps` calls of fn, bracketed by synchronisation and CUDA events."""
     import torch
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(steps)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    for a, b in evs:
-        flush()
-        a.record(stream)
-        graph.replay()
-        b.record(stream)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
     torch.cuda.synchronize()
-    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    return a.elapsed_time(b)
 
 
-def run_case(w, steps: int, warmup: int, device, flush, e2e: bool = False):
-    """Times `steps` forwards (quantize + GEMM) replayed from CUDA graphs, so the numbers are
-    device time without host launch gaps.  Also times each kernel alone the same way, and (e2e)
-    the public forward call from pinned host memory with the copies inside the timed region."""
+def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes: int = 0):
+    """Device time per step (ms) of w's forwards (every M of w["Ms"] per step), replayed from a
+    CUDA graph over R rotating weight copies with R * weight bytes > L2 (or with an explicit L2
+    flush before each replay), plus per-kernel times measured the same way, plus (e2e) the public
+    forward call from pinned host memory with the copies inside the timed region."""
     import torch
     import bit_quantized_moe_tcgen05_b200 as ql
-    lin = ql.QLinear(w["codes"], w["scales"], k_tail=w["k"])
-    M, N = w["M"], w["N"]
-    x = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).to(device)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-    ws = torch.empty(lin.workspace_bytes(M), dtype=torch.uint8, device=device)
-    for _ in range(warmup):                       # eager warm-up (also sets kernel attributes)
-        lin.quantize_input(x, ws)
-        lin.gemm(M, y, ws)
+    R = 1 if flush_bytes else min(64, L2_BYTES // w["weight_bytes"] + 2)
+    layers = [w["make"]() for _ in range(R)]
+    Ms = w["Ms"]
+    xs = {M: torch.from_numpy(w["xs"][M].view(np.int16)).view(torch.bfloat16).to(device) for M in Ms}
+    ys = {M: torch.empty((M, w["N"]), dtype=torch.bfloat16, device=device) for M in Ms}
+    wss = {M: torch.empty(layers[0].workspace_bytes(M), dtype=torch.uint8, device=device) for M in Ms}
+    flush_buf = torch.empty(flush_bytes, dtype=torch.uint8, device=device) if flush_bytes else None
+
+    def fwd(layer, M):
+        layer.quantize_input(xs[M], wss[M])
+        layer.gemm(M, ys[M], wss[M])
+
+    for _ in range(warmup):
+        for layer in layers:
+            for M in Ms:
+                fwd(layer, M)
     ql.check()
-    g_step, g_q, g_g = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):
-        lin.quantize_input(x, ws)
-        lin.gemm(M, y, ws)
-    with torch.cuda.graph(g_q):
-        lin.quantize_input(x, ws)
-    with torch.cuda.graph(g_g):
-        lin.gemm(M, y, ws)
     stream = torch.cuda.current_stream(device)
-    for g in (g_step, g_q, g_g):
+    g_all, g_q, g_g = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all):
+        for layer in layers:
+            for M in Ms:
+                fwd(layer, M)
+    with torch.cuda.graph(g_q):
+        for layer in layers:
+            for M in Ms:
+                layer.quantize_input(xs[M], wss[M])
+    with torch.cuda.graph(g_g):
+        for layer in layers:
+            for M in Ms:
+                layer.gemm(M, ys[M], wss[M])
+    for g in (g_all, g_q, g_g):
         for _ in range(warmup):
             g.replay()
     ql.check()
-    step_ms = _time_graph(g_step, steps, flush, stream)
-    q_ms = _time_graph(g_q, steps, flush, stream)
-    g_ms = _time_graph(g_g, steps, flush, stream)
+    reps = max(1, -(-steps // R))                    # graph replays so that >= steps steps run
+
+    def timed(graph):
+        if flush_buf is None:
+            return _elapsed(graph.replay, reps, stream) / (reps * R)
+        tot = 0.0
+        for _ in range(reps):
+            flush_buf.fill_(1)
+            tot += _elapsed(graph.replay, 1, stream)
+        return tot / (reps * R)
+
+    out = dict(R=R, step_ms=timed(g_all), quant_ms=timed(g_q), gemm_ms=timed(g_g), steps=reps * R)
     ql.check()
-    out = dict(step_ms=step_ms, quant_ms=q_ms, gemm_ms=g_ms, launches=2 * steps)
     if e2e:
-        xh = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
-        yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-        xd = torch.empty_like(x)
+        xh = {M: torch.from_numpy(w["xs"][M].view(np.int16)).view(torch.bfloat16).pin_memory()
+              for M in Ms}
+        yh = {M: torch.empty((M, w["N"]), dtype=torch.bfloat16).pin_memory() for M in Ms}
+        xd = {M: torch.empty_like(xs[M]) for M in Ms}
+        count = [0]
+
+        def e2e_step():
+            layer = layers[count[0] % R]
+            count[0] += 1
+            for M in Ms:
+                xd[M].copy_(xh[M], non_blocking=True)
+                layer.forward(xd[M], out=ys[M], ws=wss[M])
+                yh[M].copy_(ys[M], non_blocking=True)
+
         for _ in range(warmup):
-            xd.copy_(xh, non_blocking=True)
-            lin.forward(xd, out=y, ws=ws)
-            yh.copy_(y, non_blocking=True)
-        torch.cuda.synchronize(device)
-        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-        for i in range(steps):
-            flush()
-            e0[i].record(stream)
-            xd.copy_(xh, non_blocking=True)
-            lin.forward(xd, out=y, ws=ws)
-            yh.copy_(y, non_blocking=True)
-            e1[i].record(stream)
-        torch.cuda.synchronize(device)
+            e2e_step()
+        out["e2e_ms"] = _elapsed(e2e_step, reps * R, stream) / (reps * R)
+        out["h2d"] = sum(M * w["C"] * 2 for M in Ms)
+        out["d2h"] = sum(M * w["N"] * 2 for M in Ms)
         ql.check()
-        out["e2e_ms"] = float(np.mean([e0[i].elapsed_time(e1[i]) for i in range(steps)]))
-        out["h2d"] = M * w["C"] * 2
-        out["d2h"] = M * N * 2
-        out["launches"] += 2 * steps
-    del g_step, g_q, g_g
-    lin.close()
+    del g_all, g_q, g_g
+    for layer in layers:
+        layer.close()
     return out
 
 
-def cpu_baseline(w, budget_s: float = 15.0) -> dict:
-    """The oracle as it stands (numpy, fp64) on a bounded sample of the same workload: the first
-    m_s tokens through quantize + augmented GEMM against the full weight."""
-    from oracle import formats as F, mx, gemm as G
+# ------------------------------------------------------------------------------ CPU baseline
+def cpu_baseline_vq(w, budget_s: float = 20.0) -> dict:
+    """The oracle as it stands (numpy, fp64) on a bounded sample of the headline workload: whole
+    forwards (E4M3-B16 activation quantization, codebook decode, dequantized fp64 GEMM) at the
+    workload's batch sizes, as many as fit the time budget."""
+    from oracle import vq
     import synth
-    N, C, k = w["N"], w["C"], w["k"]
-    codes = F.unpack_nibbles(w["codes"])
-    m_s = 1
-    xd_all = synth.bf16_bits_to_f64(w["x"])
-    best = None
-    while True:
-        t0 = time.perf_counter()
-        xd = xd_all[:m_s]
-        xc, xs = mx.quantize_e8m0_b32(xd)
-        if k:
-            xc = np.concatenate([xc, xc[:, C - k:]], axis=1)
-            xs = np.concatenate([xs, xs[:, (C - k) // 32:]], axis=1)
-        y = G.gemm_ref(mx.dequant_e8m0_b32(xc, xs), mx.dequant_e8m0_b32(codes, w["scales"]))
-        dt = time.perf_counter() - t0
-        best = (m_s, dt)
-        if dt > budget_s / 3 or m_s >= w["M"]:
+    o = w["oracle"]
+    cb = np.empty(o["cb"].shape[:-1] + (4,), np.uint8)
+    cb[..., 0::2] = o["cb"] & 0xF
+    cb[..., 1::2] = o["cb"] >> 4
+    prep = dict(ts=o["ts"], sb=o["sb"], idx=o["idx"])
+    done, t0 = [], time.perf_counter()
+    for M in w["Ms"] * 4:
+        vq.forward(synth.bf16_bits_to_f64(w["xs"][M]), prep, cb)
+        done.append(M)
+        if time.perf_counter() - t0 > budget_s:
             break
-        m_s = min(w["M"], m_s * 4)
-    m_s, dt = best
-    flops = 2.0 * m_s * N * (C + k)
-    cores = len(os.sched_getaffinity(0))
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{m_s} of {w['M']} tokens of {w['name']} (quantize + fp64 GEMM incl. weight "
-                      f"dequant), {dt:.2f} s; numpy BLAS may use every core"}
+    dt = time.perf_counter() - t0
+    return {"value": len(done) * w["weight_bytes"] / dt / 1e9, "unit": "GB/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"{len(done)} forwards (M = {done}) of {w['name']}, {dt:.1f} s; "
+                      "numpy fp64, BLAS may use every core"}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="qlinear", choices=["qlinear", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cases", default="all", choices=["all", "headline"])
-    ap.add_argument("--workload", default="prquant_m2048",
-                    choices=["prquant_m2048", "prquant_m512", "prquant_m16", "mxfp4_m16"],
-                    help="headline workload (default: the PRQuant prefill case)")
+    ap.add_argument("--cases", default="all", choices=["all", "none"])
+    ap.add_argument("--workload", default="vq", choices=["vq", "prquant_m2048", "prquant_m512",
+                                                         "prquant_m16", "mxfp4_m16"])
     args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
-
+    args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    head = {"prquant_m2048": lambda: prquant_workload(2048),
-            "prquant_m512": lambda: prquant_workload(512),
-            "prquant_m16": lambda: prquant_workload(16),
-            "mxfp4_m16": lambda: mxfp4_workload(16)}[args.workload]()
-    wk = work_of(head)
+    builders = {"vq": make_vq, "prquant_m2048": lambda: make_prquant(2048),
+                "prquant_m512": lambda: make_prquant(512), "prquant_m16": lambda: make_prquant(16),
+                "mxfp4_m16": lambda: make_mxfp4(16)}
+    head = builders[args.workload]()
+    decode = head["kind"] == "vq" or max(head["Ms"]) <= 64
+    unit = "GB/s" if decode else "TFLOP/s"
+
+    def per_step_units(w):
+        if decode:
+            return len(w["Ms"]) * w["weight_bytes"] / 1e9
+        return sum(flops_of(w, M) for M in w["Ms"]) / 1e12
+
+    config = {"workload": head["name"], "N": head["N"], "K": head["K"], "M": head["Ms"],
+              "parallelism": "replicas" if world > 1 else "single",
+              "l2": ("rotating weight copies totalling > 126 MB L2 (no flush)" if decode
+                     else "flushed before each step (256 MiB write)")}
 
     if args.impl == "reference":
         if rank != 0:
             return
-        cb = cpu_baseline(head)
-        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "TFLOP/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": wk["flops"] / (cb["value"] * 1e12) * 1e3,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": head["name"], "M": head["M"],
-                                                "N": head["N"], "K_aug": head["C"] + head["k"],
-                                                "parallelism": "replicas"},
-                "cpu_baseline": cb,
-                "e2e": {"value": cb["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line))
+        if head["kind"] != "vq":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the "
+                              "oracle on the headline VQ workload only"}))
+            return
+        cb = cpu_baseline_vq(head)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": cb["unit"],
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_step_units(head) / cb["value"] * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config, "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": cb["unit"], "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
         return
 
     import torch
@@ -291,11 +341,6 @@ def main():
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    peaks = measured_peaks()
-    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
-
-    def flush():
-        flush_buf.fill_(1)
 
     def barrier():
         if world > 1:
@@ -303,67 +348,79 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(device)
 
-    # warm up + headline timing (device) with clock sampling
+    peaks = measured_peaks()
     barrier()
     with ClockSampler(local) as clk:
-        res = run_case(head, args.steps, args.warmup, device, flush, e2e=True)
+        res = run_case(head, args.steps, args.warmup, device, e2e=True,
+                       flush_bytes=0 if decode else 256 << 20)
     barrier()
-    step_ms = res["step_ms"]
-    e2e_ms = res["e2e_ms"]
+    step_ms, e2e_ms = res["step_ms"], res["e2e_ms"]
     if world > 1:
         import torch.distributed as dist
         t = torch.tensor([step_ms, e2e_ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         step_ms, e2e_ms = float(t[0]), float(t[1])
-    value = world * wk["flops"] / (step_ms * 1e-3) / 1e12
-    e2e_val = world * wk["flops"] / (e2e_ms * 1e-3) / 1e12
+    units = per_step_units(head)
+    value = world * units / (step_ms * 1e-3)
+    e2e_val = world * units / (e2e_ms * 1e-3)
 
     fp4_peak = peaks["bf16"] * NOMINAL_FP4_OVER_BF16
-    gemm_tflops = wk["flops"] / (res["gemm_ms"] * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                "frac": gemm_tflops / fp4_peak, "traffic": None,
-                "kernel": "fp4_gemm_kernel (tcgen05.mma kind::mxf4 block32)",
-                "peak_source": f"{peaks['src']} bf16 burst {peaks['bf16']} x {NOMINAL_FP4_OVER_BF16}"
-                               " (nominal FP4/bf16 dense ratio)"}
+    nl = len(head["Ms"])
+    if decode:
+        alg = sum(gemm_bytes_of(head, M) for M in head["Ms"]) / nl
+        ach = alg / (res["gemm_ms"] / nl * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm"], "traffic": None,
+                    "kernel": "fp4_gemm_kernel (block16 MMA, VQ decode)" if head["kind"] == "vq"
+                    else "fp4_gemm_kernel (mxf4)",
+                    "algorithmic_bytes_per_launch": alg,
+                    "peak_source": f"{peaks['src']} HBM copy bandwidth"}
+    else:
+        alg = sum(flops_of(head, M) for M in head["Ms"]) / nl
+        ach = alg / (res["gemm_ms"] / nl * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s",
+                    "frac": ach / fp4_peak, "traffic": None, "kernel": "fp4_gemm_kernel (mxf4)",
+                    "algorithmic_flops_per_launch": alg,
+                    "peak_source": f"{peaks['src']} bf16 burst {peaks['bf16']} x 4 (nominal FP4/bf16)"}
 
     cases = {}
     if args.cases == "all":
-        for wl in (prquant_workload(16), prquant_workload(512), mxfp4_workload(16)):
-            r = run_case(wl, args.steps, args.warmup, device, flush)
-            wkk = work_of(wl)
+        for wl, flush in ((make_prquant(2048), 256 << 20), (make_prquant(512), 0),
+                          (make_prquant(16), 0), (make_mxfp4(16), 0)):
+            r = run_case(wl, 8, args.warmup, device, flush_bytes=flush)
+            M = wl["Ms"][0]
             cases[wl["name"]] = {
                 "step_us": r["step_ms"] * 1e3, "gemm_us": r["gemm_ms"] * 1e3,
                 "quant_us": r["quant_ms"] * 1e3,
-                "tflops": wkk["flops"] / (r["step_ms"] * 1e-3) / 1e12,
-                "weight_stream_gbs": wkk["weight_bytes"] / (r["gemm_ms"] * 1e-3) / 1e9,
-                "gemm_hbm_frac": wkk["gemm_bytes"] / (r["gemm_ms"] * 1e-3) / 1e9 / peaks["hbm"],
-                "gemm_tensor_frac": wkk["flops"] / (r["gemm_ms"] * 1e-3) / 1e12 / fp4_peak,
-            }
+                "tflops": flops_of(wl, M) / (r["step_ms"] * 1e-3) / 1e12,
+                "gemm_tflops": flops_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e12,
+                "gemm_tensor_frac": flops_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e12 / fp4_peak,
+                "weight_stream_gbs": wl["weight_bytes"] / (r["gemm_ms"] * 1e-3) / 1e9,
+                "gemm_hbm_frac": gemm_bytes_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e9 / peaks["hbm"],
+                "l2": "flushed (256 MiB write)" if flush else f"{r['R']} rotating weight copies"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
+    kernels_per_fwd = 3 if head["kind"] == "vq" else 2
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": res["steps"],
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp4-e2m1/e8m0 (fp32 accumulate, bf16 out)",
-        "data": "synthetic",
-        "config": {"workload": head["name"], "M": head["M"], "N": head["N"], "K": head["C"],
-                   "k_tail": head["k"], "K_aug": head["C"] + head["k"],
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "flushed between steps (256 MiB write)"},
-        "roofline": roofline,
-        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": res["h2d"],
+        "vs_baseline": None,
+        "dtype": ("fp4-e2m1 E4M3-B16 (+fp32 tensor scales), fp32 accumulate, bf16 out"
+                  if head["kind"] == "vq" else "fp4-e2m1 E8M0-B32, fp32 accumulate, bf16 out"),
+        "data": "synthetic", "config": config, "roofline": roofline,
+        "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
-        "gpu_launches": res["launches"],
+        "gpu_launches": kernels_per_fwd * nl * res["steps"],
         "clocks": clk.summary(),
-        "kernel_us": {"quant_mx_e8m0_b32": res["quant_ms"] * 1e3, "fp4_gemm": res["gemm_ms"] * 1e3},
+        "kernel_us_per_step": {"quantize": res["quant_ms"] * 1e3, "gemm": res["gemm_ms"] * 1e3},
         "cases": cases,
     }
-    if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(head)
+    if not args.no_cpu_baseline and head["kind"] == "vq":
+        line["cpu_baseline"] = cpu_baseline_vq(head)
     print(json.dumps(line))
 
 

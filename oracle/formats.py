@@ -133,3 +133,10 @@ def int4_encode(q: np.ndarray) -> np.ndarray:
     q = np.asarray(q).astype(np.int64)
     assert np.all(np.abs(q) <= 7)
     return (q & 0xF).astype(np.uint8)
+
+
+# --- bf16 ---------------------------------------------------------------------------------
+def bf16_decode(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64 (exact: the upper half of an IEEE binary32)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)

@@ -119,3 +119,54 @@ def vq_codebooks(seed: int, w: np.ndarray, qn: int = 64, qk: int = 64, entries: 
         snap = np.abs(cent[..., None] - _E2M1_GRID).argmin(-1)
         out[c0:c0 + B] = _E2M1_CODE[snap]
     return out.reshape(QR, QC, entries, 4)
+
+
+def zipf_router_logits(seed: int, T: int, E: int = 128, s: float = 1.1) -> np.ndarray:
+    """Router logits [T, E] fp32 for a Zipf(s) expert popularity: p_e ~ r_e^-s with r a seeded
+    permutation of the ranks 1..E; logit = ln p_e + Gumbel(0, 1) noise, so that the top-k of a
+    token is a Gumbel-top-k draw from p without replacement."""
+    g = rng(seed * 13 + 5)
+    ranks = g.permutation(E) + 1.0
+    p = ranks ** -s
+    p /= p.sum()
+    u = g.random((T, E))
+    u = np.clip(u, 1e-300, 1.0 - 1e-16)
+    return (np.log(p)[None, :] - np.log(-np.log(u))).astype(np.float32)
+
+
+def cluster_rows(seed: int, rows: int, K: int, nu: float = 4.0, C: int = 16,
+                 iters: int = 6) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row C-centroid codebooks fit by 1-D k-means (Lloyd, quantile start) on Student-t(nu)
+    weights [rows, K] (data synthesis only).  Returns (centroids as bf16 bits [rows, C], ascending;
+    4-bit indices [rows, K] of the nearest bf16 centroid, ties to the lower index)."""
+    w = student_t(seed, (rows, K), nu).astype(np.float64)
+    srt = np.sort(w, axis=1)
+    lo, hi = srt[:, :1], srt[:, -1:]
+    span = float((hi - lo).max()) * 2.0 + 1.0
+    key = (np.arange(rows)[:, None] * span + (srt - lo)).reshape(-1)     # row-major ascending
+    cs = np.concatenate([np.zeros((rows, 1)), np.cumsum(srt, axis=1)], axis=1)
+    q = (np.arange(C) + 0.5) / C
+    cent = srt[:, np.minimum((q * K).astype(int), K - 1)]
+    rows_off = np.arange(rows)[:, None]
+    for _ in range(iters):
+        mids = 0.5 * (cent[:, 1:] + cent[:, :-1])
+        pos = np.searchsorted(key, (rows_off * span + (mids - lo)).reshape(-1), side="left")
+        pos = pos.reshape(rows, C - 1) - rows_off * K
+        b = np.concatenate([np.zeros((rows, 1), int), pos, np.full((rows, 1), K)], axis=1)
+        cnt = np.diff(b, axis=1)
+        sums = np.take_along_axis(cs, b[:, 1:], 1) - np.take_along_axis(cs, b[:, :-1], 1)
+        cent = np.where(cnt > 0, sums / np.maximum(cnt, 1), cent)
+        cent = np.sort(cent, axis=1)
+    cbits = to_bf16_bits(cent)
+    cq = bf16_bits_to_f64(cbits)
+    order = np.argsort(cq, axis=1, kind="stable")
+    cbits = np.take_along_axis(cbits, order, 1)
+    cq = np.take_along_axis(cq, order, 1)
+    # nearest centroid in the original order: number of midpoints strictly below the value
+    mids = 0.5 * (cq[:, 1:] + cq[:, :-1])
+    lo2 = np.minimum(w.min(axis=1, keepdims=True), cq[:, :1])
+    span2 = float((np.maximum(w.max(axis=1, keepdims=True), cq[:, -1:]) - lo2).max()) * 2.0 + 1.0
+    mkey = (rows_off * span2 + (mids - lo2)).reshape(-1)
+    idx = np.searchsorted(mkey, (rows_off * span2 + (w - lo2)).reshape(-1), side="left")
+    idx = idx.reshape(rows, K) - rows_off * (C - 1)
+    return cbits, np.clip(idx, 0, C - 1).astype(np.uint8)
