@@ -32,7 +32,8 @@ EXPORTED_SYMBOLS = (
     "ql_version", "ql_last_error", "qlinear_create", "qlinear_destroy", "qlinear_workspace_bytes",
     "qlinear_forward", "quantize_act", "ql_check", "qlinear_prepare_prquant",
     "qlinear_quantize_input", "qlinear_gemm", "qlinear_forward_fixed_scratch",
-    "qlinear_prepare_vq_prescale",
+    "qlinear_prepare_vq_prescale", "moe_create", "moe_destroy", "moe_capture_intermediate",
+    "moe_workspace_bytes", "moe_workspace_layout", "moe_grouped_forward",
 )
 
 
@@ -56,6 +57,12 @@ class WeightDesc(ctypes.Structure):
     ]
 
 
+class MoeWsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "counts", "offsets", "entries", "ids", "gates", "x_codes", "x_scales", "x_dq", "h_codes",
+        "h_scales", "h_dq", "h32", "yslot", "total")]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing; build it with "
@@ -76,6 +83,13 @@ def _load() -> ctypes.CDLL:
         "ql_check": [vp],
         "qlinear_prepare_prquant": [vp, i64, i64, i32, vp, vp, vp],
         "qlinear_prepare_vq_prescale": [vp, i64, i64, vp, i32, i32, vp, vp, vp],
+        "moe_create": [ctypes.POINTER(WeightDesc), ctypes.POINTER(WeightDesc), i32, i32, vp,
+                       ctypes.POINTER(vp)],
+        "moe_destroy": [vp],
+        "moe_capture_intermediate": [vp, i32],
+        "moe_workspace_bytes": [vp, i64, ctypes.POINTER(sz)],
+        "moe_workspace_layout": [vp, i64, ctypes.POINTER(MoeWsLayout)],
+        "moe_grouped_forward": [vp, vp, i64, vp, vp, vp, vp, vp, vp, sz, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -264,3 +278,80 @@ def prepare_vq_prescale(w_bf16_bits: np.ndarray, codebooks_packed: np.ndarray, q
                                         scales.ctypes.data, idx.ctypes.data),
         "qlinear_prepare_vq_prescale")
     return np.float32(ts[0]), scales, idx
+
+
+def _pack4(idx: np.ndarray) -> np.ndarray:
+    idx = np.ascontiguousarray(idx, dtype=np.uint8)
+    return ((idx[..., 0::2] & 0xF) | ((idx[..., 1::2] & 0xF) << 4)).astype(np.uint8)
+
+
+class MoE:
+    """Routed MoE FFN with CodeQuant-style cluster-codebook experts (see moe_create in qlinear.h).
+
+    gu_idx uint8 [E*2I, H] 4-bit indices (values 0..15), gu_cent bf16 bit patterns [E*2I, 16];
+    dn_idx [E*H, I], dn_cent [E*H, 16]; per expert the gate rows come first, then the up rows."""
+
+    def __init__(self, gu_idx, gu_cent, dn_idx, dn_cent, E: int, top_k: int, stream=None):
+        gi, di = _pack4(gu_idx), _pack4(dn_idx)
+        gc = np.ascontiguousarray(gu_cent, dtype=np.uint16)
+        dc = np.ascontiguousarray(dn_cent, dtype=np.uint16)
+        self.E, self.k = E, top_k
+        self.H = gu_idx.shape[1]
+        self.I = dn_idx.shape[1]
+        g = WeightDesc(wfmt=QL_W_CLUSTER4_ROW16_BF16, N=gu_idx.shape[0], K=self.H,
+                       codes=gi.ctypes.data, codebooks=gc.ctypes.data)
+        d = WeightDesc(wfmt=QL_W_CLUSTER4_ROW16_BF16, N=dn_idx.shape[0], K=self.I,
+                       codes=di.ctypes.data, codebooks=dc.ctypes.data)
+        h = ctypes.c_void_p()
+        _ok(lib.moe_create(ctypes.byref(g), ctypes.byref(d), E, top_k, _stream(stream),
+                           ctypes.byref(h)), "moe_create")
+        self._h = h
+        self._ws = None
+
+    def capture_intermediate(self, enable: bool = True) -> None:
+        _ok(lib.moe_capture_intermediate(self._h, 1 if enable else 0), "moe_capture_intermediate")
+
+    def workspace_bytes(self, T: int) -> int:
+        n = ctypes.c_size_t()
+        _ok(lib.moe_workspace_bytes(self._h, T, ctypes.byref(n)), "moe_workspace_bytes")
+        return n.value
+
+    def layout(self, T: int) -> dict:
+        lay = MoeWsLayout()
+        _ok(lib.moe_workspace_layout(self._h, T, ctypes.byref(lay)), "moe_workspace_layout")
+        return {n: getattr(lay, n) for n, _ in MoeWsLayout._fields_}
+
+    def workspace(self, T: int, device):
+        import torch
+        need = self.workspace_bytes(T)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=device)
+        return self._ws
+
+    def forward(self, x, logits, out=None, out_f32=None, ids_out=None, gates_out=None, ws=None,
+                stream=None):
+        import torch
+        assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()
+        assert logits.is_cuda and logits.dtype == torch.float32 and logits.is_contiguous()
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.bfloat16, device=x.device)
+        if ws is None:
+            ws = self.workspace(T, x.device)
+        _ok(lib.moe_grouped_forward(self._h, x.data_ptr(), T, logits.data_ptr(), out.data_ptr(),
+                                    _ptr(out_f32), _ptr(ids_out), _ptr(gates_out), ws.data_ptr(),
+                                    ws.numel(), _stream(stream)), "moe_grouped_forward")
+        return out
+
+    __call__ = forward
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib.moe_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -17,6 +17,7 @@
 #include "ptx.cuh"
 #include "quant_act.cuh"
 #include "gemm_fp4.cuh"
+#include "moe.cuh"
 
 namespace {
 
@@ -73,6 +74,22 @@ ql_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner_bytes, u
                   swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return QL_OK;
+}
+
+// 2-D bf16 tensor [rows, cols] with a 128-byte swizzled box [box_rows, 64 elements].
+ql_status make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                         uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled (bf16) failed (%d)", int(r));
   return QL_OK;
 }
 
@@ -200,7 +217,7 @@ void repack_sf_tiled(const uint8_t* plain, int64_t rows, int64_t cols, int atoms
 
 ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
                           uint8_t* st, int st_atoms, int* zero_words, int nzero,
-                          cudaStream_t s) {
+                          cudaStream_t s, __nv_bfloat16* deq = nullptr) {
   const long total = static_cast<long>(M) * (K / 32);
   const long threads = std::max<long>(total, nzero);
   if (threads == 0) return QL_OK;
@@ -209,7 +226,7 @@ ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, u
   ql::quant_mx_e8m0_b32_kernel<<<static_cast<unsigned>(grid), block, 0, s>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K),
       static_cast<int>(K), codes, static_cast<int>(K / 2), sp, static_cast<int>(K / 32), st,
-      st_atoms, zero_words, nzero);
+      st_atoms, zero_words, nzero, deq);
   QL_CUDA(cudaGetLastError());
   return QL_OK;
 }
@@ -446,6 +463,223 @@ ql_status ql_check(ql_stream_t stream) {
     QL_CUDA(cudaMemcpyToSymbol(ql::g_dev_error, &zero, sizeof(int)));
     return fail(QL_ERR_TIMEOUT, "device wait expired (code %d, site %d)", err, site);
   }
+  return QL_OK;
+}
+
+}  // extern "C"
+
+// ========================================================================= MoE
+struct ql_moe {
+  int E, k, H, I;
+  uint8_t* d_idx_gu = nullptr;        // [E*2I, H/2] 4-bit indices, kernel row order
+  uint8_t* d_idx_d = nullptr;         // [E*H, I/2]
+  __nv_bfloat16* d_cent_gu = nullptr; // [E*2I][16]
+  __nv_bfloat16* d_cent_d = nullptr;  // [E*H][16]
+  CUtensorMap tm_idx_gu, tm_idx_d;
+  bool capture_h32 = false;
+};
+
+namespace {
+
+constexpr int kMoeBN = 128;
+
+struct MoePlan {
+  size_t counts, offsets, entries, ids, gates, x_codes, x_scales, x_dq, h_codes, h_scales, h_dq,
+      h32, yslot, total;
+};
+
+MoePlan plan_moe(const ql_moe* m, int64_t T) {
+  MoePlan p{};
+  const size_t P = static_cast<size_t>(T) * m->k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + std::max<size_t>(bytes, 1), 256);
+    return o;
+  };
+  p.counts = take(sizeof(int) * m->E);
+  p.offsets = take(sizeof(int) * (m->E + 1));
+  p.entries = take(sizeof(int) * P);
+  p.ids = take(sizeof(int) * P);
+  p.gates = take(sizeof(float) * P);
+  p.x_codes = take(static_cast<size_t>(T) * m->H / 2);
+  p.x_scales = take(static_cast<size_t>(T) * m->H / 32);
+  p.x_dq = take(static_cast<size_t>(T) * m->H * 2);
+  p.h_codes = take(P * m->I / 2);
+  p.h_scales = take(P * m->I / 32);
+  p.h_dq = take(P * m->I * 2);
+  p.h32 = take(m->capture_h32 ? P * m->I * 4 : 0);
+  p.yslot = take(P * m->H * 4);
+  p.total = off;
+  return p;
+}
+
+template <int BN, bool GATEUP>
+ql_status launch_moe_gemm(const CUtensorMap& ti, const CUtensorMap& tb, const ql::MoeGemmArgs& a,
+                          int grid, cudaStream_t s) {
+  using Cfg = ql::MoeCfg<BN>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    QL_CUDA(cudaFuncSetAttribute(ql::moe_gemm_kernel<BN, GATEUP>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+    attr_done[dev] = true;
+  }
+  ql::moe_gemm_kernel<BN, GATEUP><<<grid, 192, Cfg::kSmemBytes, s>>>(ti, tb, a);
+  QL_CUDA(cudaGetLastError());
+  return QL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ql_status moe_create(const ql_weight_desc* gu, const ql_weight_desc* dn, int32_t E, int32_t top_k,
+                     ql_stream_t stream, ql_moe** out) {
+  if (gu == nullptr || dn == nullptr || out == nullptr) return fail(QL_ERR_INVALID_ARG, "null args");
+  *out = nullptr;
+  if (gu->wfmt != QL_W_CLUSTER4_ROW16_BF16 || dn->wfmt != QL_W_CLUSTER4_ROW16_BF16)
+    return fail(QL_ERR_UNSUPPORTED, "MoE experts must use QL_W_CLUSTER4_ROW16_BF16");
+  if (E <= 0 || E > 256 || top_k <= 0 || top_k > 16 || top_k > E)
+    return fail(QL_ERR_UNSUPPORTED, "need 0 < top_k <= 16, top_k <= E <= 256");
+  if (gu->codes == nullptr || gu->codebooks == nullptr || dn->codes == nullptr ||
+      dn->codebooks == nullptr)
+    return fail(QL_ERR_INVALID_ARG, "codes and codebooks must be non-null host pointers");
+  if (gu->N % E != 0 || dn->N % E != 0) return fail(QL_ERR_INVALID_ARG, "N must be E * rows");
+  const int64_t two_i = gu->N / E, H = gu->K, I = dn->K;
+  if (dn->N / E != H || two_i != 2 * I)
+    return fail(QL_ERR_INVALID_ARG, "gate/up must be [E*2I, H] and down [E*H, I]");
+  if (I % 64 != 0 || H % 128 != 0 || H % 64 != 0 || I < 64)
+    return fail(QL_ERR_UNSUPPORTED, "MoE needs I %% 64 == 0 and H %% 128 == 0");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto* m = new ql_moe();
+  m->E = E; m->k = top_k; m->H = static_cast<int>(H); m->I = static_cast<int>(I);
+  // gate/up rows in kernel order: per expert, per 128-row tile: 64 gate rows then the 64 up
+  // rows with the same intermediate index, so SwiGLU pairs sit in one accumulator tile.
+  const size_t rgu = static_cast<size_t>(E) * two_i;
+  std::vector<uint8_t> idx_gu(rgu * (H / 2));
+  std::vector<uint16_t> cent_gu(rgu * 16);
+  const uint8_t* src_idx = static_cast<const uint8_t*>(gu->codes);
+  const uint16_t* src_c = static_cast<const uint16_t*>(gu->codebooks);
+  for (int64_t e = 0; e < E; ++e)
+    for (int64_t r = 0; r < two_i; ++r) {
+      const int64_t tile = r / 128, w = r % 128;
+      const int64_t srow = (w < 64) ? tile * 64 + w : I + tile * 64 + (w - 64);
+      const size_t d = e * two_i + r, sr = e * two_i + srow;
+      std::memcpy(&idx_gu[d * (H / 2)], src_idx + sr * (H / 2), H / 2);
+      std::memcpy(&cent_gu[d * 16], src_c + sr * 16, 32);
+    }
+  const size_t rd = static_cast<size_t>(E) * H;
+  auto cleanup = [&](ql_status st) {
+    cudaFree(m->d_idx_gu); cudaFree(m->d_idx_d); cudaFree(m->d_cent_gu); cudaFree(m->d_cent_d);
+    delete m;
+    return st;
+  };
+  if (cudaMalloc(&m->d_idx_gu, idx_gu.size()) != cudaSuccess ||
+      cudaMalloc(&m->d_idx_d, rd * (I / 2)) != cudaSuccess ||
+      cudaMalloc(&m->d_cent_gu, cent_gu.size() * 2) != cudaSuccess ||
+      cudaMalloc(&m->d_cent_d, rd * 32) != cudaSuccess)
+    return cleanup(fail(QL_ERR_OOM, "cudaMalloc of MoE weights failed"));
+  if (cudaMemcpyAsync(m->d_idx_gu, idx_gu.data(), idx_gu.size(), cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(m->d_idx_d, dn->codes, rd * (I / 2), cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(m->d_cent_gu, cent_gu.data(), cent_gu.size() * 2, cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(m->d_cent_d, dn->codebooks, rd * 32, cudaMemcpyHostToDevice, s) ||
+      cudaStreamSynchronize(s))
+    return cleanup(fail(QL_ERR_CUDA, "MoE weight upload failed"));
+  ql_status st = make_tmap_u8(&m->tm_idx_gu, m->d_idx_gu, H / 2, rgu, H / 2, 32, 128, false);
+  if (st == QL_OK) st = make_tmap_u8(&m->tm_idx_d, m->d_idx_d, I / 2, rd, I / 2, 32, 128, false);
+  if (st != QL_OK) return cleanup(st);
+  *out = m;
+  return QL_OK;
+}
+
+ql_status moe_destroy(ql_moe* m) {
+  if (m == nullptr) return QL_OK;
+  cudaFree(m->d_idx_gu); cudaFree(m->d_idx_d); cudaFree(m->d_cent_gu); cudaFree(m->d_cent_d);
+  delete m;
+  return QL_OK;
+}
+
+ql_status moe_capture_intermediate(ql_moe* m, int32_t enable) {
+  if (m == nullptr) return fail(QL_ERR_INVALID_ARG, "null moe");
+  m->capture_h32 = enable != 0;
+  return QL_OK;
+}
+
+ql_status moe_workspace_bytes(const ql_moe* m, int64_t T, size_t* bytes) {
+  if (m == nullptr || bytes == nullptr || T < 0) return fail(QL_ERR_INVALID_ARG, "bad args");
+  *bytes = plan_moe(m, T).total;
+  return QL_OK;
+}
+
+ql_status moe_workspace_layout(const ql_moe* m, int64_t T, ql_moe_ws_layout* out) {
+  if (m == nullptr || out == nullptr || T < 0) return fail(QL_ERR_INVALID_ARG, "bad args");
+  const MoePlan p = plan_moe(m, T);
+  out->counts = p.counts; out->offsets = p.offsets; out->entries = p.entries; out->ids = p.ids;
+  out->gates = p.gates; out->x_codes = p.x_codes; out->x_scales = p.x_scales; out->x_dq = p.x_dq;
+  out->h_codes = p.h_codes; out->h_scales = p.h_scales; out->h_dq = p.h_dq;
+  out->h32 = m->capture_h32 ? p.h32 : SIZE_MAX; out->yslot = p.yslot; out->total = p.total;
+  return QL_OK;
+}
+
+ql_status moe_grouped_forward(const ql_moe* m, const void* x, int64_t T, const float* logits,
+                              void* y, float* y32, int32_t* ids_out, float* gates_out, void* ws,
+                              size_t ws_bytes, ql_stream_t stream) {
+  if (m == nullptr || T < 0) return fail(QL_ERR_INVALID_ARG, "null moe or negative T");
+  if (T == 0) return QL_OK;
+  if (x == nullptr || logits == nullptr || y == nullptr)
+    return fail(QL_ERR_INVALID_ARG, "null x/logits/y");
+  if (T > (1 << 20)) return fail(QL_ERR_UNSUPPORTED, "T too large");
+  if ((reinterpret_cast<uintptr_t>(x) & 15) != 0 || (reinterpret_cast<uintptr_t>(y) & 15) != 0)
+    return fail(QL_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+  const MoePlan p = plan_moe(m, T);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0 || ws_bytes < p.total)
+    return fail(QL_ERR_WORKSPACE, "workspace needs %zu bytes, 256-aligned", p.total);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  int* counts = reinterpret_cast<int*>(w8 + p.counts);
+  int* offsets = reinterpret_cast<int*>(w8 + p.offsets);
+  int* entries = reinterpret_cast<int*>(w8 + p.entries);
+  int* ids = reinterpret_cast<int*>(w8 + p.ids);
+  float* gates = reinterpret_cast<float*>(w8 + p.gates);
+  const int total = static_cast<int>(T * m->k);
+  QL_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * m->E, s));
+  ql::moe_topk_kernel<<<static_cast<unsigned>((T * 32 + 255) / 256), 256, 0, s>>>(
+      logits, static_cast<int>(T), m->E, m->k, ids, gates, counts);
+  QL_CUDA(cudaGetLastError());
+  ql::moe_scatter_kernel<<<m->E, 256, 0, s>>>(ids, total, m->E, counts, offsets, entries);
+  QL_CUDA(cudaGetLastError());
+  __nv_bfloat16* x_dq = reinterpret_cast<__nv_bfloat16*>(w8 + p.x_dq);
+  ql_status st = launch_quant_mx(x, T, m->H, w8 + p.x_codes, w8 + p.x_scales, nullptr, 0, nullptr,
+                                 0, s, x_dq);
+  if (st != QL_OK) return st;
+  CUtensorMap tm_x, tm_h;
+  __nv_bfloat16* h_dq = reinterpret_cast<__nv_bfloat16*>(w8 + p.h_dq);
+  st = make_tmap_bf16(&tm_x, x_dq, m->H, T, 1);
+  if (st == QL_OK) st = make_tmap_bf16(&tm_h, h_dq, m->I, total, kMoeBN);
+  if (st != QL_OK) return st;
+  ql::MoeGemmArgs a{};
+  a.E = m->E; a.k = m->k; a.counts = counts; a.offsets = offsets; a.entries = entries;
+  a.gates = gates; a.I = m->I; a.H = m->H;
+  a.h_codes = w8 + p.h_codes; a.h_scales = w8 + p.h_scales; a.h_dq = h_dq;
+  a.h32 = m->capture_h32 ? reinterpret_cast<float*>(w8 + p.h32) : nullptr;
+  a.yslot = reinterpret_cast<float*>(w8 + p.yslot);
+  const int max_mtiles = m->E + (total + kMoeBN - 1) / kMoeBN;   // >= sum_e ceil(count_e / BN)
+  a.rows_per_expert = 2 * m->I; a.kdim = m->H; a.n_tiles = 2 * m->I / 128; a.cent = m->d_cent_gu;
+  st = launch_moe_gemm<kMoeBN, true>(m->tm_idx_gu, tm_x, a, a.n_tiles * max_mtiles, s);
+  if (st != QL_OK) return st;
+  a.rows_per_expert = m->H; a.kdim = m->I; a.n_tiles = m->H / 128; a.cent = m->d_cent_d;
+  st = launch_moe_gemm<kMoeBN, false>(m->tm_idx_d, tm_h, a, a.n_tiles * max_mtiles, s);
+  if (st != QL_OK) return st;
+  const long n4 = T * m->H / 4;
+  ql::moe_combine_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
+      a.yslot, static_cast<int>(T), m->H, m->k, static_cast<__nv_bfloat16*>(y), y32);
+  QL_CUDA(cudaGetLastError());
+  if (ids_out != nullptr)
+    QL_CUDA(cudaMemcpyAsync(ids_out, ids, sizeof(int) * total, cudaMemcpyDeviceToDevice, s));
+  if (gates_out != nullptr)
+    QL_CUDA(cudaMemcpyAsync(gates_out, gates, sizeof(float) * total, cudaMemcpyDeviceToDevice, s));
   return QL_OK;
 }
 

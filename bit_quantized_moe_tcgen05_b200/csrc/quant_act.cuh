@@ -57,6 +57,25 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&f)[8]) {
   return out;
 }
 
+// Two E2M1 codes (lo -> low nibble, hi -> high nibble), RNE, satfinite; no sign fix-up.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.u32.u8 %0, b0;\n\t}"
+      : "=r"(out)
+      : "f"(lo), "f"(hi));
+  return out;
+}
+
+// Value of an E2M1 code (bit 3 = sign).
+__device__ __forceinline__ float e2m1_code_value(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const float mag = m < 2 ? 0.5f * static_cast<float>(m)
+                          : __uint_as_float(((126u + (m >> 1)) << 23) | ((m & 1u) << 22));
+  return (c & 8u) ? -mag : mag;
+}
+
 // Sign bits of eight bf16 values packed in four words (element 2i low half of word i) placed at
 // bit 3 of each nibble of the matching code word.
 __device__ __forceinline__ uint32_t bf16x8_sign_nibbles(const uint32_t (&w)[4]) {
@@ -71,10 +90,12 @@ __device__ __forceinline__ uint32_t bf16x8_sign_nibbles(const uint32_t (&w)[4]) 
 // x: bf16 [M, K] with row stride ldx (elements).  codes: [M, K/2] bytes (row stride ldc),
 // low nibble = even k.  Scales go to the plain [M, K/32] layout and/or the tiled layout.
 // The first `nzero` ints of `zero_words` are cleared (scratch the consumer expects zeroed).
+// deq_out (optional, [M, K] bf16) receives the exact value of every quantized element.
 __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, uint8_t* __restrict__ codes,
     int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
-    int sf_atoms_per_row, int* __restrict__ zero_words, int nzero) {
+    int sf_atoms_per_row, int* __restrict__ zero_words, int nzero,
+    __nv_bfloat16* __restrict__ deq_out = nullptr) {
   const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (zero_words != nullptr && gtid < nzero) zero_words[gtid] = 0;
   const int nblk = K >> 5;
@@ -114,6 +135,20 @@ __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
   const uint8_t b = static_cast<uint8_t>(e + 127);
   if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = b;
   if (scales_tiled != nullptr) scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row)] = b;
+  if (deq_out != nullptr) {
+    uint32_t o[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t c0 = (packed[i >> 2] >> (8 * (i & 3))) & 15u;
+      const uint32_t c1 = (packed[i >> 2] >> (8 * (i & 3) + 4)) & 15u;
+      const __nv_bfloat162 v = __floats2bfloat162_rn(ldexpf(e2m1_code_value(c0), e),
+                                                     ldexpf(e2m1_code_value(c1), e));
+      o[i] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(deq_out + static_cast<size_t>(m) * K + j * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  }
 }
 
 // ------------------------------------------------------------------ E4M3-B16 + FP32 tensor scale

@@ -173,6 +173,46 @@ ql_status ql_check(ql_stream_t stream);
 ql_status qlinear_prepare_prquant(const uint16_t* w_bf16, int64_t N, int64_t C, int32_t k,
                                   int32_t* perm_out, uint8_t* codes_out, uint8_t* scales_out);
 
+/* ---- MoE grouped FFN (CodeQuant-style cluster-codebook experts) ----------------------------
+ * CodeQuant abstract and Figure 4 (table in SM shared memory); gated FFN of PRQuant's Eq. (1).
+ * gate_up: wfmt QL_W_CLUSTER4_ROW16_BF16, N = E*2I rows (per expert: gate rows 0..I-1, then up
+ *          rows I..2I-1), K = H; codes = 4-bit indices [N, H/2] (element 2j in the low nibble),
+ *          codebooks = bf16 [N][16] centroids.
+ * down:    same format, N = E*H rows, K = I.
+ * Requirements: E <= 256, top_k <= 16, I % 64 == 0, H % 128 == 0.  Weights are copied (and the
+ * gate/up rows reordered for the fused SwiGLU) into library-owned device memory. */
+ql_status moe_create(const ql_weight_desc* gate_up, const ql_weight_desc* down, int32_t E,
+                     int32_t top_k, ql_stream_t stream, ql_moe** out);
+ql_status moe_destroy(ql_moe* moe);
+/* When enabled, moe_grouped_forward also writes the fp32 intermediate h (before its MXFP4
+ * requantization) into the workspace (for inspection and stage-wise testing). */
+ql_status moe_capture_intermediate(ql_moe* moe, int32_t enable);
+ql_status moe_workspace_bytes(const ql_moe* moe, int64_t T, size_t* bytes);
+
+/* Byte offsets, inside the workspace, of the forward's stage buffers (SIZE_MAX if absent):
+ * counts int[E], offsets int[E+1], entries int[T*k] (routed entries f = t*k+s, expert by expert,
+ * ascending f inside an expert), ids int[T,k], gates float[T,k], x_codes [T,H/2], x_scales
+ * [T,H/32] (MXFP4 of x), x_dq bf16 [T,H] (its exact values), h_codes [T*k,I/2], h_scales
+ * [T*k,I/32] (MXFP4 of h, rows in entry order), h_dq bf16 [T*k,I], h32 float [T*k,I] (only when
+ * captured), yslot float [T*k,H] (gate-weighted expert outputs by entry f). */
+typedef struct ql_moe_ws_layout {
+  size_t counts, offsets, entries, ids, gates, x_codes, x_scales, x_dq, h_codes, h_scales, h_dq,
+      h32, yslot, total;
+} ql_moe_ws_layout;
+ql_status moe_workspace_layout(const ql_moe* moe, int64_t T, ql_moe_ws_layout* out);
+
+/* out[T,H] = sum_s gate[t,s] * down_e(MXFP4(silu(gate_e(x_q)) * up_e(x_q))), e = ids[t,s]:
+ * router logits fp32 [T,E] (device) -> top-k (descending logit, ties to the lower id), gate
+ * weights = softmax of the k logits (fp32); x bf16 [T,H] (device) quantized to MXFP4 E8M0-B32;
+ * per expert a grouped bf16 tcgen05 GEMM over its routed tokens with weights decoded from the
+ * row codebooks in shared memory; SwiGLU and the MXFP4 requantization of h fused into the
+ * gate/up epilogue; the down epilogue writes gate-weighted slot outputs; the slots are summed in
+ * slot order.  y bf16 [T,H]; y_f32, ids_out int32 [T,k] and gates_out float [T,k] may be NULL. */
+ql_status moe_grouped_forward(const ql_moe* moe, const void* x_bf16, int64_t T,
+                              const float* router_logits, void* y_bf16, float* y_f32,
+                              int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                              ql_stream_t stream);
+
 /* MXCode PreScale VQ preparation (MXCode abstract: PreScale extracts the MX scales before the
  * codebook is learned; Table 1 row E4M3-B16-FP4).  w_bf16 [N,K]; codebooks = packed E2M1 entries
  * [N/64][K/64][256][2] (entry element 2i in the low nibble of byte i); outputs: the FP32 tensor
