@@ -27,7 +27,14 @@
 namespace ql {
 
 // Largest cluster of K-splits: bigger clusters co-schedule poorly (few fit on the GPU at once).
-constexpr int kMaxClusterSplits = 4;
+#ifndef QL_MAX_CLUSTER_SPLITS
+#define QL_MAX_CLUSTER_SPLITS 4
+#endif
+constexpr int kMaxClusterSplits = QL_MAX_CLUSTER_SPLITS;
+// Shared-memory budget (KB) of the operand ring for narrow token tiles (decode).
+#ifndef QL_NARROW_RING_KB
+#define QL_NARROW_RING_KB 100
+#endif
 
 struct Fp4GemmArgs {
   int M, N;                 // tokens, output features
@@ -46,6 +53,9 @@ struct Fp4GemmArgs {
   int ldy;
   const uint8_t* lut;       // VQ: packed E2M1 codebooks [N/64][K/64][256][2]
   int lut_qc;               // VQ: QBlocks along K (K / 64)
+  const uint8_t* wt;        // weight operand blocks [N/128][n_stages_total][block bytes]:
+                            // FP4 codes 128 rows x 128 B, 128-byte swizzle pre-applied (16 KB),
+                            // or VQ indices 128 rows x 64 B (8 KB)
 };
 
 template <int BN, bool E8M0, bool VQ = false>
@@ -60,25 +70,27 @@ struct Fp4Cfg {
   static constexpr int kIdxBytes = VQ ? 128 * 64 : 0;   // VQ: 8-bit indices, 128 rows x 64
   static constexpr int kLutBytes = VQ ? 8 * 512 : 0;    // VQ: 2 x 4 QBlock codebooks of 512 B
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kIdxBytes + kLutBytes;
-  static constexpr int kBudget = (BN <= 64 && !VQ) ? 100 * 1024 : 212 * 1024;
+  static constexpr int kBudget = (BN <= 64 && !VQ) ? QL_NARROW_RING_KB * 1024 : 212 * 1024;
   static constexpr int kStagesRaw = kBudget / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : (kStagesRaw < 2 ? 2 : kStagesRaw);
+  static constexpr int kStages = kStagesRaw > 12 ? 12 : (kStagesRaw < 2 ? 2 : kStagesRaw);
   static constexpr int kSfaCols = kAtoms * 4;          // TMEM columns per stage
   static constexpr int kSfbCols = kAtoms * 4 * kG;
   static constexpr int kColsNeeded = BN + kStages * (kSfaCols + kSfbCols);
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                  : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
   static_assert(kColsNeeded <= 512, "TMEM budget");
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-  static_assert(BN * 128 * 4 <= kStages * kStageBytes, "split-K partial tile must fit the ring");
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/;
+  static_assert(BN * 128 * 4 <= kStages * kStageBytes, "output staging must fit the ring");
 };
 
-// VQ = true (MXCode PreScale weights): tm_w maps the 8-bit index matrix [N, K/4] instead of the
-// weight codes; warps 2..5 decode each stage's operand tile from the shared-memory codebooks.
+// The weight operand of each (128-row tile, K stage) is one contiguous block in HBM, laid out at
+// create time exactly as the stage buffer wants it, and arrives by one 1-D bulk copy.
+// VQ = true (MXCode PreScale weights): the blocks hold 8-bit indices; warps 2..5 decode each
+// stage's operand tile from the shared-memory codebooks.
 template <int BN, bool E8M0, bool VQ = false>
 __global__ void __launch_bounds__(192, 1)
-    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
-                    const __grid_constant__ CUtensorMap tm_x, const Fp4GemmArgs a) {
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
+                    const __grid_constant__ CUtensorMap tm_y32, const Fp4GemmArgs a) {
   using Cfg = Fp4Cfg<BN, E8M0, VQ>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -110,10 +122,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(accf, 1);
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_w);
-    prefetch_tmap(&tm_x);
-  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tm_x);
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
@@ -151,15 +160,17 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t wbytes = VQ ? Cfg::kIdxBytes + Cfg::kLutBytes : Cfg::kABytes;
         const uint32_t bytes = wbytes + Cfg::kBBytes + nat * 512 * (1 + Cfg::kG);
         mbar_arrive_expect_tx(&full[st], bytes);
+        const uint8_t* wblk = a.wt + (static_cast<size_t>(blockIdx.x) * a.n_stages_total + i) *
+                                         (VQ ? Cfg::kIdxBytes : Cfg::kABytes);
         if constexpr (VQ) {
-          tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_w, &full[st], kw >> 2, n0);
+          bulk_load(sIdx + st * Cfg::kIdxBytes, wblk, Cfg::kIdxBytes, &full[st]);
 #pragma unroll
           for (int g2 = 0; g2 < 2; ++g2)
             bulk_load(sLut + st * Cfg::kLutBytes + g2 * 2048,
                       a.lut + (static_cast<size_t>((n0 >> 6) + g2) * a.lut_qc + (kw >> 6)) * 512,
                       2048, &full[st]);
         } else {
-          tma_load_2d(sA + st * Cfg::kABytes, &tm_w, &full[st], kw >> 1, n0);
+          bulk_load(sA + st * Cfg::kABytes, wblk, Cfg::kABytes, &full[st]);
         }
         tma_load_2d(sB + st * Cfg::kBBytes, &tm_x, &full[st], kx >> 1, m0);
         bulk_load(sSfa + st * Cfg::kSfaBytes,
@@ -251,37 +262,69 @@ __global__ void __launch_bounds__(192, 1)
     }
     // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
     const int q = warp & 3;
-    const int n = n0 + q * 32 + lane;
     const int splits = gridDim.z;   // == cluster size along z
     const bool have_acc = (s_end > s_begin);
     float alpha = a.alpha;
     if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
     if (have_acc) ok = mbar_wait(accf, 0, 3);
     tc_fence_after();
-    const int mcount = min(BN, a.M - m0);
-    if (ok) {
+    // Without split-K the tile is staged in the idle operand ring as y[m][n] and written by one
+    // TMA tensor store (which clips rows past M and columns past N): first the bf16 tile, then,
+    // when requested, the fp32 tile in the same buffer once the first store has read it.  With
+    // split-K each rank parks its fp32 partial tile there instead.
+    if (splits == 1) {
+      __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(smem);               // [BN][128]
+      float* y32buf = reinterpret_cast<float*>(smem);                             // [BN][128]
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 8) {
+          uint32_t r[8];
+          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            ybuf[(c + j) * 128 + q * 32 + lane] =
+                __float2bfloat16_rn((have_acc ? __uint_as_float(r[j]) : 0.f) * alpha);
+        }
+      }
+      fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 64 && ok) {
+        tma_store_2d(&tm_y, ybuf, n0, m0);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+      if (a.y32 != nullptr) {
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok) {
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 8) {
+            uint32_t r[8];
+            tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              y32buf[(c + j) * 128 + q * 32 + lane] = (have_acc ? __uint_as_float(r[j]) : 0.f) * alpha;
+          }
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x == 64 && ok) {
+          tma_store_2d(&tm_y32, y32buf, n0, m0);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+      }
+    } else if (ok) {
+      float* part = reinterpret_cast<float*>(smem);   // [BN][128] fp32, column = token
 #pragma unroll 1
       for (int c = 0; c < BN; c += 8) {
         uint32_t r[8];
         tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int mm = c + j;
-          if (mm >= mcount || n >= a.N) continue;
-          const float v = have_acc ? __uint_as_float(r[j]) : 0.f;
-          const size_t o = static_cast<size_t>(m0 + mm) * a.ldy + n;
-          if (splits == 1) {
-            a.y[o] = __float2bfloat16_rn(v * alpha);
-            if (a.y32 != nullptr) a.y32[o] = v * alpha;
-          }
-        }
-        if (splits > 1) {
-          float* part = reinterpret_cast<float*>(smem);   // [BN][128] fp32, column = token
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            part[(c + j) * 128 + q * 32 + lane] = have_acc ? __uint_as_float(r[j]) : 0.f;
-        }
+        for (int j = 0; j < 8; ++j)
+          part[(c + j) * 128 + q * 32 + lane] = have_acc ? __uint_as_float(r[j]) : 0.f;
       }
     }
   }

@@ -93,6 +93,24 @@ ql_status make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64
   return QL_OK;
 }
 
+// Output tensor [rows, cols] (bf16 or fp32, row-major, no swizzle), box [box_rows, 128 cols].
+ql_status make_tmap_out(CUtensorMap* m, const void* base, bool f32, uint64_t cols, uint64_t rows,
+                        uint64_t ld, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * es};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QL_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", int(r));
+  return QL_OK;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -102,8 +120,8 @@ int sm_count() {
 
 // ----------------------------------------------------------------------- GEMM launch
 template <int BN, bool E8M0, bool VQ>
-ql_status launch_fp4_bn(const CUtensorMap& tw, const CUtensorMap& tx, const ql::Fp4GemmArgs& a,
-                        dim3 grid, cudaStream_t s) {
+ql_status launch_fp4_bn(const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& ty32,
+                        const ql::Fp4GemmArgs& a, dim3 grid, cudaStream_t s) {
   using Cfg = ql::Fp4Cfg<BN, E8M0, VQ>;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -126,19 +144,19 @@ ql_status launch_fp4_bn(const CUtensorMap& tw, const CUtensorMap& tx, const ql::
   attr[0].val.clusterDim.z = grid.z;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_gemm_kernel<BN, E8M0, VQ>, tw, tx, a));
+  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_gemm_kernel<BN, E8M0, VQ>, tx, ty, ty32, a));
   return QL_OK;
 }
 
 template <bool E8M0, bool VQ>
-ql_status launch_fp4(int BN, const CUtensorMap& tw, const CUtensorMap& tx,
+ql_status launch_fp4(int BN, const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& ty32,
                      const ql::Fp4GemmArgs& a, dim3 grid, cudaStream_t s) {
   switch (BN) {
-    case 16: return launch_fp4_bn<16, E8M0, VQ>(tw, tx, a, grid, s);
-    case 32: return launch_fp4_bn<32, E8M0, VQ>(tw, tx, a, grid, s);
-    case 64: return launch_fp4_bn<64, E8M0, VQ>(tw, tx, a, grid, s);
-    case 128: return launch_fp4_bn<128, E8M0, VQ>(tw, tx, a, grid, s);
-    case 256: return launch_fp4_bn<256, E8M0, VQ>(tw, tx, a, grid, s);
+    case 16: return launch_fp4_bn<16, E8M0, VQ>(tx, ty, ty32, a, grid, s);
+    case 32: return launch_fp4_bn<32, E8M0, VQ>(tx, ty, ty32, a, grid, s);
+    case 64: return launch_fp4_bn<64, E8M0, VQ>(tx, ty, ty32, a, grid, s);
+    case 128: return launch_fp4_bn<128, E8M0, VQ>(tx, ty, ty32, a, grid, s);
+    case 256: return launch_fp4_bn<256, E8M0, VQ>(tx, ty, ty32, a, grid, s);
   }
   return fail(QL_ERR_UNSUPPORTED, "no GEMM tile for BN=%d", BN);
 }
@@ -158,13 +176,12 @@ struct ql_linear {
   int32_t k_tail;
   bool e8m0 = true;            // E8M0-B32 scales (else E4M3-B16 + tensor scales)
   bool vq = false;             // MXCode PreScale VQ weight
-  uint8_t* d_codes = nullptr;  // [N, K/2] codes, or [N, K/4] indices for VQ
+  uint8_t* d_codes = nullptr;  // weight operand blocks [N/128][stages][16 KB codes | 8 KB indices]
   uint8_t* d_lut = nullptr;    // VQ codebooks [N/64][K/64][256][2]
   uint8_t* d_sf = nullptr;     // tiled scale atoms
   int sf_atoms = 0;            // atoms per 128-row group of the weight
   int lut_qc = 0;
   float w_ts = 1.f;
-  CUtensorMap tm_w;
   int n_base_stages = 0, n_stages_total = 0;
 };
 
@@ -186,7 +203,7 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   const int tiles = p.tiles_n * p.tiles_m;
   const int total = L->n_stages_total;
   // Narrow token tiles (decode) run two CTAs per SM; split K until the grid fills the GPU.
-  const int target = sm_count() * ((p.BN <= 64 && !L->vq) ? 2 : 1);
+  const int target = sm_count() * ((p.BN <= 64 && !L->vq && QL_NARROW_RING_KB <= 110) ? 2 : 1);
   int splits = 1;
   if (tiles < target) splits = std::max(1, std::min({total, target / tiles, kMaxSplits}));
   p.spp = static_cast<int>(cdiv(total, splits));
@@ -213,6 +230,44 @@ void repack_sf_tiled(const uint8_t* plain, int64_t rows, int64_t cols, int atoms
     for (int64_t j = 0; j < cols; ++j)
       out[ql::sf_tiled_offset(static_cast<int>(r), static_cast<int>(j), atoms_per_row)] =
           plain[r * cols + j];
+}
+
+// Weight operand blocks for the FP4 GEMM: for every 128-row tile and every K stage of 256
+// elements (the base stages over [0, C), then the tail stages over [C, C + k_tail)), one block
+// laid out as the stage buffer: FP4 codes as 128 rows x 128 B with 16-byte chunk c of row r at
+// chunk c ^ (r % 8) (the 128-byte swizzle), or VQ indices as 128 rows x 64 B.  Rows past N and
+// elements past a partial stage are zero.
+void repack_weight_blocks(const uint8_t* src, int64_t N, int64_t K, int64_t C, int64_t k_tail,
+                          bool vq, std::vector<uint8_t>& out) {
+  const int64_t nb = cdiv(C, 256), nt = cdiv(k_tail, 256), stages = nb + nt;
+  const int64_t tiles = cdiv(N, 128);
+  const int row_bytes = vq ? 64 : 128;       // one stage of one row
+  const int64_t src_row = vq ? K / 4 : K / 2;
+  const int per_byte = vq ? 4 : 2;           // elements per source byte
+  out.assign(static_cast<size_t>(tiles) * stages * 128 * row_bytes, 0);
+  for (int64_t t = 0; t < tiles; ++t)
+    for (int64_t i = 0; i < stages; ++i) {
+      int64_t kw, valid;
+      if (i < nb) {
+        kw = i * 256;
+        valid = std::min<int64_t>(256, C - kw);
+      } else {
+        const int64_t j = (i - nb) * 256;
+        kw = C + j;
+        valid = std::min<int64_t>(256, k_tail - j);
+      }
+      uint8_t* blk = out.data() + (static_cast<size_t>(t) * stages + i) * 128 * row_bytes;
+      for (int r = 0; r < 128; ++r) {
+        const int64_t n = t * 128 + r;
+        if (n >= N) break;
+        const uint8_t* srow = src + n * src_row + kw / per_byte;
+        const int nbytes = static_cast<int>(valid / per_byte);
+        for (int b = 0; b < nbytes; ++b) {
+          const int dst = vq ? b : ((((b >> 4) ^ (r & 7)) << 4) | (b & 15));
+          blk[r * row_bytes + dst] = srow[b];
+        }
+      }
+    }
 }
 
 ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
@@ -301,7 +356,11 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
   L->n_stages_total = L->n_base_stages + static_cast<int>(cdiv(L->k_tail, 256));
   std::vector<uint8_t> sf;
   repack_sf_tiled(static_cast<const uint8_t*>(d->scales), d->N, d->K / sf_block, L->sf_atoms, sf);
-  const size_t code_bytes = static_cast<size_t>(d->N) * (vq ? d->K / 4 : d->K / 2);
+  std::vector<uint8_t> blocks;
+  repack_weight_blocks(vq ? static_cast<const uint8_t*>(d->indices)
+                          : static_cast<const uint8_t*>(d->codes),
+                       d->N, d->K, L->C, L->k_tail, vq, blocks);
+  const size_t code_bytes = blocks.size();
   const size_t lut_bytes = vq ? static_cast<size_t>(d->N / 64) * (d->K / 64) * 512 : 0;
   L->lut_qc = vq ? static_cast<int>(d->K / 64) : 0;
   auto cleanup = [&](ql_status st) {
@@ -316,16 +375,13 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
       (vq && cudaMalloc(&L->d_lut, lut_bytes) != cudaSuccess))
     return cleanup(fail(QL_ERR_OOM, "cudaMalloc of %zu weight bytes failed",
                         code_bytes + sf.size() + lut_bytes));
-  const void* src = vq ? static_cast<const void*>(d->indices) : d->codes;
-  if (cudaMemcpyAsync(L->d_codes, src, code_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+  if (cudaMemcpyAsync(L->d_codes, blocks.data(), code_bytes, cudaMemcpyHostToDevice, s) !=
+          cudaSuccess ||
       cudaMemcpyAsync(L->d_sf, sf.data(), sf.size(), cudaMemcpyHostToDevice, s) != cudaSuccess ||
       (vq && cudaMemcpyAsync(L->d_lut, d->codebooks, lut_bytes, cudaMemcpyHostToDevice, s) !=
                  cudaSuccess) ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return cleanup(fail(QL_ERR_CUDA, "weight upload failed"));
-  ql_status st = vq ? make_tmap_u8(&L->tm_w, L->d_codes, d->K / 4, d->N, d->K / 4, 64, 128, false)
-                    : make_tmap_u8(&L->tm_w, L->d_codes, d->K / 2, d->N, d->K / 2, 128, 128);
-  if (st != QL_OK) return cleanup(st);
   *out = L;
   return QL_OK;
 }
@@ -404,11 +460,20 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   a.ldy = static_cast<int>(L->N);
   a.lut = L->d_lut;
   a.lut_qc = L->lut_qc;
+  a.wt = L->d_codes;
   dim3 grid(p.tiles_n, p.tiles_m, p.splits);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (L->vq) return launch_fp4<false, true>(p.BN, L->tm_w, tm_x, a, grid, cs);
-  if (!L->e8m0) return launch_fp4<false, false>(p.BN, L->tm_w, tm_x, a, grid, cs);
-  return launch_fp4<true, false>(p.BN, L->tm_w, tm_x, a, grid, cs);
+  if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (y32 && (reinterpret_cast<uintptr_t>(y32) & 15)) ||
+      (L->N * 2) % 16 != 0)
+    return fail(QL_ERR_INVALID_ARG, "y / y_f32 must be 16-byte aligned");
+  CUtensorMap tm_y, tm_y32;
+  st = make_tmap_out(&tm_y, y, false, L->N, M, L->N, p.BN);
+  if (st == QL_OK) st = make_tmap_out(&tm_y32, y32 ? static_cast<const void*>(y32) : y, y32 != nullptr,
+                                      L->N, M, L->N, p.BN);
+  if (st != QL_OK) return st;
+  if (L->vq) return launch_fp4<false, true>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
+  if (!L->e8m0) return launch_fp4<false, false>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
+  return launch_fp4<true, false>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
 }
 
 ql_status qlinear_forward(const ql_linear* L, const void* x, int64_t M, void* y, float* y32,
