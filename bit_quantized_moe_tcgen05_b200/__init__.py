@@ -34,6 +34,7 @@ EXPORTED_SYMBOLS = (
     "qlinear_quantize_input", "qlinear_gemm", "qlinear_forward_fixed_scratch",
     "qlinear_prepare_vq_prescale", "moe_create", "moe_destroy", "moe_capture_intermediate",
     "moe_workspace_bytes", "moe_workspace_layout", "moe_grouped_forward",
+    "qlinear_prepare_int4_bsr",
 )
 
 
@@ -90,6 +91,8 @@ def _load() -> ctypes.CDLL:
         "moe_workspace_bytes": [vp, i64, ctypes.POINTER(sz)],
         "moe_workspace_layout": [vp, i64, ctypes.POINTER(MoeWsLayout)],
         "moe_grouped_forward": [vp, vp, i64, vp, vp, vp, vp, vp, vp, sz, vp],
+        "qlinear_prepare_int4_bsr": [vp, i64, i64, vp, i64, ctypes.c_float, vp, vp, vp, vp, vp, vp,
+                                     i32, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -355,3 +358,27 @@ class MoE:
             self.close()
         except Exception:
             pass
+
+
+def prepare_int4_bsr(w_bf16_bits: np.ndarray, x_calib_bf16_bits: np.ndarray,
+                     density: float = 0.02) -> dict:
+    """Offline INT4 dense + block-sparse residual preparation on the host (library C++ code).
+    Returns codes [N,K/2], fp16 scale bits [N,K/128], rowptr, col, residual codes/scale bits."""
+    w = np.ascontiguousarray(w_bf16_bits, dtype=np.uint16)
+    x = np.ascontiguousarray(x_calib_bf16_bits, dtype=np.uint16)
+    N, K = w.shape
+    cap = int(round(density * (N // 16) * (K // 128))) + 1
+    codes = np.empty((N, K // 2), np.uint8)
+    scales = np.empty((N, K // 128), np.uint16)
+    rowptr = np.empty(N // 16 + 1, np.int32)
+    col = np.empty(cap, np.int16)
+    rcodes = np.empty((cap, 16, 64), np.uint8)
+    rscales = np.empty((cap, 16), np.uint16)
+    nnzb = np.zeros(1, np.int32)
+    _ok(lib.qlinear_prepare_int4_bsr(w.ctypes.data, N, K, x.ctypes.data, x.shape[0], density,
+                                     codes.ctypes.data, scales.ctypes.data, rowptr.ctypes.data,
+                                     col.ctypes.data, rcodes.ctypes.data, rscales.ctypes.data, cap,
+                                     nnzb.ctypes.data), "qlinear_prepare_int4_bsr")
+    n = int(nnzb[0])
+    return dict(codes=codes, scales=scales, rowptr=rowptr, col=col[:n], rcodes=rcodes[:n],
+                rscales=rscales[:n])

@@ -202,3 +202,140 @@ extern "C" ql_status qlinear_prepare_vq_prescale(const uint16_t* w_bf16, int64_t
   }
   return QL_OK;
 }
+
+// MosaicQuant-style INT4 dense base + block-sparse INT4 residual ("Dense Base and Sparse
+// Residuals", "Activation-aware Delta-Hessian Block Selection").  Per (row, 128-group) the base
+// scale is fp16(amax/7) and codes clamp(rint(w/s), -7, 7); dW = W - base; the score of a 16 x 128
+// block is the sum over its rows, then columns, of abar_k |dW| with abar_k = mean_t |x_t,k| over
+// the calibration rows; the round(density * blocks) best blocks (ties to the lower id) keep a
+// residual quantized like the base on fp32(dW).
+namespace {
+
+uint16_t f32_to_f16_rne(float f) {
+  const uint32_t x = f32_bits(f);
+  const uint32_t sign = (x >> 16) & 0x8000u;
+  if ((x & 0x7FFFFFFFu) == 0) return static_cast<uint16_t>(sign);
+  const int exp = static_cast<int>((x >> 23) & 0xFF) - 127 + 15;
+  uint32_t mant = x & 0x7FFFFFu;
+  if (exp >= 31) return static_cast<uint16_t>(sign | 0x7C00u);           // overflow -> inf
+  if (exp <= 0) {                                                          // fp16 subnormal
+    if (exp < -10) return static_cast<uint16_t>(sign);
+    mant |= 0x800000u;
+    const int shift = 14 - exp;
+    uint32_t h = mant >> shift;
+    const uint32_t rem = mant & ((1u << shift) - 1u), half = 1u << (shift - 1);
+    if (rem > half || (rem == half && (h & 1u))) ++h;
+    return static_cast<uint16_t>(sign | h);
+  }
+  uint32_t h = sign | (static_cast<uint32_t>(exp) << 10) | (mant >> 13);
+  const uint32_t rem = mant & 0x1FFFu;
+  if (rem > 0x1000u || (rem == 0x1000u && (h & 1u))) ++h;
+  return static_cast<uint16_t>(h);
+}
+
+float f16_to_f32(uint16_t h) {
+  const uint32_t s = (h & 0x8000u) << 16, e = (h >> 10) & 0x1F, m = h & 0x3FF;
+  if (e == 0) {
+    const float v = std::ldexp(static_cast<float>(m), -24);
+    return s ? -v : v;
+  }
+  if (e == 31) {
+    uint32_t u = s | 0x7F800000u | (m << 13);
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+  }
+  uint32_t u = s | ((e + 112) << 23) | (m << 13);
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+// INT4 codes of one 128-group with an fp16 scale; returns the scale bits.
+uint16_t quant_group_int4(const float* w, int8_t* q) {
+  float amax = 0.f;
+  for (int i = 0; i < 128; ++i) amax = std::max(amax, std::fabs(w[i]));
+  const uint16_t s16 = f32_to_f16_rne(amax / 7.0f);
+  const float sf = f16_to_f32(s16);
+  for (int i = 0; i < 128; ++i) {
+    if (sf == 0.f) { q[i] = 0; continue; }
+    const float r = std::nearbyint(w[i] / sf);
+    q[i] = static_cast<int8_t>(std::min(7.f, std::max(-7.f, r)));
+  }
+  return s16;
+}
+
+}  // namespace
+
+extern "C" ql_status qlinear_prepare_int4_bsr(const uint16_t* w_bf16, int64_t N, int64_t K,
+                                              const uint16_t* x_calib_bf16, int64_t T,
+                                              float density, uint8_t* codes_out,
+                                              uint16_t* scales_out, int32_t* rowptr_out,
+                                              int16_t* col_out, uint8_t* rcodes_out,
+                                              uint16_t* rscales_out, int32_t capacity,
+                                              int32_t* nnzb_out) {
+  if (!w_bf16 || !x_calib_bf16 || !codes_out || !scales_out || !rowptr_out || !col_out ||
+      !rcodes_out || !rscales_out || !nnzb_out)
+    return QL_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || T <= 0 || N % 16 != 0 || K % 128 != 0 || !(density >= 0.f && density <= 1.f))
+    return QL_ERR_INVALID_ARG;
+  const int64_t G = K / 128, NB = N / 16;
+  std::vector<double> dw(static_cast<size_t>(N) * K);
+  std::vector<float> row(K);
+  std::vector<int8_t> q(128);
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) row[k] = bf16_to_f32(w_bf16[n * K + k]);
+    for (int64_t g = 0; g < G; ++g) {
+      const uint16_t s16 = quant_group_int4(&row[g * 128], q.data());
+      scales_out[n * G + g] = s16;
+      const double sf = f16_to_f32(s16);
+      for (int i = 0; i < 128; ++i) {
+        const int64_t k = g * 128 + i;
+        dw[n * K + k] = static_cast<double>(row[k]) - static_cast<double>(q[i]) * sf;
+        const uint8_t nib = static_cast<uint8_t>(q[i]) & 0xF;
+        uint8_t& b = codes_out[n * (K / 2) + k / 2];
+        b = (k & 1) ? static_cast<uint8_t>((b & 0x0F) | (nib << 4)) : nib;
+      }
+    }
+  }
+  std::vector<double> abar(K, 0.0);
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t k = 0; k < K; ++k) abar[k] += std::fabs(static_cast<double>(bf16_to_f32(x_calib_bf16[t * K + k])));
+  for (int64_t k = 0; k < K; ++k) abar[k] /= static_cast<double>(T);
+  std::vector<double> score(static_cast<size_t>(NB) * G, 0.0);
+  for (int64_t nb = 0; nb < NB; ++nb)
+    for (int64_t g = 0; g < G; ++g) {
+      double s = 0.0;
+      for (int r = 0; r < 16; ++r)
+        for (int i = 0; i < 128; ++i) {
+          const int64_t k = g * 128 + i;
+          s += std::fabs(dw[(nb * 16 + r) * K + k]) * abar[k];
+        }
+      score[nb * G + g] = s;
+    }
+  const int64_t keep = static_cast<int64_t>(std::llround(static_cast<double>(density) * NB * G));
+  if (keep > capacity) return QL_ERR_INVALID_ARG;
+  std::vector<int64_t> order(NB * G);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int64_t a, int64_t b) { return score[a] > score[b]; });
+  std::vector<int64_t> sel(order.begin(), order.begin() + keep);
+  std::sort(sel.begin(), sel.end());
+  std::fill(rowptr_out, rowptr_out + NB + 1, 0);
+  std::vector<float> seg(128);
+  for (int64_t i = 0; i < keep; ++i) {
+    const int64_t nb = sel[i] / G, g = sel[i] % G;
+    rowptr_out[nb + 1] += 1;
+    col_out[i] = static_cast<int16_t>(g);
+    for (int r = 0; r < 16; ++r) {
+      for (int j = 0; j < 128; ++j) seg[j] = static_cast<float>(dw[(nb * 16 + r) * K + g * 128 + j]);
+      rscales_out[i * 16 + r] = quant_group_int4(seg.data(), q.data());
+      for (int j = 0; j < 64; ++j)
+        rcodes_out[(i * 16 + r) * 64 + j] = static_cast<uint8_t>((static_cast<uint8_t>(q[2 * j]) & 0xF) |
+                                                                 ((static_cast<uint8_t>(q[2 * j + 1]) & 0xF) << 4));
+    }
+  }
+  for (int64_t nb = 0; nb < NB; ++nb) rowptr_out[nb + 1] += rowptr_out[nb];
+  *nnzb_out = static_cast<int32_t>(keep);
+  return QL_OK;
+}

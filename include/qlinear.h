@@ -224,6 +224,22 @@ ql_status qlinear_prepare_vq_prescale(const uint16_t* w_bf16, int64_t N, int64_t
                                       const uint8_t* codebooks, int32_t qn, int32_t qk,
                                       float* ts_out, uint8_t* scales_out, uint8_t* idx_out);
 
+/* MosaicQuant-style INT4 dense + block-sparse residual preparation (MosaicQuant, "Dense Base and
+ * Sparse Residuals" and "Activation-aware Delta-Hessian Block Selection"; formulas are readings).
+ * w_bf16 [N,K] (N % 16 == 0, K % 128 == 0), calibration activations x_calib_bf16 [T,K].
+ * Base per (row, 128-group): s = fp16_RNE(amax/7) (fp32 divide), q = clamp(rint(w/s), -7, 7).
+ * dW = W - base; block (nb, g) of 16 rows x 128 columns scores sum_rows sum_cols abar_k |dW|
+ * (abar_k = mean_t |x[t,k]|; sums in that order, double); the round(density * N/16 * K/128)
+ * best blocks (ties to the lower id nb*(K/128)+g) keep a residual quantized per row like the
+ * base on fp32(dW).  Outputs: codes [N,K/2] (two's-complement nibbles, element 2j low), fp16
+ * scale bits [N,K/128], rowptr int32 [N/16+1], col int16 [nnzb] (group index), residual codes
+ * [nnzb][16][64], residual fp16 scale bits [nnzb][16]; nnzb <= capacity. Host, CPU. */
+ql_status qlinear_prepare_int4_bsr(const uint16_t* w_bf16, int64_t N, int64_t K,
+                                   const uint16_t* x_calib_bf16, int64_t T, float density,
+                                   uint8_t* codes_out, uint16_t* scales_out, int32_t* rowptr_out,
+                                   int16_t* col_out, uint8_t* rcodes_out, uint16_t* rscales_out,
+                                   int32_t capacity, int32_t* nnzb_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -72,3 +72,20 @@ def test_vq_prescale_host_preparation_matches_oracle(N, K):
     assert ts == ref["ts"]
     assert np.array_equal(sb, ref["sb"])
     assert np.array_equal(idx, ref["idx"])
+
+
+@pytest.mark.parametrize("N,K,T", [(64, 512, 32), (128, 1024, 16)])
+def test_int4_bsr_host_preparation_matches_oracle(N, K, T):
+    import bit_quantized_moe_tcgen05_b200 as ql
+    from oracle import formats as F, int4bsr
+    wb = synth.to_bf16_bits(synth.student_t(23 + K, (N, K), 4.0))
+    xb, _ = synth.activations_bf16(23, T, K, 0.01 * 8, 30.0)
+    got = ql.prepare_int4_bsr(wb, xb, density=0.05)
+    ref = int4bsr.prepare(synth.bf16_bits_to_f64(wb), synth.bf16_bits_to_f64(xb), density=0.05)
+    assert np.array_equal(got["codes"], F.pack_nibbles(F.int4_encode(ref["q"])))
+    assert np.array_equal(got["scales"], ref["sw"].view(np.uint16))
+    assert np.array_equal(got["rowptr"], ref["rowptr"])
+    assert np.array_equal(got["col"], ref["col"])
+    assert np.array_equal(got["rcodes"].reshape(len(ref["sel"]), 16, 64),
+                          F.pack_nibbles(F.int4_encode(ref["rq"])))
+    assert np.array_equal(got["rscales"], ref["rs"].view(np.uint16))
