@@ -137,6 +137,11 @@ def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None):
         _ok(lib.quantize_act(fmt, x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), None,
                              _stream(stream)), "quantize_act")
         return codes, scales
+    if fmt == QL_A_INT4_TOK_G128:
+        scales = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+        _ok(lib.quantize_act(fmt, x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), None,
+                             _stream(stream)), "quantize_act")
+        return codes, scales
     if fmt == QL_A_FP4_E4M3_B16_TS:
         scales = torch.empty((M, K // 16), dtype=torch.uint8, device=x.device)
         ts = torch.empty(1, dtype=torch.float32, device=x.device)
@@ -158,12 +163,33 @@ class QLinear:
     def __init__(self, codes: np.ndarray | None, scales: np.ndarray, k_tail: int = 0,
                  wfmt: int = QL_W_MXFP4_E8M0_B32, w_tensor_scale: float = 1.0,
                  indices: np.ndarray | None = None, codebooks: np.ndarray | None = None,
-                 stream=None):
+                 bsr: dict | None = None, stream=None):
         """MXFP4: codes [N, K/2] + E8M0 scales [N, K/32] (+ k_tail).  NVFP4 (E4M3-B16): codes +
         E4M3 scales [N, K/16] + w_tensor_scale.  VQ PreScale: indices [N, K/4] + packed codebooks
-        [N/64, K/64, 256, 2] + E4M3 scales [N, K/16] + w_tensor_scale (codes = None)."""
-        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        [N/64, K/64, 256, 2] + E4M3 scales [N, K/16] + w_tensor_scale (codes = None).
+        INT4 + block-sparse residual: codes [N, K/2], fp16 scale bits [N, K/128] and
+        bsr = {rowptr, col, rcodes, rscales} as returned by prepare_int4_bsr."""
+        scales = np.ascontiguousarray(scales, dtype=np.uint8 if wfmt != QL_W_INT4_G128_BSR else np.uint16)
         keep = [scales]
+        if wfmt == QL_W_INT4_G128_BSR:
+            codes = np.ascontiguousarray(codes, dtype=np.uint8)
+            N, K = codes.shape[0], 2 * codes.shape[1]
+            b = bsr or {}
+            rowptr = np.ascontiguousarray(b.get("rowptr", np.zeros(N // 16 + 1)), dtype=np.int32)
+            col = np.ascontiguousarray(b.get("col", np.zeros(0)), dtype=np.int16)
+            rcodes = np.ascontiguousarray(b.get("rcodes", np.zeros((0, 16, 64))), dtype=np.uint8)
+            rscales = np.ascontiguousarray(b.get("rscales", np.zeros((0, 16))), dtype=np.uint16)
+            keep += [codes, rowptr, col, rcodes, rscales]
+            self.N, self.K, self.k_tail, self.C, self.wfmt = N, K, 0, K, wfmt
+            d = WeightDesc(wfmt=wfmt, N=N, K=K, codes=codes.ctypes.data, scales=scales.ctypes.data,
+                           bsr_rowptr=rowptr.ctypes.data, bsr_col=col.ctypes.data,
+                           bsr_codes=rcodes.ctypes.data, bsr_scales=rscales.ctypes.data,
+                           bsr_block_n=16, bsr_block_k=128, bsr_nnzb=len(col))
+            h = ctypes.c_void_p()
+            _ok(lib.qlinear_create(ctypes.byref(d), _stream(stream), ctypes.byref(h)), "qlinear_create")
+            self._h = h
+            self._ws = None
+            return
         if wfmt == QL_W_VQ_PRESCALE_E4M3_B16:
             indices = np.ascontiguousarray(indices, dtype=np.uint8)
             codebooks = np.ascontiguousarray(codebooks, dtype=np.uint8)

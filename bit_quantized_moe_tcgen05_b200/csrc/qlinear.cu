@@ -18,6 +18,7 @@
 #include "quant_act.cuh"
 #include "gemm_fp4.cuh"
 #include "moe.cuh"
+#include "int4_gemm.cuh"
 
 namespace {
 
@@ -183,6 +184,11 @@ struct ql_linear {
   int lut_qc = 0;
   float w_ts = 1.f;
   int n_base_stages = 0, n_stages_total = 0;
+  // INT4 dense + block-sparse residual
+  bool int4 = false;
+  int* d_stage_start = nullptr;   // [N/128 + 1]
+  int* d_stage_group = nullptr;   // [stages]
+  int max_tile_stages = 0;
 };
 
 namespace {
@@ -195,7 +201,31 @@ struct FwdPlan {
 
 constexpr int kMaxSplits = ql::kMaxClusterSplits;  // the K-splits of a tile form one cluster
 
+FwdPlan plan_forward_int4(const ql_linear* L, int64_t M) {
+  FwdPlan p{};
+  p.BN = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.tiles_n = static_cast<int>(L->N / 128);
+  p.tiles_m = static_cast<int>(cdiv(std::max<int64_t>(M, 1), p.BN));
+  const int tiles = p.tiles_n * p.tiles_m;
+  const int total = L->max_tile_stages;
+  int splits = 1;
+  const int target = sm_count();
+  if (tiles < target) splits = std::max(1, std::min({total, target / tiles, ql::kMaxClusterSplits}));
+  p.spp = static_cast<int>(cdiv(total, splits));
+  p.splits = static_cast<int>(cdiv(total, p.spp));
+  p.sfb_atoms = p.tiles_m * p.BN;                       // ldt of the transposed scales
+  size_t off = 0;
+  p.codes_off = off;                                    // int8 activation [M, K]
+  off = align_up(off + static_cast<size_t>(M) * L->K, 256);
+  p.sf_off = off;                                       // scales [K/128][ldt]
+  off = align_up(off + static_cast<size_t>(L->K / 128) * p.sfb_atoms * 4, 256);
+  p.scal_off = off;
+  p.total = off;
+  return p;
+}
+
 FwdPlan plan_forward(const ql_linear* L, int64_t M) {
+  if (L->int4) return plan_forward_int4(L, M);
   FwdPlan p{};
   p.BN = pick_bn(M);
   p.tiles_n = static_cast<int>(cdiv(L->N, 128));
@@ -270,6 +300,57 @@ void repack_weight_blocks(const uint8_t* src, int64_t N, int64_t K, int64_t C, i
     }
 }
 
+float half_bits_to_float(uint16_t h) {
+  const uint32_t sgn = (h & 0x8000u) << 16, e = (h >> 10) & 0x1F, m = h & 0x3FF;
+  float f;
+  if (e == 0) {
+    f = std::ldexp(static_cast<float>(m), -24);
+    return sgn ? -f : f;
+  }
+  const uint32_t u = sgn | (e == 31 ? (0xFFu << 23) : ((e + 112) << 23)) | (m << 13);
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+template <int BN>
+ql_status launch_int4_bn(const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& ty32,
+                         const ql::Int4GemmArgs& a, dim3 grid, cudaStream_t s) {
+  using Cfg = ql::Int4Cfg<BN>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    QL_CUDA(cudaFuncSetAttribute(ql::int4_gemm_kernel<BN>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+    attr_done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(320, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = grid.z;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::int4_gemm_kernel<BN>, tx, ty, ty32, a));
+  return QL_OK;
+}
+
+ql_status launch_quant_int4(const void* x, int64_t M, int64_t K, int8_t* q8, uint8_t* q4, float* sc,
+                            float* sct, int ldt, cudaStream_t s) {
+  const long warps = M * (K / 128);
+  if (warps == 0) return QL_OK;
+  ql::quant_int4_g128_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K), q8, q4, sc,
+      sct, ldt);
+  QL_CUDA(cudaGetLastError());
+  return QL_OK;
+}
+
 ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
                           uint8_t* st, int st_atoms, int* zero_words, int nzero,
                           cudaStream_t s, __nv_bfloat16* deq = nullptr) {
@@ -313,9 +394,96 @@ extern "C" {
 const char* ql_version(void) { return "qlinear-b200 0.1 (sm_100a)"; }
 const char* ql_last_error(void) { return g_last_error.c_str(); }
 
+static ql_status create_int4_bsr(const ql_weight_desc* d, cudaStream_t s, ql_linear** out) {
+  if (d->codes == nullptr || d->scales == nullptr)
+    return fail(QL_ERR_INVALID_ARG, "INT4 layer needs codes and scales");
+  if (d->N <= 0 || d->K <= 0 || d->N % 128 != 0 || d->K % 128 != 0 || d->k_tail != 0)
+    return fail(QL_ERR_UNSUPPORTED, "INT4 layer needs N %% 128 == 0, K %% 128 == 0, no tail");
+  if (d->bsr_nnzb < 0 || (d->bsr_nnzb > 0 && (d->bsr_rowptr == nullptr || d->bsr_col == nullptr ||
+                                             d->bsr_codes == nullptr || d->bsr_scales == nullptr)))
+    return fail(QL_ERR_INVALID_ARG, "bad block-sparse residual description");
+  if (d->bsr_nnzb > 0 && (d->bsr_block_n != 16 || d->bsr_block_k != 128))
+    return fail(QL_ERR_UNSUPPORTED, "residual blocks must be 16 x 128");
+  const int64_t N = d->N, K = d->K, G = K / 128, tiles = N / 128;
+  const uint8_t* codes = static_cast<const uint8_t*>(d->codes);
+  const uint16_t* sc = static_cast<const uint16_t*>(d->scales);
+  const uint8_t* rcodes = static_cast<const uint8_t*>(d->bsr_codes);
+  const uint16_t* rsc = static_cast<const uint16_t*>(d->bsr_scales);
+  std::vector<int> start(tiles + 1, 0), group;
+  std::vector<uint8_t> blocks;
+  blocks.reserve(static_cast<size_t>(tiles) * (G + 8) * ql::kInt4WBlock);
+  int max_st = 0;
+  for (int64_t t = 0; t < tiles; ++t) {
+    start[t] = static_cast<int>(group.size());
+    auto add_block = [&](int g) {
+      group.push_back(g);
+      const size_t at = blocks.size();
+      blocks.resize(at + ql::kInt4WBlock, 0);
+      return blocks.data() + at;
+    };
+    for (int g = 0; g < G; ++g) {
+      uint8_t* b = add_block(g);
+      float* rs = reinterpret_cast<float*>(b + 128 * 64);
+      for (int r = 0; r < 128; ++r) {
+        const int64_t n = t * 128 + r;
+        std::memcpy(b + r * 64, codes + n * (K / 2) + g * 64, 64);
+        rs[r] = half_bits_to_float(sc[n * G + g]);
+      }
+    }
+    if (d->bsr_nnzb > 0) {
+      std::vector<int> gs;
+      for (int nb = static_cast<int>(t * 8); nb < t * 8 + 8; ++nb)
+        for (int i = d->bsr_rowptr[nb]; i < d->bsr_rowptr[nb + 1]; ++i) {
+          if (i < 0 || i >= d->bsr_nnzb || d->bsr_col[i] < 0 || d->bsr_col[i] >= G)
+            return fail(QL_ERR_INVALID_ARG, "residual block index out of range");
+          gs.push_back(d->bsr_col[i]);
+        }
+      std::sort(gs.begin(), gs.end());
+      gs.erase(std::unique(gs.begin(), gs.end()), gs.end());
+      for (int g : gs) {
+        uint8_t* b = add_block(g);
+        float* rs = reinterpret_cast<float*>(b + 128 * 64);
+        for (int nb = static_cast<int>(t * 8); nb < t * 8 + 8; ++nb)
+          for (int i = d->bsr_rowptr[nb]; i < d->bsr_rowptr[nb + 1]; ++i) {
+            if (d->bsr_col[i] != g) continue;
+            for (int r = 0; r < 16; ++r) {
+              const int row = (nb - static_cast<int>(t * 8)) * 16 + r;
+              std::memcpy(b + row * 64, rcodes + (static_cast<size_t>(i) * 16 + r) * 64, 64);
+              rs[row] = half_bits_to_float(rsc[static_cast<size_t>(i) * 16 + r]);
+            }
+          }
+      }
+    }
+    max_st = std::max(max_st, static_cast<int>(group.size()) - start[t]);
+  }
+  start[tiles] = static_cast<int>(group.size());
+  auto* L = new ql_linear();
+  L->wfmt = d->wfmt;
+  L->N = N; L->K = K; L->C = K; L->k_tail = 0;
+  L->e8m0 = false; L->int4 = true; L->max_tile_stages = max_st;
+  auto cleanup = [&](ql_status st) {
+    cudaFree(L->d_codes); cudaFree(L->d_stage_start); cudaFree(L->d_stage_group);
+    delete L;
+    return st;
+  };
+  if (cudaMalloc(&L->d_codes, blocks.size()) != cudaSuccess ||
+      cudaMalloc(&L->d_stage_start, start.size() * sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&L->d_stage_group, group.size() * sizeof(int)) != cudaSuccess)
+    return cleanup(fail(QL_ERR_OOM, "cudaMalloc of INT4 weight blocks failed"));
+  if (cudaMemcpyAsync(L->d_codes, blocks.data(), blocks.size(), cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(L->d_stage_start, start.data(), start.size() * sizeof(int), cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(L->d_stage_group, group.data(), group.size() * sizeof(int), cudaMemcpyHostToDevice, s) ||
+      cudaStreamSynchronize(s))
+    return cleanup(fail(QL_ERR_CUDA, "INT4 weight upload failed"));
+  *out = L;
+  return QL_OK;
+}
+
 ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear** out) {
   if (d == nullptr || out == nullptr) return fail(QL_ERR_INVALID_ARG, "null descriptor/out");
   *out = nullptr;
+  if (d->wfmt == QL_W_INT4_G128_BSR)
+    return create_int4_bsr(d, reinterpret_cast<cudaStream_t>(stream), out);
   const bool mx = d->wfmt == QL_W_MXFP4_E8M0_B32;
   const bool nv = d->wfmt == QL_W_NVFP4_E4M3_B16;
   const bool vq = d->wfmt == QL_W_VQ_PRESCALE_E4M3_B16;
@@ -390,6 +558,8 @@ ql_status qlinear_destroy(ql_linear* L) {
   if (L == nullptr) return QL_OK;
   if (L->d_codes) cudaFree(L->d_codes);
   if (L->d_lut) cudaFree(L->d_lut);
+  if (L->d_stage_start) cudaFree(L->d_stage_start);
+  if (L->d_stage_group) cudaFree(L->d_stage_group);
   if (L->d_sf) cudaFree(L->d_sf);
   delete L;
   return QL_OK;
@@ -420,6 +590,10 @@ ql_status qlinear_quantize_input(const ql_linear* L, const void* x, int64_t M, v
   if ((reinterpret_cast<uintptr_t>(x) & 15) != 0)
     return fail(QL_ERR_INVALID_ARG, "x must be 16-byte aligned");
   uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (L->int4)
+    return launch_quant_int4(x, M, L->K, reinterpret_cast<int8_t*>(w8 + p.codes_off), nullptr,
+                             nullptr, reinterpret_cast<float*>(w8 + p.sf_off), p.sfb_atoms,
+                             reinterpret_cast<cudaStream_t>(stream));
   if (!L->e8m0) {
     unsigned* scal = reinterpret_cast<unsigned*>(w8 + p.scal_off);
     return launch_quant_e4m3(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
@@ -438,6 +612,34 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   if (st != QL_OK) return st;
   if (y == nullptr) return fail(QL_ERR_INVALID_ARG, "null y");
   uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (L->int4) {
+    if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (y32 && (reinterpret_cast<uintptr_t>(y32) & 15)))
+      return fail(QL_ERR_INVALID_ARG, "y / y_f32 must be 16-byte aligned");
+    CUtensorMap tx, ty, ty32;
+    st = make_tmap_u8(&tx, w8 + p.codes_off, L->K, M, L->K, 128, p.BN);
+    if (st == QL_OK) st = make_tmap_out(&ty, y, false, L->N, M, L->N, p.BN);
+    if (st == QL_OK) st = make_tmap_out(&ty32, y32 ? static_cast<const void*>(y32) : y, y32 != nullptr,
+                                        L->N, M, L->N, p.BN);
+    if (st != QL_OK) return st;
+    ql::Int4GemmArgs a{};
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(L->N);
+    a.wblocks = L->d_codes;
+    a.stage_start = L->d_stage_start;
+    a.stage_group = L->d_stage_group;
+    a.sx_t = reinterpret_cast<const float*>(w8 + p.sf_off);
+    a.ldt = p.sfb_atoms;
+    a.stages_per_split = p.spp;
+    a.y = static_cast<__nv_bfloat16*>(y);
+    a.y32 = y32;
+    dim3 grid(p.tiles_n, p.tiles_m, p.splits);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    switch (p.BN) {
+      case 16: return launch_int4_bn<16>(tx, ty, ty32, a, grid, cs);
+      case 32: return launch_int4_bn<32>(tx, ty, ty32, a, grid, cs);
+      default: return launch_int4_bn<64>(tx, ty, ty32, a, grid, cs);
+    }
+  }
   CUtensorMap tm_x;
   st = make_tmap_u8(&tm_x, w8 + p.codes_off, L->C / 2, M, L->C / 2, 128, p.BN);
   if (st != QL_OK) return st;
@@ -513,6 +715,10 @@ ql_status quantize_act(ql_aformat fmt, const void* x, int64_t M, int64_t K, void
       QL_CUDA(cudaGetLastError());
       return QL_OK;
     }
+    case QL_A_INT4_TOK_G128:
+      if (K % 128 != 0) return fail(QL_ERR_UNSUPPORTED, "INT4 activations need K %% 128 == 0");
+      return launch_quant_int4(x, M, K, nullptr, static_cast<uint8_t*>(codes),
+                               static_cast<float*>(scales), nullptr, 0, s);
     default:
       return fail(QL_ERR_UNSUPPORTED, "activation format %d not supported", int(fmt));
   }

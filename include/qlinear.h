@@ -107,6 +107,12 @@ const char* ql_last_error(void);
  *   QL_W_VQ_PRESCALE_E4M3_B16  N % 128 == 0, K % 256 == 0, 64 x 64 QBlocks, no tail; indices,
  *                              codebooks, E4M3 scales [N,K/16] and w_tensor_scale; the weight
  *                              operand is rebuilt from the codebooks inside the GEMM.
+ *   QL_W_INT4_G128_BSR         N % 128 == 0, K % 128 == 0, no tail; codes [N,K/2] (INT4, two's
+ *                              complement nibbles), fp16 scales [N,K/128], and a 16 x 128
+ *                              block-sparse INT4 residual (bsr_*: rowptr [N/16+1], col = group,
+ *                              codes [nnzb][16][64], fp16 scales [nnzb][16]); activations INT4
+ *                              per (token, 128-group); y = sum_g sx*sw*I_g + residual terms,
+ *                              both branches in one fused tcgen05 kind::i8 GEMM.
  * Synchronous with respect to `stream` (uses it for the uploads). */
 ql_status qlinear_create(const ql_weight_desc* desc, ql_stream_t stream, ql_linear** out);
 ql_status qlinear_destroy(ql_linear* layer);
@@ -155,7 +161,10 @@ ql_status qlinear_forward_fixed_scratch(const ql_linear* layer, const void* x_bf
  * QL_A_FP4_E4M3_B16_TS: K % 16 == 0; codes [M,K/2], E4M3 scales [M,K/16], *tensor_scale (device
  * float) receives ts = amax(x)/2688 (1 for an all-zero x); per 16 elements
  * s = E4M3_RNE_satfinite((amax/6)/ts), code = E2M1 RNE of x/(dec(s)*ts) (MXCode Table 1 row
- * E4M3-B16-FP4), each step an IEEE fp32 operation. */
+ * E4M3-B16-FP4), each step an IEEE fp32 operation.
+ * QL_A_INT4_TOK_G128: K % 128 == 0; codes [M,K/2] (two's-complement nibbles), scales float
+ * [M,K/128]: per (token, 128-group) s = amax/7 (fp32), q = clamp(rint(x/s), -7, 7) (MosaicQuant's
+ * W4A4 INT4 path; the granularity is a reading). */
 ql_status quantize_act(ql_aformat fmt, const void* x_bf16, int64_t M, int64_t K, void* codes,
                        void* scales, float* tensor_scale, ql_stream_t stream);
 
