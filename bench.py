@@ -70,14 +70,25 @@ def make_vq(Ms=(1, 8, 64), seed: int = 2) -> dict:
                 oracle=dict(ts=ts, sb=sb, idx=idx, cb=cb))
 
 
+_PRQ_CACHE = {}
+
+
+def _prquant_weight(seed: int):
+    if seed not in _PRQ_CACHE:
+        import synth
+        import bit_quantized_moe_tcgen05_b200 as ql
+        wb = synth.to_bf16_bits(synth.student_t(seed, (2560, 9728), 3.0))
+        _PRQ_CACHE[seed] = ql.prepare_prquant(wb, 128)
+    return _PRQ_CACHE[seed]
+
+
 def make_prquant(M: int, seed: int = 3) -> dict:
     """PRQuant tail-residual layer: W [2560, 9728] bf16 Student-t(3), k = 128 tail channels
     (library host preparation); X [M, 9728] N(0,1) with 0.5% outlier channels x50, permuted."""
     import synth
     import bit_quantized_moe_tcgen05_b200 as ql
     N, C, k = 2560, 9728, 128
-    wb = synth.to_bf16_bits(synth.student_t(seed, (N, C), 3.0))
-    perm, codes, scales = ql.prepare_prquant(wb, k)
+    perm, codes, scales = _prquant_weight(seed)
     xb, _ = synth.activations_bf16(seed, M, C, 0.005, 50.0)
     xb = np.ascontiguousarray(xb[:, perm])
     return dict(name=f"prquant_tail_n{N}_c{C}_k{k}_m{M}", kind="mx", N=N, K=C + k, C=C, Ms=[M],
@@ -99,14 +110,82 @@ def make_mxfp4(M: int = 16, seed: int = 1) -> dict:
                 make=lambda: ql.QLinear(codes, scales))
 
 
+def make_int4(M: int, seed: int = 5) -> dict:
+    """MosaicQuant-style layer: W [8192, 8192] Student-t(4) -> INT4 per 128-group + 655 residual
+    blocks of 16 x 128 chosen over the 4096-token calibration X (library host preparation);
+    X [M, 8192] = the first M calibration rows (N(0,1), 1% outlier channels x30)."""
+    import synth
+    import bit_quantized_moe_tcgen05_b200 as ql
+    N = K = 8192
+    wb = synth.to_bf16_bits(synth.student_t(seed, (N, K), 4.0))
+    xcal, _ = synth.activations_bf16(seed, 4096, K, 0.01, 30.0)
+    p = ql.prepare_int4_bsr(wb, xcal, 0.02)
+    wbytes = p["codes"].nbytes + p["scales"].nbytes + p["rowptr"].nbytes + p["col"].nbytes + \
+        p["rcodes"].nbytes + p["rscales"].nbytes
+    bsr = dict(rowptr=p["rowptr"], col=p["col"], rcodes=p["rcodes"], rscales=p["rscales"])
+    nnz = len(p["col"])
+    return dict(name=f"int4_bsr_n{N}_k{K}_nnzb{nnz}_m{M}", kind="int4", N=N, K=K, C=K, Ms=[M],
+                xs={M: np.ascontiguousarray(xcal[:M])}, weight_bytes=wbytes,
+                extra_flops_per_token=2.0 * nnz * 16 * 128,
+                make=lambda: ql.QLinear(p["codes"], p["scales"], wfmt=ql.QL_W_INT4_G128_BSR, bsr=bsr))
+
+
 def flops_of(w, M) -> float:
-    return 2.0 * M * w["N"] * w["K"]
+    return 2.0 * M * w["N"] * w["K"] + M * w.get("extra_flops_per_token", 0.0)
 
 
 def gemm_bytes_of(w, M) -> float:
     """Algorithmic bytes of one GEMM launch: weight payload + quantized activation + bf16 y."""
+    if w["kind"] == "int4":
+        return w["weight_bytes"] + M * w["C"] + M * w["C"] / 32 + 2.0 * M * w["N"]
     sf = 16 if w["kind"] == "vq" else 32
     return w["weight_bytes"] + M * w["C"] / 2 + M * w["C"] / sf + 2.0 * M * w["N"]
+
+
+def make_moe(seed: int = 4) -> dict:
+    """MoE grouped FFN: 128 experts, top-8, hidden 2048, intermediate 768, per-row 16-centroid
+    bf16 codebooks with 4-bit indices (seeded 1-D k-means on Student-t(4)), 2048 tokens N(0,1),
+    Zipf(1.1) router logits."""
+    import synth
+    E, H, I, T, k = 128, 2048, 768, 2048, 8
+    gi, gc, di, dc = [], [], [], []
+    for e in range(E):
+        c, i = synth.cluster_rows(seed * 1000 + e, 2 * I, H)
+        gc.append(c); gi.append(i)
+        c, i = synth.cluster_rows(seed * 1000 + 500 + e, H, I)
+        dc.append(c); di.append(i)
+    xb, _ = synth.activations_bf16(seed, T, H, 0.0, 1.0)
+    logits = synth.zipf_router_logits(seed, T, E)
+    flops = 2.0 * T * k * (2 * I * H + H * I)
+    wbytes = E * (2 * I * H + H * I) // 2 + E * (2 * I + H) * 32
+    return dict(name=f"moe_e{E}_top{k}_h{H}_i{I}_t{T}", E=E, H=H, I=I, T=T, k=k, x=xb,
+                logits=logits, gi=np.concatenate(gi), gc=np.concatenate(gc),
+                di=np.concatenate(di), dc=np.concatenate(dc), flops=flops, weight_bytes=wbytes)
+
+
+def run_moe(w, steps: int, warmup: int, device) -> dict:
+    """Device time of the whole routed FFN forward (routing, x quantization, gate/up GEMM with
+    SwiGLU + requantization, down GEMM, combine), replayed from a CUDA graph."""
+    import torch
+    import bit_quantized_moe_tcgen05_b200 as ql
+    layer = ql.MoE(w["gi"], w["gc"], w["di"], w["dc"], w["E"], w["k"])
+    x = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).to(device)
+    lg = torch.from_numpy(w["logits"]).to(device)
+    y = torch.empty((w["T"], w["H"]), dtype=torch.bfloat16, device=device)
+    ws = layer.workspace(w["T"], device)
+    for _ in range(warmup):
+        layer(x, lg, out=y, ws=ws)
+    ql.check()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer(x, lg, out=y, ws=ws)
+    for _ in range(warmup):
+        g.replay()
+    ms = _elapsed(g.replay, steps, torch.cuda.current_stream(device)) / steps
+    ql.check()
+    del g
+    layer.close()
+    return dict(step_ms=ms, steps=steps)
 
 
 # ------------------------------------------------------------------------------ clocks
@@ -292,16 +371,35 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cases", default="all", choices=["all", "none"])
     ap.add_argument("--workload", default="vq", choices=["vq", "prquant_m2048", "prquant_m512",
-                                                         "prquant_m16", "mxfp4_m16"])
+                                                         "prquant_m16", "mxfp4_m16", "int4_m4096",
+                                                         "int4_m256", "int4_m16", "int4_m1", "moe"])
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.workload == "moe":
+        import torch
+        w = make_moe()
+        torch.cuda.set_device(local)
+        r = run_moe(w, args.steps, args.warmup, torch.device("cuda", local))
+        peaks = measured_peaks()
+        tf = w["flops"] / (r["step_ms"] * 1e-3) / 1e12
+        print(json.dumps({"metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["step_ms"],
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "bf16 MMA on exact MXFP4 / codebook values, fp32 accumulate",
+                          "data": "synthetic", "config": {"workload": w["name"]},
+                          "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16"],
+                                       "unit": "TFLOP/s", "frac": tf / peaks["bf16"],
+                                       "traffic": None, "kernel": "whole routed FFN forward"}}))
+        return
     builders = {"vq": make_vq, "prquant_m2048": lambda: make_prquant(2048),
                 "prquant_m512": lambda: make_prquant(512), "prquant_m16": lambda: make_prquant(16),
-                "mxfp4_m16": lambda: make_mxfp4(16)}
+                "mxfp4_m16": lambda: make_mxfp4(16), "int4_m4096": lambda: make_int4(4096),
+                "int4_m256": lambda: make_int4(256), "int4_m16": lambda: make_int4(16),
+                "int4_m1": lambda: make_int4(1)}
     head = builders[args.workload]()
     decode = head["kind"] == "vq" or max(head["Ms"]) <= 64
     unit = "GB/s" if decode else "TFLOP/s"
@@ -385,8 +483,13 @@ def main():
 
     cases = {}
     if args.cases == "all":
+        int4_4096 = make_int4(4096)
+        int4_cases = [dict(int4_4096, name=int4_4096["name"].replace("_m4096", f"_m{M}"), Ms=[M],
+                           xs={M: np.ascontiguousarray(int4_4096["xs"][4096][:M])})
+                      for M in (256, 16, 1)]
         for wl, flush in ((make_prquant(2048), 256 << 20), (make_prquant(512), 0),
-                          (make_prquant(16), 0), (make_mxfp4(16), 0)):
+                          (make_prquant(16), 0), (make_mxfp4(16), 0), (int4_4096, 256 << 20),
+                          *[(c, 0) for c in int4_cases]):
             r = run_case(wl, 8, args.warmup, device, flush_bytes=flush)
             M = wl["Ms"][0]
             cases[wl["name"]] = {
@@ -394,10 +497,20 @@ def main():
                 "quant_us": r["quant_ms"] * 1e3,
                 "tflops": flops_of(wl, M) / (r["step_ms"] * 1e-3) / 1e12,
                 "gemm_tflops": flops_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e12,
-                "gemm_tensor_frac": flops_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e12 / fp4_peak,
+                "gemm_tensor_frac": flops_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e12 /
+                                    (2 * peaks["bf16"] if wl["kind"] == "int4" else fp4_peak),
+                "tensor_peak": "int8 = 2 x measured bf16 (nominal ratio)" if wl["kind"] == "int4"
+                               else "fp4 = 4 x measured bf16 (nominal ratio)",
                 "weight_stream_gbs": wl["weight_bytes"] / (r["gemm_ms"] * 1e-3) / 1e9,
                 "gemm_hbm_frac": gemm_bytes_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e9 / peaks["hbm"],
                 "l2": "flushed (256 MiB write)" if flush else f"{r['R']} rotating weight copies"}
+        mw = make_moe()
+        r = run_moe(mw, 10, args.warmup, device)
+        tf = mw["flops"] / (r["step_ms"] * 1e-3) / 1e12
+        cases[mw["name"]] = {"step_us": r["step_ms"] * 1e3, "tflops": tf,
+                             "bf16_tensor_frac": tf / peaks["bf16"],
+                             "fp4_tensor_frac": tf / fp4_peak,
+                             "l2": "weights 317 MB > L2"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -4,37 +4,34 @@
 //
 // over packed E2M1 operands with per-32 E8M0 scales (kind::mxf4) or per-16 UE4M3 scales
 // (kind::mxf4nvf4, alpha = product of the two FP32 tensor scales).  The weight is the MMA's
-// 128-row "A" operand and the tokens are the "B" operand of width BN (8..256), so one kernel
-// serves decode (M = 1..16, with split-K over CTAs) and prefill (M up to thousands).
+// 128-row "A" operand and the tokens are the "B" operand of width BN (16..256), so one kernel
+// serves decode (M = 1..64, with split-K over CTAs) and prefill (M up to thousands).
 //
 // PRQuant ("Kernel design for efficient inference"): the weight is W_aug = Q([W~, R_W]) with
 // reduction width C + k; the activation is quantized once over its C channels and its last k
 // channels are read a second time for the tail stages (activation coordinate C - k + j while
 // the weight coordinate is C + j).  No tail copy is materialised.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + single-thread
-// MMA issuer, warps 2..5 = epilogue (TMEM -> registers -> global).  Split-K (decode): the
-// gridDim.z K-splits of one output tile form a thread-block cluster; each CTA parks its fp32
-// partial tile in its own (now idle) operand ring; then each rank sums a share of the token
-// columns over distributed shared memory, adding the ranks in rank order, so the reduction is
-// deterministic and never leaves the chip.  A STAGES-deep ring of
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer (one
+// lane issues), warps 2..5 = (VQ weights: codebook decode, then) epilogue.  A STAGES-deep ring of
 // shared-memory stages, each 256 K-elements deep, is guarded by full/empty mbarriers; MMA
 // completion is signalled by tcgen05.commit.  Every wait is bounded (see ptx.cuh).
+//
+// Weight streaming starts before the activations exist: the kernel is launched with programmatic
+// stream serialization behind the activation quantizer, the producer first issues the weight
+// copies of the whole first ring fill (and the VQ warps decode them), and only then waits for the
+// quantizer grid (griddepcontrol.wait) before it loads activation tiles.  Split-K (decode): the
+// gridDim.z K-splits of one output tile each write an fp32 partial tile to a global workspace;
+// the last split to finish (an atomic ticket per tile) adds the partials in split order, so the
+// result is deterministic, writes y and re-arms the ticket for the next launch.
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
 
 namespace ql {
 
-// Largest cluster of K-splits: bigger clusters co-schedule poorly (few fit on the GPU at once).
-#ifndef QL_MAX_CLUSTER_SPLITS
-#define QL_MAX_CLUSTER_SPLITS 4
-#endif
-constexpr int kMaxClusterSplits = QL_MAX_CLUSTER_SPLITS;
-// Shared-memory budget (KB) of the operand ring for narrow token tiles (decode).
-#ifndef QL_NARROW_RING_KB
-#define QL_NARROW_RING_KB 100
-#endif
+// Most K-splits of one output tile (bounds the per-thread partial loads of the reduction).
+constexpr int kMaxSplits = 16;
 
 struct Fp4GemmArgs {
   int M, N;                 // tokens, output features
@@ -56,6 +53,8 @@ struct Fp4GemmArgs {
   const uint8_t* wt;        // weight operand blocks [N/128][n_stages_total][block bytes]:
                             // FP4 codes 128 rows x 128 B, 128-byte swizzle pre-applied (16 KB),
                             // or VQ indices 128 rows x 64 B (8 KB)
+  float* partials;          // split-K: [tiles][splits][BN][128] fp32 (tile = y-tile * gridDim.x + x-tile)
+  int* tickets;             // split-K: [tiles] arrival counters, zero between launches
 };
 
 template <int BN, bool E8M0, bool VQ = false>
@@ -70,7 +69,7 @@ struct Fp4Cfg {
   static constexpr int kIdxBytes = VQ ? 128 * 64 : 0;   // VQ: 8-bit indices, 128 rows x 64
   static constexpr int kLutBytes = VQ ? 8 * 512 : 0;    // VQ: 2 x 4 QBlock codebooks of 512 B
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kIdxBytes + kLutBytes;
-  static constexpr int kBudget = (BN <= 64 && !VQ) ? QL_NARROW_RING_KB * 1024 : 212 * 1024;
+  static constexpr int kBudget = 212 * 1024;
   static constexpr int kStagesRaw = kBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : (kStagesRaw < 2 ? 2 : kStagesRaw);
   static constexpr int kSfaCols = kAtoms * 4;          // TMEM columns per stage
@@ -105,19 +104,23 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sLut + S * Cfg::kLutBytes);
   uint64_t* empty = full + S;
   uint64_t* decd = empty + S;   // VQ: operand tile decoded (count 128)
-  uint64_t* accf = decd + S;
+  uint64_t* wfull = decd + S;   // VQ: indices + codebooks landed
+  uint64_t* accf = wfull + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  __shared__ int s_last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN;
   const int s_begin = blockIdx.z * a.stages_per_split;
   const int s_end = min(a.n_stages_total, s_begin + a.stages_per_split);
+  const int n_it = max(0, s_end - s_begin);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&decd[s], 128);
+      mbar_init(&wfull[s], 1);
     }
     mbar_init(accf, 1);
     fence_mbar_init();
@@ -149,97 +152,133 @@ __global__ void __launch_bounds__(192, 1)
 
   bool ok = true;
   if (warp == 0) {
-    if (lane == 0) {
-      for (int i = s_begin, it = 0; i < s_end && ok; ++i, ++it) {
-        const int st = it % S;
-        const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait(&empty[st], ph ^ 1, 1)) { ok = false; break; }
-        int kw, kx, valid;
-        stage_coords(i, kw, kx, valid);
-        const int nat = valid / Cfg::kAtomK;
-        const uint32_t wbytes = VQ ? Cfg::kIdxBytes + Cfg::kLutBytes : Cfg::kABytes;
-        const uint32_t bytes = wbytes + Cfg::kBBytes + nat * 512 * (1 + Cfg::kG);
-        mbar_arrive_expect_tx(&full[st], bytes);
-        const uint8_t* wblk = a.wt + (static_cast<size_t>(blockIdx.x) * a.n_stages_total + i) *
-                                         (VQ ? Cfg::kIdxBytes : Cfg::kABytes);
-        if constexpr (VQ) {
-          bulk_load(sIdx + st * Cfg::kIdxBytes, wblk, Cfg::kIdxBytes, &full[st]);
+    // ---------------- producer: the whole warp runs the loop; one elected lane issues copies.
+    // Weight part of stage it (independent of earlier grids): codes or indices + codebooks, SFA.
+    auto issue_weight = [&](int it) {
+      const int i = s_begin + it, st = it % S;
+      int kw, kx, valid;
+      stage_coords(i, kw, kx, valid);
+      const int nat = valid / Cfg::kAtomK;
+      const uint32_t act_bytes = Cfg::kBBytes + nat * 512 * Cfg::kG;
+      const uint8_t* wblk = a.wt + (static_cast<size_t>(blockIdx.x) * a.n_stages_total + i) *
+                                       (VQ ? Cfg::kIdxBytes : Cfg::kABytes);
+      if constexpr (VQ) {
+        mbar_arrive_expect_tx(&wfull[st], Cfg::kIdxBytes + Cfg::kLutBytes);
+        mbar_arrive_expect_tx(&full[st], nat * 512 + act_bytes);
+        bulk_load(sIdx + st * Cfg::kIdxBytes, wblk, Cfg::kIdxBytes, &wfull[st]);
 #pragma unroll
-          for (int g2 = 0; g2 < 2; ++g2)
-            bulk_load(sLut + st * Cfg::kLutBytes + g2 * 2048,
-                      a.lut + (static_cast<size_t>((n0 >> 6) + g2) * a.lut_qc + (kw >> 6)) * 512,
-                      2048, &full[st]);
-        } else {
-          bulk_load(sA + st * Cfg::kABytes, wblk, Cfg::kABytes, &full[st]);
-        }
-        tma_load_2d(sB + st * Cfg::kBBytes, &tm_x, &full[st], kx >> 1, m0);
-        bulk_load(sSfa + st * Cfg::kSfaBytes,
-                  a.sfa + (static_cast<size_t>(n0 >> 7) * a.sfa_atoms + kw / Cfg::kAtomK) * 512,
-                  nat * 512, &full[st]);
-#pragma unroll
-        for (int g = 0; g < Cfg::kG; ++g)
-          bulk_load(sSfb + st * Cfg::kSfbBytes + g * Cfg::kAtoms * 512,
-                    a.sfb + (static_cast<size_t>((m0 >> 7) + g) * a.sfb_atoms + kx / Cfg::kAtomK) * 512,
-                    nat * 512, &full[st]);
+        for (int g2 = 0; g2 < 2; ++g2)
+          bulk_load(sLut + st * Cfg::kLutBytes + g2 * 2048,
+                    a.lut + (static_cast<size_t>((n0 >> 6) + g2) * a.lut_qc + (kw >> 6)) * 512,
+                    2048, &wfull[st]);
+      } else {
+        mbar_arrive_expect_tx(&full[st], Cfg::kABytes + nat * 512 + act_bytes);
+        bulk_load(sA + st * Cfg::kABytes, wblk, Cfg::kABytes, &full[st]);
       }
+      bulk_load(sSfa + st * Cfg::kSfaBytes,
+                a.sfa + (static_cast<size_t>(n0 >> 7) * a.sfa_atoms + kw / Cfg::kAtomK) * 512,
+                nat * 512, &full[st]);
+    };
+    // Activation part of stage it (written by the quantizer grid): B codes and SFB.
+    auto issue_act = [&](int it) {
+      const int i = s_begin + it, st = it % S;
+      int kw, kx, valid;
+      stage_coords(i, kw, kx, valid);
+      const int nat = valid / Cfg::kAtomK;
+      tma_load_2d(sB + st * Cfg::kBBytes, &tm_x, &full[st], kx >> 1, m0);
+#pragma unroll
+      for (int g = 0; g < Cfg::kG; ++g)
+        bulk_load(sSfb + st * Cfg::kSfbBytes + g * Cfg::kAtoms * 512,
+                  a.sfb + (static_cast<size_t>((m0 >> 7) + g) * a.sfb_atoms + kx / Cfg::kAtomK) * 512,
+                  nat * 512, &full[st]);
+    };
+    const int pre = min(n_it, S);   // the first ring fill needs no empty-slot wait
+    if (elect_one())
+      for (int it = 0; it < pre; ++it) issue_weight(it);
+    __syncwarp();
+    griddep_wait();
+    if (elect_one())
+      for (int it = 0; it < pre; ++it) issue_act(it);
+    __syncwarp();
+    for (int it = pre; it < n_it && ok; ++it) {
+      const int st = it % S;
+      const uint32_t ph = (it / S) & 1;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 1));
+      if (!ok) break;
+      if (elect_one()) {
+        issue_weight(it);
+        issue_act(it);
+      }
+      __syncwarp();
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc0 = idesc_fp4_block(BN, E8M0);
-      bool first = true;
-      for (int i = s_begin, it = 0; i < s_end && ok; ++i, ++it) {
-        const int st = it % S;
-        const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait(&full[st], ph, 2)) { ok = false; break; }
-        if constexpr (VQ) {
-          if (!mbar_wait(&decd[st], ph, 4)) { ok = false; break; }
-        }
-        tc_fence_after();
-        int kw, kx, valid;
-        stage_coords(i, kw, kx, valid);
-        const int nat = valid / Cfg::kAtomK;
-        const uint32_t ta = tmem + sfa_col0 + st * Cfg::kSfaCols;
-        const uint32_t tb = tmem + sfb_col0 + st * Cfg::kSfbCols;
-        for (int at = 0; at < nat; ++at) {
-          tc_cp_32x128b_warpx4(ta + at * 4,
-                               make_sdesc(smem_u32(sSfa + st * Cfg::kSfaBytes + at * 512), 0, 128, kLayoutNone));
+    // ---------------- MMA issuer: converged warp, one lane issues the tcgen05 instructions
+    const uint32_t idesc0 = idesc_fp4_block(BN, E8M0);
+    bool first = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int i = s_begin + it, st = it % S;
+      const uint32_t ph = (it / S) & 1;
+      bool w = mbar_wait(&full[st], ph, 2);
+      if constexpr (VQ) w = w && mbar_wait(&decd[st], ph, 4);
+      ok = __all_sync(0xFFFFFFFFu, w);
+      if (!ok) break;
+      tc_fence_after();
+      int kw, kx, valid;
+      stage_coords(i, kw, kx, valid);
+      const int nat = valid / Cfg::kAtomK;
+      const uint32_t ta = tmem + sfa_col0 + st * Cfg::kSfaCols;
+      const uint32_t tb = tmem + sfb_col0 + st * Cfg::kSfbCols;
+      const uint32_t sfa_s = smem_u32(sSfa + st * Cfg::kSfaBytes);
+      const uint32_t sfb_s = smem_u32(sSfb + st * Cfg::kSfbBytes);
+      const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
+      const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
+      const int nk = valid / 64;
+      if (lane == 0) {   // the same lane issues every MMA and the commits that track them
 #pragma unroll
-          for (int g = 0; g < Cfg::kG; ++g)
-            tc_cp_32x128b_warpx4(tb + at * 4 * Cfg::kG + g * 4,
-                                 make_sdesc(smem_u32(sSfb + st * Cfg::kSfbBytes + g * Cfg::kAtoms * 512 + at * 512),
-                                            0, 128, kLayoutNone));
+        for (int at = 0; at < Cfg::kAtoms; ++at) {
+          if (at < nat) {
+            tc_cp_32x128b_warpx4(ta + at * 4, make_sdesc(sfa_s + at * 512, 0, 128, kLayoutNone));
+#pragma unroll
+            for (int g = 0; g < Cfg::kG; ++g)
+              tc_cp_32x128b_warpx4(tb + at * 4 * Cfg::kG + g * 4,
+                                   make_sdesc(sfb_s + g * Cfg::kAtoms * 512 + at * 512, 0, 128, kLayoutNone));
+          }
         }
-        const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
-        const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
-        const int nk = valid / 64;
-        for (int kk = 0; kk < nk; ++kk) {
-          const int at = (kk * 64) / Cfg::kAtomK;
-          const uint32_t byte = E8M0 ? static_cast<uint32_t>((kk & 1) * 2) : 0u;
-          const uint64_t adesc = make_sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128);
-          const uint64_t bdesc = make_sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128);
-          const uint32_t idesc = idesc0 | (byte << 29) | (byte << 4);
-          const uint32_t sfa_t = (ta + at * 4) | (byte << 30);
-          const uint32_t sfb_t = (tb + at * 4 * Cfg::kG) | (byte << 30);
-          if (E8M0)
-            mma_mxf4_block32(tmem, adesc, bdesc, idesc, sfa_t, sfb_t, first ? 0u : 1u);
-          else
-            mma_nvf4_block16(tmem, adesc, bdesc, idesc, sfa_t, sfb_t, first ? 0u : 1u);
-          first = false;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          if (kk < nk) {
+            const int at = (kk * 64) / Cfg::kAtomK;
+            const uint32_t byte = E8M0 ? static_cast<uint32_t>((kk & 1) * 2) : 0u;
+            const uint64_t ad = make_sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bd = make_sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128);
+            const uint32_t idd = idesc0 | (byte << 29) | (byte << 4);
+            const uint32_t sa = (ta + at * 4) | (byte << 30);
+            const uint32_t sb = (tb + at * 4 * Cfg::kG) | (byte << 30);
+            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+            if (E8M0)
+              mma_mxf4_block32(tmem, ad, bd, idd, sa, sb, acc);
+            else
+              mma_nvf4_block16(tmem, ad, bd, idd, sa, sb, acc);
+          }
         }
         tc_commit(&empty[st]);
       }
-      tc_commit(accf);
+      first = false;
+      __syncwarp();
     }
+    if (lane == 0) tc_commit(accf);
+    __syncwarp();
   } else {
     if constexpr (VQ) {
       // ---------------- VQ decode (warps 2..5, 128 threads): for each stage rebuild the
       // 128 x 256 E2M1 operand tile from 8-bit indices and the QBlock codebooks, in the
       // 128-byte-swizzled K-major layout the MMA reads (16-byte chunk kc of row r at kc ^ (r%8)).
+      // Only weights are read, so this runs ahead of the activation quantizer.
       const int t = threadIdx.x - 64;
-      for (int i = s_begin, it = 0; i < s_end && ok; ++i, ++it) {
+      for (int it = 0; it < n_it && ok; ++it) {
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait(&full[st], ph, 5)) { ok = false; break; }
+        if (!mbar_wait(&wfull[st], ph, 5)) { ok = false; break; }
         const uint8_t* idx_s = sIdx + st * Cfg::kIdxBytes;
         const uint16_t* lut = reinterpret_cast<const uint16_t*>(sLut + st * Cfg::kLutBytes);
         uint8_t* a_s = sA + st * Cfg::kABytes;
@@ -262,17 +301,17 @@ __global__ void __launch_bounds__(192, 1)
     }
     // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
     const int q = warp & 3;
-    const int splits = gridDim.z;   // == cluster size along z
-    const bool have_acc = (s_end > s_begin);
+    const int splits = gridDim.z;
+    const bool have_acc = n_it > 0;
+    griddep_wait();   // alpha_dev, the workspace and y belong to / follow earlier grids
     float alpha = a.alpha;
     if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
-    if (have_acc) ok = mbar_wait(accf, 0, 3);
+    if (have_acc && ok) ok = mbar_wait(accf, 0, 3);
     tc_fence_after();
-    // Without split-K the tile is staged in the idle operand ring as y[m][n] and written by one
-    // TMA tensor store (which clips rows past M and columns past N): first the bf16 tile, then,
-    // when requested, the fp32 tile in the same buffer once the first store has read it.  With
-    // split-K each rank parks its fp32 partial tile there instead.
     if (splits == 1) {
+      // The tile is staged in the idle operand ring as y[m][n] and written by one TMA tensor
+      // store (which clips rows past M and columns past N): first the bf16 tile, then, when
+      // requested, the fp32 tile in the same buffer once the first store has read it.
       __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(smem);               // [BN][128]
       float* y32buf = reinterpret_cast<float*>(smem);                             // [BN][128]
       if (ok) {
@@ -315,60 +354,52 @@ __global__ void __launch_bounds__(192, 1)
           bulk_wait_group_read0();
         }
       }
-    } else if (ok) {
-      float* part = reinterpret_cast<float*>(smem);   // [BN][128] fp32, column = token
+    } else {
+      // Split-K: park this split's fp32 partial tile [BN tokens][128 rows] in the workspace
+      // (lanes cover consecutive rows: coalesced), then take a ticket; the last split reduces.
+      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+      const int nl = q * 32 + lane;
+      const int mcount = min(BN, a.M - m0);
+      float* part = a.partials + static_cast<size_t>(tile) * splits * BN * 128;
+      if (ok) {
+        float* mine = part + static_cast<size_t>(blockIdx.z) * BN * 128;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 8) {
-        uint32_t r[8];
-        tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
-        tmem_ld_wait();
+        for (int c = 0; c < mcount; c += 8) {
+          uint32_t r[8];
+          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          part[(c + j) * 128 + q * 32 + lane] = have_acc ? __uint_as_float(r[j]) : 0.f;
-      }
-    }
-  }
-  // ---- split-K reduction across the cluster (all threads take part in the barriers)
-  __syncwarp();
-  cluster_sync_all();
-  if (gridDim.z > 1 && warp >= 2) {
-    // Columns are reduced in chunks of 8 tokens; chunk c belongs to rank c % nsplit, which
-    // loads that chunk from every rank (all loads in flight) and sums them in rank order.
-    const int q = warp & 3;
-    const int n = n0 + q * 32 + lane;
-    const int nsplit = gridDim.z;
-    const int rank = static_cast<int>(cluster_ctarank());
-    float alpha = a.alpha;
-    if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
-    const int mcount = min(BN, a.M - m0);
-    const uint32_t base = smem_u32(smem) + (q * 32 + lane) * 4;
-    for (int c = rank * 8; c < mcount; c += nsplit * 8) {
-      float v[kMaxClusterSplits][8];
-#pragma unroll
-      for (int r = 0; r < kMaxClusterSplits; ++r) {
-        if (r < nsplit) {
-          const uint32_t remote = map_shared_rank(base + c * 512, r);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) v[r][j] = ld_shared_cluster_f32(remote + j * 512);
+          for (int j = 0; j < 8; ++j)
+            if (c + j < mcount) __stcg(mine + (c + j) * 128 + nl, have_acc ? __uint_as_float(r[j]) : 0.f);
         }
       }
-      if (n < a.N) {
+      __threadfence();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 64) s_last = ok ? (atomicAdd(a.tickets + tile, 1) == splits - 1) : 0;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (s_last) {
+        __threadfence();
+        const int n = n0 + nl;
+#pragma unroll 1
+        for (int c = 0; c < mcount; ++c) {
+          float v[kMaxSplits];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+          for (int r = 0; r < kMaxSplits; ++r)
+            if (r < splits) v[r] = __ldcg(part + (static_cast<size_t>(r) * BN + c) * 128 + nl);
           float acc = 0.f;
 #pragma unroll
-          for (int r = 0; r < kMaxClusterSplits; ++r)
-            if (r < nsplit) acc += v[r][j];
-          if (c + j < mcount) {
-            const size_t o = static_cast<size_t>(m0 + c + j) * a.ldy + n;
+          for (int r = 0; r < kMaxSplits; ++r)
+            if (r < splits) acc += v[r];
+          if (n < a.N) {
+            const size_t o = static_cast<size_t>(m0 + c) * a.ldy + n;
             a.y[o] = __float2bfloat16_rn(acc * alpha);
             if (a.y32 != nullptr) a.y32[o] = acc * alpha;
           }
         }
+        if (threadIdx.x == 64) a.tickets[tile] = 0;   // re-armed for the next launch
       }
     }
   }
-  cluster_sync_all();   // every rank keeps its shared memory until all peers have read it
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);

@@ -20,6 +20,9 @@
 
 namespace ql {
 
+// Most K-splits of one INT4 output tile; the splits form one thread-block cluster.
+constexpr int kInt4MaxClusterSplits = 4;
+
 // ------------------------------------------------------------------ INT4 activation quantizer
 // One warp per (token, 128-group): s = amax / 7 (fp32), q = clamp(rint(x / s), -7, 7) (fp32
 // divide, ties to even), q = 0 when s == 0.  Outputs (each optional): int8 codes [M, K] (row

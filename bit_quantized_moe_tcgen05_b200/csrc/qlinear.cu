@@ -120,6 +120,9 @@ int sm_count() {
 }
 
 // ----------------------------------------------------------------------- GEMM launch
+// The GEMM is launched with programmatic stream serialization: it may start while the kernel
+// before it on the stream (the activation quantizer) is still running, and streams (and, for VQ,
+// decodes) weights until its griddepcontrol.wait.
 template <int BN, bool E8M0, bool VQ>
 ql_status launch_fp4_bn(const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& ty32,
                         const ql::Fp4GemmArgs& a, dim3 grid, cudaStream_t s) {
@@ -132,17 +135,14 @@ ql_status launch_fp4_bn(const CUtensorMap& tx, const CUtensorMap& ty, const CUte
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
     attr_done[dev] = true;
   }
-  // K-splits of one output tile form a cluster along z (reduced over DSMEM in the kernel).
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = grid.z;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_gemm_kernel<BN, E8M0, VQ>, tx, ty, ty32, a));
@@ -196,10 +196,10 @@ namespace {
 struct FwdPlan {
   int BN, splits, spp, tiles_n, tiles_m;
   int sfb_atoms;
-  size_t codes_off, sf_off, scal_off, total;
+  size_t codes_off, sf_off, scal_off, tick_off, part_off, total;
+  int n_tickets;   // split-K tickets (zeroed by the quantizer, re-armed by the GEMM)
 };
 
-constexpr int kMaxSplits = ql::kMaxClusterSplits;  // the K-splits of a tile form one cluster
 
 FwdPlan plan_forward_int4(const ql_linear* L, int64_t M) {
   FwdPlan p{};
@@ -210,7 +210,7 @@ FwdPlan plan_forward_int4(const ql_linear* L, int64_t M) {
   const int total = L->max_tile_stages;
   int splits = 1;
   const int target = sm_count();
-  if (tiles < target) splits = std::max(1, std::min({total, target / tiles, ql::kMaxClusterSplits}));
+  if (tiles < target) splits = std::max(1, std::min({total, target / tiles, ql::kInt4MaxClusterSplits}));
   p.spp = static_cast<int>(cdiv(total, splits));
   p.splits = static_cast<int>(cdiv(total, p.spp));
   p.sfb_atoms = p.tiles_m * p.BN;                       // ldt of the transposed scales
@@ -232,10 +232,10 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   p.tiles_m = static_cast<int>(cdiv(std::max<int64_t>(M, 1), p.BN));
   const int tiles = p.tiles_n * p.tiles_m;
   const int total = L->n_stages_total;
-  // Narrow token tiles (decode) run two CTAs per SM; split K until the grid fills the GPU.
-  const int target = sm_count() * ((p.BN <= 64 && !L->vq && QL_NARROW_RING_KB <= 110) ? 2 : 1);
+  // One CTA per SM: split K until the grid covers the SMs (at most kMaxSplits ways).
+  const int target = sm_count();
   int splits = 1;
-  if (tiles < target) splits = std::max(1, std::min({total, target / tiles, kMaxSplits}));
+  if (tiles < target) splits = std::max(1, std::min({total, target / tiles, ql::kMaxSplits}));
   p.spp = static_cast<int>(cdiv(total, splits));
   p.splits = static_cast<int>(cdiv(total, p.spp));
   const int atomK = L->e8m0 ? 128 : 64;  // K elements covered by one 512-byte scale atom
@@ -246,8 +246,14 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   off = align_up(off + static_cast<size_t>(M) * (L->C / 2), 256);
   p.sf_off = off;
   off = align_up(off + static_cast<size_t>(rows_pad / 128) * p.sfb_atoms * 512, 256);
-  p.scal_off = off;  // E4M3-B16 activations: [0] amax bit pattern, [1] tensor scale
-  off = align_up(off + 2 * sizeof(float), 256);
+  // [0] amax bit pattern and [1] tensor scale of E4M3-B16 activations, then the split-K tickets
+  // (one memset or the quantizer clears the whole run before the GEMM).
+  p.scal_off = off;
+  p.tick_off = off + 2 * sizeof(float);
+  p.n_tickets = p.splits > 1 ? tiles : 0;
+  off = align_up(p.tick_off + static_cast<size_t>(p.n_tickets) * sizeof(int), 256);
+  p.part_off = off;
+  if (p.splits > 1) off = align_up(off + static_cast<size_t>(tiles) * p.splits * p.BN * 128 * 4, 256);
   p.total = off;
   return p;
 }
@@ -367,22 +373,79 @@ ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, u
   return QL_OK;
 }
 
+// Cluster size for the one-launch small-tensor quantizer: 16 CTAs where the device can
+// co-schedule such a cluster, else the portable 8.
+int e4m3_cluster_size() {
+  static int size[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64) return 8;
+  if (size[dev] == 0) {
+    int want = 8;
+    if (cudaFuncSetAttribute(ql::quant_e4m3_b16_cluster_kernel,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16, 1, 1);
+      cfg.blockDim = dim3(1024, 1, 1);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, ql::quant_e4m3_b16_cluster_kernel, &cfg) == cudaSuccess &&
+          n > 0)
+        want = 16;
+    }
+    cudaGetLastError();
+    size[dev] = want;
+  }
+  return size[dev];
+}
+
+// Tensors up to this many elements are quantized by one cluster in one launch.
+constexpr int64_t kE4m3ClusterMaxElems = int64_t(1) << 21;
+
+// E4M3-B16 activation quantizer.  amax_slot: device word for the reduced amax bit pattern (the
+// two-launch path max-reduces into it; it is followed by the tensor-scale word and then
+// n_tickets split-K tickets, all cleared here).  ts_out: where ts goes (may be null).
 ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
                             uint8_t* st, int st_atoms, unsigned* amax_slot, float* ts_out,
-                            cudaStream_t s) {
-  QL_CUDA(cudaMemsetAsync(amax_slot, 0, sizeof(unsigned), s));
+                            cudaStream_t s, int n_tickets = 0) {
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  int* tickets = n_tickets > 0 ? reinterpret_cast<int*>(amax_slot + 2) : nullptr;
+  if (M * K <= kE4m3ClusterMaxElems) {
+    const int cs = e4m3_cluster_size();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs, 1, 1);
+    cfg.blockDim = dim3(1024, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    QL_CUDA(cudaLaunchKernelEx(&cfg, ql::quant_e4m3_b16_cluster_kernel, xb, static_cast<int>(M),
+                               static_cast<int>(K), static_cast<int>(K), amax_slot, ts_out, codes,
+                               static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms,
+                               tickets, n_tickets));
+    return QL_OK;
+  }
+  QL_CUDA(cudaMemsetAsync(amax_slot, 0, sizeof(unsigned) + (n_tickets > 0 ? sizeof(float) + n_tickets * sizeof(int) : 0), s));
   const long n8 = static_cast<long>(M) * K / 8;
   const int block = 256;
   const long want = (n8 + block - 1) / block;
   const int grid_a = static_cast<int>(std::max<long>(1, std::min<long>(want, 4L * sm_count())));
-  ql::absmax_bf16_kernel<<<grid_a, block, 0, s>>>(static_cast<const __nv_bfloat16*>(x), n8,
-                                                  amax_slot);
+  ql::absmax_bf16_kernel<<<grid_a, block, 0, s>>>(xb, n8, amax_slot);
   QL_CUDA(cudaGetLastError());
   const long total = static_cast<long>(M) * (K / 16);
   ql::quant_e4m3_b16_kernel<<<static_cast<unsigned>((total + block - 1) / block), block, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K),
-      static_cast<int>(K), amax_slot, ts_out, codes, static_cast<int>(K / 2), sp,
-      static_cast<int>(K / 16), st, st_atoms);
+      xb, static_cast<int>(M), static_cast<int>(K), static_cast<int>(K), amax_slot, ts_out, codes,
+      static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms);
   QL_CUDA(cudaGetLastError());
   return QL_OK;
 }
@@ -598,10 +661,11 @@ ql_status qlinear_quantize_input(const ql_linear* L, const void* x, int64_t M, v
     unsigned* scal = reinterpret_cast<unsigned*>(w8 + p.scal_off);
     return launch_quant_e4m3(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
                              scal, reinterpret_cast<float*>(scal + 1),
-                             reinterpret_cast<cudaStream_t>(stream));
+                             reinterpret_cast<cudaStream_t>(stream), p.n_tickets);
   }
   return launch_quant_mx(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
-                         nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+                         reinterpret_cast<int*>(w8 + p.tick_off), p.n_tickets,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void* ws,
@@ -663,6 +727,8 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   a.lut = L->d_lut;
   a.lut_qc = L->lut_qc;
   a.wt = L->d_codes;
+  a.partials = reinterpret_cast<float*>(w8 + p.part_off);
+  a.tickets = reinterpret_cast<int*>(w8 + p.tick_off);
   dim3 grid(p.tiles_n, p.tiles_m, p.splits);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (y32 && (reinterpret_cast<uintptr_t>(y32) & 15)) ||
@@ -708,6 +774,9 @@ ql_status quantize_act(ql_aformat fmt, const void* x, int64_t M, int64_t K, void
       if (tensor_scale == nullptr)
         return fail(QL_ERR_INVALID_ARG, "E4M3-B16 needs a device tensor_scale pointer");
       unsigned* slot = reinterpret_cast<unsigned*>(tensor_scale);
+      if (M * K <= kE4m3ClusterMaxElems)   // one launch writes ts directly
+        return launch_quant_e4m3(x, M, K, static_cast<uint8_t*>(codes),
+                                 static_cast<uint8_t*>(scales), nullptr, 0, nullptr, tensor_scale, s);
       ql_status st = launch_quant_e4m3(x, M, K, static_cast<uint8_t*>(codes),
                                        static_cast<uint8_t*>(scales), nullptr, 0, slot, nullptr, s);
       if (st != QL_OK) return st;

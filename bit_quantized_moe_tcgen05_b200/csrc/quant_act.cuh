@@ -13,6 +13,8 @@
 #include <cuda_fp8.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace ql {
 
 // Round an (exactly scaled) fp32 value to the nearest E2M1 code, ties to the even code,
@@ -96,6 +98,7 @@ __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
     int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
     int sf_atoms_per_row, int* __restrict__ zero_words, int nzero,
     __nv_bfloat16* __restrict__ deq_out = nullptr) {
+  griddep_launch_dependents();   // a GEMM launched behind this grid may start streaming weights
   const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (zero_words != nullptr && gtid < nzero) zero_words[gtid] = 0;
   const int nblk = K >> 5;
@@ -195,20 +198,12 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
   return e == 0 ? static_cast<float>(m) * 0x1p-9f : __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-// One thread per 16-element block.  codes [M, K/2] (row stride ldc), scales plain [M, K/16]
-// and/or tiled (atoms of 64 K).  Thread 0 stores ts to *ts_out when ts_out is not null.
-__global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
-    const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, const unsigned* __restrict__ amax16,
-    float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
-    uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
+// Quantize the 16-element block j of row m with tensor scale ts: codes [M, K/2] (row stride
+// ldc), scales plain [M, K/16] and/or tiled (atoms of 64 K).
+__device__ __forceinline__ void quant_e4m3_block(
+    const __nv_bfloat16* __restrict__ x, int m, int j, int ldx, float ts, uint8_t* __restrict__ codes,
+    int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
     int sf_atoms_per_row) {
-  const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const float ts = tensor_scale_from_amax16(*amax16);
-  if (gtid == 0 && ts_out != nullptr) *ts_out = ts;
-  const int nblk = K >> 4;
-  if (gtid >= static_cast<long>(M) * nblk) return;
-  const int m = static_cast<int>(gtid / nblk);
-  const int j = static_cast<int>(gtid - static_cast<long>(m) * nblk);
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
   const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
   const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -237,6 +232,88 @@ __global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
   if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = static_cast<uint8_t>(sb);
   if (scales_tiled != nullptr)
     scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row)] = static_cast<uint8_t>(sb);
+}
+
+// One thread per 16-element block, tensor scale from the amax that absmax_bf16_kernel reduced.
+// Thread 0 stores ts to *ts_out when ts_out is not null.
+__global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
+    const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, const unsigned* __restrict__ amax16,
+    float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
+    uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
+    int sf_atoms_per_row) {
+  griddep_launch_dependents();   // a GEMM launched behind this grid may start streaming weights
+  const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const float ts = tensor_scale_from_amax16(*amax16);
+  if (gtid == 0 && ts_out != nullptr) *ts_out = ts;
+  const int nblk = K >> 4;
+  if (gtid >= static_cast<long>(M) * nblk) return;
+  const int m = static_cast<int>(gtid / nblk);
+  const int j = static_cast<int>(gtid - static_cast<long>(m) * nblk);
+  quant_e4m3_block(x, m, j, ldx, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+}
+
+// Small tensors (decode): one thread-block cluster does the whole job in one launch.  Pass 1
+// reduces amax over the cluster (each CTA's maximum is read by rank 0..n-1 over distributed
+// shared memory), pass 2 quantizes.  No memset, no second launch.  The amax bit pattern goes to
+// *amax_out and ts to *ts_out (either may be null); the first nzero ints of zero_words are cleared.
+__global__ void __launch_bounds__(1024) quant_e4m3_b16_cluster_kernel(
+    const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, unsigned* __restrict__ amax_out,
+    float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
+    uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
+    int sf_atoms_per_row, int* __restrict__ zero_words, int nzero) {
+  griddep_launch_dependents();
+  __shared__ uint32_t red[32];
+  __shared__ uint32_t s_cta_amax, s_amax;
+  const int ncta = static_cast<int>(gridDim.x);   // the grid is one cluster
+  const long tid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long nthr = static_cast<long>(ncta) * blockDim.x;
+  const int nblk = K >> 4;
+  const long total = static_cast<long>(M) * nblk;
+  uint32_t mx = 0;
+  for (long b = tid; b < total; b += nthr) {
+    const int m = static_cast<int>(b / nblk);
+    const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
+    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+    mx = __vmaxu2(mx, v0.x & 0x7FFF7FFFu); mx = __vmaxu2(mx, v0.y & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v0.z & 0x7FFF7FFFu); mx = __vmaxu2(mx, v0.w & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v1.x & 0x7FFF7FFFu); mx = __vmaxu2(mx, v1.y & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v1.z & 0x7FFF7FFFu); mx = __vmaxu2(mx, v1.w & 0x7FFF7FFFu);
+  }
+  uint32_t m16 = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m16;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    if (threadIdx.x == 0) s_cta_amax = v;
+  }
+  cluster_sync_all();
+  if (threadIdx.x < 32) {
+    uint32_t v = 0;
+    if (static_cast<int>(threadIdx.x) < ncta)
+      v = ld_shared_cluster_u32(map_shared_rank(smem_u32(&s_cta_amax), threadIdx.x));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    if (threadIdx.x == 0) s_amax = v;
+  }
+  cluster_sync_all();   // every rank has read every other rank's maximum
+  const uint32_t amax16 = s_amax;
+  const float ts = tensor_scale_from_amax16(amax16);
+  if (tid == 0) {
+    if (amax_out != nullptr) *amax_out = amax16;
+    if (ts_out != nullptr) *ts_out = ts;
+  }
+  if (zero_words != nullptr)
+    for (long i = tid; i < nzero; i += nthr) zero_words[i] = 0;
+  for (long b = tid; b < total; b += nthr) {
+    const int m = static_cast<int>(b / nblk);
+    const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
+    quant_e4m3_block(x, m, j, ldx, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+  }
 }
 
 // Replace the amax bit pattern stored in *slot by the tensor scale it implies (single thread).

@@ -173,3 +173,25 @@ def test_forward_is_deterministic_and_reentrant():
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
     lin.close()
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_gemm_repeat_without_requantize(M):
+    """The GEMM run again on the same quantized input (its split-K tickets re-armed by the kernel
+    itself, not by the quantizer) reproduces the forward's output bit for bit."""
+    ql = _ql()
+    codes, sb = random_mx_weight(17, 2560, 2048)
+    xb, _ = synth.activations_bf16(17, M, 2048, 0.01, 20.0)
+    lin = ql.QLinear(codes, sb)
+    x = dev_bf16(xb)
+    ws = torch.empty(lin.workspace_bytes(M), dtype=torch.uint8, device="cuda")
+    ref = lin.forward(x, ws=ws).clone()
+    outs = []
+    for _ in range(3):
+        y = torch.empty_like(ref)
+        lin.gemm(M, y, ws)
+        outs.append(y)
+    ql.check()
+    for o in outs:
+        assert torch.equal(o, ref)
+    lin.close()
