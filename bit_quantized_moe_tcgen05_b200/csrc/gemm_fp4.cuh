@@ -20,10 +20,12 @@
 // Weight streaming starts before the activations exist: the kernel is launched with programmatic
 // stream serialization behind the activation quantizer, the producer first issues the weight
 // copies of the whole first ring fill (and the VQ warps decode them), and only then waits for the
-// quantizer grid (griddepcontrol.wait) before it loads activation tiles.  Split-K (decode): the
-// gridDim.z K-splits of one output tile each write an fp32 partial tile to a global workspace;
-// the last split to finish (an atomic ticket per tile) adds the partials in split order, so the
-// result is deterministic, writes y and re-arms the ticket for the next launch.
+// quantizer grid (griddepcontrol.wait) before it loads activation tiles.  In decode launches the
+// activation tiles and scale atoms of every stage go by cp.async from the producer warp, so they
+// do not queue behind the weight blocks in the bulk-copy engine.  Split-K (decode): the gridDim.z
+// K-splits of one output tile each write an fp32 partial tile to a global workspace; the last
+// split to finish (an atomic ticket per tile) bulk-copies the partials into its idle ring and
+// adds them in split order, so the result is deterministic, writes y and re-arms the ticket.
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -31,7 +33,7 @@
 namespace ql {
 
 // Most K-splits of one output tile (bounds the per-thread partial loads of the reduction).
-constexpr int kMaxSplits = 16;
+constexpr int kMaxSplits = 8;
 
 struct Fp4GemmArgs {
   int M, N;                 // tokens, output features
@@ -39,8 +41,6 @@ struct Fp4GemmArgs {
   int n_base_stages;        // ceil(C / 256)
   int n_stages_total;       // n_base_stages + ceil(k_tail / 256)
   int stages_per_split;     // K stages handled by one CTA (gridDim.z = splits)
-  const uint8_t* sfa;       // weight scales, tiled atoms
-  int sfa_atoms;            // atoms per 128-row group of the weight
   const uint8_t* sfb;       // activation scales, tiled atoms
   int sfb_atoms;            // atoms per 128-row group of the activation
   const float* alpha_dev;   // optional device scalar multiplied into alpha (tensor scale of x)
@@ -48,17 +48,22 @@ struct Fp4GemmArgs {
   __nv_bfloat16* y;         // [M, ldy] bf16 output
   float* y32;               // optional [M, ldy] fp32 output
   int ldy;
-  const uint8_t* lut;       // VQ: packed E2M1 codebooks [N/64][K/64][256][2]
-  int lut_qc;               // VQ: QBlocks along K (K / 64)
-  const uint8_t* wt;        // weight operand blocks [N/128][n_stages_total][block bytes]:
-                            // FP4 codes 128 rows x 128 B, 128-byte swizzle pre-applied (16 KB),
-                            // or VQ indices 128 rows x 64 B (8 KB)
-  float* partials;          // split-K: [tiles][splits][BN][128] fp32 (tile = y-tile * gridDim.x + x-tile)
-  int* tickets;             // split-K: [tiles] arrival counters, zero between launches
+  const uint8_t* wt;        // weight blocks [N/128][n_stages_total][Fp4Cfg::kWBytes], one per
+                            // (128-row tile, 256-wide K stage), laid out as the stage buffer:
+                            // FP4 codes 128 rows x 128 B with the 128-byte swizzle applied, or VQ
+                            // indices 128 rows x 64 B + the stage's 8 QBlock codebooks; then the
+                            // stage's weight scale atoms
+  float* partials;          // split-K: fp32 [tiles][splits][BN][128] (tile = blockIdx.y * gridDim.x
+                            // + blockIdx.x)
+  const uint8_t* xq;        // quantized activation codes [M, C/2] (read directly by decode launches)
+  int* tickets;             // [tiles] arrival counters, zero between launches
 };
 
 template <int BN, bool E8M0, bool VQ = false>
 struct Fp4Cfg {
+  // warps: 0 producer, 1 MMA, 2..5 epilogue; VQ adds decoders so that warps 2..9 decode
+  static constexpr int kDecWarps = VQ ? 8 : 0;
+  static constexpr int kThreads = VQ ? 320 : 192;
   static constexpr int kAtomK = E8M0 ? 128 : 64;      // K elements covered by one SF atom
   static constexpr int kAtoms = 256 / kAtomK;         // SF atoms per stage per 128 rows
   static constexpr int kG = (BN + 127) / 128;          // 128-row groups of the B operand
@@ -68,7 +73,11 @@ struct Fp4Cfg {
   static constexpr int kSfbBytes = kAtoms * kG * 512;
   static constexpr int kIdxBytes = VQ ? 128 * 64 : 0;   // VQ: 8-bit indices, 128 rows x 64
   static constexpr int kLutBytes = VQ ? 8 * 512 : 0;    // VQ: 2 x 4 QBlock codebooks of 512 B
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kIdxBytes + kLutBytes;
+  // The weight block of one stage, as stored in HBM and copied by one bulk copy:
+  // FP4: [codes 16 KB][SFA atoms]; VQ: [indices 8 KB][codebooks 4 KB][SFA atoms].
+  static constexpr int kWBytes = (VQ ? kIdxBytes + kLutBytes : kABytes) + kSfaBytes;
+  static constexpr int kSfaOff = VQ ? kIdxBytes + kLutBytes : kABytes;
+  static constexpr int kStageBytes = kWBytes + kBBytes + kSfbBytes + (VQ ? kABytes : 0);
   static constexpr int kBudget = 212 * 1024;
   static constexpr int kStagesRaw = kBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : (kStagesRaw < 2 ? 2 : kStagesRaw);
@@ -87,7 +96,7 @@ struct Fp4Cfg {
 // VQ = true (MXCode PreScale weights): the blocks hold 8-bit indices; warps 2..5 decode each
 // stage's operand tile from the shared-memory codebooks.
 template <int BN, bool E8M0, bool VQ = false>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
                     const __grid_constant__ CUtensorMap tm_y32, const Fp4GemmArgs a) {
   using Cfg = Fp4Cfg<BN, E8M0, VQ>;
@@ -95,34 +104,42 @@ __global__ void __launch_bounds__(192, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + S * Cfg::kABytes;
-  uint8_t* sSfa = sB + S * Cfg::kBBytes;
-  uint8_t* sSfb = sSfa + S * Cfg::kSfaBytes;
-  uint8_t* sIdx = sSfb + S * Cfg::kSfbBytes;
-  uint8_t* sLut = sIdx + S * Cfg::kIdxBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sLut + S * Cfg::kLutBytes);
+  // ring layout (every region 1 KB aligned): weight blocks, B tiles, SFB atoms, decoded A (VQ)
+  uint8_t* sW = smem;
+  uint8_t* sB = sW + S * Cfg::kWBytes;
+  uint8_t* sSfb = sB + S * Cfg::kBBytes;
+  uint8_t* sAdec = sSfb + S * Cfg::kSfbBytes;
+  auto sA = [&](int st) { return VQ ? sAdec + st * Cfg::kABytes : sW + st * Cfg::kWBytes; };
+  uint64_t* full = reinterpret_cast<uint64_t*>(sAdec + (VQ ? S * Cfg::kABytes : 0));
   uint64_t* empty = full + S;
-  uint64_t* decd = empty + S;   // VQ: operand tile decoded (count 128)
-  uint64_t* wfull = decd + S;   // VQ: indices + codebooks landed
-  uint64_t* accf = wfull + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* decd = empty + S;   // VQ: operand tile decoded
+  uint64_t* wfull = decd + S;   // VQ: indices + codebooks + SFA landed
+  uint64_t* afull = wfull + S;  // decode: activation tile + SFB landed by cp.async (count 32)
+  uint64_t* accf = afull + S;   // accumulator complete
+  uint64_t* rbar = accf + 1;    // split-K: the splits' partials landed in the idle ring
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 1);
   __shared__ int s_last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN;
+  const int tile = blockIdx.y * gridDim.x + blockIdx.x;
   const int s_begin = blockIdx.z * a.stages_per_split;
   const int s_end = min(a.n_stages_total, s_begin + a.stages_per_split);
   const int n_it = max(0, s_end - s_begin);
+  const int splits = gridDim.z;
+  // decode launches whose stages all fit the ring take activations by cp.async
+  const bool lsu_act = BN <= 64 && n_it <= S;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&decd[s], 128);
+      mbar_init(&decd[s], VQ ? Cfg::kDecWarps * 32 : 1);
       mbar_init(&wfull[s], 1);
+      mbar_init(&afull[s], 32);
     }
     mbar_init(accf, 1);
+    mbar_init(rbar, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) prefetch_tmap(&tm_x);
@@ -153,33 +170,24 @@ __global__ void __launch_bounds__(192, 1)
   bool ok = true;
   if (warp == 0) {
     // ---------------- producer: the whole warp runs the loop; one elected lane issues copies.
-    // Weight part of stage it (independent of earlier grids): codes or indices + codebooks, SFA.
+    // Weight part of stage it (independent of earlier grids): one bulk copy of the stage block.
     auto issue_weight = [&](int it) {
       const int i = s_begin + it, st = it % S;
       int kw, kx, valid;
       stage_coords(i, kw, kx, valid);
       const int nat = valid / Cfg::kAtomK;
-      const uint32_t act_bytes = Cfg::kBBytes + nat * 512 * Cfg::kG;
-      const uint8_t* wblk = a.wt + (static_cast<size_t>(blockIdx.x) * a.n_stages_total + i) *
-                                       (VQ ? Cfg::kIdxBytes : Cfg::kABytes);
+      const uint32_t act_bytes = lsu_act ? 0u : Cfg::kBBytes + nat * 512 * Cfg::kG;
+      const uint8_t* wblk = a.wt + (static_cast<size_t>(blockIdx.x) * a.n_stages_total + i) * Cfg::kWBytes;
       if constexpr (VQ) {
-        mbar_arrive_expect_tx(&wfull[st], Cfg::kIdxBytes + Cfg::kLutBytes);
-        mbar_arrive_expect_tx(&full[st], nat * 512 + act_bytes);
-        bulk_load(sIdx + st * Cfg::kIdxBytes, wblk, Cfg::kIdxBytes, &wfull[st]);
-#pragma unroll
-        for (int g2 = 0; g2 < 2; ++g2)
-          bulk_load(sLut + st * Cfg::kLutBytes + g2 * 2048,
-                    a.lut + (static_cast<size_t>((n0 >> 6) + g2) * a.lut_qc + (kw >> 6)) * 512,
-                    2048, &wfull[st]);
+        mbar_arrive_expect_tx(&wfull[st], Cfg::kWBytes);
+        if (!lsu_act) mbar_arrive_expect_tx(&full[st], act_bytes);
+        bulk_load(sW + st * Cfg::kWBytes, wblk, Cfg::kWBytes, &wfull[st]);
       } else {
-        mbar_arrive_expect_tx(&full[st], Cfg::kABytes + nat * 512 + act_bytes);
-        bulk_load(sA + st * Cfg::kABytes, wblk, Cfg::kABytes, &full[st]);
+        mbar_arrive_expect_tx(&full[st], Cfg::kWBytes + act_bytes);
+        bulk_load(sW + st * Cfg::kWBytes, wblk, Cfg::kWBytes, &full[st]);
       }
-      bulk_load(sSfa + st * Cfg::kSfaBytes,
-                a.sfa + (static_cast<size_t>(n0 >> 7) * a.sfa_atoms + kw / Cfg::kAtomK) * 512,
-                nat * 512, &full[st]);
     };
-    // Activation part of stage it (written by the quantizer grid): B codes and SFB.
+    // Activation part (written by the quantizer grid): B codes and SFB, by the bulk-copy engine.
     auto issue_act = [&](int it) {
       const int i = s_begin + it, st = it % S;
       int kw, kx, valid;
@@ -197,29 +205,56 @@ __global__ void __launch_bounds__(192, 1)
       for (int it = 0; it < pre; ++it) issue_weight(it);
     __syncwarp();
     griddep_wait();
-    if (elect_one())
-      for (int it = 0; it < pre; ++it) issue_act(it);
-    __syncwarp();
-    for (int it = pre; it < n_it && ok; ++it) {
-      const int st = it % S;
-      const uint32_t ph = (it / S) & 1;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 1));
-      if (!ok) break;
-      if (elect_one()) {
-        issue_weight(it);
-        issue_act(it);
+    if (lsu_act) {
+      // Every stage's activation tile (BN rows x 128 B, stored with the 128-byte swizzle) and its
+      // scale atoms, 16 bytes per cp.async from all 32 lanes; rows past M are zero-filled.
+      for (int it = 0; it < n_it; ++it) {
+        int kw, kx, valid;
+        stage_coords(s_begin + it, kw, kx, valid);
+        const int nat = valid / Cfg::kAtomK;
+        const uint32_t bdst = smem_u32(sB + it * Cfg::kBBytes);
+        for (int c = lane; c < BN * 8; c += 32) {
+          const int r = c >> 3, kc = c & 7;
+          const bool in = m0 + r < a.M;
+          const uint8_t* src = a.xq + static_cast<size_t>(in ? m0 + r : 0) * (a.C / 2) + (kx >> 1) + kc * 16;
+          cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4), src, in ? 16u : 0u);
+        }
+        const uint8_t* sfsrc = a.sfb + (static_cast<size_t>(m0 >> 7) * a.sfb_atoms + kx / Cfg::kAtomK) * 512;
+        const uint32_t sfdst = smem_u32(sSfb + it * Cfg::kSfbBytes);
+        for (int c = lane; c < nat * 32; c += 32) cp_async16(sfdst + c * 16, sfsrc + c * 16, 16u);
+        cp_async_commit();
       }
+      for (int it = 0; it < n_it; ++it) {   // stage it complete -> visible to the tensor core
+        cp_async_wait_pending(n_it - 1 - it);
+        fence_proxy_async_smem();
+        mbar_arrive(&afull[it]);
+      }
+    } else {
+      if (elect_one())
+        for (int it = 0; it < pre; ++it) issue_act(it);
       __syncwarp();
+      for (int it = pre; it < n_it && ok; ++it) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 1));
+        if (!ok) break;
+        if (elect_one()) {
+          issue_weight(it);
+          issue_act(it);
+        }
+        __syncwarp();
+      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer: converged warp, one lane issues the tcgen05 instructions
     const uint32_t idesc0 = idesc_fp4_block(BN, E8M0);
-    bool first = true;
     for (int it = 0; it < n_it && ok; ++it) {
       const int i = s_begin + it, st = it % S;
       const uint32_t ph = (it / S) & 1;
-      bool w = mbar_wait(&full[st], ph, 2);
-      if constexpr (VQ) w = w && mbar_wait(&decd[st], ph, 4);
+      bool w = true;
+      if (!VQ || !lsu_act) w = mbar_wait(&full[st], ph, 2);
+      if constexpr (VQ) w = w && mbar_wait(&wfull[st], ph, 6) && mbar_wait(&decd[st], ph, 4);
+      if (lsu_act) w = w && mbar_wait(&afull[st], 0, 9);
       ok = __all_sync(0xFFFFFFFFu, w);
       if (!ok) break;
       tc_fence_after();
@@ -228,9 +263,9 @@ __global__ void __launch_bounds__(192, 1)
       const int nat = valid / Cfg::kAtomK;
       const uint32_t ta = tmem + sfa_col0 + st * Cfg::kSfaCols;
       const uint32_t tb = tmem + sfb_col0 + st * Cfg::kSfbCols;
-      const uint32_t sfa_s = smem_u32(sSfa + st * Cfg::kSfaBytes);
+      const uint32_t sfa_s = smem_u32(sW + st * Cfg::kWBytes + Cfg::kSfaOff);
       const uint32_t sfb_s = smem_u32(sSfb + st * Cfg::kSfbBytes);
-      const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
+      const uint32_t a_base = smem_u32(sA(st));
       const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
       const int nk = valid / 64;
       if (lane == 0) {   // the same lane issues every MMA and the commits that track them
@@ -239,9 +274,9 @@ __global__ void __launch_bounds__(192, 1)
           if (at < nat) {
             tc_cp_32x128b_warpx4(ta + at * 4, make_sdesc(sfa_s + at * 512, 0, 128, kLayoutNone));
 #pragma unroll
-            for (int g = 0; g < Cfg::kG; ++g)
-              tc_cp_32x128b_warpx4(tb + at * 4 * Cfg::kG + g * 4,
-                                   make_sdesc(sfb_s + g * Cfg::kAtoms * 512 + at * 512, 0, 128, kLayoutNone));
+            for (int gg = 0; gg < Cfg::kG; ++gg)
+              tc_cp_32x128b_warpx4(tb + at * 4 * Cfg::kG + gg * 4,
+                                   make_sdesc(sfb_s + gg * Cfg::kAtoms * 512 + at * 512, 0, 128, kLayoutNone));
           }
         }
 #pragma unroll
@@ -254,7 +289,7 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t idd = idesc0 | (byte << 29) | (byte << 4);
             const uint32_t sa = (ta + at * 4) | (byte << 30);
             const uint32_t sb = (tb + at * 4 * Cfg::kG) | (byte << 30);
-            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+            const uint32_t acc = (it == 0 && kk == 0) ? 0u : 1u;
             if (E8M0)
               mma_mxf4_block32(tmem, ad, bd, idd, sa, sb, acc);
             else
@@ -263,28 +298,28 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_commit(&empty[st]);
       }
-      first = false;
       __syncwarp();
     }
     if (lane == 0) tc_commit(accf);
     __syncwarp();
   } else {
     if constexpr (VQ) {
-      // ---------------- VQ decode (warps 2..5, 128 threads): for each stage rebuild the
-      // 128 x 256 E2M1 operand tile from 8-bit indices and the QBlock codebooks, in the
-      // 128-byte-swizzled K-major layout the MMA reads (16-byte chunk kc of row r at kc ^ (r%8)).
-      // Only weights are read, so this runs ahead of the activation quantizer.
+      // ---------------- VQ decode (warps 2..9): for each stage rebuild the 128 x 256 E2M1 operand
+      // tile from 8-bit indices and the QBlock codebooks, in the 128-byte-swizzled K-major layout
+      // the MMA reads (16-byte chunk kc of row r at kc ^ (r%8)).  Only weights are read, so this
+      // runs ahead of the activation quantizer.
       const int t = threadIdx.x - 64;
+      constexpr int kDT = Cfg::kDecWarps * 32;
       for (int it = 0; it < n_it && ok; ++it) {
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
         if (!mbar_wait(&wfull[st], ph, 5)) { ok = false; break; }
-        const uint8_t* idx_s = sIdx + st * Cfg::kIdxBytes;
-        const uint16_t* lut = reinterpret_cast<const uint16_t*>(sLut + st * Cfg::kLutBytes);
-        uint8_t* a_s = sA + st * Cfg::kABytes;
-#pragma unroll 4
-        for (int j = 0; j < 8; ++j) {
-          const int c = t + 128 * j;             // 16-byte output chunk: row r, chunk kc
+        const uint8_t* idx_s = sW + st * Cfg::kWBytes;
+        const uint16_t* lut = reinterpret_cast<const uint16_t*>(idx_s + Cfg::kIdxBytes);
+        uint8_t* a_s = sA(st);
+#pragma unroll
+        for (int j = 0; j < 1024 / kDT; ++j) {
+          const int c = t + kDT * j;             // 16-byte output chunk: row r, chunk kc
           const int r = c >> 3, kc = c & 7;
           const uint2 iv = *reinterpret_cast<const uint2*>(idx_s + r * 64 + kc * 8);
           const uint16_t* L = lut + ((((r >> 6) << 2) + (kc >> 1)) << 8);
@@ -299,104 +334,122 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(&decd[st]);
       }
     }
-    // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
-    const int q = warp & 3;
-    const int splits = gridDim.z;
-    const bool have_acc = n_it > 0;
-    griddep_wait();   // alpha_dev, the workspace and y belong to / follow earlier grids
-    float alpha = a.alpha;
-    if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
-    if (have_acc && ok) ok = mbar_wait(accf, 0, 3);
-    tc_fence_after();
-    if (splits == 1) {
-      // The tile is staged in the idle operand ring as y[m][n] and written by one TMA tensor
-      // store (which clips rows past M and columns past N): first the bf16 tile, then, when
-      // requested, the fp32 tile in the same buffer once the first store has read it.
-      __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(smem);               // [BN][128]
-      float* y32buf = reinterpret_cast<float*>(smem);                             // [BN][128]
-      if (ok) {
+    if (warp < 6) {   // (extra VQ decoders, warps 6..9, take no part in the epilogue)
+      // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+      const int q = warp & 3;
+      const int nl = q * 32 + lane;
+      const int n = n0 + nl;
+      const int mcount = min(BN, a.M - m0);
+      const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      griddep_wait();   // alpha_dev, the workspace and y belong to / follow earlier grids
+      float alpha = a.alpha;
+      if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
+      if (n_it > 0) ok = bar_and(1, 128, ok && mbar_wait(accf, 0, 3));   // the 128 agree
+      tc_fence_after();
+      if (ok && splits == 1) {
+        // The tile is staged in the idle operand ring as y[m][n] and written by one TMA tensor
+        // store (which clips rows past M and columns past N): first the bf16 tile, then, when
+        // requested, the fp32 tile in the same buffer once the first store has read it.
+        __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(smem);               // [BN][128]
+        float* y32buf = reinterpret_cast<float*>(smem);                             // [BN][128]
 #pragma unroll 1
         for (int c = 0; c < BN; c += 8) {
           uint32_t r[8];
-          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+          tmem_ld8(trow + c, r);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            ybuf[(c + j) * 128 + q * 32 + lane] =
-                __float2bfloat16_rn((have_acc ? __uint_as_float(r[j]) : 0.f) * alpha);
-        }
-      }
-      fence_proxy_async_smem();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (threadIdx.x == 64 && ok) {
-        tma_store_2d(&tm_y, ybuf, n0, m0);
-        bulk_commit_group();
-        bulk_wait_group_read0();
-      }
-      if (a.y32 != nullptr) {
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (ok) {
-#pragma unroll 1
-          for (int c = 0; c < BN; c += 8) {
-            uint32_t r[8];
-            tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              y32buf[(c + j) * 128 + q * 32 + lane] = (have_acc ? __uint_as_float(r[j]) : 0.f) * alpha;
-          }
+            ybuf[(c + j) * 128 + nl] = __float2bfloat16_rn((n_it > 0 ? __uint_as_float(r[j]) : 0.f) * alpha);
         }
         fence_proxy_async_smem();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (threadIdx.x == 64 && ok) {
-          tma_store_2d(&tm_y32, y32buf, n0, m0);
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) {
+          tma_store_2d(&tm_y, ybuf, n0, m0);
           bulk_commit_group();
           bulk_wait_group_read0();
         }
-      }
-    } else {
-      // Split-K: park this split's fp32 partial tile [BN tokens][128 rows] in the workspace
-      // (lanes cover consecutive rows: coalesced), then take a ticket; the last split reduces.
-      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-      const int nl = q * 32 + lane;
-      const int mcount = min(BN, a.M - m0);
-      float* part = a.partials + static_cast<size_t>(tile) * splits * BN * 128;
-      if (ok) {
+        if (a.y32 != nullptr) {
+          named_bar_sync(1, 128);
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 8) {
+            uint32_t r[8];
+            tmem_ld8(trow + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) y32buf[(c + j) * 128 + nl] = (n_it > 0 ? __uint_as_float(r[j]) : 0.f) * alpha;
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (threadIdx.x == 64) {
+            tma_store_2d(&tm_y32, y32buf, n0, m0);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+        }
+      } else if (ok) {
+        // Split-K: park this split's fp32 partial [BN tokens][128 rows] in the workspace (lanes
+        // cover consecutive rows: coalesced) and take a ticket; the last split reduces.
+        float* part = a.partials + static_cast<size_t>(tile) * splits * BN * 128;
         float* mine = part + static_cast<size_t>(blockIdx.z) * BN * 128;
 #pragma unroll 1
         for (int c = 0; c < mcount; c += 8) {
           uint32_t r[8];
-          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+          tmem_ld8(trow + c, r);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            if (c + j < mcount) __stcg(mine + (c + j) * 128 + nl, have_acc ? __uint_as_float(r[j]) : 0.f);
+            if (c + j < mcount) mine[(c + j) * 128 + nl] = n_it > 0 ? __uint_as_float(r[j]) : 0.f;
         }
-      }
-      __threadfence();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (threadIdx.x == 64) s_last = ok ? (atomicAdd(a.tickets + tile, 1) == splits - 1) : 0;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (s_last) {
-        __threadfence();
-        const int n = n0 + nl;
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) {
+          __threadfence();   // release the whole CTA's partial (ordered before by the barrier)
+          s_last = (atomicAdd(a.tickets + tile, 1) == splits - 1);
+          if (s_last) __threadfence();   // acquire every other split's partial
+        }
+        named_bar_sync(1, 128);
+        if (s_last) {
+          // The ring is idle: bulk-copy every split's partial for a run of tokens into it (all
+          // copies in flight at once), then each thread adds its row in split order, 4 tokens at
+          // a time with every split's value of them loaded before the adds.
+          float* stg = reinterpret_cast<float*>(smem);
+          constexpr int kRing = S * Cfg::kStageBytes;
+          const int cc = min(mcount, (kRing / (splits * 512)) & ~7);
 #pragma unroll 1
-        for (int c = 0; c < mcount; ++c) {
-          float v[kMaxSplits];
+          for (int c0 = 0, rnd = 0; c0 < mcount && ok; c0 += cc, ++rnd) {
+            const int cn = min(cc, mcount - c0);
+            if (threadIdx.x == 64) {
+              fence_proxy_async_global();
+              mbar_arrive_expect_tx(rbar, splits * cn * 512);
+              for (int r = 0; r < splits; ++r)
+                bulk_load(stg + r * cc * 128, part + (static_cast<size_t>(r) * BN + c0) * 128, cn * 512, rbar);
+            }
+            ok = bar_and(1, 128, mbar_wait(rbar, rnd & 1, 8));
+            if (!ok) break;
+#pragma unroll 1
+            for (int c = 0; c < cn; c += 4) {
+              float v[kMaxSplits][4];
 #pragma unroll
-          for (int r = 0; r < kMaxSplits; ++r)
-            if (r < splits) v[r] = __ldcg(part + (static_cast<size_t>(r) * BN + c) * 128 + nl);
-          float acc = 0.f;
+              for (int r = 0; r < kMaxSplits; ++r)
 #pragma unroll
-          for (int r = 0; r < kMaxSplits; ++r)
-            if (r < splits) acc += v[r];
-          if (n < a.N) {
-            const size_t o = static_cast<size_t>(m0 + c) * a.ldy + n;
-            a.y[o] = __float2bfloat16_rn(acc * alpha);
-            if (a.y32 != nullptr) a.y32[o] = acc * alpha;
+                for (int j = 0; j < 4; ++j)
+                  v[r][j] = (r < splits && c + j < cn) ? stg[(r * cc + c + j) * 128 + nl] : 0.f;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                float acc = 0.f;
+#pragma unroll
+                for (int r = 0; r < kMaxSplits; ++r)
+                  if (r < splits) acc += v[r][j];
+                if (c + j < cn && n < a.N) {
+                  const size_t o = static_cast<size_t>(m0 + c0 + c + j) * a.ldy + n;
+                  a.y[o] = __float2bfloat16_rn(acc * alpha);
+                  if (a.y32 != nullptr) a.y32[o] = acc * alpha;
+                }
+              }
+            }
+            named_bar_sync(1, 128);   // before the next run overwrites stg
           }
+          if (threadIdx.x == 64) a.tickets[tile] = 0;   // re-armed for the next launch
         }
-        if (threadIdx.x == 64) a.tickets[tile] = 0;   // re-armed for the next launch
       }
     }
   }

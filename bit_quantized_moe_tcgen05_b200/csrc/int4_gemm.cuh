@@ -80,6 +80,11 @@ constexpr int kInt4WBlock = 128 * 64 + 128 * 4;   // 8704 B
 
 template <int BN>
 struct Int4Cfg {
+  // warps: 0 producer, 1 MMA, then kFoldWarps fold/epilogue warps, then 4 decode warps
+  static constexpr int kFoldWarps = BN >= 128 ? 8 : 4;
+  static constexpr int kCols = BN * 4 / kFoldWarps;   // accumulator columns per fold thread
+  static constexpr int kDecWarps = 4;
+  static constexpr int kThreads = (2 + kFoldWarps + kDecWarps) * 32;
   static constexpr int kRawBytes = kInt4WBlock;
   static constexpr int kABytes = 128 * 128;        // int8 tile, 128 rows x 128 B
   static constexpr int kBBytes = BN * 128;
@@ -90,14 +95,52 @@ struct Int4Cfg {
   static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 512;
   static_assert(BN * 128 * 4 <= kStages * kStageBytes, "output staging must fit the ring");
+  static_assert(kCols % 8 == 0, "fold columns come in tcgen05.ld groups of 8");
 };
 
+// Packed fp32 pair arithmetic (sm_100 f32x2 instructions): d = a * b + c, d = a + b, d = a * b,
+// each element rounded to nearest even exactly as the scalar instruction would.
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// Exact float of an int32 x with |x| < 2^22: in [2^23, 2^24) the float grid is the integers, so
+// the bit pattern of 1.5 * 2^23 plus x is the float 1.5 * 2^23 + x; the subtraction is exact.
+__device__ __forceinline__ float2 small_ints_to_float2(uint32_t x0, uint32_t x1) {
+  return f2_add(make_float2(__uint_as_float(x0 + 0x4B400000u), __uint_as_float(x1 + 0x4B400000u)),
+                make_float2(-12582912.0f, -12582912.0f));
+}
+
 template <int BN>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
     int4_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
                      const __grid_constant__ CUtensorMap tm_y32, const Int4GemmArgs a) {
   using Cfg = Int4Cfg<BN>;
   constexpr int S = Cfg::kStages;
+  constexpr int kFoldThreads = Cfg::kFoldWarps * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -121,12 +164,17 @@ __global__ void __launch_bounds__(320, 1)
   const int s_begin = blockIdx.z * a.stages_per_split;
   const int s_end = min(st_n, s_begin + a.stages_per_split);
   const int nst = max(0, s_end - s_begin);
+  const bool fold_warp = warp >= 2 && warp < 2 + Cfg::kFoldWarps;
+  const int fthread = threadIdx.x - 64;                       // 0.. fold threads - 1
+  const int q = warp & 3;                                     // TMEM lane quadrant of a fold warp
+  const int row = q * 32 + lane;                              // weight row of a fold thread
+  const int col0 = (fthread / 128) * Cfg::kCols;              // its accumulator columns
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 2);     // MMA commit + fold release
-      mbar_init(&decd[s], 128);
+      mbar_init(&decd[s], Cfg::kDecWarps * 32);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accf[b], 1);
@@ -145,9 +193,9 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
-  float acc[BN];
+  float2 acc[Cfg::kCols / 2];
 #pragma unroll
-  for (int c = 0; c < BN; ++c) acc[c] = 0.f;
+  for (int c = 0; c < Cfg::kCols / 2; ++c) acc[c] = make_float2(0.f, 0.f);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -181,9 +229,9 @@ __global__ void __launch_bounds__(320, 1)
         tc_commit(&accf[b]);
       }
     }
-  } else if (warp >= 6) {
+  } else if (!fold_warp) {
     // ---------------- decode: packed INT4 -> int8, 128-byte swizzled K-major tile
-    const int t = threadIdx.x - 192;
+    const int t = threadIdx.x - (2 + Cfg::kFoldWarps) * 32;
     for (int j = 0; j < nst && ok; ++j) {
       const int st = j % S;
       const uint32_t ph = (j / S) & 1;
@@ -210,62 +258,71 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(&decd[st]);
     }
   } else {
-    // ---------------- fold: warps 2..5 own TMEM lane quadrant q (weight rows 32q..32q+31)
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    // The loop count is the same for all 128 fold threads (named barrier inside); a thread whose
-    // wait expired skips the work but keeps taking the barriers.
+    // ---------------- fold: acc += I * (s_w * s_x) per 128-input group, on packed fp32 pairs.
+    // Fold warps own TMEM lane quadrant warp % 4 (weight rows) and a run of kCols columns.
+    // The loop count is the same for all fold threads (named barrier inside); a thread whose wait
+    // expired skips the work but keeps taking the barriers.
     for (int j = 0; j < nst; ++j) {
       const int st = j % S, b = j & 1;
       if (ok) ok = mbar_wait(&accf[b], (j >> 1) & 1, 26);
       tc_fence_after();
       if (ok) {
         const float rs = reinterpret_cast<const float*>(sRaw(st) + 128 * 64)[row];
-        const float* sx = sSx(st);
+        const float2 rs2 = make_float2(rs, rs);
+        const float* sx = sSx(st) + col0;
 #pragma unroll
-        for (int c = 0; c < BN; c += 8) {
+        for (int c = 0; c < Cfg::kCols; c += 8) {
           uint32_t r[8];
-          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN + c, r);
+          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN + col0 + c, r);
+          const float4 s0 = *reinterpret_cast<const float4*>(sx + c);
+          const float4 s1 = *reinterpret_cast<const float4*>(sx + c + 4);
           tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            acc[c + e] = fmaf(static_cast<float>(static_cast<int>(r[e])), rs * sx[c + e], acc[c + e]);
+          const float2 w0 = f2_mul(rs2, make_float2(s0.x, s0.y)), w1 = f2_mul(rs2, make_float2(s0.z, s0.w));
+          const float2 w2 = f2_mul(rs2, make_float2(s1.x, s1.y)), w3 = f2_mul(rs2, make_float2(s1.z, s1.w));
+          acc[c / 2 + 0] = f2_fma(small_ints_to_float2(r[0], r[1]), w0, acc[c / 2 + 0]);
+          acc[c / 2 + 1] = f2_fma(small_ints_to_float2(r[2], r[3]), w1, acc[c / 2 + 1]);
+          acc[c / 2 + 2] = f2_fma(small_ints_to_float2(r[4], r[5]), w2, acc[c / 2 + 2]);
+          acc[c / 2 + 3] = f2_fma(small_ints_to_float2(r[6], r[7]), w3, acc[c / 2 + 3]);
         }
       }
       tc_fence_before();
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      if (threadIdx.x == 64) {
+      named_bar_sync(2, kFoldThreads);
+      if (fthread == 0) {
         mbar_arrive(&acce[b]);
         mbar_arrive(&empty[st]);
       }
     }
   }
 
-  // ---------------- epilogue (warps 2..5): one tile, or a cluster of K-splits
+  // ---------------- epilogue (fold warps): one tile, or a cluster of K-splits
   const int splits = gridDim.z;
-  if (warp >= 2 && warp < 6) {
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    asm volatile("bar.sync 2, 128;" ::: "memory");   // every fold thread is past the ring
+  if (fold_warp) {
+    named_bar_sync(2, kFoldThreads);   // every fold thread is past the ring
     if (splits == 1) {
       __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(smem);
 #pragma unroll
-      for (int c = 0; c < BN; ++c) ybuf[c * 128 + row] = __float2bfloat16_rn(acc[c]);
+      for (int c = 0; c < Cfg::kCols / 2; ++c) {
+        ybuf[(col0 + 2 * c) * 128 + row] = __float2bfloat16_rn(acc[c].x);
+        ybuf[(col0 + 2 * c + 1) * 128 + row] = __float2bfloat16_rn(acc[c].y);
+      }
       fence_proxy_async_smem();
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      if (threadIdx.x == 64 && ok) {
+      named_bar_sync(2, kFoldThreads);
+      if (fthread == 0 && ok) {
         tma_store_2d(&tm_y, ybuf, n0, m0);
         bulk_commit_group();
         bulk_wait_group_read0();
       }
       if (a.y32 != nullptr) {
-        asm volatile("bar.sync 2, 128;" ::: "memory");
+        named_bar_sync(2, kFoldThreads);
         float* y32buf = reinterpret_cast<float*>(smem);
 #pragma unroll
-        for (int c = 0; c < BN; ++c) y32buf[c * 128 + row] = acc[c];
+        for (int c = 0; c < Cfg::kCols / 2; ++c) {
+          y32buf[(col0 + 2 * c) * 128 + row] = acc[c].x;
+          y32buf[(col0 + 2 * c + 1) * 128 + row] = acc[c].y;
+        }
         fence_proxy_async_smem();
-        asm volatile("bar.sync 2, 128;" ::: "memory");
-        if (threadIdx.x == 64 && ok) {
+        named_bar_sync(2, kFoldThreads);
+        if (fthread == 0 && ok) {
           tma_store_2d(&tm_y32, y32buf, n0, m0);
           bulk_commit_group();
           bulk_wait_group_read0();
@@ -274,21 +331,24 @@ __global__ void __launch_bounds__(320, 1)
     } else {
       float* part = reinterpret_cast<float*>(smem);
 #pragma unroll
-      for (int c = 0; c < BN; ++c) part[c * 128 + row] = acc[c];
+      for (int c = 0; c < Cfg::kCols / 2; ++c) {
+        part[(col0 + 2 * c) * 128 + row] = acc[c].x;
+        part[(col0 + 2 * c + 1) * 128 + row] = acc[c].y;
+      }
     }
   }
   __syncwarp();
   cluster_sync_all();
   if (splits > 1 && warp >= 2 && warp < 6) {
-    const int q = warp & 3;
-    const int n = n0 + q * 32 + lane;
+    const int qq = warp & 3;
+    const int n = n0 + qq * 32 + lane;
     const int rank = static_cast<int>(cluster_ctarank());
     const int mcount = min(BN, a.M - m0);
-    const uint32_t base = smem_u32(smem) + (q * 32 + lane) * 4;
+    const uint32_t base = smem_u32(smem) + (qq * 32 + lane) * 4;
     for (int c = rank * 8; c < mcount; c += splits * 8) {
-      float v[4][8];
+      float v[kInt4MaxClusterSplits][8];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < kInt4MaxClusterSplits; ++r)
         if (r < splits) {
           const uint32_t remote = map_shared_rank(base + c * 512, r);
 #pragma unroll
@@ -297,14 +357,14 @@ __global__ void __launch_bounds__(320, 1)
       if (n < a.N) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          float s = 0.f;
+          float sacc = 0.f;
 #pragma unroll
-          for (int r = 0; r < 4; ++r)
-            if (r < splits) s += v[r][e];
+          for (int r = 0; r < kInt4MaxClusterSplits; ++r)
+            if (r < splits) sacc += v[r][e];
           if (c + e < mcount) {
             const size_t o = static_cast<size_t>(m0 + c + e) * a.N + n;
-            a.y[o] = __float2bfloat16_rn(s);
-            if (a.y32 != nullptr) a.y32[o] = s;
+            a.y[o] = __float2bfloat16_rn(sacc);
+            if (a.y32 != nullptr) a.y32[o] = sacc;
           }
         }
       }

@@ -158,11 +158,16 @@ struct MoeCfg {
   static constexpr int kBBytes = BN * 128;        // BN rows x 64 bf16
   static constexpr int kIdxBytes = 128 * 32;      // 128 rows x 64 4-bit indices
   static constexpr int kStageBytes = kABytes + kBBytes + kIdxBytes;
-  static constexpr int kStages = (180 * 1024) / kStageBytes > 6 ? 6 : (180 * 1024) / kStageBytes;
+  static constexpr int kStages = 4;
   static constexpr int kCentBytes = 128 * 16 * 2;
-  static constexpr int kTmemCols = BN < 32 ? 32 : BN;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kCentBytes + BN * 8 + 1024 + 256;
-  static_assert(BN * 64 * 4 <= kStages * kStageBytes, "SwiGLU staging must fit the ring");
+  static constexpr int kHalf = BN / 2;            // tokens per epilogue pass
+  static constexpr int kStgLd = 129;              // padded row of the transposed staging tile
+  static constexpr int kStgBytes = kHalf * kStgLd * 4;
+  static constexpr int kTmemCols = 2 * BN;        // two accumulators (ping-pong across items)
+  static constexpr int kDecWarps = 8;
+  static constexpr int kThreads = (2 + kDecWarps + 4) * 32;
+  static constexpr int kSmemBytes =
+      kStages * kStageBytes + 2 * kCentBytes + kStgBytes + 2 * BN * 4 + 1024 + 512;
 };
 
 __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
@@ -175,12 +180,16 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-
-// One CTA per work item (expert e, 128-row weight tile nt, BN-token tile mt), items enumerated
-// expert by expert, nt fastest.  GATEUP: weight rows of a tile are 64 gate rows then the 64
-// matching up rows (repacked at create time), so the SwiGLU pairs meet inside one tile.
+// Persistent grouped GEMM.  Work items (expert e, 128-row weight tile nt, BN-token tile mt) are
+// enumerated expert by expert, nt fastest; CTA c takes items c, c + gridDim.x, ...  Warp roles:
+// 0 producer (TMA: index tile, B rows -- gathered token rows for gate/up, contiguous h rows for
+// down -- and the item's 128 centroid rows), 1 TMEM allocator + MMA issuer (kind::f16, N = the
+// item's token count rounded up to 16), 2..9 decode (4-bit indices -> bf16 operand tile),
+// 10..13 epilogue.  Two TMEM accumulators alternate between items, so the epilogue of one item
+// overlaps the main loop of the next.  GATEUP: the weight rows of a tile are 64 gate rows then
+// the 64 matching up rows (repacked at create time), so the SwiGLU pairs meet inside one tile.
 template <int BN, bool GATEUP>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_idx,
                     const __grid_constant__ CUtensorMap tm_b, const MoeGemmArgs a) {
   using Cfg = MoeCfg<BN>;
@@ -191,192 +200,294 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sA = smem;
   uint8_t* sB = sA + S * Cfg::kABytes;
   uint8_t* sIdx = sB + S * Cfg::kBBytes;
-  __nv_bfloat16* sCent = reinterpret_cast<__nv_bfloat16*>(sIdx + S * Cfg::kIdxBytes);
-  int* sRow = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(sCent) + Cfg::kCentBytes);  // [BN]
-  float* sGate = reinterpret_cast<float*>(sRow + BN);                                         // [BN]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sGate + BN);
+  __nv_bfloat16* sCent = reinterpret_cast<__nv_bfloat16*>(sIdx + S * Cfg::kIdxBytes);    // [2][128][16]
+  float* sStg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sCent) + 2 * Cfg::kCentBytes);
+  int* sRow = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(sStg) + Cfg::kStgBytes);  // [2][BN]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sRow + 2 * BN);
   uint64_t* empty = full + S;
   uint64_t* decd = empty + S;
-  uint64_t* cfull = decd + S;
-  uint64_t* accf = cfull + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
-  int* s_item = reinterpret_cast<int*>(tmem_slot + 1);   // e, nt, mt, count in tile, p0
+  uint64_t* cfull = decd + S;     // [2] centroids + row list of an item landed
+  uint64_t* cempty = cfull + 2;   // [2] decoders done with them
+  uint64_t* accf = cempty + 2;    // [2] accumulator complete
+  uint64_t* acce = accf + 2;      // [2] accumulator drained by the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  __shared__ int s_pre[257];      // first item of each expert; s_pre[E] = number of items
+  __shared__ int s_cnt[256], s_off[256];   // routed token count and first entry of each expert
+  __shared__ int s_f[BN];         // down epilogue: routed entry of each token of the item
+  __shared__ float s_g[BN];       //                and its gate weight
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    int item = blockIdx.x, base = 0, e = 0;
-    for (; e < a.E; ++e) {
-      const int it = a.n_tiles * ((a.counts[e] + BN - 1) / BN);
-      if (item < base + it) break;
-      base += it;
-    }
-    s_item[0] = e;
-    if (e < a.E) {
-      const int local = item - base;
-      s_item[1] = local % a.n_tiles;
-      s_item[2] = local / a.n_tiles;
-      s_item[3] = min(BN, a.counts[e] - s_item[2] * BN);
-      s_item[4] = a.offsets[e] + s_item[2] * BN;
-    }
-  }
-  __syncthreads();
-  const int e = s_item[0];
-  if (e >= a.E) return;                                  // past the last item: whole CTA leaves
-  const int nt = s_item[1], cnt = s_item[3], p0 = s_item[4];
-  const int row0 = e * a.rows_per_expert + nt * 128;
-  for (int j = threadIdx.x; j < BN; j += blockDim.x) {
-    const int f = j < cnt ? a.entries[p0 + j] : a.entries[p0];
-    sRow[j] = GATEUP ? f / a.k : f;
-    sGate[j] = GATEUP ? 0.f : a.gates[f];
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    const int c = a.counts[e];
+    s_cnt[e] = c;
+    s_off[e] = a.offsets[e];
+    s_pre[e + 1] = a.n_tiles * ((c + BN - 1) / BN);
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&decd[s], 128);
+      mbar_init(&decd[s], Cfg::kDecWarps * 32);
     }
-    mbar_init(cfull, 1);
-    mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&cfull[b], 1);
+      mbar_init(&cempty[b], Cfg::kDecWarps * 32);
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 128);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_pre[0] = 0;
+    for (int e = 0; e < a.E; ++e) s_pre[e + 1] += s_pre[e];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int n_items = s_pre[a.E];
   const int nstages = a.kdim / 64;
+
+  struct Item { int e, nt, cnt, p0; };
+  auto item_of = [&](int id) {
+    int lo = 0, hi = a.E - 1;                 // last expert with s_pre[e] <= id
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] <= id) lo = mid; else hi = mid - 1;
+    }
+    Item it;
+    it.e = lo;
+    const int local = id - s_pre[lo];
+    it.nt = local % a.n_tiles;
+    const int mt = local / a.n_tiles;
+    it.cnt = min(BN, s_cnt[lo] - mt * BN);
+    it.p0 = s_off[lo] + mt * BN;
+    return it;
+  };
 
   bool ok = true;
   if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(cfull, Cfg::kCentBytes);
-      bulk_load(sCent, a.cent + static_cast<size_t>(row0) * 16, Cfg::kCentBytes, cfull);
-      for (int i = 0, it = 0; i < nstages && ok; ++i, ++it) {
+    // ---------------- producer
+    int it = 0;   // global stage counter
+    for (int id = blockIdx.x, j = 0; id < n_items && ok; id += gridDim.x, ++j) {
+      const Item I = item_of(id);
+      const int b = j & 1;
+      const int row0 = I.e * a.rows_per_expert + I.nt * 128;
+      const int nrow = min(BN, (I.cnt + 15) & ~15);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&cempty[b], ((j >> 1) & 1) ^ 1, 11));
+      if (!ok) break;
+      int* rows = sRow + b * BN;
+      int fv[BN / 32];
+#pragma unroll
+      for (int u = 0; u < BN / 32; ++u) {   // all loads in flight, then the stores
+        const int c = lane + 32 * u;
+        fv[u] = a.entries[I.p0 + (c < I.cnt ? c : 0)];
+      }
+#pragma unroll
+      for (int u = 0; u < BN / 32; ++u) rows[lane + 32 * u] = GATEUP ? fv[u] / a.k : fv[u];
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&cfull[b], Cfg::kCentBytes);
+        bulk_load(sCent + b * 128 * 16, a.cent + static_cast<size_t>(row0) * 16, Cfg::kCentBytes, &cfull[b]);
+      }
+      for (int i = 0; i < nstages && ok; ++i, ++it) {
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait(&empty[st], ph ^ 1, 11)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[st], Cfg::kIdxBytes + Cfg::kBBytes);
-        tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_idx, &full[st], i * 32, row0);
-        if constexpr (GATEUP) {
-#pragma unroll 4
-          for (int g = 0; g < BN / 4; ++g)
-            tma_gather4(sB + st * Cfg::kBBytes + g * 512, &tm_b, &full[st], i * 64, sRow[4 * g],
-                        sRow[4 * g + 1], sRow[4 * g + 2], sRow[4 * g + 3]);
-        } else {
-          tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, p0);
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 12));
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[st], Cfg::kIdxBytes + (GATEUP ? nrow * 128 : Cfg::kBBytes));
+          tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_idx, &full[st], i * 32, row0);
+          if constexpr (GATEUP) {
+            for (int g = 0; g < nrow / 4; ++g)
+              tma_gather4(sB + st * Cfg::kBBytes + g * 512, &tm_b, &full[st], i * 64, rows[4 * g],
+                          rows[4 * g + 1], rows[4 * g + 2], rows[4 * g + 3]);
+          } else {
+            tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, I.p0);
+          }
         }
+        __syncwarp();
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(BN);
-      for (int i = 0, it = 0; i < nstages && ok; ++i, ++it) {
+    // ---------------- MMA issuer
+    int it = 0;
+    for (int id = blockIdx.x, j = 0; id < n_items && ok; id += gridDim.x, ++j) {
+      const Item I = item_of(id);
+      const int b = j & 1;
+      const int nrow = min(BN, (I.cnt + 15) & ~15);
+      const uint32_t idesc = idesc_bf16(nrow);
+      const uint32_t acc = tmem + b * BN;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acce[b], ((j >> 1) & 1) ^ 1, 17));
+      if (!ok) break;
+      tc_fence_after();
+      for (int i = 0; i < nstages && ok; ++i, ++it) {
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait(&full[st], ph, 12) || !mbar_wait(&decd[st], ph, 13)) { ok = false; break; }
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[st], ph, 13) && mbar_wait(&decd[st], ph, 14));
+        if (!ok) break;
         tc_fence_after();
         const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
         const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
+        if (lane == 0) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16(tmem, make_sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128),
-                  make_sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128), idesc,
-                  (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&empty[st]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(acc, make_sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128),
+                    make_sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128), idesc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&empty[st]);
+          if (i == nstages - 1) tc_commit(&accf[b]);
+        }
+        __syncwarp();
       }
-      tc_commit(accf);
     }
-  } else {
+  } else if (warp < 2 + Cfg::kDecWarps) {
     // ---------------- decode: 4-bit indices -> bf16 operand tile through the row centroids
     const int t = threadIdx.x - 64;
-    if (!mbar_wait(cfull, 0, 14)) ok = false;
-    for (int i = 0, it = 0; i < nstages && ok; ++i, ++it) {
-      const int st = it % S;
-      const uint32_t ph = (it / S) & 1;
-      if (!mbar_wait(&full[st], ph, 15)) { ok = false; break; }
-      const uint8_t* idx_s = sIdx + st * Cfg::kIdxBytes;
-      uint8_t* a_s = sA + st * Cfg::kABytes;
-#pragma unroll 2
-      for (int j = 0; j < 8; ++j) {
-        const int c = t + 128 * j;
-        const int r = c >> 3, kc = c & 7;
-        const uint32_t iv = *reinterpret_cast<const uint32_t*>(idx_s + r * 32 + kc * 4);
-        const uint16_t* L = reinterpret_cast<const uint16_t*>(sCent) + r * 16;
-        uint4 o;
-        o.x = L[iv & 15u] | (static_cast<uint32_t>(L[(iv >> 4) & 15u]) << 16);
-        o.y = L[(iv >> 8) & 15u] | (static_cast<uint32_t>(L[(iv >> 12) & 15u]) << 16);
-        o.z = L[(iv >> 16) & 15u] | (static_cast<uint32_t>(L[(iv >> 20) & 15u]) << 16);
-        o.w = L[(iv >> 24) & 15u] | (static_cast<uint32_t>(L[iv >> 28]) << 16);
-        *reinterpret_cast<uint4*>(a_s + r * 128 + ((kc ^ (r & 7)) << 4)) = o;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&decd[st]);
-    }
-    // ---------------- epilogue
-    const int q = warp & 3;
-    if (ok) ok = mbar_wait(accf, 0, 16);
-    tc_fence_after();
-    if constexpr (GATEUP) {
-      float* ubuf = reinterpret_cast<float*>(smem);            // [BN][64] up values
-      if (q >= 2 && ok) {
-        for (int c = 0; c < BN; c += 8) {
-          uint32_t r[8];
-          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
-          tmem_ld_wait();
+    constexpr int kDT = Cfg::kDecWarps * 32;
+    int it = 0;
+    for (int id = blockIdx.x, j = 0; id < n_items && ok; id += gridDim.x, ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(&cfull[b], (j >> 1) & 1, 15)) { ok = false; break; }
+      const uint16_t* cent = reinterpret_cast<const uint16_t*>(sCent + b * 128 * 16);
+      for (int i = 0; i < nstages && ok; ++i, ++it) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait(&full[st], ph, 16)) { ok = false; break; }
+        const uint8_t* idx_s = sIdx + st * Cfg::kIdxBytes;
+        uint8_t* a_s = sA + st * Cfg::kABytes;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) ubuf[(c + j) * 64 + (q - 2) * 32 + lane] = __uint_as_float(r[j]);
+        for (int jj = 0; jj < 1024 / kDT; ++jj) {
+          const int c = t + kDT * jj;
+          const int r = c >> 3, kc = c & 7;
+          const uint32_t iv = *reinterpret_cast<const uint32_t*>(idx_s + r * 32 + kc * 4);
+          const uint16_t* L = cent + r * 16;
+          uint4 o;
+          o.x = L[iv & 15u] | (static_cast<uint32_t>(L[(iv >> 4) & 15u]) << 16);
+          o.y = L[(iv >> 8) & 15u] | (static_cast<uint32_t>(L[(iv >> 12) & 15u]) << 16);
+          o.z = L[(iv >> 16) & 15u] | (static_cast<uint32_t>(L[(iv >> 20) & 15u]) << 16);
+          o.w = L[(iv >> 24) & 15u] | (static_cast<uint32_t>(L[iv >> 28]) << 16);
+          *reinterpret_cast<uint4*>(a_s + r * 128 + ((kc ^ (r & 7)) << 4)) = o;
         }
+        fence_proxy_async_smem();
+        mbar_arrive(&decd[st]);
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (q < 2 && ok) {
-        const int jf = nt * 64 + q * 32 + lane;                 // intermediate feature
-        for (int c = 0; c < BN; c += 8) {
-          uint32_t r[8];
-          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
-          tmem_ld_wait();
+      if (ok) mbar_arrive(&cempty[b]);
+    }
+  } else {
+    // ---------------- epilogue (4 warps; TMEM lane quadrant = warp % 4)
+    const int q = warp & 3;
+    const int et = threadIdx.x - (2 + Cfg::kDecWarps) * 32;   // 0..127
+    const int row = q * 32 + lane;                             // accumulator row of this thread
+    for (int id = blockIdx.x, j = 0; id < n_items && ok; id += gridDim.x, ++j) {
+      const Item I = item_of(id);
+      const int b = j & 1;
+      ok = bar_and(2, 128, mbar_wait(&accf[b], (j >> 1) & 1, 18));   // all 128 agree
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + b * BN + (static_cast<uint32_t>(q * 32) << 16);
+      if constexpr (GATEUP) {
+        // Transpose half a tile at a time through shared memory ([token][row], padded), then
+        // thread et handles token et % kHalf and MX block et / kHalf (32 intermediate features):
+        // h = silu(g) * u, MXFP4 requantization, the exact bf16 of the quantized h.
+        constexpr int H2 = Cfg::kHalf;
+        for (int h0 = 0; h0 < BN; h0 += H2) {
+          if (h0 < I.cnt) {
+#pragma unroll 1
+            for (int c = 0; c < H2; c += 8) {
+              uint32_t r[8];
+              tmem_ld8(acc + h0 + c, r);
+              tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (c + j >= cnt) break;
-            const float g = __uint_as_float(r[j]);
-            const float u = ubuf[(c + j) * 64 + q * 32 + lane];
-            const float h = g / (1.0f + expf(-g)) * u;
-            const size_t p = static_cast<size_t>(p0 + c + j);
-            if (a.h32 != nullptr) a.h32[p * a.I + jf] = h;
-            // MXFP4 requantization of h over this warp's 32 features
-            uint32_t am = __float_as_uint(h) & 0x7FFFFFFFu;
+              for (int jj = 0; jj < 8; ++jj) sStg[(c + jj) * Cfg::kStgLd + row] = __uint_as_float(r[jj]);
+            }
+          }
+          if (h0 + H2 >= BN) {   // last read of this accumulator
+            tc_fence_before();
+            mbar_arrive(&acce[b]);
+          }
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+          const int c = et % H2, blk = et / H2;
+          if (h0 + c < I.cnt && blk < 2) {
+            const float* gr = sStg + c * Cfg::kStgLd + 32 * blk;
+            const float* ur = gr + 64;
+            float hv[32];
+            uint32_t am = 0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+            for (int i = 0; i < 32; ++i) {
+              const float g = gr[i];
+              hv[i] = g / (1.0f + expf(-g)) * ur[i];
+              am = max(am, __float_as_uint(hv[i]) & 0x7FFFFFFFu);
+            }
             const int E8 = static_cast<int>(am >> 23);
             const int ex = (E8 == 0) ? -127 : max(E8 - 129, -127);
             const float inv = __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
-            const float hn = __shfl_xor_sync(0xFFFFFFFFu, h, 1);
-            uint32_t byte = e2m1x2(h * inv, hn * inv);                  // even lane: (h, next)
-            byte |= ((__float_as_uint(h) >> 28) & 8u) | ((__float_as_uint(hn) >> 24) & 0x80u);
-            const uint32_t nb = __shfl_xor_sync(0xFFFFFFFFu, byte, 1);
-            const uint32_t mycode = (lane & 1) ? ((nb >> 4) & 15u) : (byte & 15u);
-            if ((lane & 1) == 0) a.h_codes[p * (a.I / 2) + (jf >> 1)] = static_cast<uint8_t>(byte);
-            if (lane == 0) a.h_scales[p * (a.I / 32) + (jf >> 5)] = static_cast<uint8_t>(ex + 127);
-            // exact value of the quantized element (power-of-two scaling; 2^-127 is subnormal)
-            a.h_dq[p * a.I + jf] = __float2bfloat16_rn(ldexpf(e2m1_code_value(mycode), ex));
+            uint32_t code[4];
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4) {
+              float f[8];
+              uint32_t sgn = 0;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                f[i] = hv[8 * w4 + i] * inv;
+                sgn |= ((__float_as_uint(hv[8 * w4 + i]) >> 31) << (4 * i + 3));
+              }
+              code[w4] = e2m1x8(f) | sgn;
+            }
+            const size_t p = static_cast<size_t>(I.p0 + h0 + c);
+            const int jf0 = I.nt * 64 + 32 * blk;                  // first intermediate feature
+            *reinterpret_cast<uint4*>(a.h_codes + p * (a.I / 2) + jf0 / 2) =
+                make_uint4(code[0], code[1], code[2], code[3]);
+            a.h_scales[p * (a.I / 32) + jf0 / 32] = static_cast<uint8_t>(ex + 127);
+            uint32_t dq[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint32_t c0 = (code[i >> 2] >> (8 * (i & 3))) & 15u;
+              const uint32_t c1 = (code[i >> 2] >> (8 * (i & 3) + 4)) & 15u;
+              const __nv_bfloat162 v = __floats2bfloat162_rn(ldexpf(e2m1_code_value(c0), ex),
+                                                             ldexpf(e2m1_code_value(c1), ex));
+              dq[i] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(a.h_dq + p * a.I + jf0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(dq[4 * i], dq[4 * i + 1], dq[4 * i + 2], dq[4 * i + 3]);
+            if (a.h32 != nullptr) {
+              float4* d32 = reinterpret_cast<float4*>(a.h32 + p * a.I + jf0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) d32[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+            }
           }
+          asm volatile("bar.sync 2, 128;" ::: "memory");
         }
-      }
-    } else {
-      if (ok) {
-        const int n = nt * 128 + q * 32 + lane;                 // output feature of the expert
-        for (int c = 0; c < BN; c += 8) {
+      } else {
+        // down: y_e[token, n] * gate, scattered to the token's slot row (coalesced along n).
+        // The item's routed entries and gates are fetched once, in parallel, into shared memory.
+        if (et < I.cnt) {
+          const int f = a.entries[I.p0 + et];
+          s_f[et] = f;
+          s_g[et] = a.gates[f];
+        }
+        named_bar_sync(2, 128);
+        const int n = I.nt * 128 + row;
+#pragma unroll 1
+        for (int c = 0; c < I.cnt; c += 8) {
           uint32_t r[8];
-          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+          tmem_ld8(acc + c, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (c + j >= cnt) break;
-            a.yslot[static_cast<size_t>(sRow[c + j]) * a.H + n] = __uint_as_float(r[j]) * sGate[c + j];
+          for (int jj = 0; jj < 8; ++jj) {
+            if (c + jj < I.cnt)
+              a.yslot[static_cast<size_t>(s_f[c + jj]) * a.H + n] = __uint_as_float(r[jj]) * s_g[c + jj];
           }
         }
+        tc_fence_before();
+        mbar_arrive(&acce[b]);
+        named_bar_sync(2, 128);   // s_f / s_g are rewritten by the next item
       }
     }
   }

@@ -94,10 +94,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int si
   }
 }
 
+// Named barrier `id` over `n` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Named barrier `id` over `n` threads that also ANDs a predicate across them (so that a group of
+// warps leaves a loop together when one of its bounded waits expired).
+__device__ __forceinline__ bool bar_and(int id, int n, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred P, Q;\n\t"
+      "setp.ne.u32 P, %1, 0;\n\t"
+      "bar.red.and.pred Q, %2, %3, P;\n\t"
+      "selp.u32 %0, 1, 0, Q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(p)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA,
 // tcgen05.mma operand reads) before it signals a consumer.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Order this thread's earlier generic-proxy accesses of global memory (including what it acquired
+// from other CTAs) before its later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- clusters
@@ -145,6 +170,37 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// 16-byte global -> shared copy through the load/store path (cp.async), completing in the
+// thread's current async group; src_bytes < 16 zero-fills the rest (0: nothing is read).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most n (0..15) of this thread's committed cp.async groups are still pending.
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    case 7: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+    case 8: asm volatile("cp.async.wait_group 8;" ::: "memory"); break;
+    case 9: asm volatile("cp.async.wait_group 9;" ::: "memory"); break;
+    case 10: asm volatile("cp.async.wait_group 10;" ::: "memory"); break;
+    case 11: asm volatile("cp.async.wait_group 11;" ::: "memory"); break;
+    case 12: asm volatile("cp.async.wait_group 12;" ::: "memory"); break;
+    case 13: asm volatile("cp.async.wait_group 13;" ::: "memory"); break;
+    case 14: asm volatile("cp.async.wait_group 14;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 15;" ::: "memory"); break;
+  }
+}
+
 // Shared -> global tensor store of a 2-D box; completion tracked by the bulk async-group.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
   asm volatile(

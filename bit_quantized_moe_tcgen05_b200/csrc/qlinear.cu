@@ -137,7 +137,7 @@ ql_status launch_fp4_bn(const CUtensorMap& tx, const CUtensorMap& ty, const CUte
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -177,11 +177,8 @@ struct ql_linear {
   int32_t k_tail;
   bool e8m0 = true;            // E8M0-B32 scales (else E4M3-B16 + tensor scales)
   bool vq = false;             // MXCode PreScale VQ weight
-  uint8_t* d_codes = nullptr;  // weight operand blocks [N/128][stages][16 KB codes | 8 KB indices]
-  uint8_t* d_lut = nullptr;    // VQ codebooks [N/64][K/64][256][2]
-  uint8_t* d_sf = nullptr;     // tiled scale atoms
-  int sf_atoms = 0;            // atoms per 128-row group of the weight
-  int lut_qc = 0;
+  uint8_t* d_codes = nullptr;  // weight blocks [N/128][stages][codes or indices + codebooks, scales]
+  size_t weight_bytes = 0;
   float w_ts = 1.f;
   int n_base_stages = 0, n_stages_total = 0;
   // INT4 dense + block-sparse residual
@@ -203,7 +200,7 @@ struct FwdPlan {
 
 FwdPlan plan_forward_int4(const ql_linear* L, int64_t M) {
   FwdPlan p{};
-  p.BN = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.BN = M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
   p.tiles_n = static_cast<int>(L->N / 128);
   p.tiles_m = static_cast<int>(cdiv(std::max<int64_t>(M, 1), p.BN));
   const int tiles = p.tiles_n * p.tiles_m;
@@ -253,34 +250,36 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   p.n_tickets = p.splits > 1 ? tiles : 0;
   off = align_up(p.tick_off + static_cast<size_t>(p.n_tickets) * sizeof(int), 256);
   p.part_off = off;
-  if (p.splits > 1) off = align_up(off + static_cast<size_t>(tiles) * p.splits * p.BN * 128 * 4, 256);
+  if (p.splits > 1)
+    off = align_up(off + static_cast<size_t>(tiles) * p.splits * p.BN * 128 * 4, 256);
   p.total = off;
   return p;
 }
 
-void repack_sf_tiled(const uint8_t* plain, int64_t rows, int64_t cols, int atoms_per_row,
-                     std::vector<uint8_t>& out) {
-  const int64_t groups = cdiv(rows, 128);
-  out.assign(static_cast<size_t>(groups) * atoms_per_row * 512, 0);
-  for (int64_t r = 0; r < rows; ++r)
-    for (int64_t j = 0; j < cols; ++j)
-      out[ql::sf_tiled_offset(static_cast<int>(r), static_cast<int>(j), atoms_per_row)] =
-          plain[r * cols + j];
-}
-
-// Weight operand blocks for the FP4 GEMM: for every 128-row tile and every K stage of 256
-// elements (the base stages over [0, C), then the tail stages over [C, C + k_tail)), one block
-// laid out as the stage buffer: FP4 codes as 128 rows x 128 B with 16-byte chunk c of row r at
-// chunk c ^ (r % 8) (the 128-byte swizzle), or VQ indices as 128 rows x 64 B.  Rows past N and
-// elements past a partial stage are zero.
-void repack_weight_blocks(const uint8_t* src, int64_t N, int64_t K, int64_t C, int64_t k_tail,
-                          bool vq, std::vector<uint8_t>& out) {
+// Weight blocks for the FP4 GEMM: for every 128-row tile and every K stage of 256 elements (the
+// base stages over [0, C), then the tail stages over [C, C + k_tail)), one block laid out exactly
+// as the kernel's stage buffer, so that one bulk copy moves it:
+//   FP4: codes as 128 rows x 128 B, 16-byte chunk c of row r stored at chunk c ^ (r % 8) (the
+//        128-byte swizzle the MMA reads);
+//   VQ:  indices as 128 rows x 64 B, then the 2 x 4 QBlock codebooks the stage touches (512 B
+//        each, row QBlock major);
+// then the stage's weight scales as 512-byte atoms of 128 rows x 4 scale columns (row r at
+// (r%32)*16 + ((r/32)%4)*4, column j at j%4; the layout tcgen05.cp moves into TMEM).  Rows past N
+// and elements past a partial stage are zero.  Returns the block size.
+size_t repack_weight_blocks(const uint8_t* src, const uint8_t* scales, const uint8_t* lut,
+                            int64_t N, int64_t K, int64_t C, int64_t k_tail, bool vq, bool e8m0,
+                            std::vector<uint8_t>& out) {
   const int64_t nb = cdiv(C, 256), nt = cdiv(k_tail, 256), stages = nb + nt;
   const int64_t tiles = cdiv(N, 128);
   const int row_bytes = vq ? 64 : 128;       // one stage of one row
   const int64_t src_row = vq ? K / 4 : K / 2;
   const int per_byte = vq ? 4 : 2;           // elements per source byte
-  out.assign(static_cast<size_t>(tiles) * stages * 128 * row_bytes, 0);
+  const int sfb = e8m0 ? 32 : 16;            // elements per scale
+  const int atoms = 256 / (4 * sfb);         // scale atoms per stage
+  const size_t code_bytes = static_cast<size_t>(128) * row_bytes;
+  const size_t lut_bytes = vq ? 8 * 512 : 0;
+  const size_t blk_bytes = code_bytes + lut_bytes + static_cast<size_t>(atoms) * 512;
+  out.assign(static_cast<size_t>(tiles) * stages * blk_bytes, 0);
   for (int64_t t = 0; t < tiles; ++t)
     for (int64_t i = 0; i < stages; ++i) {
       int64_t kw, valid;
@@ -292,7 +291,8 @@ void repack_weight_blocks(const uint8_t* src, int64_t N, int64_t K, int64_t C, i
         kw = C + j;
         valid = std::min<int64_t>(256, k_tail - j);
       }
-      uint8_t* blk = out.data() + (static_cast<size_t>(t) * stages + i) * 128 * row_bytes;
+      uint8_t* blk = out.data() + (static_cast<size_t>(t) * stages + i) * blk_bytes;
+      uint8_t* sfa = blk + code_bytes + lut_bytes;
       for (int r = 0; r < 128; ++r) {
         const int64_t n = t * 128 + r;
         if (n >= N) break;
@@ -302,8 +302,20 @@ void repack_weight_blocks(const uint8_t* src, int64_t N, int64_t K, int64_t C, i
           const int dst = vq ? b : ((((b >> 4) ^ (r & 7)) << 4) | (b & 15));
           blk[r * row_bytes + dst] = srow[b];
         }
+        for (int jl = 0; jl < valid / sfb; ++jl)
+          sfa[(jl >> 2) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (jl & 3)] =
+              scales[n * (K / sfb) + kw / sfb + jl];
       }
+      if (vq)
+        for (int g2 = 0; g2 < 2; ++g2)
+          for (int q = 0; q < 4; ++q) {
+            const int64_t qr = t * 2 + g2, qc = kw / 64 + q;
+            if (qr * 64 < N && qc * 64 < K)
+              std::memcpy(blk + code_bytes + g2 * 2048 + q * 512,
+                          lut + (static_cast<size_t>(qr) * (K / 64) + qc) * 512, 512);
+          }
     }
+  return blk_bytes;
 }
 
 float half_bits_to_float(uint16_t h) {
@@ -332,7 +344,7 @@ ql_status launch_int4_bn(const CUtensorMap& tx, const CUtensorMap& ty, const CUt
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(320, 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -373,8 +385,8 @@ ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, u
   return QL_OK;
 }
 
-// Cluster size for the one-launch small-tensor quantizer: 16 CTAs where the device can
-// co-schedule such a cluster, else the portable 8.
+// Cluster size for the one-launch quantizer: 16 CTAs where the device can co-schedule such a
+// cluster, else the portable 8.
 int e4m3_cluster_size() {
   static int size[64] = {};
   int dev = 0;
@@ -405,8 +417,10 @@ int e4m3_cluster_size() {
   return size[dev];
 }
 
-// Tensors up to this many elements are quantized by one cluster in one launch.
+// Tensors up to this many elements are quantized in one launch: one CTA up to 2^14 elements (a
+// single decode token), else one cluster.
 constexpr int64_t kE4m3ClusterMaxElems = int64_t(1) << 21;
+constexpr int64_t kE4m3OneCtaMaxElems = int64_t(1) << 14;
 
 // E4M3-B16 activation quantizer.  amax_slot: device word for the reduced amax bit pattern (the
 // two-launch path max-reduces into it; it is followed by the tensor-scale word and then
@@ -417,7 +431,7 @@ ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes,
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   int* tickets = n_tickets > 0 ? reinterpret_cast<int*>(amax_slot + 2) : nullptr;
   if (M * K <= kE4m3ClusterMaxElems) {
-    const int cs = e4m3_cluster_size();
+    const int cs = M * K <= kE4m3OneCtaMaxElems ? 1 : e4m3_cluster_size();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cs, 1, 1);
     cfg.blockDim = dim3(1024, 1, 1);
@@ -580,39 +594,33 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
   L->e8m0 = mx;
   L->vq = vq;
   L->w_ts = mx ? 1.f : d->w_tensor_scale;
-  const int atomK = mx ? 128 : 64;
-  const int sf_block = mx ? 32 : 16;
-  L->sf_atoms = static_cast<int>(cdiv(d->K, atomK));
   L->n_base_stages = static_cast<int>(cdiv(L->C, 256));
   L->n_stages_total = L->n_base_stages + static_cast<int>(cdiv(L->k_tail, 256));
-  std::vector<uint8_t> sf;
-  repack_sf_tiled(static_cast<const uint8_t*>(d->scales), d->N, d->K / sf_block, L->sf_atoms, sf);
   std::vector<uint8_t> blocks;
-  repack_weight_blocks(vq ? static_cast<const uint8_t*>(d->indices)
+  const size_t blk = repack_weight_blocks(vq ? static_cast<const uint8_t*>(d->indices)
                           : static_cast<const uint8_t*>(d->codes),
-                       d->N, d->K, L->C, L->k_tail, vq, blocks);
+                       static_cast<const uint8_t*>(d->scales),
+                       vq ? static_cast<const uint8_t*>(d->codebooks) : nullptr, d->N, d->K, L->C,
+                       L->k_tail, vq, mx, blocks);
+  const size_t want = vq ? ql::Fp4Cfg<16, false, true>::kWBytes
+                         : (mx ? ql::Fp4Cfg<16, true, false>::kWBytes : ql::Fp4Cfg<16, false, false>::kWBytes);
+  if (blk != want) {
+    delete L;
+    return fail(QL_ERR_UNSUPPORTED, "internal: weight block of %zu bytes, kernel expects %zu", blk, want);
+  }
   const size_t code_bytes = blocks.size();
-  const size_t lut_bytes = vq ? static_cast<size_t>(d->N / 64) * (d->K / 64) * 512 : 0;
-  L->lut_qc = vq ? static_cast<int>(d->K / 64) : 0;
   auto cleanup = [&](ql_status st) {
     if (L->d_codes) cudaFree(L->d_codes);
-    if (L->d_lut) cudaFree(L->d_lut);
-    if (L->d_sf) cudaFree(L->d_sf);
     delete L;
     return st;
   };
-  if (cudaMalloc(&L->d_codes, code_bytes) != cudaSuccess ||
-      cudaMalloc(&L->d_sf, sf.size()) != cudaSuccess ||
-      (vq && cudaMalloc(&L->d_lut, lut_bytes) != cudaSuccess))
-    return cleanup(fail(QL_ERR_OOM, "cudaMalloc of %zu weight bytes failed",
-                        code_bytes + sf.size() + lut_bytes));
+  if (cudaMalloc(&L->d_codes, code_bytes) != cudaSuccess)
+    return cleanup(fail(QL_ERR_OOM, "cudaMalloc of %zu weight bytes failed", code_bytes));
   if (cudaMemcpyAsync(L->d_codes, blocks.data(), code_bytes, cudaMemcpyHostToDevice, s) !=
           cudaSuccess ||
-      cudaMemcpyAsync(L->d_sf, sf.data(), sf.size(), cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      (vq && cudaMemcpyAsync(L->d_lut, d->codebooks, lut_bytes, cudaMemcpyHostToDevice, s) !=
-                 cudaSuccess) ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return cleanup(fail(QL_ERR_CUDA, "weight upload failed"));
+  L->weight_bytes = code_bytes;
   *out = L;
   return QL_OK;
 }
@@ -620,10 +628,8 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
 ql_status qlinear_destroy(ql_linear* L) {
   if (L == nullptr) return QL_OK;
   if (L->d_codes) cudaFree(L->d_codes);
-  if (L->d_lut) cudaFree(L->d_lut);
   if (L->d_stage_start) cudaFree(L->d_stage_start);
   if (L->d_stage_group) cudaFree(L->d_stage_group);
-  if (L->d_sf) cudaFree(L->d_sf);
   delete L;
   return QL_OK;
 }
@@ -701,7 +707,8 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
     switch (p.BN) {
       case 16: return launch_int4_bn<16>(tx, ty, ty32, a, grid, cs);
       case 32: return launch_int4_bn<32>(tx, ty, ty32, a, grid, cs);
-      default: return launch_int4_bn<64>(tx, ty, ty32, a, grid, cs);
+      case 64: return launch_int4_bn<64>(tx, ty, ty32, a, grid, cs);
+      default: return launch_int4_bn<128>(tx, ty, ty32, a, grid, cs);
     }
   }
   CUtensorMap tm_x;
@@ -715,8 +722,6 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   a.n_base_stages = L->n_base_stages;
   a.n_stages_total = L->n_stages_total;
   a.stages_per_split = p.spp;
-  a.sfa = L->d_sf;
-  a.sfa_atoms = L->sf_atoms;
   a.sfb = w8 + p.sf_off;
   a.sfb_atoms = p.sfb_atoms;
   a.alpha_dev = L->e8m0 ? nullptr : reinterpret_cast<const float*>(w8 + p.scal_off) + 1;
@@ -724,11 +729,10 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   a.y = static_cast<__nv_bfloat16*>(y);
   a.y32 = y32;
   a.ldy = static_cast<int>(L->N);
-  a.lut = L->d_lut;
-  a.lut_qc = L->lut_qc;
   a.wt = L->d_codes;
   a.partials = reinterpret_cast<float*>(w8 + p.part_off);
   a.tickets = reinterpret_cast<int*>(w8 + p.tick_off);
+  a.xq = w8 + p.codes_off;
   dim3 grid(p.tiles_n, p.tiles_m, p.splits);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (y32 && (reinterpret_cast<uintptr_t>(y32) & 15)) ||
@@ -856,7 +860,7 @@ MoePlan plan_moe(const ql_moe* m, int64_t T) {
 
 template <int BN, bool GATEUP>
 ql_status launch_moe_gemm(const CUtensorMap& ti, const CUtensorMap& tb, const ql::MoeGemmArgs& a,
-                          int grid, cudaStream_t s) {
+                          int max_items, cudaStream_t s) {
   using Cfg = ql::MoeCfg<BN>;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -866,7 +870,9 @@ ql_status launch_moe_gemm(const CUtensorMap& ti, const CUtensorMap& tb, const ql
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
     attr_done[dev] = true;
   }
-  ql::moe_gemm_kernel<BN, GATEUP><<<grid, 192, Cfg::kSmemBytes, s>>>(ti, tb, a);
+  // persistent: one CTA per SM (the item count is only known on the device)
+  const int grid = std::max(1, std::min(max_items, sm_count()));
+  ql::moe_gemm_kernel<BN, GATEUP><<<grid, Cfg::kThreads, Cfg::kSmemBytes, s>>>(ti, tb, a);
   QL_CUDA(cudaGetLastError());
   return QL_OK;
 }

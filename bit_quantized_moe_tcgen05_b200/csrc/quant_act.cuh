@@ -214,18 +214,48 @@ __device__ __forceinline__ void quant_e4m3_block(
   const float r = __fdiv_rn(__fdiv_rn(amax_b, 6.0f), ts);
   const uint32_t sb = static_cast<uint32_t>(__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3));
   const float S = __fmul_rn(e4m3_value(sb), ts);
+  // Codes of the fp32 quotients q = RN(|x| / S), without a division per element: with
+  // inv = RN(1/S) and r = RN(|x| * inv), r is within 2^-22 (relative) of q, so
+  //   RN(r * (1 - 2^-21)) < q < RN(r * (1 + 2^-21))
+  // (the constants are exact in fp32).  E2M1 round-to-nearest-even is monotone in q, so when the
+  // codes of both bounds agree they are the code of q.  Otherwise -- a bound straddles a
+  // rounding threshold, which almost never happens -- q is computed by the correctly rounded
+  // division.  The bound needs S normal (so 1/S is finite); subnormal S takes the exact path.
+  // Codes are formed from magnitudes and the sign of x is or-ed in (a negative x that rounds
+  // to zero keeps code 0x8).
+  const bool fast = S >= 0x1p-126f;
+  const float inv = fast ? __frcp_rn(S) : 0.f;
   uint32_t packed[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    float f[8];
     const uint32_t ww[4] = {w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]};
+    float a[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float lo = __uint_as_float(ww[i] << 16), hi = __uint_as_float(ww[i] & 0xFFFF0000u);
-      f[2 * i] = S == 0.f ? 0.f : __fdiv_rn(lo, S);
-      f[2 * i + 1] = S == 0.f ? 0.f : __fdiv_rn(hi, S);
+      a[2 * i] = __uint_as_float((ww[i] << 16) & 0x7FFF0000u);
+      a[2 * i + 1] = __uint_as_float(ww[i] & 0x7FFF0000u);
     }
-    packed[h] = e2m1x8(f) | bf16x8_sign_nibbles(ww);
+    uint32_t code = 0;
+    bool done = false;
+    if (fast) {
+      float lo[8], hi[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float r = __fmul_rn(a[i], inv);
+        lo[i] = __fmul_rn(r, 0x1.fffffp-1f);   // 1 - 2^-21
+        hi[i] = __fmul_rn(r, 0x1.00001p+0f);   // 1 + 2^-21
+      }
+      const uint32_t cl = e2m1x8(lo), ch = e2m1x8(hi);
+      done = (cl == ch);
+      code = cl;
+    }
+    if (!done) {
+      float f[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] = S == 0.f ? 0.f : __fdiv_rn(a[i], S);
+      code = e2m1x8(f);
+    }
+    packed[h] = code | bf16x8_sign_nibbles(ww);
   }
   *reinterpret_cast<uint2*>(codes + static_cast<size_t>(m) * ldc + j * 8) =
       make_uint2(packed[0], packed[1]);

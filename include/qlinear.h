@@ -131,7 +131,12 @@ ql_status qlinear_forward(const ql_linear* layer, const void* x_bf16, int64_t M,
  * (MXFP4 codes and tiled scales); qlinear_gemm runs
  * the tcgen05 GEMM from that workspace.  Called in this order on one stream with the same M and
  * workspace they equal qlinear_forward.  A caller whose several layers share one input (gate and
- * up projections, say) can quantize once; the split also lets a profiler time the GEMM alone. */
+ * up projections, say) can quantize once; the split also lets a profiler time the GEMM alone.
+ * qlinear_gemm may be repeated on one quantized workspace: the split-K arrival counters it keeps
+ * there are cleared by qlinear_quantize_input and left cleared by every qlinear_gemm.  The GEMM
+ * is launched with programmatic stream serialization: it may start while the kernel before it on
+ * the stream is still running, streams (and decodes) weights meanwhile, and waits for that kernel
+ * to complete before it reads the workspace, writes y or reads the activation tensor scale. */
 ql_status qlinear_quantize_input(const ql_linear* layer, const void* x_bf16, int64_t M, void* ws,
                                  size_t ws_bytes, ql_stream_t stream);
 ql_status qlinear_gemm(const ql_linear* layer, int64_t M, void* y_bf16, float* y_f32, void* ws,

@@ -125,3 +125,64 @@ def test_vq_workload_full_size(M):
     ref, t = vq.forward(synth.bf16_bits_to_f64(xb), c["prep"], c["cb"])
     check_fp32(y32, ref, t, f"C2 M={M}")
     check_bf16(y, ref, t, f"C2 M={M}")
+
+
+def test_nvfp4_weight_linear_prefill():
+    """E4M3-B16 weights at a prefill shape (256-token tiles, split-K)."""
+    ql = _ql()
+    N, K, M = 2560, 2048, 300
+    codes = synth.uniform_nibble_bytes(60, N, K)
+    sb = synth.uniform_bytes(61, (N, K // 16), 0x28, 0x48)
+    ts_w = np.float32(0.0123)
+    lin = ql.QLinear(codes, sb, wfmt=ql.QL_W_NVFP4_E4M3_B16, w_tensor_scale=float(ts_w))
+    xb, _ = synth.activations_bf16(62, M, K, 0.01, 30.0)
+    y, y32 = _run(lin, xb)
+    lin.close()
+    xd = _x_deq(xb)
+    wd = mx.dequant_e4m3_b16(F.unpack_nibbles(codes), sb, ts_w)
+    ref, t = G.gemm_ref(xd, wd), G.abs_scale(xd, wd)
+    check_fp32(y32, ref, t, "nvfp4 prefill")
+    check_bf16(y, ref, t, "nvfp4 prefill")
+
+
+@pytest.mark.parametrize("M", [300, 16])
+def test_vq_linear_random_codebooks(M):
+    """VQ weights with random indices, codebooks and scales at N = 2560, K = 2048: M = 300 as a
+    prefill tile, M = 16 as split-K with the decode running ahead of the activation quantizer."""
+    g = np.random.default_rng(70 + M)
+    N, K = 2560, 2048
+    cb = g.integers(0, 16, (N // 64, K // 64, 256, 4), dtype=np.uint8)
+    prep = dict(ts=np.float32(0.0071), sb=g.integers(0x28, 0x48, (N, K // 16), dtype=np.uint8),
+                idx=g.integers(0, 256, (N, K // 4), dtype=np.uint8))
+    lin = _vq_layer(None, cb, prep)
+    xb, _ = synth.activations_bf16(71, M, K, 0.01, 30.0)
+    y, y32 = _run(lin, xb)
+    lin.close()
+    ref, t = vq.forward(synth.bf16_bits_to_f64(xb), prep, cb)
+    check_fp32(y32, ref, t, f"vq random M={M}")
+    check_bf16(y, ref, t, f"vq random M={M}")
+
+
+def test_quant_e4m3_b16_rounding_thresholds():
+    """Quotients x/S at and next to every E2M1 rounding threshold (ties included), which the
+    quantizer must resolve exactly as the fp32 division does; plus blocks whose scale product S
+    is an fp32 subnormal."""
+    thr = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    rows = []
+    for j in range(-3, 4):                        # S = 2^j: ts = 1 (amax 2688), s = 2^j
+        row = [2688.0] + [0.0] * 15               # block 0 fixes the tensor scale
+        for t in thr:
+            blk = [6.0 * 2.0 ** j]                # block amax -> E4M3 scale 2^j exactly
+            v = t * 2.0 ** j
+            up, dn = np.nextafter(np.float32(v), np.float32(np.inf)), np.nextafter(np.float32(v), np.float32(0))
+            blk += [v, -v, float(up), float(dn), v * (1 + 2 ** -8), v * (1 - 2 ** -8), -v * (1 + 2 ** -8)]
+            blk += [0.0] * (16 - len(blk))
+            row += blk
+        rows.append(row)
+    width = max(len(r) for r in rows)
+    x = np.array([r + [0.0] * (width - len(r)) for r in rows])
+    _check_quant(synth.to_bf16_bits(x))
+    g = np.random.default_rng(5)
+    tiny = g.standard_normal((2, 128)) * 1e-39    # subnormal block scales
+    tiny[:, 0] = 3e-36
+    _check_quant(synth.to_bf16_bits(tiny))
