@@ -142,6 +142,7 @@ struct MoeGemmArgs {
   const int* offsets;             // [E+1]
   const int* entries;             // [T*k] routed entries, expert-sorted
   const __nv_bfloat16* cent;      // [E*rows_per_expert][16] centroids (kernel row order)
+  const __nv_bfloat16* x_dq;      // [T, H] exact bf16 of the quantized x (gate/up B rows)
   const float* gates;             // [T*k] gate weights by entry (down)
   int I;                          // intermediate width
   uint8_t* h_codes;               // [T*k, I/2] MXFP4 codes of h, sorted order (gate/up)
@@ -151,6 +152,9 @@ struct MoeGemmArgs {
   float* yslot;                   // [T*k, H] gate * y per entry (down)
   int H;
 };
+
+// Stages of token-row gathers the gate/up producer keeps in flight before signalling one.
+constexpr int kGatherLag = 2;
 
 template <int BN>
 struct MoeCfg {
@@ -225,7 +229,7 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], GATEUP ? 33 : 1);   // gate/up: + one arrival per producer lane
       mbar_init(&empty[s], 1);
       mbar_init(&decd[s], Cfg::kDecWarps * 32);
     }
@@ -301,17 +305,35 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 12));
         if (!ok) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[st], Cfg::kIdxBytes + (GATEUP ? nrow * 128 : Cfg::kBBytes));
+          mbar_arrive_expect_tx(&full[st], Cfg::kIdxBytes + (GATEUP ? 0 : Cfg::kBBytes));
           tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_idx, &full[st], i * 32, row0);
-          if constexpr (GATEUP) {
-            for (int g = 0; g < nrow / 4; ++g)
-              tma_gather4(sB + st * Cfg::kBBytes + g * 512, &tm_b, &full[st], i * 64, rows[4 * g],
-                          rows[4 * g + 1], rows[4 * g + 2], rows[4 * g + 3]);
-          } else {
-            tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, I.p0);
+          if constexpr (!GATEUP) tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, I.p0);
+        }
+        if constexpr (GATEUP) {
+          // Gather the item's token rows (64 bf16 of each, in the 128-byte-swizzled K-major
+          // layout) with 16-byte cp.async from all lanes; a stage is signalled kGatherLag stages
+          // later, once its copies have landed, so that several stages are in flight.
+          const uint32_t bdst = smem_u32(sB + st * Cfg::kBBytes);
+          for (int c = lane; c < nrow * 8; c += 32) {
+            const int r = c >> 3, kc = c & 7;
+            cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4),
+                       a.x_dq + static_cast<size_t>(rows[r]) * a.kdim + i * 64 + kc * 8, 16u);
+          }
+          cp_async_commit();
+          if (it >= kGatherLag) {
+            cp_async_wait_pending(kGatherLag);
+            fence_proxy_async_smem();
+            mbar_arrive(&full[(it - kGatherLag) % S]);
           }
         }
         __syncwarp();
+      }
+    }
+    if constexpr (GATEUP) {   // signal the stages still in flight
+      for (int k = max(0, it - kGatherLag); k < it; ++k) {
+        cp_async_wait_pending(it - 1 - k);
+        fence_proxy_async_smem();
+        mbar_arrive(&full[k % S]);
       }
     }
   } else if (warp == 1) {

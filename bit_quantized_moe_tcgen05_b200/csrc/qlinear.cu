@@ -398,7 +398,7 @@ int e4m3_cluster_size() {
                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(16, 1, 1);
-      cfg.blockDim = dim3(1024, 1, 1);
+      cfg.blockDim = dim3(ql::kE4m3ClusterThreads, 1, 1);
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
       attr[0].val.clusterDim.x = 16;
@@ -417,10 +417,14 @@ int e4m3_cluster_size() {
   return size[dev];
 }
 
-// Tensors up to this many elements are quantized in one launch: one CTA up to 2^14 elements (a
-// single decode token), else one cluster.
-constexpr int64_t kE4m3ClusterMaxElems = int64_t(1) << 21;
+// Tensors whose 16-element blocks fit the registers of one cluster (kE4m3RegBlocks per thread)
+// are quantized in one launch: by one CTA up to 2^14 elements (a single decode token), else by
+// one cluster.
 constexpr int64_t kE4m3OneCtaMaxElems = int64_t(1) << 14;
+bool e4m3_one_launch(int64_t M, int64_t K) {
+  const int64_t cap = int64_t(ql::kE4m3RegBlocks) * ql::kE4m3ClusterThreads * 16;   // elements per CTA
+  return M * K <= kE4m3OneCtaMaxElems || M * K <= cap * e4m3_cluster_size();
+}
 
 // E4M3-B16 activation quantizer.  amax_slot: device word for the reduced amax bit pattern (the
 // two-launch path max-reduces into it; it is followed by the tensor-scale word and then
@@ -430,19 +434,21 @@ ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes,
                             cudaStream_t s, int n_tickets = 0) {
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   int* tickets = n_tickets > 0 ? reinterpret_cast<int*>(amax_slot + 2) : nullptr;
-  if (M * K <= kE4m3ClusterMaxElems) {
+  if (e4m3_one_launch(M, K)) {
     const int cs = M * K <= kE4m3OneCtaMaxElems ? 1 : e4m3_cluster_size();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cs, 1, 1);
-    cfg.blockDim = dim3(1024, 1, 1);
+    cfg.blockDim = dim3(ql::kE4m3ClusterThreads, 1, 1);
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may start early; waits
+    attr[1].val.programmaticStreamSerializationAllowed = 1;            // for x in-kernel
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     QL_CUDA(cudaLaunchKernelEx(&cfg, ql::quant_e4m3_b16_cluster_kernel, xb, static_cast<int>(M),
                                static_cast<int>(K), static_cast<int>(K), amax_slot, ts_out, codes,
                                static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms,
@@ -778,7 +784,7 @@ ql_status quantize_act(ql_aformat fmt, const void* x, int64_t M, int64_t K, void
       if (tensor_scale == nullptr)
         return fail(QL_ERR_INVALID_ARG, "E4M3-B16 needs a device tensor_scale pointer");
       unsigned* slot = reinterpret_cast<unsigned*>(tensor_scale);
-      if (M * K <= kE4m3ClusterMaxElems)   // one launch writes ts directly
+      if (e4m3_one_launch(M, K))   // one launch writes ts directly
         return launch_quant_e4m3(x, M, K, static_cast<uint8_t*>(codes),
                                  static_cast<uint8_t*>(scales), nullptr, 0, nullptr, tensor_scale, s);
       ql_status st = launch_quant_e4m3(x, M, K, static_cast<uint8_t*>(codes),
@@ -1007,7 +1013,7 @@ ql_status moe_grouped_forward(const ql_moe* m, const void* x, int64_t T, const f
   if (st != QL_OK) return st;
   ql::MoeGemmArgs a{};
   a.E = m->E; a.k = m->k; a.counts = counts; a.offsets = offsets; a.entries = entries;
-  a.gates = gates; a.I = m->I; a.H = m->H;
+  a.gates = gates; a.I = m->I; a.H = m->H; a.x_dq = x_dq;
   a.h_codes = w8 + p.h_codes; a.h_scales = w8 + p.h_scales; a.h_dq = h_dq;
   a.h32 = m->capture_h32 ? reinterpret_cast<float*>(w8 + p.h32) : nullptr;
   a.yslot = reinterpret_cast<float*>(w8 + p.yslot);

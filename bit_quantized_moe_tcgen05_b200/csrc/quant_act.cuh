@@ -200,13 +200,11 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
 
 // Quantize the 16-element block j of row m with tensor scale ts: codes [M, K/2] (row stride
 // ldc), scales plain [M, K/16] and/or tiled (atoms of 64 K).
-__device__ __forceinline__ void quant_e4m3_block(
-    const __nv_bfloat16* __restrict__ x, int m, int j, int ldx, float ts, uint8_t* __restrict__ codes,
-    int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
+// The same from the block's 16 bf16 values already in registers (element 2i low half of w[i]).
+__device__ __forceinline__ void quant_e4m3_regs(
+    const uint32_t (&w)[8], int m, int j, float ts, uint8_t* __restrict__ codes, int ldc,
+    uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
     int sf_atoms_per_row) {
-  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
-  const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
   uint32_t mx = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
@@ -264,6 +262,16 @@ __device__ __forceinline__ void quant_e4m3_block(
     scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row)] = static_cast<uint8_t>(sb);
 }
 
+__device__ __forceinline__ void quant_e4m3_block(
+    const __nv_bfloat16* __restrict__ x, int m, int j, int ldx, float ts, uint8_t* __restrict__ codes,
+    int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
+    int sf_atoms_per_row) {
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
+  const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  quant_e4m3_regs(w, m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+}
+
 // One thread per 16-element block, tensor scale from the amax that absmax_bf16_kernel reduced.
 // Thread 0 stores ts to *ts_out when ts_out is not null.
 __global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
@@ -282,33 +290,44 @@ __global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
   quant_e4m3_block(x, m, j, ldx, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
 }
 
-// Small tensors (decode): one thread-block cluster does the whole job in one launch.  Pass 1
-// reduces amax over the cluster (each CTA's maximum is read by rank 0..n-1 over distributed
-// shared memory), pass 2 quantizes.  No memset, no second launch.  The amax bit pattern goes to
+// Small tensors (decode): one thread-block cluster does the whole job in one launch.  Each thread
+// loads its (at most kE4m3RegBlocks) 16-element blocks once and keeps them in registers; every CTA
+// pushes its maximum into a slot of every CTA's shared memory (distributed shared memory), one
+// cluster barrier later each CTA has all maxima locally, and the blocks are quantized from
+// registers.  Launched with programmatic stream serialization: it waits for the grid before it
+// (which may produce x), then lets the GEMM behind it start.  The amax bit pattern goes to
 // *amax_out and ts to *ts_out (either may be null); the first nzero ints of zero_words are cleared.
-__global__ void __launch_bounds__(1024) quant_e4m3_b16_cluster_kernel(
+constexpr int kE4m3RegBlocks = 12;
+constexpr int kE4m3ClusterThreads = 256;
+__global__ void __launch_bounds__(kE4m3ClusterThreads) quant_e4m3_b16_cluster_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, unsigned* __restrict__ amax_out,
     float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
     uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
     int sf_atoms_per_row, int* __restrict__ zero_words, int nzero) {
+  griddep_wait();
   griddep_launch_dependents();
-  __shared__ uint32_t red[32];
-  __shared__ uint32_t s_cta_amax, s_amax;
-  const int ncta = static_cast<int>(gridDim.x);   // the grid is one cluster
+  __shared__ uint32_t red[kE4m3ClusterThreads / 32];
+  __shared__ uint32_t s_slot[16];   // CTA maxima of the cluster's ranks
+  const int ncta = static_cast<int>(gridDim.x);   // the grid is one cluster (<= 16 CTAs)
   const long tid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long nthr = static_cast<long>(ncta) * blockDim.x;
   const int nblk = K >> 4;
   const long total = static_cast<long>(M) * nblk;
+  uint32_t w[kE4m3RegBlocks][8];
   uint32_t mx = 0;
-  for (long b = tid; b < total; b += nthr) {
-    const int m = static_cast<int>(b / nblk);
-    const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
-    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-    mx = __vmaxu2(mx, v0.x & 0x7FFF7FFFu); mx = __vmaxu2(mx, v0.y & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, v0.z & 0x7FFF7FFFu); mx = __vmaxu2(mx, v0.w & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, v1.x & 0x7FFF7FFFu); mx = __vmaxu2(mx, v1.y & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, v1.z & 0x7FFF7FFFu); mx = __vmaxu2(mx, v1.w & 0x7FFF7FFFu);
+#pragma unroll
+  for (int k = 0; k < kE4m3RegBlocks; ++k) {
+    const long b = tid + k * nthr;
+    if (b < total) {
+      const int m = static_cast<int>(b / nblk);
+      const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
+      const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
+      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+      w[k][0] = v0.x; w[k][1] = v0.y; w[k][2] = v0.z; w[k][3] = v0.w;
+      w[k][4] = v1.x; w[k][5] = v1.y; w[k][6] = v1.z; w[k][7] = v1.w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[k][i] & 0x7FFF7FFFu);
+    }
   }
   uint32_t m16 = max(mx & 0xFFFFu, mx >> 16);
 #pragma unroll
@@ -319,19 +338,12 @@ __global__ void __launch_bounds__(1024) quant_e4m3_b16_cluster_kernel(
     uint32_t v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0u;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-    if (threadIdx.x == 0) s_cta_amax = v;
+    if (static_cast<int>(threadIdx.x) < ncta)   // lane t pushes this CTA's maximum to rank t
+      st_shared_cluster_u32(map_shared_rank(smem_u32(&s_slot[blockIdx.x]), threadIdx.x), v);
   }
   cluster_sync_all();
-  if (threadIdx.x < 32) {
-    uint32_t v = 0;
-    if (static_cast<int>(threadIdx.x) < ncta)
-      v = ld_shared_cluster_u32(map_shared_rank(smem_u32(&s_cta_amax), threadIdx.x));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-    if (threadIdx.x == 0) s_amax = v;
-  }
-  cluster_sync_all();   // every rank has read every other rank's maximum
-  const uint32_t amax16 = s_amax;
+  uint32_t amax16 = 0;
+  for (int r = 0; r < ncta; ++r) amax16 = max(amax16, s_slot[r]);
   const float ts = tensor_scale_from_amax16(amax16);
   if (tid == 0) {
     if (amax_out != nullptr) *amax_out = amax16;
@@ -339,10 +351,14 @@ __global__ void __launch_bounds__(1024) quant_e4m3_b16_cluster_kernel(
   }
   if (zero_words != nullptr)
     for (long i = tid; i < nzero; i += nthr) zero_words[i] = 0;
-  for (long b = tid; b < total; b += nthr) {
-    const int m = static_cast<int>(b / nblk);
-    const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
-    quant_e4m3_block(x, m, j, ldx, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+#pragma unroll
+  for (int k = 0; k < kE4m3RegBlocks; ++k) {
+    const long b = tid + k * nthr;
+    if (b < total) {
+      const int m = static_cast<int>(b / nblk);
+      const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
+      quant_e4m3_regs(w[k], m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+    }
   }
 }
 
