@@ -36,6 +36,12 @@ NOMINAL_FP4_OVER_BF16 = 4.0      # 9 PFLOP/s dense FP4 / 2.25 PFLOP/s dense bf16
 L2_BYTES = 126 * 1024 * 1024
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the timed GEMM
+# kernel, from an ncu --set full capture of that kernel (the VQ layer's M = 64 launch; the PRQuant
+# M = 2048 launch).  Set an entry to None whenever its kernel changes until it is captured again.
+NCU_TRAFFIC_PER_LAUNCH = {"vq": 11.33e6, "prquant_m2048": 24.19e6}
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -468,7 +474,7 @@ def main():
         alg = sum(gemm_bytes_of(head, M) for M in head["Ms"]) / nl
         ach = alg / (res["gemm_ms"] / nl * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm"], "traffic": None,
+                    "frac": ach / peaks["hbm"], "traffic": NCU_TRAFFIC_PER_LAUNCH.get(args.workload),
                     "kernel": "fp4_gemm_kernel (block16 MMA, VQ decode)" if head["kind"] == "vq"
                     else "fp4_gemm_kernel (mxf4)",
                     "algorithmic_bytes_per_launch": alg,
@@ -477,7 +483,8 @@ def main():
         alg = sum(flops_of(head, M) for M in head["Ms"]) / nl
         ach = alg / (res["gemm_ms"] / nl * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s",
-                    "frac": ach / fp4_peak, "traffic": None, "kernel": "fp4_gemm_kernel (mxf4)",
+                    "frac": ach / fp4_peak, "traffic": NCU_TRAFFIC_PER_LAUNCH.get(args.workload),
+                    "kernel": "fp4_gemm_kernel (mxf4)",
                     "algorithmic_flops_per_launch": alg,
                     "peak_source": f"{peaks['src']} bf16 burst {peaks['bf16']} x 4 (nominal FP4/bf16)"}
 

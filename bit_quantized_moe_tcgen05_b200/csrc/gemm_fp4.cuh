@@ -22,10 +22,15 @@
 // copies of the whole first ring fill (and the VQ warps decode them), and only then waits for the
 // quantizer grid (griddepcontrol.wait) before it loads activation tiles.  In decode launches the
 // activation tiles and scale atoms of every stage go by cp.async from the producer warp, so they
-// do not queue behind the weight blocks in the bulk-copy engine.  Split-K (decode): the gridDim.z
-// K-splits of one output tile each write an fp32 partial tile to a global workspace; the last
-// split to finish (an atomic ticket per tile) bulk-copies the partials into its idle ring and
-// adds them in split order, so the result is deterministic, writes y and re-arms the ticket.
+// do not queue behind the weight blocks in the bulk-copy engine.
+//
+// Work: a 1-D grid.  Tiles (128 weight rows x BN tokens, weight tile fastest) [0, full_tiles) get
+// one CTA each over all K; the remaining tiles are split along K over `splits` CTAs each.
+// Decode launches split every tile (full_tiles = 0) so that the grid covers the SMs; prefill
+// launches whose tiles overfill the last wave split only that wave's leftover tiles.  The K-splits
+// of a tile each write an fp32 partial tile to a global workspace; the last split to finish (an
+// atomic ticket per tile) bulk-copies the partials into its idle ring and adds them in split
+// order, so the result is deterministic, writes y and re-arms the ticket.
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -40,7 +45,10 @@ struct Fp4GemmArgs {
   int C, k_tail;            // activation width; tail width (weight width K' = C + k_tail)
   int n_base_stages;        // ceil(C / 256)
   int n_stages_total;       // n_base_stages + ceil(k_tail / 256)
-  int stages_per_split;     // K stages handled by one CTA (gridDim.z = splits)
+  int stages_per_split;     // K stages handled by one CTA of a split tile
+  int tiles_n;              // 128-row weight tiles
+  int full_tiles;           // tiles [0, full_tiles) are not split
+  int splits;               // K-splits of every other tile
   const uint8_t* sfb;       // activation scales, tiled atoms
   int sfb_atoms;            // atoms per 128-row group of the activation
   const float* alpha_dev;   // optional device scalar multiplied into alpha (tensor scale of x)
@@ -53,10 +61,9 @@ struct Fp4GemmArgs {
                             // FP4 codes 128 rows x 128 B with the 128-byte swizzle applied, or VQ
                             // indices 128 rows x 64 B + the stage's 8 QBlock codebooks; then the
                             // stage's weight scale atoms
-  float* partials;          // split-K: fp32 [tiles][splits][BN][128] (tile = blockIdx.y * gridDim.x
-                            // + blockIdx.x)
+  float* partials;          // split tiles: fp32 [tile - full_tiles][splits][BN][128]
   const uint8_t* xq;        // quantized activation codes [M, C/2] (read directly by decode launches)
-  int* tickets;             // [tiles] arrival counters, zero between launches
+  int* tickets;             // [split tiles] arrival counters, zero between launches
 };
 
 template <int BN, bool E8M0, bool VQ = false>
@@ -121,12 +128,22 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
   __shared__ int s_last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN;
-  const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-  const int s_begin = blockIdx.z * a.stages_per_split;
-  const int s_end = min(a.n_stages_total, s_begin + a.stages_per_split);
+  int tile, zsplit, splits;
+  if (static_cast<int>(blockIdx.x) < a.full_tiles) {
+    tile = blockIdx.x;
+    zsplit = 0;
+    splits = 1;
+  } else {
+    const int r = blockIdx.x - a.full_tiles;
+    tile = a.full_tiles + r / a.splits;
+    zsplit = r % a.splits;
+    splits = a.splits;
+  }
+  const int wtile = tile % a.tiles_n;
+  const int n0 = wtile * 128, m0 = (tile / a.tiles_n) * BN;
+  const int s_begin = splits == 1 ? 0 : zsplit * a.stages_per_split;
+  const int s_end = splits == 1 ? a.n_stages_total : min(a.n_stages_total, s_begin + a.stages_per_split);
   const int n_it = max(0, s_end - s_begin);
-  const int splits = gridDim.z;
   // decode launches whose stages all fit the ring take activations by cp.async
   const bool lsu_act = BN <= 64 && n_it <= S;
 
@@ -177,7 +194,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
       stage_coords(i, kw, kx, valid);
       const int nat = valid / Cfg::kAtomK;
       const uint32_t act_bytes = lsu_act ? 0u : Cfg::kBBytes + nat * 512 * Cfg::kG;
-      const uint8_t* wblk = a.wt + (static_cast<size_t>(blockIdx.x) * a.n_stages_total + i) * Cfg::kWBytes;
+      const uint8_t* wblk = a.wt + (static_cast<size_t>(wtile) * a.n_stages_total + i) * Cfg::kWBytes;
       if constexpr (VQ) {
         mbar_arrive_expect_tx(&wfull[st], Cfg::kWBytes);
         if (!lsu_act) mbar_arrive_expect_tx(&full[st], act_bytes);
@@ -389,8 +406,9 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
       } else if (ok) {
         // Split-K: park this split's fp32 partial [BN tokens][128 rows] in the workspace (lanes
         // cover consecutive rows: coalesced) and take a ticket; the last split reduces.
-        float* part = a.partials + static_cast<size_t>(tile) * splits * BN * 128;
-        float* mine = part + static_cast<size_t>(blockIdx.z) * BN * 128;
+        const int stile = tile - a.full_tiles;   // index among the split tiles
+        float* part = a.partials + static_cast<size_t>(stile) * splits * BN * 128;
+        float* mine = part + static_cast<size_t>(zsplit) * BN * 128;
 #pragma unroll 1
         for (int c = 0; c < mcount; c += 8) {
           uint32_t r[8];
@@ -403,7 +421,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
         named_bar_sync(1, 128);
         if (threadIdx.x == 64) {
           __threadfence();   // release the whole CTA's partial (ordered before by the barrier)
-          s_last = (atomicAdd(a.tickets + tile, 1) == splits - 1);
+          s_last = (atomicAdd(a.tickets + stile, 1) == splits - 1);
           if (s_last) __threadfence();   // acquire every other split's partial
         }
         named_bar_sync(1, 128);
@@ -448,7 +466,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
             }
             named_bar_sync(1, 128);   // before the next run overwrites stg
           }
-          if (threadIdx.x == 64) a.tickets[tile] = 0;   // re-armed for the next launch
+          if (threadIdx.x == 64) a.tickets[stile] = 0;   // re-armed for the next launch
         }
       }
     }

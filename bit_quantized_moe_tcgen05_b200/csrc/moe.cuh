@@ -153,7 +153,10 @@ struct MoeGemmArgs {
   int H;
 };
 
-// Stages of token-row gathers the gate/up producer keeps in flight before signalling one.
+// Stages of token-row gathers the gate/up producer keeps in flight before signalling one.  A
+// stage's slot can only be refilled after it was signalled and consumed, so the consumers can
+// run at most kStages - kGatherLag stages ahead of the gathers: the lag trades latency hiding
+// for consumer slack.
 constexpr int kGatherLag = 2;
 
 template <int BN>
@@ -162,7 +165,7 @@ struct MoeCfg {
   static constexpr int kBBytes = BN * 128;        // BN rows x 64 bf16
   static constexpr int kIdxBytes = 128 * 32;      // 128 rows x 64 4-bit indices
   static constexpr int kStageBytes = kABytes + kBBytes + kIdxBytes;
-  static constexpr int kStages = 4;
+  static constexpr int kStages = 5;
   static constexpr int kCentBytes = 128 * 16 * 2;
   static constexpr int kHalf = BN / 2;            // tokens per epilogue pass
   static constexpr int kStgLd = 129;              // padded row of the transposed staging tile
@@ -172,6 +175,8 @@ struct MoeCfg {
   static constexpr int kThreads = (2 + kDecWarps + 4) * 32;
   static constexpr int kSmemBytes =
       kStages * kStageBytes + 2 * kCentBytes + kStgBytes + 2 * BN * 4 + 1024 + 512;
+  static_assert(kSmemBytes + 4200 <= 227 * 1024, "dynamic + static shared memory per block");
+  static_assert(kGatherLag < kStages, "gathers must be signalled before their slot comes round");
 };
 
 __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
@@ -207,8 +212,9 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
   __nv_bfloat16* sCent = reinterpret_cast<__nv_bfloat16*>(sIdx + S * Cfg::kIdxBytes);    // [2][128][16]
   float* sStg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sCent) + 2 * Cfg::kCentBytes);
   int* sRow = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(sStg) + Cfg::kStgBytes);  // [2][BN]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sRow + 2 * BN);
-  uint64_t* empty = full + S;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sRow + 2 * BN);   // B rows (and indices) landed
+  uint64_t* ifull = full + S;                                       // index tile landed
+  uint64_t* empty = ifull + S;
   uint64_t* decd = empty + S;
   uint64_t* cfull = decd + S;     // [2] centroids + row list of an item landed
   uint64_t* cempty = cfull + 2;   // [2] decoders done with them
@@ -229,7 +235,8 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], GATEUP ? 33 : 1);   // gate/up: + one arrival per producer lane
+      mbar_init(&full[s], GATEUP ? 32 : 1);   // gate/up: one arrival per producer lane
+      mbar_init(&ifull[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&decd[s], Cfg::kDecWarps * 32);
     }
@@ -305,9 +312,12 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 12));
         if (!ok) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[st], Cfg::kIdxBytes + (GATEUP ? 0 : Cfg::kBBytes));
-          tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_idx, &full[st], i * 32, row0);
-          if constexpr (!GATEUP) tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, I.p0);
+          mbar_arrive_expect_tx(&ifull[st], Cfg::kIdxBytes);
+          tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_idx, &ifull[st], i * 32, row0);
+          if constexpr (!GATEUP) {
+            mbar_arrive_expect_tx(&full[st], Cfg::kBBytes);
+            tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, I.p0);
+          }
         }
         if constexpr (GATEUP) {
           // Gather the item's token rows (64 bf16 of each, in the 128-byte-swizzled K-major
@@ -380,7 +390,7 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       for (int i = 0; i < nstages && ok; ++i, ++it) {
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait(&full[st], ph, 16)) { ok = false; break; }
+        if (!mbar_wait(&ifull[st], ph, 16)) { ok = false; break; }   // indices only: runs ahead of B
         const uint8_t* idx_s = sIdx + st * Cfg::kIdxBytes;
         uint8_t* a_s = sA + st * Cfg::kABytes;
 #pragma unroll

@@ -192,6 +192,7 @@ namespace {
 
 struct FwdPlan {
   int BN, splits, spp, tiles_n, tiles_m;
+  int full_tiles;   // FP4 GEMM: tiles [0, full_tiles) unsplit, the rest split `splits` ways
   int sfb_atoms;
   size_t codes_off, sf_off, scal_off, tick_off, part_off, total;
   int n_tickets;   // split-K tickets (zeroed by the quantizer, re-armed by the GEMM)
@@ -229,10 +230,17 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   p.tiles_m = static_cast<int>(cdiv(std::max<int64_t>(M, 1), p.BN));
   const int tiles = p.tiles_n * p.tiles_m;
   const int total = L->n_stages_total;
-  // One CTA per SM: split K until the grid covers the SMs (at most kMaxSplits ways).
+  // One CTA per SM.  With at least as many tiles as SMs every tile runs unsplit.  With fewer,
+  // every tile is split along K so that the grid covers the SMs; the number of ways is bounded
+  // by kMaxSplits and by the volume of fp32 partials one tile's last split must add up (about
+  // 512 KB).  (Splitting only the tiles left over after the last whole wave was measured too:
+  // at 160 prefill tiles on 148 SMs the split tiles' reduction cost more than the idle SMs.)
   const int target = sm_count();
+  p.full_tiles = tiles >= target ? tiles : 0;
+  const int rest = tiles - p.full_tiles;
   int splits = 1;
-  if (tiles < target) splits = std::max(1, std::min({total, target / tiles, ql::kMaxSplits}));
+  if (rest > 0)
+    splits = std::max(1, std::min({total, target / rest, ql::kMaxSplits, std::max(1, 1024 / p.BN)}));
   p.spp = static_cast<int>(cdiv(total, splits));
   p.splits = static_cast<int>(cdiv(total, p.spp));
   const int atomK = L->e8m0 ? 128 : 64;  // K elements covered by one 512-byte scale atom
@@ -247,11 +255,11 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   // (one memset or the quantizer clears the whole run before the GEMM).
   p.scal_off = off;
   p.tick_off = off + 2 * sizeof(float);
-  p.n_tickets = p.splits > 1 ? tiles : 0;
+  p.n_tickets = p.splits > 1 ? rest : 0;
   off = align_up(p.tick_off + static_cast<size_t>(p.n_tickets) * sizeof(int), 256);
   p.part_off = off;
   if (p.splits > 1)
-    off = align_up(off + static_cast<size_t>(tiles) * p.splits * p.BN * 128 * 4, 256);
+    off = align_up(off + static_cast<size_t>(rest) * p.splits * p.BN * 128 * 4, 256);
   p.total = off;
   return p;
 }
@@ -739,7 +747,10 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   a.partials = reinterpret_cast<float*>(w8 + p.part_off);
   a.tickets = reinterpret_cast<int*>(w8 + p.tick_off);
   a.xq = w8 + p.codes_off;
-  dim3 grid(p.tiles_n, p.tiles_m, p.splits);
+  a.tiles_n = p.tiles_n;
+  a.full_tiles = p.full_tiles;
+  a.splits = p.splits;
+  dim3 grid(p.full_tiles + (p.tiles_n * p.tiles_m - p.full_tiles) * p.splits, 1, 1);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (y32 && (reinterpret_cast<uintptr_t>(y32) & 15)) ||
       (L->N * 2) % 16 != 0)

@@ -297,8 +297,8 @@ __global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
 // registers.  Launched with programmatic stream serialization: it waits for the grid before it
 // (which may produce x), then lets the GEMM behind it start.  The amax bit pattern goes to
 // *amax_out and ts to *ts_out (either may be null); the first nzero ints of zero_words are cleared.
-constexpr int kE4m3RegBlocks = 12;
-constexpr int kE4m3ClusterThreads = 256;
+constexpr int kE4m3RegBlocks = 3;
+constexpr int kE4m3ClusterThreads = 1024;
 __global__ void __launch_bounds__(kE4m3ClusterThreads) quant_e4m3_b16_cluster_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, unsigned* __restrict__ amax_out,
     float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
