@@ -22,7 +22,11 @@
 // copies of the whole first ring fill (and the VQ warps decode them), and only then waits for the
 // quantizer grid (griddepcontrol.wait) before it loads activation tiles.  In decode launches the
 // activation tiles and scale atoms of every stage go by cp.async from the producer warp, so they
-// do not queue behind the weight blocks in the bulk-copy engine.
+// do not queue behind the weight blocks in the bulk-copy engine.  Every CTA also releases the
+// next programmatic grid at once (griddepcontrol.launch_dependents): the next layer's quantizer
+// and GEMM then take SMs as this grid's CTAs retire and start their weight streams during this
+// grid's split-K tail.  Whatever they read of this grid's results (y, the workspace) they read
+// after their own griddepcontrol.wait, which returns only once this grid has completed.
 //
 // Work: a 1-D grid.  Tiles (128 weight rows x BN tokens, weight tile fastest) [0, full_tiles) get
 // one CTA each over all K; the remaining tiles are split along K over `splits` CTAs each.
@@ -78,10 +82,10 @@ struct Fp4Cfg {
   static constexpr int kBBytes = BN * 128;
   static constexpr int kSfaBytes = kAtoms * 512;
   static constexpr int kSfbBytes = kAtoms * kG * 512;
-  static constexpr int kIdxBytes = VQ ? 128 * 64 : 0;   // VQ: 8-bit indices, 128 rows x 64
+  static constexpr int kIdxBytes = VQ ? 128 * 64 : 0;   // VQ: 8-bit indices [chunk 8][row 128][8]
   static constexpr int kLutBytes = VQ ? 8 * 512 : 0;    // VQ: 2 x 4 QBlock codebooks of 512 B
   // The weight block of one stage, as stored in HBM and copied by one bulk copy:
-  // FP4: [codes 16 KB][SFA atoms]; VQ: [indices 8 KB][codebooks 4 KB][SFA atoms].
+  // FP4: [codes 16 KB][SFA atoms]; VQ: [indices 8 KB, chunk-major][codebooks 4 KB][SFA atoms].
   static constexpr int kWBytes = (VQ ? kIdxBytes + kLutBytes : kABytes) + kSfaBytes;
   static constexpr int kSfaOff = VQ ? kIdxBytes + kLutBytes : kABytes;
   static constexpr int kStageBytes = kWBytes + kBBytes + kSfbBytes + (VQ ? kABytes : 0);
@@ -126,6 +130,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
   uint64_t* rbar = accf + 1;    // split-K: the splits' partials landed in the idle ring
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 1);
   __shared__ int s_last;
+  griddep_launch_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int tile, zsplit, splits;
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&decd[s], VQ ? Cfg::kDecWarps * 32 : 1);
+      mbar_init(&decd[s], VQ ? Cfg::kDecWarps : 1);
       mbar_init(&wfull[s], 1);
       mbar_init(&afull[s], 32);
     }
@@ -324,9 +329,13 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
       // ---------------- VQ decode (warps 2..9): for each stage rebuild the 128 x 256 E2M1 operand
       // tile from 8-bit indices and the QBlock codebooks, in the 128-byte-swizzled K-major layout
       // the MMA reads (16-byte chunk kc of row r at kc ^ (r%8)).  Only weights are read, so this
-      // runs ahead of the activation quantizer.
+      // runs ahead of the activation quantizer.  One warp instruction covers 32 consecutive rows
+      // of one 32-element chunk: its index loads are 256 contiguous bytes (the block stores the
+      // indices chunk-major), its lookups all fall in one 512-byte codebook, and its 16-byte
+      // stores hit every bank once per 8 rows.
       const int t = threadIdx.x - 64;
       constexpr int kDT = Cfg::kDecWarps * 32;
+      static_assert(1024 % kDT == 0 && kDT % 256 == 0, "decoder threads tile the 1024 chunks");
       for (int it = 0; it < n_it && ok; ++it) {
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
@@ -336,9 +345,9 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
         uint8_t* a_s = sA(st);
 #pragma unroll
         for (int j = 0; j < 1024 / kDT; ++j) {
-          const int c = t + kDT * j;             // 16-byte output chunk: row r, chunk kc
-          const int r = c >> 3, kc = c & 7;
-          const uint2 iv = *reinterpret_cast<const uint2*>(idx_s + r * 64 + kc * 8);
+          const int c = t + kDT * j;
+          const int kc = (c >> 5) & 7, r = (c & 31) | ((c >> 8) << 5);
+          const uint2 iv = *reinterpret_cast<const uint2*>(idx_s + kc * 1024 + r * 8);
           const uint16_t* L = lut + ((((r >> 6) << 2) + (kc >> 1)) << 8);
           uint4 o;
           o.x = L[iv.x & 255u] | (static_cast<uint32_t>(L[(iv.x >> 8) & 255u]) << 16);
@@ -347,8 +356,9 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
           o.w = L[(iv.y >> 16) & 255u] | (static_cast<uint32_t>(L[iv.y >> 24]) << 16);
           *reinterpret_cast<uint4*>(a_s + r * 128 + ((kc ^ (r & 7)) << 4)) = o;
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&decd[st]);
+        fence_proxy_async_smem();   // every writer orders its stores for the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&decd[st]);
       }
     }
     if (warp < 6) {   // (extra VQ decoders, warps 6..9, take no part in the epilogue)
@@ -420,9 +430,10 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
         }
         named_bar_sync(1, 128);
         if (threadIdx.x == 64) {
-          __threadfence();   // release the whole CTA's partial (ordered before by the barrier)
-          s_last = (atomicAdd(a.tickets + stile, 1) == splits - 1);
-          if (s_last) __threadfence();   // acquire every other split's partial
+          // releases the whole CTA's partial (ordered before by the barrier); the last split
+          // acquires every other split's
+          s_last = atom_add_acq_rel_gpu(reinterpret_cast<uint32_t*>(a.tickets + stile), 1u) ==
+                   static_cast<uint32_t>(splits - 1);
         }
         named_bar_sync(1, 128);
         if (s_last) {

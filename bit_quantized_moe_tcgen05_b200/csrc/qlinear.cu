@@ -307,8 +307,11 @@ size_t repack_weight_blocks(const uint8_t* src, const uint8_t* scales, const uin
         const uint8_t* srow = src + n * src_row + kw / per_byte;
         const int nbytes = static_cast<int>(valid / per_byte);
         for (int b = 0; b < nbytes; ++b) {
-          const int dst = vq ? b : ((((b >> 4) ^ (r & 7)) << 4) | (b & 15));
-          blk[r * row_bytes + dst] = srow[b];
+          // VQ: indices chunk-major, [32-element chunk][row][8]; FP4: row-major with the
+          // 128-byte swizzle the MMA expects
+          const int dst = vq ? ((b >> 3) * 1024 + r * 8 + (b & 7))
+                             : (r * row_bytes + ((((b >> 4) ^ (r & 7)) << 4) | (b & 15)));
+          blk[dst] = srow[b];
         }
         for (int jl = 0; jl < valid / sfb; ++jl)
           sfa[(jl >> 2) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (jl & 3)] =

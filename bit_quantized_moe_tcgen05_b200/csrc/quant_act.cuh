@@ -294,9 +294,11 @@ __global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
 // loads its (at most kE4m3RegBlocks) 16-element blocks once and keeps them in registers; every CTA
 // pushes its maximum into a slot of every CTA's shared memory (distributed shared memory), one
 // cluster barrier later each CTA has all maxima locally, and the blocks are quantized from
-// registers.  Launched with programmatic stream serialization: it waits for the grid before it
-// (which may produce x), then lets the GEMM behind it start.  The amax bit pattern goes to
-// *amax_out and ts to *ts_out (either may be null); the first nzero ints of zero_words are cleared.
+// registers.  Launched with programmatic stream serialization: it first lets the GEMM behind it
+// launch (that grid streams weights until its own griddepcontrol.wait, which returns only after
+// this grid completes), then waits for the grid before it (which may produce x).  The amax bit
+// pattern goes to *amax_out and ts to *ts_out (either may be null); the first nzero ints of
+// zero_words are cleared.
 constexpr int kE4m3RegBlocks = 3;
 constexpr int kE4m3ClusterThreads = 1024;
 __global__ void __launch_bounds__(kE4m3ClusterThreads) quant_e4m3_b16_cluster_kernel(
@@ -304,8 +306,8 @@ __global__ void __launch_bounds__(kE4m3ClusterThreads) quant_e4m3_b16_cluster_ke
     float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
     uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
     int sf_atoms_per_row, int* __restrict__ zero_words, int nzero) {
-  griddep_wait();
   griddep_launch_dependents();
+  griddep_wait();
   __shared__ uint32_t red[kE4m3ClusterThreads / 32];
   __shared__ uint32_t s_slot[16];   // CTA maxima of the cluster's ranks
   const int ncta = static_cast<int>(gridDim.x);   // the grid is one cluster (<= 16 CTAs)
