@@ -113,8 +113,9 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
   using Cfg = Fp4Cfg<BN, E8M0, VQ>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1 KB aligned by offsetting the shared array itself, so that every pointer derived from it
+  // stays a shared-space pointer (plain ld/st.shared, not generic accesses)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   // ring layout (every region 1 KB aligned): weight blocks, B tiles, SFB atoms, decoded A (VQ)
   uint8_t* sW = smem;
   uint8_t* sB = sW + S * Cfg::kWBytes;

@@ -142,8 +142,9 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
   constexpr int S = Cfg::kStages;
   constexpr int kFoldThreads = Cfg::kFoldWarps * 32;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1 KB aligned by offsetting the shared array itself, so that every pointer derived from it
+  // stays a shared-space pointer (plain ld/st.shared, not generic accesses)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   // stage st: [A int8 tile 16 KB][B tile][raw weight block][sx]  (A and B 1024-aligned)
   auto sA = [&](int st) { return smem + st * Cfg::kStageBytes; };
   auto sB = [&](int st) { return smem + st * Cfg::kStageBytes + Cfg::kABytes; };

@@ -125,6 +125,16 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// 64-bit release store / acquire load at GPU scope (flags that publish data to other CTAs).
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Fetch-and-add with acquire-release semantics at GPU scope: publishes the writes that happen
 // before it (including other CTA threads' writes ordered by a barrier) and, for the caller,
 // orders later reads after every earlier release on the same counter.

@@ -364,6 +364,135 @@ __global__ void __launch_bounds__(kE4m3ClusterThreads) quant_e4m3_b16_cluster_ke
   }
 }
 
+// Mid-size tensors (a few decode tokens up to ~1.8 M elements): one grid of small CTAs, at most one
+// per SM, so that all of them are resident at once, also beside a running GEMM CTA.  Each thread
+// keeps its (at most kE4m3RegBlocks) 16-element blocks in registers.  The tensor amax is agreed on
+// through the workspace block `sync`: word 0 a launch counter, bytes 8..15 a result word, then one
+// 64-bit slot per CTA.  Every CTA reads the counter c once and publishes its maximum in its slot,
+// tagged with c + 1 (release).  CTA 0 waits (bounded) until every slot carries the tag (acquire),
+// stores the tagged maximum of all of them in the result word and advances the counter; the other
+// CTAs wait for the tagged result (one word, so the polling does not pile onto the slots' cache
+// lines).  No word needs clearing between launches; a stale word would have to repeat a 48-bit tag
+// to be taken for a fresh one.  Launched with programmatic stream serialization like the cluster
+// kernel.  On a timeout the error word is set and no codes are written.
+constexpr int kE4m3GridThreads = 256;
+constexpr int kE4m3GridMaxCtas = 256;   // CTA 0 polls one slot per thread
+constexpr int kE4m3SyncBytes = 16 + 8 * kE4m3GridMaxCtas;
+
+__device__ __forceinline__ unsigned long long e4m3_grid_tag(uint32_t c) {
+  return (static_cast<unsigned long long>(c) << 32) |
+         (static_cast<unsigned long long>((c * 0x9E37u + 0x5A3Cu) & 0xFFFFu) << 16);
+}
+
+// Bounded wait until *p carries `tag` in its upper 48 bits; returns the word (0 on a timeout).
+__device__ __forceinline__ unsigned long long wait_tagged_u64(const unsigned long long* p,
+                                                              unsigned long long tag, bool& ok) {
+  unsigned long long s = ld_acquire_gpu_u64(p);
+  if ((s & ~0xFFFFull) == tag) return s;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(64);
+    s = ld_acquire_gpu_u64(p);
+    if ((s & ~0xFFFFull) == tag) return s;
+    if (globaltimer_ns() - t0 > 2000000000ull) {
+      record_error(DEV_TIMEOUT, 30);
+      ok = false;
+      return 0;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kE4m3GridThreads) quant_e4m3_b16_grid_kernel(
+    const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, unsigned* __restrict__ amax_out,
+    float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
+    uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
+    int sf_atoms_per_row, int* __restrict__ zero_words, int nzero, uint32_t* __restrict__ sync) {
+  griddep_launch_dependents();
+  griddep_wait();
+  __shared__ uint32_t red[kE4m3GridThreads / 32];
+  __shared__ uint32_t s_count, s_amax;
+  __shared__ int s_ok;
+  unsigned long long* result = reinterpret_cast<unsigned long long*>(sync + 2);
+  unsigned long long* slots = result + 1;
+  if (threadIdx.x == 0) s_count = *reinterpret_cast<volatile uint32_t*>(sync) + 1u;
+  const long tid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long nthr = static_cast<long>(gridDim.x) * blockDim.x;
+  const int nblk = K >> 4;
+  const long total = static_cast<long>(M) * nblk;
+  uint32_t w[kE4m3RegBlocks][8];
+  uint32_t mx = 0;
+#pragma unroll
+  for (int k = 0; k < kE4m3RegBlocks; ++k) {
+    const long b = tid + k * nthr;
+    if (b < total) {
+      const int m = static_cast<int>(b / nblk);
+      const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
+      const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
+      const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+      w[k][0] = v0.x; w[k][1] = v0.y; w[k][2] = v0.z; w[k][3] = v0.w;
+      w[k][4] = v1.x; w[k][5] = v1.y; w[k][6] = v1.z; w[k][7] = v1.w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[k][i] & 0x7FFF7FFFu);
+    }
+  }
+  if (zero_words != nullptr)
+    for (long i = tid; i < nzero; i += nthr) zero_words[i] = 0;
+  uint32_t m16 = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m16;
+  __syncthreads();   // also publishes s_count
+  const uint32_t cnt = s_count;
+  const unsigned long long tag = e4m3_grid_tag(cnt);
+  if (threadIdx.x == 0) {
+    uint32_t v = 0;
+    for (int i = 0; i < kE4m3GridThreads / 32; ++i) v = max(v, red[i]);
+    st_release_gpu_u64(&slots[blockIdx.x], tag | v);
+  }
+  bool ok = true;
+  if (blockIdx.x == 0) {
+    uint32_t a16 = 0;
+    if (threadIdx.x < gridDim.x)
+      a16 = static_cast<uint32_t>(wait_tagged_u64(&slots[threadIdx.x], tag, ok) & 0xFFFFull);
+    __syncthreads();   // red[] is reused
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a16 = max(a16, __shfl_xor_sync(0xFFFFFFFFu, a16, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a16;
+    ok = __syncthreads_and(ok);
+    if (threadIdx.x == 0) {
+      uint32_t v = 0;
+      for (int i = 0; i < kE4m3GridThreads / 32; ++i) v = max(v, red[i]);
+      s_amax = v;
+      if (ok) {
+        st_release_gpu_u64(result, tag | v);
+        *sync = cnt;
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    s_ok = 1;
+    s_amax = static_cast<uint32_t>(wait_tagged_u64(result, tag, ok) & 0xFFFFull);
+    s_ok = ok;
+  }
+  __syncthreads();
+  if (blockIdx.x != 0) ok = s_ok != 0;
+  if (!ok) return;
+  const uint32_t amax16 = s_amax;
+  const float ts = tensor_scale_from_amax16(amax16);
+  if (tid == 0) {
+    if (amax_out != nullptr) *amax_out = amax16;
+    if (ts_out != nullptr) *ts_out = ts;
+  }
+#pragma unroll
+  for (int k = 0; k < kE4m3RegBlocks; ++k) {
+    const long b = tid + k * nthr;
+    if (b < total) {
+      const int m = static_cast<int>(b / nblk);
+      const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
+      quant_e4m3_regs(w[k], m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+    }
+  }
+}
+
 // Replace the amax bit pattern stored in *slot by the tensor scale it implies (single thread).
 __global__ void amax_to_tensor_scale_kernel(unsigned* slot) {
   const float ts = tensor_scale_from_amax16(*slot);

@@ -186,3 +186,42 @@ def test_quant_e4m3_b16_rounding_thresholds():
     tiny = g.standard_normal((2, 128)) * 1e-39    # subnormal block scales
     tiny[:, 0] = 3e-36
     _check_quant(synth.to_bf16_bits(tiny))
+
+
+def test_e4m3_grid_quantizer_shared_workspace():
+    """The grid-wide E4M3-B16 quantizer (more 16-element blocks than a cluster has threads)
+    agrees on the tensor amax through tagged words in the caller's workspace: it must work on a
+    workspace full of random bytes, when two layers of different shapes take turns on one
+    workspace, and give identical results when repeated."""
+    ql = _ql()
+    g = np.random.default_rng(90)
+    layers, refs, xs = [], [], []
+    for N, K, M in ((256, 8192, 64), (384, 4096, 80)):   # 32768 and 20480 blocks of 16
+        codes = synth.uniform_nibble_bytes(91 + N, N, K)
+        sb = synth.uniform_bytes(92 + N, (N, K // 16), 0x28, 0x48)
+        ts_w = np.float32(0.0123)
+        lin = ql.QLinear(codes, sb, wfmt=ql.QL_W_NVFP4_E4M3_B16, w_tensor_scale=float(ts_w))
+        xb, _ = synth.activations_bf16(93 + N, M, K, 0.01, 30.0)
+        xd = _x_deq(xb)
+        wd = mx.dequant_e4m3_b16(F.unpack_nibbles(codes), sb, ts_w)
+        layers.append(lin)
+        xs.append(dev_bf16(xb))
+        refs.append((G.gemm_ref(xd, wd), G.abs_scale(xd, wd)))
+    need = max(l.workspace_bytes(x.shape[0]) for l, x in zip(layers, xs))
+    ws = torch.from_numpy(g.integers(0, 256, need, dtype=np.uint8)).cuda()
+    first = {}
+    for rnd in range(3):
+        for i, (lin, x) in enumerate(zip(layers, xs)):
+            y32 = torch.empty((x.shape[0], lin.N), dtype=torch.float32, device="cuda")
+            y = lin(x, out_f32=y32, ws=ws)
+            ql.check()
+            yb, y32h = y.float().cpu().numpy(), y32.cpu().numpy()
+            ref, t = refs[i]
+            check_fp32(y32h, ref, t, f"shared ws layer {i} round {rnd}")
+            check_bf16(yb, ref, t, f"shared ws layer {i} round {rnd}")
+            if rnd == 0:
+                first[i] = y32h
+            else:
+                assert np.array_equal(first[i], y32h), f"layer {i} round {rnd} not repeatable"
+    for lin in layers:
+        lin.close()
