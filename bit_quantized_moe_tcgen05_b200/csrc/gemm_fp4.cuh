@@ -153,29 +153,6 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
   // decode launches whose stages all fit the ring take activations by cp.async
   const bool lsu_act = BN <= 64 && n_it <= S;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-      mbar_init(&decd[s], VQ ? Cfg::kDecWarps : 1);
-      mbar_init(&wfull[s], 1);
-      mbar_init(&afull[s], 32);
-    }
-    mbar_init(accf, 1);
-    mbar_init(rbar, 1);
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) prefetch_tmap(&tm_x);
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t sfa_col0 = BN, sfb_col0 = BN + S * Cfg::kSfaCols;
-
   // K stage i -> (weight element offset, activation element offset, valid elements)
   auto stage_coords = [&](int i, int& kw, int& kx, int& valid) {
     if (i < a.n_base_stages) {
@@ -189,27 +166,60 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
       valid = min(256, a.k_tail - j);
     }
   };
+  // Weight part of stage it (independent of earlier grids): one bulk copy of the stage block.
+  auto issue_weight = [&](int it) {
+    const int i = s_begin + it, st = it % S;
+    int kw, kx, valid;
+    stage_coords(i, kw, kx, valid);
+    const int nat = valid / Cfg::kAtomK;
+    const uint32_t act_bytes = lsu_act ? 0u : Cfg::kBBytes + nat * 512 * Cfg::kG;
+    const uint8_t* wblk = a.wt + (static_cast<size_t>(wtile) * a.n_stages_total + i) * Cfg::kWBytes;
+    if constexpr (VQ) {
+      mbar_arrive_expect_tx(&wfull[st], Cfg::kWBytes);
+      if (!lsu_act) mbar_arrive_expect_tx(&full[st], act_bytes);
+      bulk_load(sW + st * Cfg::kWBytes, wblk, Cfg::kWBytes, &wfull[st]);
+    } else {
+      mbar_arrive_expect_tx(&full[st], Cfg::kWBytes + act_bytes);
+      bulk_load(sW + st * Cfg::kWBytes, wblk, Cfg::kWBytes, &full[st]);
+    }
+  };
+  const int pre = min(n_it, S);   // the first ring fill needs no empty-slot wait
+
+  // Warp 0 initialises the barriers (lane s: stage s) and, before the block-wide barrier, its lane
+  // 0 already issues the weight copies of the first ring fill, so that they are in flight while
+  // the TMEM allocation and the rest of the set-up run.
+  if (warp == 0) {
+    for (int s = lane; s < S; s += 32) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&decd[s], VQ ? Cfg::kDecWarps : 1);
+      mbar_init(&wfull[s], 1);
+      mbar_init(&afull[s], 32);
+    }
+    if (lane == 0) {
+      mbar_init(accf, 1);
+      mbar_init(rbar, 1);
+    }
+    fence_mbar_init();
+    __syncwarp();
+    if (lane == 0) {
+      for (int it = 0; it < pre; ++it) issue_weight(it);
+      prefetch_tmap(&tm_x);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sfa_col0 = BN, sfb_col0 = BN + S * Cfg::kSfaCols;
 
   bool ok = true;
   if (warp == 0) {
     // ---------------- producer: the whole warp runs the loop; one elected lane issues copies.
-    // Weight part of stage it (independent of earlier grids): one bulk copy of the stage block.
-    auto issue_weight = [&](int it) {
-      const int i = s_begin + it, st = it % S;
-      int kw, kx, valid;
-      stage_coords(i, kw, kx, valid);
-      const int nat = valid / Cfg::kAtomK;
-      const uint32_t act_bytes = lsu_act ? 0u : Cfg::kBBytes + nat * 512 * Cfg::kG;
-      const uint8_t* wblk = a.wt + (static_cast<size_t>(wtile) * a.n_stages_total + i) * Cfg::kWBytes;
-      if constexpr (VQ) {
-        mbar_arrive_expect_tx(&wfull[st], Cfg::kWBytes);
-        if (!lsu_act) mbar_arrive_expect_tx(&full[st], act_bytes);
-        bulk_load(sW + st * Cfg::kWBytes, wblk, Cfg::kWBytes, &wfull[st]);
-      } else {
-        mbar_arrive_expect_tx(&full[st], Cfg::kWBytes + act_bytes);
-        bulk_load(sW + st * Cfg::kWBytes, wblk, Cfg::kWBytes, &full[st]);
-      }
-    };
     // Activation part (written by the quantizer grid): B codes and SFB, by the bulk-copy engine.
     auto issue_act = [&](int it) {
       const int i = s_begin + it, st = it % S;
@@ -223,10 +233,6 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
                   a.sfb + (static_cast<size_t>((m0 >> 7) + g) * a.sfb_atoms + kx / Cfg::kAtomK) * 512,
                   nat * 512, &full[st]);
     };
-    const int pre = min(n_it, S);   // the first ring fill needs no empty-slot wait
-    if (elect_one())
-      for (int it = 0; it < pre; ++it) issue_weight(it);
-    __syncwarp();
     griddep_wait();
     if (lsu_act) {
       // Every stage's activation tile (BN rows x 128 B, stored with the 128-byte swizzle) and its
