@@ -39,7 +39,7 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the timed GEMM
 # kernel, from an ncu --set full capture of that kernel (the VQ layer's M = 64 launch; the PRQuant
 # M = 2048 launch).  Set an entry to None whenever its kernel changes until it is captured again.
-NCU_TRAFFIC_PER_LAUNCH = {"vq": 11.33e6, "prquant_m2048": 24.19e6}
+NCU_TRAFFIC_PER_LAUNCH = {"vq": 11.33e6, "prquant_m2048": 24.58e6}
 
 
 def measured_peaks() -> dict:

@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
   }
   const int wtile = tile % a.tiles_n;
   const int n0 = wtile * 128, m0 = (tile / a.tiles_n) * BN;
+  const int sf_group0 = (tile / a.tiles_n) * Cfg::kG;   // first 128-row scale group of the tile
   const int s_begin = splits == 1 ? 0 : zsplit * a.stages_per_split;
   const int s_end = splits == 1 ? a.n_stages_total : min(a.n_stages_total, s_begin + a.stages_per_split);
   const int n_it = max(0, s_end - s_begin);
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
 #pragma unroll
       for (int g = 0; g < Cfg::kG; ++g)
         bulk_load(sSfb + st * Cfg::kSfbBytes + g * Cfg::kAtoms * 512,
-                  a.sfb + (static_cast<size_t>((m0 >> 7) + g) * a.sfb_atoms + kx / Cfg::kAtomK) * 512,
+                  a.sfb + (static_cast<size_t>(sf_group0 + g) * a.sfb_atoms + kx / Cfg::kAtomK) * 512,
                   nat * 512, &full[st]);
     };
     griddep_wait();
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
           const uint8_t* src = a.xq + static_cast<size_t>(in ? m0 + r : 0) * (a.C / 2) + (kx >> 1) + kc * 16;
           cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4), src, in ? 16u : 0u);
         }
-        const uint8_t* sfsrc = a.sfb + (static_cast<size_t>(m0 >> 7) * a.sfb_atoms + kx / Cfg::kAtomK) * 512;
+        const uint8_t* sfsrc = a.sfb + (static_cast<size_t>(sf_group0) * a.sfb_atoms + kx / Cfg::kAtomK) * 512;
         const uint32_t sfdst = smem_u32(sSfb + it * Cfg::kSfbBytes);
         for (int c = lane; c < nat * 32; c += 32) cp_async16(sfdst + c * 16, sfsrc + c * 16, 16u);
         cp_async_commit();

@@ -157,15 +157,27 @@ ql_status launch_fp4(int BN, const CUtensorMap& tx, const CUtensorMap& ty, const
     case 32: return launch_fp4_bn<32, E8M0, VQ>(tx, ty, ty32, a, grid, s);
     case 64: return launch_fp4_bn<64, E8M0, VQ>(tx, ty, ty32, a, grid, s);
     case 128: return launch_fp4_bn<128, E8M0, VQ>(tx, ty, ty32, a, grid, s);
+    case 160: return launch_fp4_bn<160, E8M0, VQ>(tx, ty, ty32, a, grid, s);
     case 256: return launch_fp4_bn<256, E8M0, VQ>(tx, ty, ty32, a, grid, s);
   }
   return fail(QL_ERR_UNSUPPORTED, "no GEMM tile for BN=%d", BN);
 }
 
-int pick_bn(int64_t M) {
+// Token-tile width: the smallest power of two >= M up to 128.  Past 128 tokens, 256-wide tiles,
+// unless the grid has at least one full wave of tiles either way and 160-wide tiles need no more
+// waves per unit of operand traffic (each stage streams 128 weight rows plus BN token rows): at
+// 2048 tokens x 20 weight tiles, 256 wide gives 160 tiles = 2 waves on 148 SMs, 160 wide gives
+// 260 tiles = also 2 waves with 25 % less operand traffic per tile.
+int pick_bn(int64_t M, int tiles_n) {
   for (int bn : {16, 32, 64, 128})
     if (M <= bn) return bn;
-  return 256;
+  const int64_t sms = sm_count();
+  auto cost = [&](int bn) -> int64_t {
+    const int64_t tiles = tiles_n * cdiv(M, bn);
+    return tiles < sms ? -1 : cdiv(tiles, sms) * (128 + bn);
+  };
+  const int64_t c256 = cost(256), c160 = cost(160);
+  return (c256 > 0 && c160 > 0 && c160 < c256) ? 160 : 256;
 }
 
 }  // namespace
@@ -194,6 +206,7 @@ struct FwdPlan {
   int BN, splits, spp, tiles_n, tiles_m;
   int full_tiles;   // FP4 GEMM: tiles [0, full_tiles) unsplit, the rest split `splits` ways
   int sfb_atoms;
+  int sf_rows;      // rows per token tile in the tiled activation-scale layout (>= 128)
   size_t sync_off;   // E4M3 grid quantizer: launch counter and per-CTA amax slots
   size_t codes_off, sf_off, scal_off, tick_off, part_off, total;
   int n_tickets;   // split-K tickets (zeroed by the quantizer, re-armed by the GEMM)
@@ -226,8 +239,8 @@ FwdPlan plan_forward_int4(const ql_linear* L, int64_t M) {
 FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   if (L->int4) return plan_forward_int4(L, M);
   FwdPlan p{};
-  p.BN = pick_bn(M);
   p.tiles_n = static_cast<int>(cdiv(L->N, 128));
+  p.BN = pick_bn(M, p.tiles_n);
   p.tiles_m = static_cast<int>(cdiv(std::max<int64_t>(M, 1), p.BN));
   const int tiles = p.tiles_n * p.tiles_m;
   const int total = L->n_stages_total;
@@ -246,14 +259,17 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   p.splits = static_cast<int>(cdiv(total, p.spp));
   const int atomK = L->e8m0 ? 128 : 64;  // K elements covered by one 512-byte scale atom
   p.sfb_atoms = static_cast<int>(cdiv(L->C, atomK));
-  const int64_t rows_pad = cdiv(std::max<int64_t>(M, 1), 256) * 256;
+  p.sf_rows = std::max(p.BN, 128);
+  // 128-row atom groups of the tiled activation scales: ceil(sf_rows / 128) per token tile
+  const int64_t sf_groups = std::max<int64_t>(cdiv(std::max<int64_t>(M, 1), 256) * 2,
+                                              static_cast<int64_t>(p.tiles_m) * cdiv(p.sf_rows, 128));
   size_t off = 0;
   p.sync_off = off;
   off = align_up(off + ql::kE4m3SyncBytes, 256);
   p.codes_off = off;
   off = align_up(off + static_cast<size_t>(M) * (L->C / 2), 256);
   p.sf_off = off;
-  off = align_up(off + static_cast<size_t>(rows_pad / 128) * p.sfb_atoms * 512, 256);
+  off = align_up(off + static_cast<size_t>(sf_groups) * p.sfb_atoms * 512, 256);
   // [0] amax bit pattern and [1] tensor scale of E4M3-B16 activations, then the split-K tickets
   // (one memset or the quantizer clears the whole run before the GEMM).
   p.scal_off = off;
@@ -385,7 +401,7 @@ ql_status launch_quant_int4(const void* x, int64_t M, int64_t K, int8_t* q8, uin
 
 ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
                           uint8_t* st, int st_atoms, int* zero_words, int nzero,
-                          cudaStream_t s, __nv_bfloat16* deq = nullptr) {
+                          cudaStream_t s, __nv_bfloat16* deq = nullptr, int st_rows = 128) {
   const long total = static_cast<long>(M) * (K / 32);
   const long threads = std::max<long>(total, nzero);
   if (threads == 0) return QL_OK;
@@ -394,7 +410,7 @@ ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, u
   ql::quant_mx_e8m0_b32_kernel<<<static_cast<unsigned>(grid), block, 0, s>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K),
       static_cast<int>(K), codes, static_cast<int>(K / 2), sp, static_cast<int>(K / 32), st,
-      st_atoms, zero_words, nzero, deq);
+      st_atoms, st_rows, zero_words, nzero, deq);
   QL_CUDA(cudaGetLastError());
   return QL_OK;
 }
@@ -445,7 +461,8 @@ bool e4m3_one_launch(int64_t M, int64_t K) {
 // n_tickets split-K tickets, all cleared here).  ts_out: where ts goes (may be null).
 ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
                             uint8_t* st, int st_atoms, unsigned* amax_slot, float* ts_out,
-                            cudaStream_t s, int n_tickets = 0, uint32_t* sync = nullptr) {
+                            cudaStream_t s, int n_tickets = 0, uint32_t* sync = nullptr,
+                            int st_rows = 128) {
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   int* tickets = n_tickets > 0 ? reinterpret_cast<int*>(amax_slot + 2) : nullptr;
   // Past one block per thread of a cluster, a grid of small co-resident CTAs when the caller's
@@ -469,7 +486,7 @@ ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes,
     cfg.numAttrs = 1;
     QL_CUDA(cudaLaunchKernelEx(&cfg, ql::quant_e4m3_b16_grid_kernel, xb, static_cast<int>(M),
                                static_cast<int>(K), static_cast<int>(K), amax_slot, ts_out, codes,
-                               static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms,
+                               static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms, st_rows,
                                tickets, n_tickets, sync));
     return QL_OK;
   }
@@ -490,7 +507,7 @@ ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes,
     cfg.numAttrs = 2;
     QL_CUDA(cudaLaunchKernelEx(&cfg, ql::quant_e4m3_b16_cluster_kernel, xb, static_cast<int>(M),
                                static_cast<int>(K), static_cast<int>(K), amax_slot, ts_out, codes,
-                               static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms,
+                               static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms, st_rows,
                                tickets, n_tickets));
     return QL_OK;
   }
@@ -504,7 +521,7 @@ ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes,
   const long total = static_cast<long>(M) * (K / 16);
   ql::quant_e4m3_b16_kernel<<<static_cast<unsigned>((total + block - 1) / block), block, 0, s>>>(
       xb, static_cast<int>(M), static_cast<int>(K), static_cast<int>(K), amax_slot, ts_out, codes,
-      static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms);
+      static_cast<int>(K / 2), sp, static_cast<int>(K / 16), st, st_atoms, st_rows);
   QL_CUDA(cudaGetLastError());
   return QL_OK;
 }
@@ -713,11 +730,11 @@ ql_status qlinear_quantize_input(const ql_linear* L, const void* x, int64_t M, v
     return launch_quant_e4m3(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
                              scal, reinterpret_cast<float*>(scal + 1),
                              reinterpret_cast<cudaStream_t>(stream), p.n_tickets,
-                             reinterpret_cast<uint32_t*>(w8 + p.sync_off));
+                             reinterpret_cast<uint32_t*>(w8 + p.sync_off), p.sf_rows);
   }
   return launch_quant_mx(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
                          reinterpret_cast<int*>(w8 + p.tick_off), p.n_tickets,
-                         reinterpret_cast<cudaStream_t>(stream));
+                         reinterpret_cast<cudaStream_t>(stream), nullptr, p.sf_rows);
 }
 
 ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void* ws,

@@ -38,9 +38,15 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 // Offset of scale (row m, scale column j) in the tiled scale-factor layout used by the
 // block-scaled MMA: 512-byte atoms of 128 rows x 4 scale columns, atoms ordered K-fastest;
 // inside an atom, row m sits at (m%32)*16 + ((m/32)%4)*4 and column j at j%4.
-__host__ __device__ __forceinline__ size_t sf_tiled_offset(int m, int j, int atoms_per_row) {
-  const size_t atom = static_cast<size_t>(m >> 7) * atoms_per_row + (j >> 2);
-  return atom * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
+// Rows are grouped by the GEMM's token tiles of tile_rows rows (128, 160 or 256): tile t owns
+// ceil(tile_rows / 128) consecutive 128-row atom groups, so that a tile's scales start on an atom
+// boundary whatever its first row; with tile_rows = 128 or 256 this is plain 128-row grouping.
+__host__ __device__ __forceinline__ size_t sf_tiled_offset(int m, int j, int atoms_per_row,
+                                                           int tile_rows) {
+  const int groups = (tile_rows + 127) >> 7;
+  const int t = m / tile_rows, r = m - t * tile_rows;
+  const size_t atom = static_cast<size_t>(t * groups + (r >> 7)) * atoms_per_row + (j >> 2);
+  return atom * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3);
 }
 
 // Eight E2M1 codes from eight exactly-scaled fp32 values (RNE, satfinite) via the hardware
@@ -96,7 +102,7 @@ __device__ __forceinline__ uint32_t bf16x8_sign_nibbles(const uint32_t (&w)[4]) 
 __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, uint8_t* __restrict__ codes,
     int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
-    int sf_atoms_per_row, int* __restrict__ zero_words, int nzero,
+    int sf_atoms_per_row, int sf_tile_rows, int* __restrict__ zero_words, int nzero,
     __nv_bfloat16* __restrict__ deq_out = nullptr) {
   griddep_launch_dependents();   // a GEMM launched behind this grid may start streaming weights
   const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -137,7 +143,7 @@ __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
       make_uint4(packed[0], packed[1], packed[2], packed[3]);
   const uint8_t b = static_cast<uint8_t>(e + 127);
   if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = b;
-  if (scales_tiled != nullptr) scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row)] = b;
+  if (scales_tiled != nullptr) scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row, sf_tile_rows)] = b;
   if (deq_out != nullptr) {
     uint32_t o[16];
 #pragma unroll
@@ -204,7 +210,7 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
 __device__ __forceinline__ void quant_e4m3_regs(
     const uint32_t (&w)[8], int m, int j, float ts, uint8_t* __restrict__ codes, int ldc,
     uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
-    int sf_atoms_per_row) {
+    int sf_atoms_per_row, int sf_tile_rows) {
   uint32_t mx = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
@@ -259,17 +265,17 @@ __device__ __forceinline__ void quant_e4m3_regs(
       make_uint2(packed[0], packed[1]);
   if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = static_cast<uint8_t>(sb);
   if (scales_tiled != nullptr)
-    scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row)] = static_cast<uint8_t>(sb);
+    scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row, sf_tile_rows)] = static_cast<uint8_t>(sb);
 }
 
 __device__ __forceinline__ void quant_e4m3_block(
     const __nv_bfloat16* __restrict__ x, int m, int j, int ldx, float ts, uint8_t* __restrict__ codes,
     int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
-    int sf_atoms_per_row) {
+    int sf_atoms_per_row, int sf_tile_rows) {
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * ldx) + j * 2;
   const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
   const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-  quant_e4m3_regs(w, m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+  quant_e4m3_regs(w, m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row, sf_tile_rows);
 }
 
 // One thread per 16-element block, tensor scale from the amax that absmax_bf16_kernel reduced.
@@ -278,7 +284,7 @@ __global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, const unsigned* __restrict__ amax16,
     float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
     uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
-    int sf_atoms_per_row) {
+    int sf_atoms_per_row, int sf_tile_rows) {
   griddep_launch_dependents();   // a GEMM launched behind this grid may start streaming weights
   const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const float ts = tensor_scale_from_amax16(*amax16);
@@ -287,7 +293,7 @@ __global__ void __launch_bounds__(256) quant_e4m3_b16_kernel(
   if (gtid >= static_cast<long>(M) * nblk) return;
   const int m = static_cast<int>(gtid / nblk);
   const int j = static_cast<int>(gtid - static_cast<long>(m) * nblk);
-  quant_e4m3_block(x, m, j, ldx, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+  quant_e4m3_block(x, m, j, ldx, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row, sf_tile_rows);
 }
 
 // Small tensors (decode): one thread-block cluster does the whole job in one launch.  Each thread
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(kE4m3ClusterThreads) quant_e4m3_b16_cluster_ke
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, unsigned* __restrict__ amax_out,
     float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
     uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
-    int sf_atoms_per_row, int* __restrict__ zero_words, int nzero) {
+    int sf_atoms_per_row, int sf_tile_rows, int* __restrict__ zero_words, int nzero) {
   griddep_launch_dependents();
   griddep_wait();
   __shared__ uint32_t red[kE4m3ClusterThreads / 32];
@@ -359,7 +365,7 @@ __global__ void __launch_bounds__(kE4m3ClusterThreads) quant_e4m3_b16_cluster_ke
     if (b < total) {
       const int m = static_cast<int>(b / nblk);
       const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
-      quant_e4m3_regs(w[k], m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+      quant_e4m3_regs(w[k], m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row, sf_tile_rows);
     }
   }
 }
@@ -406,7 +412,7 @@ __global__ void __launch_bounds__(kE4m3GridThreads) quant_e4m3_b16_grid_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, unsigned* __restrict__ amax_out,
     float* __restrict__ ts_out, uint8_t* __restrict__ codes, int ldc,
     uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
-    int sf_atoms_per_row, int* __restrict__ zero_words, int nzero, uint32_t* __restrict__ sync) {
+    int sf_atoms_per_row, int sf_tile_rows, int* __restrict__ zero_words, int nzero, uint32_t* __restrict__ sync) {
   griddep_launch_dependents();
   griddep_wait();
   __shared__ uint32_t red[kE4m3GridThreads / 32];
@@ -488,7 +494,7 @@ __global__ void __launch_bounds__(kE4m3GridThreads) quant_e4m3_b16_grid_kernel(
     if (b < total) {
       const int m = static_cast<int>(b / nblk);
       const int j = static_cast<int>(b - static_cast<long>(m) * nblk);
-      quant_e4m3_regs(w[k], m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row);
+      quant_e4m3_regs(w[k], m, j, ts, codes, ldc, scales_plain, lds, scales_tiled, sf_atoms_per_row, sf_tile_rows);
     }
   }
 }

@@ -197,10 +197,11 @@ def test_gemm_repeat_without_requantize(M):
     lin.close()
 
 
-@pytest.mark.parametrize("N,K,M", [(2560, 2048, 300), (1280, 4096, 520), (2048, 1024, 2048)])
+@pytest.mark.parametrize("N,K,M", [(2560, 2048, 300), (1280, 4096, 520), (2048, 1024, 2048),
+                                   (2560, 1024, 2000)])
 def test_fp4_gemm_prefill_shapes(N, K, M):
     """Prefill shapes: 256-token tiles, split-K across a few CTAs where the tiles alone do not fill
-    the SMs, ragged token tiles."""
+    the SMs, ragged token tiles; 2560 x 2000 runs ragged 160-token tiles."""
     codes, sb = random_mx_weight(23, N, K)
     xb, _ = synth.activations_bf16(23, M, K, 0.01, 20.0)
     check_linear(codes, sb, 0, xb, f"prefill N={N} K={K} M={M}")

@@ -127,10 +127,13 @@ def test_vq_workload_full_size(M):
     check_bf16(y, ref, t, f"C2 M={M}")
 
 
-def test_nvfp4_weight_linear_prefill():
-    """E4M3-B16 weights at a prefill shape (256-token tiles, split-K)."""
+@pytest.mark.parametrize("M", [300, 2048])
+def test_nvfp4_weight_linear_prefill(M):
+    """E4M3-B16 weights at prefill shapes: M = 300 runs 256-token tiles split along K; M = 2048
+    runs 160-token tiles (260 tiles, two full waves), whose activation scales are grouped per
+    160-row tile."""
     ql = _ql()
-    N, K, M = 2560, 2048, 300
+    N, K = 2560, 2048
     codes = synth.uniform_nibble_bytes(60, N, K)
     sb = synth.uniform_bytes(61, (N, K // 16), 0x28, 0x48)
     ts_w = np.float32(0.0123)
@@ -145,10 +148,11 @@ def test_nvfp4_weight_linear_prefill():
     check_bf16(y, ref, t, "nvfp4 prefill")
 
 
-@pytest.mark.parametrize("M", [300, 16])
+@pytest.mark.parametrize("M", [300, 16, 2048])
 def test_vq_linear_random_codebooks(M):
     """VQ weights with random indices, codebooks and scales at N = 2560, K = 2048: M = 300 as a
-    prefill tile, M = 16 as split-K with the decode running ahead of the activation quantizer."""
+    prefill tile, M = 16 as split-K with the decode running ahead of the activation quantizer,
+    M = 2048 as 160-token tiles."""
     g = np.random.default_rng(70 + M)
     N, K = 2560, 2048
     cb = g.integers(0, 16, (N // 64, K // 64, 256, 4), dtype=np.uint8)
