@@ -145,7 +145,7 @@ ql_status qlinear_gemm(const ql_linear* layer, int64_t M, void* y_bf16, float* y
 /* qlinear_forward without a caller-supplied workspace, for callers that cannot allocate device
  * memory (an engine that plans all device memory ahead and forbids allocation during a forward,
  * a plugin whose host exposes no allocator, a latency-critical loop that must not enter the
- * allocator).  The paper has no counterpart to this call; it is a packaging convenience.
+ * allocator).  No step of the method corresponds to this call; it is a packaging convenience.
  * The workspace is a fixed 8 MiB array inside the library (each GPU that loads the library keeps
  * it until the process exits); M whose qlinear_workspace_bytes exceeds 8 MiB is rejected with
  * QL_ERR_WORKSPACE.  Nothing is allocated: no cudaMalloc/cudaFree, no library allocator.
