@@ -122,8 +122,14 @@ ql_status qlinear_workspace_bytes(const ql_linear* layer, int64_t M, size_t* byt
 
 /* y[M,N] = X[M, K-k_tail] (quantized online) times the layer's weight.  x_bf16, y_bf16 and
  * the workspace are device pointers; y_f32 (device, [M,N]) may be NULL.  ws must be 256-byte
- * aligned and at least qlinear_workspace_bytes(M) long; its contents on entry do not matter.
- * Rows of x are contiguous (row stride K - k_tail elements).  M may be 0 (no-op). */
+ * aligned and at least qlinear_workspace_bytes(M) long; its contents on entry do not matter
+ * (the E4M3-B16 grid quantizer agrees on the tensor amax through words of the workspace that
+ * carry a per-launch tag, so they need no clearing; after a device timeout reported by
+ * ql_check, discard the workspace).  Calls that share a workspace must be stream-ordered.
+ * Rows of x are contiguous (row stride K - k_tail elements).  M may be 0 (no-op).
+ * Kernels are launched with programmatic stream serialization and release the next such grid
+ * at once: a following qlinear call on the stream may start streaming its weights while this
+ * one finishes, and reads this call's results only after it has completed. */
 ql_status qlinear_forward(const ql_linear* layer, const void* x_bf16, int64_t M, void* y_bf16,
                           float* y_f32, void* ws, size_t ws_bytes, ql_stream_t stream);
 
