@@ -268,6 +268,7 @@ def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes:
     forward call from pinned host memory with the copies inside the timed region."""
     import torch
     import bit_quantized_moe_tcgen05_b200 as ql
+    steps = max(1, steps)
     R = 1 if flush_bytes else min(64, L2_BYTES // w["weight_bytes"] + 2)
     layers = [w["make"]() for _ in range(R)]
     Ms = w["Ms"]
@@ -275,6 +276,9 @@ def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes:
     ys = {M: torch.empty((M, w["N"]), dtype=torch.bfloat16, device=device) for M in Ms}
     wss = {M: torch.empty(layers[0].workspace_bytes(M), dtype=torch.uint8, device=device) for M in Ms}
     flush_buf = torch.empty(flush_bytes, dtype=torch.uint8, device=device) if flush_bytes else None
+    # rotation mode: one write larger than L2 before each timed region, so that a short run
+    # (fewer steps than weight copies) starts from cold weights as well
+    evict_buf = None if flush_bytes else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
 
     def fwd(layer, M):
         layer.quantize_input(xs[M], wss[M])
@@ -299,22 +303,47 @@ def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes:
         for layer in layers:
             for M in Ms:
                 layer.gemm(M, ys[M], wss[M])
-    for g in (g_all, g_q, g_g):
-        for _ in range(warmup):
-            g.replay()
+    # Exactly `steps` steps are timed: `full` replays of the R-layer graphs, then one replay of a
+    # graph over the first `part` layers.
+    full, part = divmod(steps, R)
+    p_all = p_q = p_g = None
+    if part:
+        p_all, p_q, p_g = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(p_all):
+            for layer in layers[:part]:
+                for M in Ms:
+                    fwd(layer, M)
+        with torch.cuda.graph(p_q):
+            for layer in layers[:part]:
+                for M in Ms:
+                    layer.quantize_input(xs[M], wss[M])
+        with torch.cuda.graph(p_g):
+            for layer in layers[:part]:
+                for M in Ms:
+                    layer.gemm(M, ys[M], wss[M])
+    for g in (g_all, g_q, g_g, p_all, p_q, p_g):
+        if g is not None:
+            for _ in range(warmup):
+                g.replay()
     ql.check()
-    reps = max(1, -(-steps // R))                    # graph replays so that >= steps steps run
 
-    def timed(graph):
+    def timed(graph, pgraph):
         if flush_buf is None:
-            return _elapsed(graph.replay, reps, stream) / (reps * R)
-        tot = 0.0
-        for _ in range(reps):
+            def run():
+                for _ in range(full):
+                    graph.replay()
+                if pgraph is not None:
+                    pgraph.replay()
+            evict_buf.fill_(1)
+            return _elapsed(run, 1, stream) / steps
+        tot = 0.0                                     # R == 1: one flushed replay per step
+        for _ in range(steps):
             flush_buf.fill_(1)
             tot += _elapsed(graph.replay, 1, stream)
-        return tot / (reps * R)
+        return tot / steps
 
-    out = dict(R=R, step_ms=timed(g_all), quant_ms=timed(g_q), gemm_ms=timed(g_g), steps=reps * R)
+    out = dict(R=R, step_ms=timed(g_all, p_all), quant_ms=timed(g_q, p_q),
+               gemm_ms=timed(g_g, p_g), steps=steps)
     ql.check()
     if e2e:
         xh = {M: torch.from_numpy(w["xs"][M].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -333,11 +362,11 @@ def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes:
 
         for _ in range(warmup):
             e2e_step()
-        out["e2e_ms"] = _elapsed(e2e_step, reps * R, stream) / (reps * R)
+        out["e2e_ms"] = _elapsed(e2e_step, steps, stream) / steps
         out["h2d"] = sum(M * w["C"] * 2 for M in Ms)
         out["d2h"] = sum(M * w["N"] * 2 for M in Ms)
         ql.check()
-    del g_all, g_q, g_g
+    del g_all, g_q, g_g, p_all, p_q, p_g
     for layer in layers:
         layer.close()
     return out
