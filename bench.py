@@ -247,6 +247,25 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------------------------ ranks
+def max_over_ranks(vals, device):
+    """Element-wise maximum of a list of floats over all ranks of the default process group (the
+    slowest rank's device times); the list itself when there is no group or a single rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_throughput(units_per_step_per_rank: float, world: int, step_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own units each step (replicas), and the
+    step takes as long as the slowest rank."""
+    return world * units_per_step_per_rank / (step_ms * 1e-3)
+
+
 # ------------------------------------------------------------------------------ GPU arm
 def _elapsed(fn, reps: int, stream) -> float:
     """Device time (ms) of `reps` calls of fn, bracketed by synchronisation and CUDA events."""
@@ -487,15 +506,10 @@ def main():
         res = run_case(head, args.steps, args.warmup, device, e2e=True,
                        flush_bytes=0 if decode else 256 << 20)
     barrier()
-    step_ms, e2e_ms = res["step_ms"], res["e2e_ms"]
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([step_ms, e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, e2e_ms = float(t[0]), float(t[1])
+    step_ms, e2e_ms = max_over_ranks([res["step_ms"], res["e2e_ms"]], device)
     units = per_step_units(head)
-    value = world * units / (step_ms * 1e-3)
-    e2e_val = world * units / (e2e_ms * 1e-3)
+    value = job_throughput(units, world, step_ms)
+    e2e_val = job_throughput(units, world, e2e_ms)
 
     fp4_peak = peaks["bf16"] * NOMINAL_FP4_OVER_BF16
     nl = len(head["Ms"])
@@ -518,7 +532,7 @@ def main():
                     "peak_source": f"{peaks['src']} bf16 burst {peaks['bf16']} x 4 (nominal FP4/bf16)"}
 
     cases = {}
-    if args.cases == "all":
+    if args.cases == "all" and world == 1:
         int4_4096 = make_int4(4096)
         int4_cases = [dict(int4_4096, name=int4_4096["name"].replace("_m4096", f"_m{M}"), Ms=[M],
                            xs={M: np.ascontiguousarray(int4_4096["xs"][4096][:M])})
@@ -553,7 +567,11 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
-    kernels_per_fwd = 3 if head["kind"] == "vq" else 2
+    # library kernels per forward: the activation quantizer and the GEMM (E4M3-B16 activations
+    # past the one-launch quantizers' capacity take an amax kernel and a quantize kernel)
+    def kernels_per_fwd(M):
+        one_launch_cap = 3 * 256 * 148 * 16
+        return 3 if head["kind"] == "vq" and M * head["C"] > one_launch_cap else 2
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": res["steps"],
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -563,12 +581,12 @@ def main():
         "data": "synthetic", "config": config, "roofline": roofline,
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
-        "gpu_launches": kernels_per_fwd * nl * res["steps"],
+        "gpu_launches": sum(kernels_per_fwd(M) for M in head["Ms"]) * res["steps"],
         "clocks": clk.summary(),
         "kernel_us_per_step": {"quantize": res["quant_ms"] * 1e3, "gemm": res["gemm_ms"] * 1e3},
         "cases": cases,
     }
-    if not args.no_cpu_baseline and head["kind"] == "vq":
+    if not args.no_cpu_baseline and head["kind"] == "vq" and world == 1:
         line["cpu_baseline"] = cpu_baseline_vq(head)
     print(json.dumps(line))
 
