@@ -12,8 +12,9 @@
 // channels are read a second time for the tail stages (activation coordinate C - k + j while
 // the weight coordinate is C + j).  No tail copy is materialised.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer (one
-// lane issues), warps 2..5 = (VQ weights: codebook decode, then) epilogue.  A STAGES-deep ring of
+// Warp roles (192 threads; 320 for VQ weights): warp 0 = TMA producer, warp 1 = TMEM allocator +
+// MMA issuer (one lane issues), warps 2..5 = epilogue; with VQ weights warps 2..9 first rebuild
+// each stage's operand tile from the codebooks.  A STAGES-deep ring of
 // shared-memory stages, each 256 K-elements deep, is guarded by full/empty mbarriers; MMA
 // completion is signalled by tcgen05.commit.  Every wait is bounded (see ptx.cuh).
 //
@@ -30,8 +31,9 @@
 //
 // Work: a 1-D grid.  Tiles (128 weight rows x BN tokens, weight tile fastest) [0, full_tiles) get
 // one CTA each over all K; the remaining tiles are split along K over `splits` CTAs each.
-// Decode launches split every tile (full_tiles = 0) so that the grid covers the SMs; prefill
-// launches whose tiles overfill the last wave split only that wave's leftover tiles.  The K-splits
+// Decode launches split every tile (full_tiles = 0) so that the grid covers the SMs; launches with
+// at least a wave of tiles run them all unsplit (the kernel also accepts whole tiles followed by
+// split ones, which measured slower for the leftover tiles of the last wave).  The K-splits
 // of a tile each write an fp32 partial tile to a global workspace; the last split to finish (an
 // atomic ticket per tile) bulk-copies the partials into its idle ring and adds them in split
 // order, so the result is deterministic, writes y and re-arms the ticket.
