@@ -9,8 +9,10 @@ batch sizes M = 1, 8 and 64.  Metric: weight-stream GB/s = weight bytes streamed
 step) / step time, whole job.  Launches are replayed from CUDA graphs; each step uses the next of
 R weight copies whose total exceeds the 126 MB L2, so every pass streams from HBM.
 
-Extra cases: the PRQuant tail-residual layer at M = 2048 (prefill, TFLOP/s), 512 and 16, and the
-single MXFP4 layer at M = 16.
+Extra cases (one GPU only): the PRQuant tail-residual layer at M = 2048 (prefill, TFLOP/s), 512
+and 16; the single MXFP4 layer at M = 16; the INT4 dense + block-sparse residual layer at
+M = 4096, 256, 16 and 1; and the routed MoE FFN (128 experts, top-8, 2048 tokens).  Exactly
+`--steps` steps are timed for the headline.
 
 Multi-GPU: the layer shards into independent replicas (no collective); each rank runs the same
 workload on its own GPU and `value` sums the ranks' work over the slowest rank's time.
