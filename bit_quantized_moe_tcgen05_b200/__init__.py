@@ -34,7 +34,7 @@ EXPORTED_SYMBOLS = (
     "qlinear_quantize_input", "qlinear_gemm", "qlinear_forward_fixed_scratch",
     "qlinear_prepare_vq_prescale", "moe_create", "moe_destroy", "moe_capture_intermediate",
     "moe_workspace_bytes", "moe_workspace_layout", "moe_grouped_forward",
-    "qlinear_prepare_int4_bsr",
+    "qlinear_prepare_int4_bsr", "ql_tensor_peak",
 )
 
 
@@ -93,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "moe_grouped_forward": [vp, vp, i64, vp, vp, vp, vp, vp, vp, sz, vp],
         "qlinear_prepare_int4_bsr": [vp, i64, i64, vp, i64, ctypes.c_float, vp, vp, vp, vp, vp, vp,
                                      i32, vp],
+        "ql_tensor_peak": [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_double), vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)

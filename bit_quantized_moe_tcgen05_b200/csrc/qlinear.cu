@@ -19,6 +19,7 @@
 #include "gemm_fp4.cuh"
 #include "moe.cuh"
 #include "int4_gemm.cuh"
+#include "peak.cuh"
 
 namespace {
 
@@ -526,6 +527,18 @@ ql_status launch_quant_e4m3(const void* x, int64_t M, int64_t K, uint8_t* codes,
   return QL_OK;
 }
 
+// Tensor-pipe peak probe (measurement only).
+template <int KIND, int N>
+ql_status launch_peak(int ctas, int iters, cudaStream_t s, double* flops) {
+  using Cfg = ql::PeakCfg<KIND, N>;
+  auto k = ql::tensor_peak_kernel<KIND, N>;
+  QL_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem));
+  k<<<ctas, 128, Cfg::kSmem, s>>>(iters);
+  QL_CUDA(cudaGetLastError());
+  if (flops != nullptr)
+    *flops = Cfg::kFlopsPerMma * Cfg::kMmaPerTile * static_cast<double>(iters) * ctas;
+  return QL_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -860,6 +873,24 @@ ql_status quantize_act(ql_aformat fmt, const void* x, int64_t M, int64_t K, void
                                static_cast<float*>(scales), nullptr, 0, s);
     default:
       return fail(QL_ERR_UNSUPPORTED, "activation format %d not supported", int(fmt));
+  }
+}
+
+ql_status ql_tensor_peak(int32_t kind, int32_t n, int32_t iters, int32_t ctas,
+                         double* flops_per_launch, ql_stream_t stream) {
+  if (iters <= 0 || ctas <= 0 || ctas > 4096) return fail(QL_ERR_INVALID_ARG, "iters/ctas");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int key = kind * 1000 + n;
+  switch (key) {
+    case 0 * 1000 + 128: return launch_peak<0, 128>(ctas, iters, s, flops_per_launch);
+    case 0 * 1000 + 256: return launch_peak<0, 256>(ctas, iters, s, flops_per_launch);
+    case 1 * 1000 + 128: return launch_peak<1, 128>(ctas, iters, s, flops_per_launch);
+    case 1 * 1000 + 256: return launch_peak<1, 256>(ctas, iters, s, flops_per_launch);
+    case 2 * 1000 + 128: return launch_peak<2, 128>(ctas, iters, s, flops_per_launch);
+    case 2 * 1000 + 256: return launch_peak<2, 256>(ctas, iters, s, flops_per_launch);
+    case 3 * 1000 + 128: return launch_peak<3, 128>(ctas, iters, s, flops_per_launch);
+    case 3 * 1000 + 256: return launch_peak<3, 256>(ctas, iters, s, flops_per_launch);
+    default: return fail(QL_ERR_UNSUPPORTED, "tensor peak kind %d with N %d", int(kind), int(n));
   }
 }
 

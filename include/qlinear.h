@@ -179,6 +179,17 @@ ql_status qlinear_forward_fixed_scratch(const ql_linear* layer, const void* x_bf
 ql_status quantize_act(ql_aformat fmt, const void* x_bf16, int64_t M, int64_t K, void* codes,
                        void* scales, float* tensor_scale, ql_stream_t stream);
 
+/* Tensor-pipe throughput probe (measurement only; no step of the method).  Launches `ctas` CTAs
+ * (one per SM at most is useful) that each issue iters x 4 back-to-back tcgen05.mma instructions
+ * of one kind (kind 0: kind::mxf4.block_scale.block32; 1: kind::mxf4nvf4.block_scale.block16;
+ * 2: kind::i8; 3: kind::f16 with bf16 operands) with M = 128 and N = n (128 or 256) on operands
+ * resident in shared memory, into one TMEM accumulator; *flops_per_launch (host, may be NULL)
+ * receives 2 * 128 * n * K_mma * 4 * iters * ctas.  The caller times the launch on `stream`
+ * (CUDA events); the quotient is the peak a GEMM of that kind can approach on this GPU, the
+ * denominator of its roofline.  Asynchronous; nothing is read back. */
+ql_status ql_tensor_peak(int32_t kind, int32_t n, int32_t iters, int32_t ctas,
+                         double* flops_per_launch, ql_stream_t stream);
+
 /* Synchronise `stream` and report (then clear) the device error word. */
 ql_status ql_check(ql_stream_t stream);
 

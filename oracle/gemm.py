@@ -6,20 +6,73 @@ inference": one MXFP4 GEMM over the quantized operands; MXCode abstract: MX-nati
 operands).  The dequantized operands are exact in float64, each product is exact, and the
 float64 sum is within K * 2^-53 relative of the exact sum, far inside the float tolerance.
 
+The sum itself is a plain C loop (``gemm_sum.c``): one running float64 total per element, terms
+added in ascending k, no blocking and no library matmul, so its rounding order is the one written
+here and not a BLAS kernel's.  The C file is compiled with gcc on first use (or by the package's
+build step) into ``oracle/_build/``; it shares nothing with the CUDA library.
+
 The tolerance scale t[m, n] = sum_k |deq x[m,k] * deq w[n,k]| bounds an fp32-accumulated
 result: |y_gpu - y| <= 1e-5 * t per element before the bf16 cast.
 """
 from __future__ import annotations
 
+import ctypes
+import os
+import subprocess
+
 import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gemm_sum.c")
+_LIB = os.path.join(_HERE, "_build", "liboracle_gemm.so")
+_lib = None
+
+
+def build_c(force: bool = False) -> str:
+    """Compile gemm_sum.c (gcc, -O2, OpenMP, no fused multiply-add) if it is newer than the
+    library; return the library path."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    os.makedirs(os.path.dirname(_LIB), exist_ok=True)
+    tmp = f"{_LIB}.{os.getpid()}.tmp"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-shared",
+                    "-fPIC", "-o", tmp, _SRC, "-lm"], check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _c():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build_c())
+        L.oracle_gemm_nt.restype = None
+        L.oracle_gemm_nt.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_void_p] * 4
+        _lib = L
+    return _lib
+
+
+def gemm_with_scale(xdeq: np.ndarray, wdeq: np.ndarray, want_scale: bool = True):
+    """(y, t): y = sum_k x[m,k] w[n,k] and t = sum_k |x[m,k] w[n,k]|, each summed in ascending k
+    in float64.  x [M, K], w [N, K]."""
+    x = np.ascontiguousarray(xdeq, dtype=np.float64)
+    w = np.ascontiguousarray(wdeq, dtype=np.float64)
+    assert x.ndim == 2 and w.ndim == 2 and x.shape[1] == w.shape[1]
+    M, K = x.shape
+    N = w.shape[0]
+    y = np.empty((M, N))
+    t = np.empty((M, N)) if want_scale else None
+    if M and N:
+        _c().oracle_gemm_nt(M, N, K, x.ctypes.data, w.ctypes.data, y.ctypes.data,
+                            t.ctypes.data if t is not None else None)
+    return y, t
 
 
 def gemm_ref(xdeq: np.ndarray, wdeq: np.ndarray) -> np.ndarray:
-    return np.asarray(xdeq, np.float64) @ np.asarray(wdeq, np.float64).T
+    return gemm_with_scale(xdeq, wdeq, want_scale=False)[0]
 
 
 def abs_scale(xdeq: np.ndarray, wdeq: np.ndarray) -> np.ndarray:
-    return np.abs(np.asarray(xdeq, np.float64)) @ np.abs(np.asarray(wdeq, np.float64)).T
+    return gemm_with_scale(xdeq, wdeq)[1]
 
 
 def naive_gemm(xdeq: np.ndarray, wdeq: np.ndarray) -> np.ndarray:

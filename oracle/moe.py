@@ -16,6 +16,7 @@ from __future__ import annotations
 import numpy as np
 
 from . import formats as F
+from . import gemm as G
 from . import mx
 
 
@@ -28,7 +29,10 @@ def route(logits: np.ndarray, k: int) -> dict:
     ids = order[:, :k].astype(np.int64)
     sel = np.take_along_axis(logits.astype(np.float64), ids, axis=1)
     ex = np.exp(sel - sel.max(axis=1, keepdims=True))
-    gates = ex / ex.sum(axis=1, keepdims=True)
+    den = np.zeros((T, 1))
+    for s in range(k):                                   # the k terms summed in slot order
+        den[:, 0] += ex[:, s]
+    gates = ex / den
     counts = np.bincount(ids.reshape(-1), minlength=E)
     offsets = np.concatenate([[0], np.cumsum(counts)])
     entries = np.argsort(ids.reshape(-1), kind="stable")
@@ -59,8 +63,7 @@ def gate_up(xq: np.ndarray, r: dict, Wgu: list, I: int, k: int) -> tuple[np.ndar
             continue
         t = r["entries"][a:b] // k
         W = Wgu[e]
-        y = xq[t] @ W.T
-        ya = np.abs(xq[t]) @ np.abs(W).T
+        y, ya = G.gemm_with_scale(xq[t], W)
         g[a:b], u[a:b] = y[:, :I], y[:, I:]
         tg[a:b], tu[a:b] = ya[:, :I], ya[:, I:]
     return g, u, swiglu(g, u), tg, tu
@@ -77,8 +80,7 @@ def down_combine(hq: np.ndarray, r: dict, Wd: list, T: int, k: int) -> tuple[np.
         if a == b:
             continue
         f = r["entries"][a:b]
-        ys[f] = hq[a:b] @ Wd[e].T
-        ts[f] = np.abs(hq[a:b]) @ np.abs(Wd[e]).T
+        ys[f], ts[f] = G.gemm_with_scale(hq[a:b], Wd[e])
     g = r["gates"].reshape(-1, 1)
     ys = (ys * g).reshape(T, k, H)
     ts = (ts * np.abs(g)).reshape(T, k, H)

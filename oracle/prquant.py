@@ -15,6 +15,7 @@ from __future__ import annotations
 
 import numpy as np
 
+from . import gemm as G
 from . import mx
 
 
@@ -77,4 +78,4 @@ def forward(xp: np.ndarray, prep: dict, k: int) -> tuple[np.ndarray, np.ndarray]
     xc, xs = quantize_activation_augmented(xp, k)
     xd = mx.dequant_e8m0_b32(xc, xs)
     wd = mx.dequant_e8m0_b32(prep["w_codes"], prep["w_sb"])
-    return xd @ wd.T, np.abs(xd) @ np.abs(wd).T
+    return G.gemm_with_scale(xd, wd)

@@ -22,6 +22,7 @@ from __future__ import annotations
 import numpy as np
 
 from . import formats as F
+from . import gemm as G
 from . import mx
 
 
@@ -99,4 +100,4 @@ def forward(x: np.ndarray, prep: dict, codebooks: np.ndarray) -> tuple[np.ndarra
     xc, xs, xts = mx.quantize_e4m3_b16(np.asarray(x, dtype=np.float32))
     xd = mx.dequant_e4m3_b16(xc, xs, xts)
     wd = dequant_weight(prep["idx"], codebooks, prep["sb"], prep["ts"])
-    return xd @ wd.T, np.abs(xd) @ np.abs(wd).T
+    return G.gemm_with_scale(xd, wd)

@@ -50,6 +50,27 @@ def test_quant_e4m3_b16_edge_values():
     _check_quant(synth.to_bf16_bits(g.standard_normal((4, 256)) * 10.0 ** g.uniform(-30, 30, (4, 1))))
 
 
+def test_quant_e4m3_b16_golden_blocks():
+    """The hand-worked E4M3-B16 blocks (MXCode Table 1, row E4M3-B16-FP4; every value bf16) through
+    the GPU quantizer: tensor scale, block bytes and codes equal the worked values."""
+    import json
+    import os
+    from tests.conftest import GOLDEN
+    with open(os.path.join(GOLDEN, "e4m3_b16_blocks.json")) as f:
+        g = json.load(f)["tensor"]
+    num = lambda s: float.fromhex(s) if "0x" in s else float(s)
+    x = np.array([[num(v) for blk in g["blocks"] for v in blk["x"]]])
+    xb = synth.to_bf16_bits(x)
+    assert np.array_equal(synth.bf16_bits_to_f64(xb), x)            # every input is a bf16 value
+    ql = _ql()
+    codes, sb, ts = ql.quantize_act(dev_bf16(xb), fmt=ql.QL_A_FP4_E4M3_B16_TS)
+    ql.check()
+    assert ts.cpu().numpy()[0] == np.float32(num(g["ts"]))
+    want_codes = np.array([[c for blk in g["blocks"] for c in blk["codes"]]], np.uint8)
+    assert sb.cpu().numpy()[0].tolist() == [blk["byte"] for blk in g["blocks"]]
+    assert np.array_equal(codes.cpu().numpy(), F.pack_nibbles(want_codes))
+
+
 def _run(lin, xb):
     x = dev_bf16(xb)
     y32 = torch.empty((x.shape[0], lin.N), dtype=torch.float32, device="cuda")

@@ -62,6 +62,27 @@ def test_single_expert_top1_is_the_dense_gated_ffn():
     np.testing.assert_allclose(res["out"], want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
 
 
+def test_gate_rows_come_first():
+    """PRQuant Eq. (1) gives the gated FFN h = act(g) * u; the fused gate/up weight holds the gate
+    rows first (reading: rows 0..I-1 gate, I..2I-1 up).  With a one-hot input the two GEMMs pick
+    out one centroid each: every gate row is -40 and every up row +40, so g = -40 and u = 40
+    exactly and h = SiLU(-40) * 40 = -1600 / (1 + e^40), about -6.8e-15.  The other row order
+    would give SiLU(40) * (-40), about -1600."""
+    H, I = 64, 32
+    bits = lambda v: synth.to_bf16_bits(np.full((1, 16), v))
+    cent = np.concatenate([np.repeat(bits(-40.0), I, 0), np.repeat(bits(40.0), I, 0)])
+    idx = np.zeros((2 * I, H), np.uint8)
+    Wgu = [moe.cluster_weight(cent, idx)]
+    Wd = [moe.cluster_weight(np.repeat(bits(1.0), H, 0), np.zeros((H, I), np.uint8))]
+    x = np.zeros((1, H))
+    x[0, 0] = 1.0                                        # MXFP4: amax 1, code 4 * 2^-2 = 1 exactly
+    res = moe.forward(x, np.zeros((1, 1), np.float32), Wgu, Wd, 1)
+    assert np.all(res["g"] == -40.0) and np.all(res["u"] == 40.0)
+    want = -1600.0 / (1.0 + np.exp(40.0))
+    np.testing.assert_allclose(res["h"], want, rtol=1e-12)
+    assert np.all(np.abs(res["h"]) < 1e-13)
+
+
 def test_expert_relabeling_invariance():
     E, H, I, T, k = 4, 64, 32, 10, 2
     Wgu, Wd, x = _model(6, E, H, I, T)

@@ -55,6 +55,21 @@ def test_mx_dequant_error_bound():
     assert np.all(err[a <= 6] <= half_step[a <= 6] + 1e-12)
 
 
+def test_e4m3_b16_golden_blocks():
+    """Hand-worked E4M3-B16 blocks (MXCode Table 1, row E4M3-B16-FP4) that tell the binary32 step
+    order apart from the plausible alternatives (6*ts formed first, one rounding of
+    amax/(6*ts), division by ts before 6, the block scale or the quotient taken in float64) and
+    drive x/S onto every E2M1 tie, a subnormal block scale and a scale that underflows."""
+    with open(os.path.join(GOLDEN, "e4m3_b16_blocks.json")) as f:
+        g = json.load(f)["tensor"]
+    x = np.array([[_num(v) for blk in g["blocks"] for v in blk["x"]]], dtype=np.float32)
+    codes, sb, ts = mx.quantize_e4m3_b16(x)
+    assert ts == np.float32(_num(g["ts"]))
+    for i, blk in enumerate(g["blocks"]):
+        assert int(sb[0, i]) == blk["byte"], blk["note"]
+        assert codes[0, 16 * i:16 * i + 16].tolist() == blk["codes"], blk["note"]
+
+
 def test_e4m3_b16_invariants():
     g = np.random.default_rng(3)
     x = (g.standard_normal((16, 256)) * 3).astype(np.float32)

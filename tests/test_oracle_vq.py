@@ -41,6 +41,24 @@ def test_prescale_scales_equal_the_e4m3_b16_rule():
     assert ts == np.float32(np.float32(np.abs(w).max()) / np.float32(2688.0))
 
 
+def test_normalized_golden():
+    """Hand-worked PreScale normalisation v = w / RN(dec(s) * ts) (MXCode abstract, Table 1):
+    values chosen so that dividing by the two scales one after the other, multiplying by the
+    reciprocal, or dividing in float64 would each give a different binary32 result; an all-zero
+    block (scale byte 0) gives v = 0."""
+    with open(os.path.join(GOLDEN, "vq_normalized.json")) as f:
+        g = json.load(f)
+    num = lambda s: float.fromhex(s) if "0x" in s else float(s)
+    w = np.array([[num(v) for v in g["w"]]], dtype=np.float32)
+    ts, sb = vq.prescale(w)
+    assert ts == np.float32(num(g["ts"])) and sb[0].tolist() == g["bytes"]
+    v = vq.normalized(w, sb, ts)
+    assert v.dtype == np.float32
+    for k, want in g["v"].items():
+        assert v[0, int(k)] == np.float32(num(want)), k
+    assert np.all(v[0, 16:32] == 0) and np.all(v[0, 35:] == 0) and np.all(v[0, 1:16] == 0)
+
+
 def test_assignment_bruteforce_tiny():
     """Nearest entry by explicit loops over every entry, first minimum wins."""
     g = np.random.default_rng(9)
