@@ -60,23 +60,41 @@ def _pack_nibbles(c: np.ndarray) -> np.ndarray:
     return ((c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)).astype(np.uint8)
 
 
-def make_vq(Ms=(1, 8, 64), seed: int = 2) -> dict:
-    """MXCode-style VQ layer: W [2560, 9728] Student-t(4) -> PreScale E4M3-B16 scales + FP32
-    tensor scale (library host preparation), seeded k-means FP4 codebooks per 64x64 QBlock
-    (256 entries of d = 4), 8-bit indices; X [M, 9728] N(0,1) for each M."""
+def _vq_weights(seed: int):
+    """W [2560, 9728] Student-t(4) as bf16 bits and its seeded k-means FP4 codebooks per 64x64
+    QBlock (256 entries of d = 4), data synthesis only."""
     import synth
-    import bit_quantized_moe_tcgen05_b200 as ql
     N, K = 2560, 9728
     wb = synth.to_bf16_bits(synth.student_t(seed, (N, K), 4.0))
-    cb = _pack_nibbles(synth.vq_codebooks(seed, synth.bf16_bits_to_f64(wb)))
-    ts, sb, idx = ql.prepare_vq_prescale(wb, cb)
+    cb = synth.vq_codebooks(seed, synth.bf16_bits_to_f64(wb))
+    return wb, cb
+
+
+def make_vq(Ms=(1, 8, 64), seed: int = 2, prep_with: str = "library") -> dict:
+    """MXCode-style VQ layer: W [2560, 9728] Student-t(4) -> PreScale E4M3-B16 scales + FP32
+    tensor scale, seeded k-means FP4 codebooks per 64x64 QBlock (256 entries of d = 4), 8-bit
+    indices; X [M, 9728] N(0,1) for each M.  prep_with = "library" prepares the weight with the
+    library's host code (GPU arm), "oracle" with the CPU oracle (reference arm and CPU baseline:
+    that arm never loads the library)."""
+    import synth
+    N, K = 2560, 9728
+    wb, cb = _vq_weights(seed)
+    cbp = _pack_nibbles(cb)
+    if prep_with == "oracle":
+        from oracle import vq as ovq
+        p = ovq.prepare(synth.bf16_bits_to_f64(wb), cb)
+        ts, sb, idx = p["ts"], p["sb"], p["idx"]
+        make = None
+    else:
+        import bit_quantized_moe_tcgen05_b200 as ql
+        ts, sb, idx = ql.prepare_vq_prescale(wb, cbp)
+        make = lambda: ql.QLinear(None, sb, wfmt=ql.QL_W_VQ_PRESCALE_E4M3_B16,
+                                  w_tensor_scale=float(ts), indices=idx, codebooks=cbp)
     xs = {M: synth.activations_bf16(seed, M, K, 0.0, 1.0)[0] for M in Ms}
-    wbytes = idx.nbytes + cb.nbytes + sb.nbytes
+    wbytes = idx.nbytes + cbp.nbytes + sb.nbytes
     return dict(name=f"mxcode_vq_n{N}_k{K}_m{'-'.join(map(str, Ms))}", kind="vq", N=N, K=K, C=K,
-                Ms=list(Ms), xs=xs, weight_bytes=wbytes,
-                make=lambda: ql.QLinear(None, sb, wfmt=ql.QL_W_VQ_PRESCALE_E4M3_B16,
-                                        w_tensor_scale=float(ts), indices=idx, codebooks=cb),
-                oracle=dict(ts=ts, sb=sb, idx=idx, cb=cb))
+                Ms=list(Ms), xs=xs, weight_bytes=wbytes, make=make, wb=wb, cb=cb,
+                oracle_prep=dict(ts=ts, sb=sb, idx=idx) if prep_with == "oracle" else None)
 
 
 _PRQ_CACHE = {}
@@ -141,6 +159,12 @@ def make_int4(M: int, seed: int = 5) -> dict:
 
 def flops_of(w, M) -> float:
     return 2.0 * M * w["N"] * w["K"] + M * w.get("extra_flops_per_token", 0.0)
+
+
+def forward_bytes_of(w, M) -> float:
+    """Algorithmic bytes of one one-launch forward (activation quantization fused into the GEMM):
+    weight payload + bf16 x read + bf16 y written."""
+    return w["weight_bytes"] + 2.0 * M * w["C"] + 2.0 * M * w["N"]
 
 
 def gemm_bytes_of(w, M) -> float:
@@ -301,9 +325,8 @@ def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes:
     # (fewer steps than weight copies) starts from cold weights as well
     evict_buf = None if flush_bytes else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
 
-    def fwd(layer, M):
-        layer.quantize_input(xs[M], wss[M])
-        layer.gemm(M, ys[M], wss[M])
+    def fwd(layer, M):   # the public call: one launch for decode sizes (quantizer fused in)
+        layer.forward(xs[M], out=ys[M], ws=wss[M])
 
     for _ in range(warmup):
         for layer in layers:
@@ -395,16 +418,16 @@ def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes:
 
 # ------------------------------------------------------------------------------ CPU baseline
 def cpu_baseline_vq(w, budget_s: float = 20.0) -> dict:
-    """The oracle as it stands (numpy, fp64) on a bounded sample of the headline workload: whole
-    forwards (E4M3-B16 activation quantization, codebook decode, dequantized fp64 GEMM) at the
-    workload's batch sizes, as many as fit the time budget."""
+    """The oracle as it stands (numpy element-wise codecs, plain C fp64 sums) on a bounded sample
+    of the headline workload: whole forwards (E4M3-B16 activation quantization, codebook decode,
+    dequantized fp64 GEMM) at the workload's batch sizes, as many as fit the time budget.  The
+    weight is prepared by the oracle too (oracle.vq.prepare), never by the library."""
     from oracle import vq
     import synth
-    o = w["oracle"]
-    cb = np.empty(o["cb"].shape[:-1] + (4,), np.uint8)
-    cb[..., 0::2] = o["cb"] & 0xF
-    cb[..., 1::2] = o["cb"] >> 4
-    prep = dict(ts=o["ts"], sb=o["sb"], idx=o["idx"])
+    cb = w["cb"]
+    if w.get("oracle_prep") is None:
+        w["oracle_prep"] = vq.prepare(synth.bf16_bits_to_f64(w["wb"]), cb)
+    prep = w["oracle_prep"]
     done, t0 = [], time.perf_counter()
     for M in w["Ms"] * 4:
         vq.forward(synth.bf16_bits_to_f64(w["xs"][M]), prep, cb)
@@ -415,7 +438,47 @@ def cpu_baseline_vq(w, budget_s: float = 20.0) -> dict:
     return {"value": len(done) * w["weight_bytes"] / dt / 1e9, "unit": "GB/s",
             "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
             "sample": f"{len(done)} forwards (M = {done}) of {w['name']}, {dt:.1f} s; "
-                      "numpy fp64, BLAS may use every core"}
+                      "fp64 C sums on every core (OpenMP)"}
+
+
+# ------------------------------------------------------------------------------ tensor peaks
+TENSOR_KINDS = {"fp4_mxf4_block32": 0, "fp4_mxf4nvf4_block16": 1, "int8": 2, "bf16": 3}
+
+
+def measure_tensor_peaks(device, burst_ms: float = 4.0, sustain_s: float = 1.5) -> dict:
+    """TFLOP/s of back-to-back tcgen05 MMAs (M = 128, N = 256) on operands resident in shared
+    memory, one CTA per SM (ql_tensor_peak): the most a GEMM of that instruction kind can reach
+    on this GPU.  burst = best single launch of ~burst_ms after a warm-up; sustained = launches
+    back to back for ~sustain_s (the clocks settle under the power cap).  The bf16 figure is the
+    same method on the pipe whose cuBLAS throughput MEASURED_PEAKS.json holds (a check)."""
+    import ctypes
+    import torch
+    import bit_quantized_moe_tcgen05_b200 as ql
+    stream = torch.cuda.current_stream(device)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    out = {}
+    for name, kind in TENSOR_KINDS.items():
+        fl = ctypes.c_double()
+
+        def launch(iters):
+            st = ql.lib.ql_tensor_peak(kind, 256, iters, sms, ctypes.byref(fl), stream.cuda_stream)
+            if st != 0:
+                raise ql.QLError(st, "ql_tensor_peak")
+            return fl.value
+
+        launch(64)
+        ql.check()
+        ms = _elapsed(lambda: launch(256), 1, stream)
+        it = max(256, int(256 * burst_ms / max(ms, 1e-3)))
+        best = 0.0
+        for _ in range(5):
+            ms = _elapsed(lambda: launch(it), 1, stream)
+            best = max(best, fl.value / (ms * 1e-3) / 1e12)
+        reps = max(2, int(sustain_s * 1e3 / max(ms, 1e-3)))
+        ms = _elapsed(lambda: launch(it), reps, stream)
+        ql.check()
+        out[name] = {"burst": best, "sustained": reps * fl.value / (ms * 1e-3) / 1e12}
+    return out
 
 
 def main():
@@ -435,11 +498,38 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.impl == "reference":
+        # The oracle on the host cores, on the headline workload prepared by the oracle itself;
+        # this arm never loads the CUDA library.  Under torchrun only rank 0 runs it.
+        if rank != 0:
+            return
+        if args.workload != "vq":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the "
+                              "oracle on the headline VQ workload only"}))
+            return
+        head = make_vq(prep_with="oracle")
+        cb = cpu_baseline_vq(head)
+        units = len(head["Ms"]) * head["weight_bytes"] / 1e9
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": cb["unit"],
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": units / cb["value"] * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": head["name"], "N": head["N"], "K": head["K"], "M": head["Ms"],
+                       "parallelism": "single",
+                       "l2": "rotating weight copies totalling > 126 MB L2 (no flush)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": cb["unit"], "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+
     if args.workload == "moe":
-        import torch
         w = make_moe()
-        torch.cuda.set_device(local)
-        r = run_moe(w, args.steps, args.warmup, torch.device("cuda", local))
+        r = run_moe(w, args.steps, args.warmup, device)
         peaks = measured_peaks()
         tf = w["flops"] / (r["step_ms"] * 1e-3) / 1e12
         print(json.dumps({"metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
@@ -469,28 +559,6 @@ def main():
               "parallelism": "replicas" if world > 1 else "single",
               "l2": ("rotating weight copies totalling > 126 MB L2 (no flush)" if decode
                      else "flushed before each step (256 MiB write)")}
-
-    if args.impl == "reference":
-        if rank != 0:
-            return
-        if head["kind"] != "vq":
-            print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the "
-                              "oracle on the headline VQ workload only"}))
-            return
-        cb = cpu_baseline_vq(head)
-        print(json.dumps({
-            "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": cb["unit"],
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": per_step_units(head) / cb["value"] * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config, "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": cb["unit"], "h2d_bytes_per_step": 0,
-                    "d2h_bytes_per_step": 0}}))
-        return
-
-    import torch
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -513,17 +581,22 @@ def main():
     value = job_throughput(units, world, step_ms)
     e2e_val = job_throughput(units, world, e2e_ms)
 
-    fp4_peak = peaks["bf16"] * NOMINAL_FP4_OVER_BF16
+    tp = measure_tensor_peaks(device)
+    fp4_peak = tp["fp4_mxf4_block32"]["burst"]
+    int8_peak = tp["int8"]["burst"]
     nl = len(head["Ms"])
+    # the dominant kernel: for decode sizes the one-launch forward (the GEMM with the activation
+    # quantizer fused in), timed by the graph of forwards; else the GEMM alone
+    one_launch = decode
     if decode:
-        alg = sum(gemm_bytes_of(head, M) for M in head["Ms"]) / nl
-        ach = alg / (res["gemm_ms"] / nl * 1e-3) / 1e9
+        alg = sum(forward_bytes_of(head, M) for M in head["Ms"]) / nl
+        ach = alg / (res["step_ms"] / nl * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
                     "frac": ach / peaks["hbm"], "traffic": NCU_TRAFFIC_PER_LAUNCH.get(args.workload),
-                    "kernel": "fp4_gemm_kernel (block16 MMA, VQ decode)" if head["kind"] == "vq"
-                    else "fp4_gemm_kernel (mxf4)",
+                    "kernel": "fp4_decode_kernel (E4M3-B16 quantizer fused, VQ decode, block16 MMA)"
+                    if head["kind"] == "vq" else "fp4_decode_kernel (mxf4)",
                     "algorithmic_bytes_per_launch": alg,
-                    "peak_source": f"{peaks['src']} HBM copy bandwidth"}
+                    "peak_source": f"{peaks['src']} HBM copy bandwidth (MEASURED_PEAKS.json)"}
     else:
         alg = sum(flops_of(head, M) for M in head["Ms"]) / nl
         ach = alg / (res["gemm_ms"] / nl * 1e-3) / 1e12
@@ -531,9 +604,28 @@ def main():
                     "frac": ach / fp4_peak, "traffic": NCU_TRAFFIC_PER_LAUNCH.get(args.workload),
                     "kernel": "fp4_gemm_kernel (mxf4)",
                     "algorithmic_flops_per_launch": alg,
-                    "peak_source": f"{peaks['src']} bf16 burst {peaks['bf16']} x 4 (nominal FP4/bf16)"}
+                    "peak_source": "measured: tcgen05 kind::mxf4 block32 MMA loop, burst"}
 
-    cases = {}
+    def case_line(wl, r, M):
+        int4 = wl["kind"] == "int4"
+        pk = int8_peak if int4 else fp4_peak
+        d = {"step_us": r["step_ms"] * 1e3, "gemm_us": r["gemm_ms"] * 1e3,
+             "quant_us": r["quant_ms"] * 1e3,
+             "tflops": flops_of(wl, M) / (r["step_ms"] * 1e-3) / 1e12,
+             "gemm_tflops": flops_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e12,
+             "tensor_peak_tflops": pk,
+             "tensor_peak": ("measured int8 (tcgen05 kind::i8 MMA loop, burst)" if int4
+                             else "measured fp4 (tcgen05 kind::mxf4 MMA loop, burst)"),
+             "weight_stream_gbs": wl["weight_bytes"] / (r["step_ms"] * 1e-3) / 1e9,
+             "l2": "flushed (256 MiB write)" if r["R"] == 1 else f"{r['R']} rotating weight copies"}
+        d["gemm_tensor_frac"] = d["gemm_tflops"] / pk
+        if M <= 64 and not int4:   # one-launch forward: its bytes against HBM
+            d["hbm_frac"] = forward_bytes_of(wl, M) / (r["step_ms"] * 1e-3) / 1e9 / peaks["hbm"]
+        else:
+            d["gemm_hbm_frac"] = gemm_bytes_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e9 / peaks["hbm"]
+        return d
+
+    cases, prefill = {}, None
     if args.cases == "all" and world == 1:
         int4_4096 = make_int4(4096)
         int4_cases = [dict(int4_4096, name=int4_4096["name"].replace("_m4096", f"_m{M}"), Ms=[M],
@@ -543,19 +635,17 @@ def main():
                           (make_prquant(16), 0), (make_mxfp4(16), 0), (int4_4096, 256 << 20),
                           *[(c, 0) for c in int4_cases]):
             r = run_case(wl, 8, args.warmup, device, flush_bytes=flush)
-            M = wl["Ms"][0]
-            cases[wl["name"]] = {
-                "step_us": r["step_ms"] * 1e3, "gemm_us": r["gemm_ms"] * 1e3,
-                "quant_us": r["quant_ms"] * 1e3,
-                "tflops": flops_of(wl, M) / (r["step_ms"] * 1e-3) / 1e12,
-                "gemm_tflops": flops_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e12,
-                "gemm_tensor_frac": flops_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e12 /
-                                    (2 * peaks["bf16"] if wl["kind"] == "int4" else fp4_peak),
-                "tensor_peak": "int8 = 2 x measured bf16 (nominal ratio)" if wl["kind"] == "int4"
-                               else "fp4 = 4 x measured bf16 (nominal ratio)",
-                "weight_stream_gbs": wl["weight_bytes"] / (r["gemm_ms"] * 1e-3) / 1e9,
-                "gemm_hbm_frac": gemm_bytes_of(wl, M) / (r["gemm_ms"] * 1e-3) / 1e9 / peaks["hbm"],
-                "l2": "flushed (256 MiB write)" if flush else f"{r['R']} rotating weight copies"}
+            cases[wl["name"]] = case_line(wl, r, wl["Ms"][0])
+            if wl["name"].endswith("_m2048") and wl["name"].startswith("prquant"):
+                c = cases[wl["name"]]
+                prefill = {"workload": wl["name"], "value": c["gemm_tflops"], "unit": "TFLOP/s",
+                           "step_tflops": c["tflops"],
+                           "roofline": {"bound": "tensor", "achieved": c["gemm_tflops"],
+                                        "peak": fp4_peak, "unit": "TFLOP/s",
+                                        "frac": c["gemm_tflops"] / fp4_peak,
+                                        "traffic": NCU_TRAFFIC_PER_LAUNCH.get("prquant_m2048"),
+                                        "kernel": "fp4_gemm_kernel (mxf4 block32, PRQuant tail)",
+                                        "peak_source": "measured"}}
         mw = make_moe()
         r = run_moe(mw, 10, args.warmup, device)
         tf = mw["flops"] / (r["step_ms"] * 1e-3) / 1e12
@@ -569,11 +659,9 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
-    # library kernels per forward: the activation quantizer and the GEMM (E4M3-B16 activations
-    # past the one-launch quantizers' capacity take an amax kernel and a quantize kernel)
-    def kernels_per_fwd(M):
-        one_launch_cap = 3 * 256 * 148 * 16
-        return 3 if head["kind"] == "vq" and M * head["C"] > one_launch_cap else 2
+
+    def kernels_per_fwd(M):   # library kernels one forward launches
+        return 1 if one_launch else 2
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": res["steps"],
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -585,11 +673,16 @@ def main():
                 "d2h_bytes_per_step": res["d2h"]},
         "gpu_launches": sum(kernels_per_fwd(M) for M in head["Ms"]) * res["steps"],
         "clocks": clk.summary(),
-        "kernel_us_per_step": {"quantize": res["quant_ms"] * 1e3, "gemm": res["gemm_ms"] * 1e3},
-        "cases": cases,
+        "kernel_us_per_step": {"forward": res["step_ms"] * 1e3,
+                               "split_api_quantize": res["quant_ms"] * 1e3,
+                               "split_api_gemm": res["gemm_ms"] * 1e3},
+        "tensor_peaks_tflops": tp,
     }
+    line["cases"] = cases
     if not args.no_cpu_baseline and head["kind"] == "vq" and world == 1:
         line["cpu_baseline"] = cpu_baseline_vq(head)
+    if prefill is not None:   # last, so that the end of the line (what log tails keep) holds it
+        line["prefill"] = prefill
     print(json.dumps(line))
 
 

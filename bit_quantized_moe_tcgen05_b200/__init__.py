@@ -14,7 +14,7 @@ import numpy as np
 
 __all__ = [
     "lib", "LIB_PATH", "QLError", "WeightDesc", "QLinear", "quantize_act", "prepare_prquant",
-    "check", "QL_W_MXFP4_E8M0_B32", "QL_A_MXFP4_E8M0_B32", "EXPORTED_SYMBOLS",
+    "check", "debug_inject", "QL_W_MXFP4_E8M0_B32", "QL_A_MXFP4_E8M0_B32", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlinear.so")
@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlinear.
 QL_OK = 0
 QL_W_MXFP4_E8M0_B32, QL_W_NVFP4_E4M3_B16, QL_W_VQ_PRESCALE_E4M3_B16 = 1, 2, 3
 QL_W_CLUSTER4_ROW16_BF16, QL_W_INT4_G128_BSR = 4, 5
+QL_W_VQ_POSTSCALE_E4M3_B16, QL_W_VQ_PRESCALE_PLUS_E4M3_B16 = 6, 7
 QL_A_MXFP4_E8M0_B32, QL_A_FP4_E4M3_B16_TS, QL_A_INT4_TOK_G128 = 1, 2, 3
 
 _STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED", 3: "QL_ERR_CUDA",
@@ -34,7 +35,8 @@ EXPORTED_SYMBOLS = (
     "qlinear_quantize_input", "qlinear_gemm", "qlinear_forward_fixed_scratch",
     "qlinear_prepare_vq_prescale", "moe_create", "moe_destroy", "moe_capture_intermediate",
     "moe_workspace_bytes", "moe_workspace_layout", "moe_grouped_forward",
-    "qlinear_prepare_int4_bsr", "ql_tensor_peak",
+    "qlinear_prepare_int4_bsr", "ql_tensor_peak", "ql_debug_inject",
+    "qlinear_prepare_vq_postscale", "qlinear_prepare_vq_prescale_plus",
 )
 
 
@@ -54,7 +56,8 @@ class WeightDesc(ctypes.Structure):
         ("bsr_rowptr", ctypes.c_void_p), ("bsr_col", ctypes.c_void_p),
         ("bsr_codes", ctypes.c_void_p), ("bsr_scales", ctypes.c_void_p),
         ("bsr_block_n", ctypes.c_int32), ("bsr_block_k", ctypes.c_int32),
-        ("bsr_nnzb", ctypes.c_int32),
+        ("bsr_nnzb", ctypes.c_int32), ("scale_codebook", ctypes.c_void_p),
+        ("scale_codebook_entries", ctypes.c_int32), ("scale_group", ctypes.c_int32),
     ]
 
 
@@ -94,6 +97,9 @@ def _load() -> ctypes.CDLL:
         "qlinear_prepare_int4_bsr": [vp, i64, i64, vp, i64, ctypes.c_float, vp, vp, vp, vp, vp, vp,
                                      i32, vp],
         "ql_tensor_peak": [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_double), vp],
+        "ql_debug_inject": [i32, ctypes.c_uint64],
+        "qlinear_prepare_vq_postscale": [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp],
+        "qlinear_prepare_vq_prescale_plus": [vp, i64, i64, vp, vp, i32, i32, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -123,6 +129,13 @@ def _ptr(t) -> int | None:
 def check(stream=None) -> None:
     """Synchronise and raise if any kernel recorded a device-side timeout."""
     _ok(lib.ql_check(_stream(stream)), "ql_check")
+
+
+def debug_inject(withhold_cta: int = -1, wait_limit_ns: int = 0) -> None:
+    """Test hook for the timeout path: lower the kernels' wait limit and withhold one CTA's
+    grid-wide publications so that the waits on them run out (see ql_debug_inject).
+    debug_inject() restores the defaults."""
+    _ok(lib.ql_debug_inject(int(withhold_cta), int(wait_limit_ns)), "ql_debug_inject")
 
 
 def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None):
@@ -164,7 +177,7 @@ class QLinear:
     def __init__(self, codes: np.ndarray | None, scales: np.ndarray, k_tail: int = 0,
                  wfmt: int = QL_W_MXFP4_E8M0_B32, w_tensor_scale: float = 1.0,
                  indices: np.ndarray | None = None, codebooks: np.ndarray | None = None,
-                 bsr: dict | None = None, stream=None):
+                 bsr: dict | None = None, scale_codebook: np.ndarray | None = None, stream=None):
         """MXFP4: codes [N, K/2] + E8M0 scales [N, K/32] (+ k_tail).  NVFP4 (E4M3-B16): codes +
         E4M3 scales [N, K/16] + w_tensor_scale.  VQ PreScale: indices [N, K/4] + packed codebooks
         [N/64, K/64, 256, 2] + E4M3 scales [N, K/16] + w_tensor_scale (codes = None).
@@ -191,12 +204,18 @@ class QLinear:
             self._h = h
             self._ws = None
             return
-        if wfmt == QL_W_VQ_PRESCALE_E4M3_B16:
+        scb_ptr = None
+        if wfmt in (QL_W_VQ_PRESCALE_E4M3_B16, QL_W_VQ_POSTSCALE_E4M3_B16,
+                    QL_W_VQ_PRESCALE_PLUS_E4M3_B16):
             indices = np.ascontiguousarray(indices, dtype=np.uint8)
             codebooks = np.ascontiguousarray(codebooks, dtype=np.uint8)
             N, K = indices.shape[0], 4 * indices.shape[1]
             keep += [indices, codebooks]
             cptr, iptr, cbptr = None, indices.ctypes.data, codebooks.ctypes.data
+            if wfmt == QL_W_VQ_PRESCALE_PLUS_E4M3_B16:
+                scb = np.ascontiguousarray(scale_codebook, dtype=np.uint8)
+                keep.append(scb)
+                scb_ptr = scb.ctypes.data
         else:
             codes = np.ascontiguousarray(codes, dtype=np.uint8)
             N, K = codes.shape[0], 2 * codes.shape[1]
@@ -207,7 +226,9 @@ class QLinear:
         self.wfmt = wfmt
         d = WeightDesc(wfmt=wfmt, N=N, K=self.K, k_tail=self.k_tail, codes=cptr,
                        scales=scales.ctypes.data, w_tensor_scale=float(w_tensor_scale),
-                       indices=iptr, codebooks=cbptr, qblock_n=64, qblock_k=64)
+                       indices=iptr, codebooks=cbptr, qblock_n=64, qblock_k=64,
+                       scale_codebook=scb_ptr, scale_codebook_entries=256 if scb_ptr else 0,
+                       scale_group=8 if scb_ptr else 0)
         h = ctypes.c_void_p()
         _ok(lib.qlinear_create(ctypes.byref(d), _stream(stream), ctypes.byref(h)), "qlinear_create")
         self._h = h
@@ -308,6 +329,42 @@ def prepare_vq_prescale(w_bf16_bits: np.ndarray, codebooks_packed: np.ndarray, q
                                         scales.ctypes.data, idx.ctypes.data),
         "qlinear_prepare_vq_prescale")
     return np.float32(ts[0]), scales, idx
+
+
+def prepare_vq_postscale(w_bf16_bits: np.ndarray, centroids: np.ndarray):
+    """Offline MXCode PostScale preparation on the host (library C++ code).  centroids: learned
+    codebooks float32 [N/64, K/64, 256, 4].  Returns (ts, packed E2M1 codebooks uint8
+    [N/64, K/64, 256, 2], QBlock E4M3 scale bytes [N/64, K/64], indices uint8 [N, K/4])."""
+    w = np.ascontiguousarray(w_bf16_bits, dtype=np.uint16)
+    c = np.ascontiguousarray(centroids, dtype=np.float32)
+    N, K = w.shape
+    ts = ctypes.c_float()
+    cb = np.empty((N // 64, K // 64, 256, 2), np.uint8)
+    qs = np.empty((N // 64, K // 64), np.uint8)
+    idx = np.empty((N, K // 4), np.uint8)
+    _ok(lib.qlinear_prepare_vq_postscale(w.ctypes.data, N, K, c.ctypes.data, 64, 64,
+                                         ctypes.addressof(ts), cb.ctypes.data, qs.ctypes.data,
+                                         idx.ctypes.data), "qlinear_prepare_vq_postscale")
+    return np.float32(ts.value), cb, qs, idx
+
+
+def prepare_vq_prescale_plus(w_bf16_bits: np.ndarray, codebooks_packed: np.ndarray,
+                             scale_codebook: np.ndarray):
+    """Offline MXCode PreScale+ preparation on the host (library C++ code).  Returns (ts,
+    compressed E4M3 scales [N, K/16], scale indices [N, K/128], weight indices [N, K/4])."""
+    w = np.ascontiguousarray(w_bf16_bits, dtype=np.uint16)
+    cb = np.ascontiguousarray(codebooks_packed, dtype=np.uint8)
+    scb = np.ascontiguousarray(scale_codebook, dtype=np.uint8)
+    N, K = w.shape
+    ts = ctypes.c_float()
+    sb = np.empty((N, K // 16), np.uint8)
+    sidx = np.empty((N, K // 128), np.uint8)
+    idx = np.empty((N, K // 4), np.uint8)
+    _ok(lib.qlinear_prepare_vq_prescale_plus(w.ctypes.data, N, K, cb.ctypes.data, scb.ctypes.data,
+                                             64, 64, ctypes.addressof(ts), sb.ctypes.data,
+                                             sidx.ctypes.data, idx.ctypes.data),
+        "qlinear_prepare_vq_prescale_plus")
+    return np.float32(ts.value), sb, sidx, idx
 
 
 def _pack4(idx: np.ndarray) -> np.ndarray:

@@ -1,0 +1,696 @@
+// Decode-size W4A4 GEMM (M <= 64 tokens) on tcgen05, with the activation quantizer fused in.
+//
+//   y[m, n] = alpha * sum_k x_q[m, k] * w_q[n, k]
+//
+// The weight forms are those of fp4_gemm_kernel: block-scaled E2M1 with E8M0-B32 scales
+// (kind::mxf4, PRQuant tail stages included), with E4M3-B16 scales (kind::mxf4nvf4, alpha = the
+// two FP32 tensor scales), or MXCode PreScale VQ indices decoded in shared memory (MXCode
+// abstract: MX-native operands rebuilt without a high-precision weight).  At decode sizes the
+// layer is bound by streaming the weight, so every CTA owns one 128-row weight tile and a range
+// of K stages (split-K), issues the bulk copies of ALL its weight stages at once, keeps them
+// resident, and the tokens are one B tile of BN = 16, 32 or 64 rows.
+//
+// Activation quantization inside the kernel (fuse = 1).  The bf16 activations of split z's
+// columns are shared out, in units of 32 elements, among the CTAs of split z; each CTA's four
+// quantizer warps quantize their units once (E8M0-B32 per the OCP MX rule PRQuant quantizes
+// with, or E4M3-B16 per MXCode Table 1) into the workspace, already in the layout of the MMA's B
+// tile of each K stage (128 B per row, 128-byte swizzle) with the stage's scale atoms beside it,
+// so that every CTA brings in the B operand of all its stages with two bulk copies.  The E4M3-B16
+// tensor scale needs the amax of the whole tensor: each CTA publishes the amax of its units in a
+// slot, CTA 0 gathers the slots and publishes the maximum in one word, which the others poll.
+// With fuse = 0 the workspace already holds the quantized activations in the plain layout
+// (qlinear_quantize_input) and the producer warp copies each stage's B tile by cp.async.
+//
+// Issuing tcgen05 instructions costs the issuing thread tens of cycles each, so the MMA issuer
+// issues MMAs only: the scale factors reach TMEM through tcgen05.st from the warps that hold them
+// (the decoder, or epilogue, warps for the weight's; the quantizer warps for the activations').
+//
+// Grid-wide agreement without clearing anything between launches.  The workspace sync block holds
+// a launch counter c.  Every CTA reads c once, after griddepcontrol.wait (so after the previous
+// launch on the workspace has completed), and tags every word it publishes with tag(c + 1): its
+// slot (E4M3: tag | amax), its "units quantized" flag, its "split-K partial written" flag, and
+// CTA 0's amax result.  Waiters compare the tag, so stale words of earlier launches never match.
+// CTA 0 advances the counter by one at its very end, once it has seen every CTA's slot (so every
+// CTA has read c).  A CTA whose bounded wait expired adds two at its end instead: a CTA that read
+// the counter late (value v, after CTA 0 gave up) leaves words tagged tag(v + 1) and then the
+// counter at v + 2 or more, so the next launch's tag matches no word any failed launch left
+// behind, and the workspace stays usable without clearing.
+//
+// Split-K reduction.  Each CTA of a tile writes its fp32 partial [M][128] to the workspace and
+// publishes its flag; every CTA of the tile waits for the tile's flags and reduces 1/S of the
+// tile's outputs, adding the splits' partials in split order (deterministic), and writes y.
+//
+// Warp roles: 0 producer (weight bulk copies, then the B tiles), 1 TMEM allocator + MMA issuer,
+// VQ: 2..9 decoders (the operand tile of each stage rebuilt from the codebooks into a ring of up
+// to eight shared-memory tiles, as many as the memory left by the resident stages holds; warps
+// 2..5 also move the stage's weight scales to TMEM), 2..5 epilogue (without VQ they move the
+// weight scales), then four quantizer warps.  Every wait is bounded and records the device error
+// word.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "ptx.cuh"
+#include "quant_act.cuh"
+
+namespace ql {
+
+constexpr int kDecMaxGrid = 256;           // CTAs of one decode launch (slots and flags)
+constexpr int kDecQUnits = 2;              // 32-element activation units per quantizer thread
+constexpr int kDecMaxSplits = 16;          // K-splits of one weight tile
+constexpr int kDecSyncBytes = 16 + 3 * 8 * kDecMaxGrid;
+
+// Workspace sync block: [0] launch counter, [8] amax result, [16..) slots, qflags, pflags (64-bit
+// words each).
+struct DecSync {
+  uint32_t* counter;
+  unsigned long long* result;   // CTA 0's published E4M3 amax (tagged)
+  unsigned long long* slots;
+  unsigned long long* qflags;
+  unsigned long long* pflags;
+};
+__host__ __device__ inline DecSync dec_sync(uint8_t* base) {
+  DecSync s;
+  s.counter = reinterpret_cast<uint32_t*>(base);
+  s.result = reinterpret_cast<unsigned long long*>(base + 8);
+  s.slots = reinterpret_cast<unsigned long long*>(base + 16);
+  s.qflags = s.slots + kDecMaxGrid;
+  s.pflags = s.qflags + kDecMaxGrid;
+  return s;
+}
+
+// 48-bit tag of a launch count (the low 16 bits of a published word carry data).
+__device__ __forceinline__ unsigned long long dec_tag(uint32_t c) {
+  return (static_cast<unsigned long long>(c) << 32) |
+         (static_cast<unsigned long long>((c * 0x6D2Bu + 0x1F35u) & 0xFFFFu) << 16);
+}
+
+// Bounded wait until *p carries `tag` in its upper 48 bits; returns the word (0 on a timeout,
+// which also sets the device error word).
+__device__ __forceinline__ unsigned long long dec_wait_tag(const unsigned long long* p,
+                                                           unsigned long long tag, int site,
+                                                           bool& ok) {
+  unsigned long long s = ld_acquire_gpu_u64(p);
+  if ((s & ~0xFFFFull) == tag) return s;
+  const uint64_t t0 = globaltimer_ns(), limit = wait_limit_ns();
+  while (true) {
+    __nanosleep(32);
+    s = ld_acquire_gpu_u64(p);
+    if ((s & ~0xFFFFull) == tag) return s;
+    if (globaltimer_ns() - t0 > limit) {
+      record_error(DEV_TIMEOUT, site);
+      ok = false;
+      return 0;
+    }
+  }
+}
+
+struct DecodeArgs {
+  int M, N;                   // tokens (<= BN), output features
+  int C, k_tail;              // activation width; PRQuant tail width (weight width C + k_tail)
+  int n_base_stages;          // ceil(C / 256)
+  int n_stages_total;         // + ceil(k_tail / 256)
+  int spp;                    // K stages per split
+  int splits;                 // CTAs per weight tile (consecutive blockIdx)
+  int fuse;                   // 1: quantize x inside the kernel
+  const __nv_bfloat16* x;     // fuse: bf16 activations [M, C]
+  uint8_t* xq;                // fuse = 0: quantized activation codes [M, C/2] (workspace)
+  uint8_t* sfb;               // fuse = 0: activation scale atoms, 128-row group 0, [C / atomK]
+  uint8_t* xt;                // fuse = 1: per K stage the B tile [BN][128 B], 128-byte swizzle
+  uint8_t* st;                // fuse = 1: per K stage its activation scale atoms
+  float* ts_x;                // E4M3: activation tensor scale (fuse: written; else read)
+  float alpha;                // host factor (weight tensor scale, or 1)
+  const uint8_t* wt;          // weight blocks [N/128][n_stages_total][kWBytes]
+  __nv_bfloat16* y;           // [M, ldy]
+  float* y32;                 // optional [M, ldy]
+  int ldy;
+  float* partials;            // splits > 1: [grid][BN][128] fp32 (rows < M written)
+  uint8_t* sync;              // DecSync block
+  const uint8_t* scb;         // VQ PreScale+: scale codebook [256][8] E4M3 bytes
+};
+
+// SF (VQ only): the weight's scales as in Fp4Cfg -- 0 PreScale atoms in the block, 1 PostScale
+// (8 QBlock bytes per stage), 2 PreScale+ (2 scale indices per row into a 256 x 8 codebook).
+template <int BN, bool E8M0, bool VQ, int SF = 0>
+struct DecCfg {
+  static constexpr int kDecWarps = VQ ? 8 : 0;
+  static constexpr int kQWarp0 = VQ ? 10 : 6;
+  static constexpr int kThreads = (kQWarp0 + 4) * 32;
+  static constexpr int kAtomK = E8M0 ? 128 : 64;     // K elements per scale atom
+  static constexpr int kAtoms = 256 / kAtomK;        // scale atoms per 256-K stage
+  static constexpr int kABytes = 128 * 128;          // decoded E2M1 tile, 128 rows x 256 K
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kSfBytes = kAtoms * 512;
+  static constexpr int kIdxBytes = VQ ? 128 * 64 : 0;
+  static constexpr int kLutBytes = VQ ? 8 * 512 : 0;
+  static_assert(SF == 0 || (VQ && !E8M0), "PostScale / PreScale+ scales: VQ E4M3-B16 weights");
+  static constexpr int kSfTail = SF == 0 ? kSfBytes : SF == 1 ? 16 : 256;
+  static constexpr int kWBytes = (VQ ? kIdxBytes + kLutBytes : kABytes) + kSfTail;   // in HBM
+  static constexpr int kWStride = (kWBytes + 1023) / 1024 * 1024;                     // in smem
+  static constexpr int kScbBytes = SF == 2 ? 2048 : 0;
+  static constexpr int kSfaOff = VQ ? kIdxBytes + kLutBytes : kABytes;
+  static constexpr int kPerStage = kWStride + kBBytes + kSfBytes;
+  static constexpr int kSmemBytes = 226 * 1024;      // dynamic shared memory of the launch
+  static constexpr int kData = kSmemBytes - 2048 - kScbBytes;   // minus slack, barriers, codebook
+  static constexpr int kMaxRing = 8;                 // VQ: decoded operand tiles in flight
+  static constexpr int kSfCols = kAtoms * 4;         // TMEM columns of one scale set
+  static constexpr int kMaxStagesTmem = (512 - BN) / (2 * kSfCols);
+  static constexpr int kMaxStagesSmem = (kData - (VQ ? kABytes : 0)) / kPerStage;
+  static constexpr int kMaxStagesRaw = kMaxStagesSmem < kMaxStagesTmem ? kMaxStagesSmem : kMaxStagesTmem;
+  static constexpr int kMaxStages = kMaxStagesRaw > 16 ? 16 : kMaxStagesRaw;
+  static_assert(kMaxStages >= 2, "decode stages");
+  static_assert(kBBytes % 1024 == 0 && kSfBytes % 1024 == 0, "1 KB regions");
+  // ring of decoded operand tiles for n_it resident stages: what the shared memory left holds
+  __host__ __device__ static constexpr int ring(int n_it) {
+    return !VQ ? 0 : ((kData - n_it * kPerStage) / kABytes < kMaxRing
+                          ? ((kData - n_it * kPerStage) / kABytes < n_it ? (kData - n_it * kPerStage) / kABytes : n_it)
+                          : (kMaxRing < n_it ? kMaxRing : n_it));
+  }
+};
+
+// MX E8M0-B32 coding of one 32-element unit held as 16 bf16x2 words: codes (16 bytes) and the
+// E8M0 byte (OCP MX: e = floor(log2 amax) - 2 from the bf16 exponent, clamped to [-127, 127]).
+__device__ __forceinline__ void dec_code_mx(const uint32_t (&w)[16], uint4& codes, uint32_t& byte) {
+  uint32_t mx = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
+  const uint32_t amax16 = max(mx & 0xFFFFu, mx >> 16);
+  const int E = static_cast<int>(amax16 >> 7);
+  const int e = (E == 0) ? -127 : max(E - 129, -127);
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
+  uint32_t packed[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float f[8];
+    const uint32_t ww[4] = {w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(ww[i] << 16) * inv;
+      f[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u) * inv;
+    }
+    packed[q] = e2m1x8(f) | bf16x8_sign_nibbles(ww);
+  }
+  codes = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  byte = static_cast<uint32_t>(e + 127);
+}
+
+template <int BN, bool E8M0, bool VQ, int SF = 0>
+__global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
+    fp4_decode_kernel(const DecodeArgs a) {
+  using Cfg = DecCfg<BN, E8M0, VQ, SF>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int tile = blockIdx.x / a.splits, z = blockIdx.x - tile * a.splits;
+  const int T = gridDim.x / a.splits;          // weight tiles
+  const int s_begin = z * a.spp;
+  const int n_it = max(0, min(a.n_stages_total, s_begin + a.spp) - s_begin);   // <= kMaxStages
+  // layout (1 KB regions): weight blocks [n_it], B tiles [n_it], SFB sets [n_it], the ring of
+  // decoded operand tiles (VQ); barriers in the last 1 KB
+  const int R = Cfg::ring(n_it);
+  uint8_t* sW = smem;
+  uint8_t* sB = sW + n_it * Cfg::kWStride;
+  uint8_t* sSfb = sB + n_it * Cfg::kBBytes;
+  uint8_t* sA = sSfb + n_it * Cfg::kSfBytes;
+  uint8_t* sScb = smem + Cfg::kData;          // SF 2: the scale codebook
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(sScb + Cfg::kScbBytes);
+  uint64_t* sfa_ok = wfull + Cfg::kMaxStages;  // weight scales of stage i in TMEM (4 warps)
+  uint64_t* decd = sfa_ok + Cfg::kMaxStages;   // VQ: ring slot decoded (8 decoder warps)
+  uint64_t* aempty = decd + Cfg::kMaxRing;     // VQ: ring slot consumed by the MMAs
+  uint64_t* accf = aempty + Cfg::kMaxRing;
+  uint64_t* xready = accf + 1;                 // quantized activations visible (quantizer warps)
+  uint64_t* bfull = xready + 1;                // every B tile + SFB set in shared memory
+  uint64_t* sfb_ok = bfull + 1;                // activation scales in TMEM (4 quantizer warps)
+  uint64_t* scbar = sfb_ok + 1;                // SF 2: the scale codebook landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(scbar + 1);
+  __shared__ uint32_t s_cnt;
+  __shared__ uint32_t s_red[4];
+  __shared__ float s_ts;
+  __shared__ int s_allseen;
+  __shared__ int s_fail;   // some bounded wait of this CTA expired
+  griddep_launch_dependents();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = tile * 128;
+  const DecSync sy = dec_sync(a.sync);
+  const uint32_t quad_lanes = static_cast<uint32_t>((warp & 3) * 32) << 16;   // TMEM lane quadrant
+
+  auto stage_coords = [&](int i, int& kw, int& kx, int& valid) {
+    if (i < a.n_base_stages) {
+      kw = i * 256;
+      kx = kw;
+      valid = min(256, a.C - kw);
+    } else {
+      const int j = (i - a.n_base_stages) * 256;
+      kw = a.C + j;
+      kx = a.C - a.k_tail + j;
+      valid = min(256, a.k_tail - j);
+    }
+  };
+  // TMEM columns: accumulator [0, BN), then per stage the weight's and the activation's scales
+  auto sfa_col = [&](int it) { return static_cast<uint32_t>(BN + it * 2 * Cfg::kSfCols); };
+  auto sfb_col = [&](int it) { return static_cast<uint32_t>(BN + it * 2 * Cfg::kSfCols + Cfg::kSfCols); };
+
+  if (warp == 0) {
+    for (int s = lane; s < Cfg::kMaxStages; s += 32) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&sfa_ok[s], 4);
+    }
+    if (lane < Cfg::kMaxRing) {
+      mbar_init(&decd[lane], Cfg::kDecWarps > 0 ? Cfg::kDecWarps : 1);
+      mbar_init(&aempty[lane], 1);
+    }
+    if (lane == 0) {
+      mbar_init(accf, 1);
+      mbar_init(xready, 1);
+      mbar_init(bfull, a.fuse ? 1 : 32);
+      mbar_init(sfb_ok, 4);
+      mbar_init(scbar, 1);
+      s_fail = 0;
+      s_allseen = 0;
+    }
+    fence_mbar_init();
+    __syncwarp();
+    if (lane == 0) {   // every weight stage of this CTA at once, before the block-wide barrier
+      if constexpr (SF == 2) {
+        mbar_arrive_expect_tx(scbar, Cfg::kScbBytes);
+        bulk_load(sScb, a.scb, Cfg::kScbBytes, scbar);
+      }
+      for (int it = 0; it < n_it; ++it) {
+        const uint8_t* blk = a.wt + (static_cast<size_t>(tile) * a.n_stages_total + s_begin + it) * Cfg::kWBytes;
+        mbar_arrive_expect_tx(&wfull[it], Cfg::kWBytes);
+        bulk_load(sW + it * Cfg::kWStride, blk, Cfg::kWBytes, &wfull[it]);
+      }
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  bool ok = true;
+  if (warp == 0) {
+    // ---------------- the B operand of every stage, once the activations are quantized
+    ok = __all_sync(0xFFFFFFFFu, mbar_wait(xready, 0, 50));
+    if (a.fuse) {
+      // stage tiles and scale sets of this CTA's stages are contiguous in the workspace
+      if (lane == 0) {
+        const uint32_t bbytes = n_it * Cfg::kBBytes, sbytes = n_it * Cfg::kSfBytes;
+        if (ok && n_it > 0) {
+          fence_proxy_async_global();   // other CTAs' generic stores, acquired, before async reads
+          mbar_arrive_expect_tx(bfull, bbytes + sbytes);
+          bulk_load(sB, a.xt + static_cast<size_t>(s_begin) * Cfg::kBBytes, bbytes, bfull);
+          bulk_load(sSfb, a.st + static_cast<size_t>(s_begin) * Cfg::kSfBytes, sbytes, bfull);
+        } else {
+          mbar_arrive(bfull);
+        }
+      }
+    } else {
+      // plain layout (qlinear_quantize_input): each stage's B tile by 16-byte cp.async from all
+      // 32 lanes into the swizzled layout (rows past M zero-filled), then its scale atoms
+      for (int it = 0; it < n_it && ok; ++it) {
+        int kw, kx, valid;
+        stage_coords(s_begin + it, kw, kx, valid);
+        const int nat = valid / Cfg::kAtomK;
+        const uint32_t bdst = smem_u32(sB + it * Cfg::kBBytes);
+        for (int c = lane; c < BN * 8; c += 32) {
+          const int r = c >> 3, kc = c & 7;
+          const bool in = r < a.M && kc * 32 < valid;
+          const uint8_t* src = a.xq + static_cast<size_t>(in ? r : 0) * (a.C / 2) + (kx >> 1) + (in ? kc * 16 : 0);
+          cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4), src, in ? 16u : 0u);
+        }
+        const uint8_t* sfsrc = a.sfb + static_cast<size_t>(kx / Cfg::kAtomK) * 512;
+        const uint32_t sfdst = smem_u32(sSfb + it * Cfg::kSfBytes);
+        for (int c = lane; c < nat * 32; c += 32) cp_async16(sfdst + c * 16, sfsrc + c * 16, 16u);
+      }
+      cp_async_commit();
+      cp_async_wait_pending(0);
+      fence_proxy_async_smem();
+      mbar_arrive(bfull);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: MMAs only (the scale factors are placed by other warps)
+    const uint32_t idesc0 = idesc_fp4_block(BN, E8M0);
+    ok = __all_sync(0xFFFFFFFFu, mbar_wait(sfb_ok, 0, 52));
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int slot = VQ ? it % R : 0;
+      bool w = mbar_wait(&sfa_ok[it], 0, 51);
+      if constexpr (VQ) w = w && mbar_wait(&decd[slot], (it / R) & 1, 53);
+      ok = __all_sync(0xFFFFFFFFu, w);
+      if (!ok) break;
+      tc_fence_after();
+      int kw, kx, valid;
+      stage_coords(s_begin + it, kw, kx, valid);
+      const uint32_t ta = tmem + sfa_col(it), tb = tmem + sfb_col(it);
+      const uint32_t a_base = VQ ? smem_u32(sA + slot * Cfg::kABytes) : smem_u32(sW + it * Cfg::kWStride);
+      const uint32_t b_base = smem_u32(sB + it * Cfg::kBBytes);
+      const int nk = valid / 64;
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          if (kk < nk) {
+            const int at = (kk * 64) / Cfg::kAtomK;
+            const uint32_t byte = E8M0 ? static_cast<uint32_t>((kk & 1) * 2) : 0u;
+            const uint64_t ad = make_sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bd = make_sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128);
+            const uint32_t idd = idesc0 | (byte << 29) | (byte << 4);
+            const uint32_t sa = (ta + at * 4) | (byte << 30);
+            const uint32_t sb = (tb + at * 4) | (byte << 30);
+            const uint32_t acc = (it == 0 && kk == 0) ? 0u : 1u;
+            if (E8M0)
+              mma_mxf4_block32(tmem, ad, bd, idd, sa, sb, acc);
+            else
+              mma_nvf4_block16(tmem, ad, bd, idd, sa, sb, acc);
+          }
+        if (VQ && it + R < n_it) tc_commit(&aempty[slot]);   // the slot may be rewritten once these complete
+      }
+      __syncwarp();
+    }
+    if (lane == 0) tc_commit(accf);
+    __syncwarp();
+  } else if (warp >= Cfg::kQWarp0) {
+    // ---------------- quantizer warps
+    const int tq = threadIdx.x - Cfg::kQWarp0 * 32;   // 0..127
+    const int G = gridDim.x;
+    griddep_wait();   // x, the workspace and the counter follow the grids before this one
+    if (tq == 0) s_cnt = *reinterpret_cast<volatile uint32_t*>(sy.counter);
+    named_bar_sync(2, 128);
+    const uint32_t cnt = s_cnt;
+    const unsigned long long tag = dec_tag(cnt + 1u);
+    // this CTA's units: the columns of split z's base stages, rows shared out over its T tiles
+    const int c0 = min(a.C, s_begin * 256);
+    const int c1 = min(a.C, min(s_begin + a.spp, a.n_base_stages) * 256);
+    const int upr = max(0, c1 - c0) >> 5;                 // 32-element units per row
+    const long U = static_cast<long>(a.M) * upr;
+    const long u0 = U * tile / T, u1 = U * (tile + 1) / T;
+    uint32_t w[kDecQUnits][16];
+    uint32_t mx = 0;
+    if (a.fuse) {
+#pragma unroll
+      for (int k = 0; k < kDecQUnits; ++k) {
+        const long u = u0 + tq + k * 128;
+        if (u < u1) {
+          const int m = static_cast<int>(u / upr), j = (c0 >> 5) + static_cast<int>(u - static_cast<long>(m) * upr);
+          const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * a.C) + j * 4;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 v = __ldg(src + i);
+            w[k][4 * i] = v.x; w[k][4 * i + 1] = v.y; w[k][4 * i + 2] = v.z; w[k][4 * i + 3] = v.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, w[k][i] & 0x7FFF7FFFu);
+        }
+      }
+    }
+    uint32_t m16 = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, o));
+    if (lane == 0) s_red[tq >> 5] = m16;
+    named_bar_sync(2, 128);
+    if (tq == 0 && !withheld(blockIdx.x))   // this CTA has read the counter; E4M3: its amax
+      st_release_gpu_u64(&sy.slots[blockIdx.x], tag | max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3])));
+    bool qok = true;
+    float ts = 1.f;
+    // CTA 0 gathers every slot: for the E4M3 tensor amax (then at once), and to know that every
+    // CTA has read the counter (without an amax to agree on, at its end)
+    const bool amax_needed = a.fuse && !E8M0;
+    if (blockIdx.x == 0 && amax_needed) {
+      uint32_t a16 = 0;
+      for (int c = tq; c < G; c += 128)
+        a16 = max(a16, static_cast<uint32_t>(dec_wait_tag(&sy.slots[c], tag, 54, qok) & 0xFFFFull));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a16 = max(a16, __shfl_xor_sync(0xFFFFFFFFu, a16, o));
+      named_bar_sync(2, 128);   // s_red was read above
+      if (lane == 0) s_red[tq >> 5] = a16;
+      qok = bar_and(2, 128, qok);
+      const uint32_t amax16 = max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3]));
+      if (tq == 0) {
+        s_allseen = qok ? 1 : 0;
+        if (qok && amax_needed && !withheld(0)) st_release_gpu_u64(sy.result, tag | amax16);
+      }
+      ts = tensor_scale_from_amax16(amax16);
+    } else if (amax_needed) {
+      if (tq == 0) s_red[0] = static_cast<uint32_t>(dec_wait_tag(sy.result, tag, 61, qok) & 0xFFFFull);
+      qok = bar_and(2, 128, qok);
+      ts = tensor_scale_from_amax16(s_red[0]);
+    }
+    if (a.fuse) {
+      if (qok) {
+        // codes and scales straight into the stage tiles: unit (m, j) of base stage i = j / 8 goes
+        // to chunk j % 8 of row m; PRQuant tail channels also to their tail stage
+#pragma unroll
+        for (int k = 0; k < kDecQUnits; ++k) {
+          const long u = u0 + tq + k * 128;
+          if (u < u1) {
+            const int m = static_cast<int>(u / upr), j = (c0 >> 5) + static_cast<int>(u - static_cast<long>(m) * upr);
+            uint4 codes;
+            uint32_t sbytes;   // E8M0: one byte; E4M3: two (blocks 2j, 2j + 1)
+            if constexpr (E8M0) {
+              dec_code_mx(w[k], codes, sbytes);
+            } else {
+              uint32_t p0[2], p1[2], b0, b1;
+              const uint32_t w0[8] = {w[k][0], w[k][1], w[k][2], w[k][3], w[k][4], w[k][5], w[k][6], w[k][7]};
+              const uint32_t w1[8] = {w[k][8], w[k][9], w[k][10], w[k][11], w[k][12], w[k][13], w[k][14], w[k][15]};
+              quant_e4m3_code_block(w0, ts, p0, b0);
+              quant_e4m3_code_block(w1, ts, p1, b1);
+              codes = make_uint4(p0[0], p0[1], p1[0], p1[1]);
+              sbytes = b0 | (b1 << 8);
+            }
+            const int c = j * 32;
+            for (int copy = 0; copy < 2; ++copy) {
+              int stage, kc;
+              if (copy == 0) {
+                stage = c >> 8;
+                kc = (c & 255) >> 5;
+              } else {
+                if (a.k_tail == 0 || c < a.C - a.k_tail) break;
+                const int t = c - (a.C - a.k_tail);
+                stage = a.n_base_stages + (t >> 8);
+                kc = (t & 255) >> 5;
+              }
+              *reinterpret_cast<uint4*>(a.xt + static_cast<size_t>(stage) * Cfg::kBBytes + m * 128 +
+                                        ((kc ^ (m & 7)) << 4)) = codes;
+              uint8_t* sft = a.st + static_cast<size_t>(stage) * Cfg::kSfBytes + (m & 31) * 16 + ((m >> 5) & 3) * 4;
+              if constexpr (E8M0) {
+                sft[(kc >> 2) * 512 + (kc & 3)] = static_cast<uint8_t>(sbytes);
+              } else {
+                const int j0 = 2 * kc;   // 16-element blocks 2kc, 2kc + 1 of the stage
+                sft[(j0 >> 2) * 512 + (j0 & 3)] = static_cast<uint8_t>(sbytes);
+                sft[((j0 + 1) >> 2) * 512 + ((j0 + 1) & 3)] = static_cast<uint8_t>(sbytes >> 8);
+              }
+            }
+          }
+        }
+        if (!E8M0 && blockIdx.x == 0 && tq == 0 && a.ts_x != nullptr) *a.ts_x = ts;
+      }
+      named_bar_sync(2, 128);   // every thread's codes are written before the release below
+      if (tq == 0 && qok && !withheld(blockIdx.x)) st_release_gpu_u64(&sy.qflags[blockIdx.x], tag | 1u);
+      // the CTAs that quantized this CTA's columns: those of split z, and for PRQuant tail stages
+      // every CTA (the tail channels sit in the last base stages)
+      const bool tail = s_begin + n_it > a.n_base_stages && a.k_tail > 0;
+      if (tail) {
+        for (int c = tq; c < G && qok; c += 128) dec_wait_tag(&sy.qflags[c], tag, 55, qok);
+      } else {
+        for (int t = tq; t < T && qok; t += 128) dec_wait_tag(&sy.qflags[t * a.splits + z], tag, 55, qok);
+      }
+      qok = bar_and(2, 128, qok);
+    } else if (!E8M0) {
+      ts = *a.ts_x;   // written by the quantizer grid, complete since griddepcontrol.wait
+    }
+    if (tq == 0) {
+      s_ts = ts;
+      if (qok) mbar_arrive(xready);   // else the producer's bounded wait records the failure
+      else s_fail = 1;
+    }
+    // the activation scales of every stage into TMEM (each warp its lane quadrant)
+    const bool bok = __all_sync(0xFFFFFFFFu, mbar_wait(bfull, 0, 62));
+    if (bok) {
+      for (int it = 0; it < n_it; ++it)
+        tmem_st_scale_atoms<Cfg::kAtoms>(tmem + quad_lanes + sfb_col(it), sSfb + it * Cfg::kSfBytes, lane);
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sfb_ok);
+    if (!bok) s_fail = 1;
+    if (blockIdx.x == 0 && !amax_needed) {
+      // CTA 0 advances the counter at its end: first every CTA's slot (each has read the counter)
+      bool sok = true;
+      for (int c = tq; c < G && sok; c += 128) dec_wait_tag(&sy.slots[c], tag, 54, sok);
+      sok = bar_and(2, 128, sok);
+      if (tq == 0) {
+        s_allseen = sok ? 1 : 0;
+        if (!sok) s_fail = 1;
+      }
+    }
+  } else {
+    if constexpr (VQ) {
+      // ---------------- VQ decode (warps 2..9) into the ring of operand tiles: one warp
+      // instruction covers 32 rows of one 32-element chunk (256 contiguous index bytes, lookups
+      // in one 512-byte codebook, 16-byte stores hitting every bank once per 8 rows); warps 2..5
+      // then put the stage's weight scales into their TMEM lane quadrant
+      const int t = threadIdx.x - 64;
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int slot = it % R;
+        bool w = mbar_wait(&wfull[it], 0, 56);
+        if (it >= R) w = w && mbar_wait(&aempty[slot], ((it / R) - 1) & 1, 57);
+        if (!__all_sync(0xFFFFFFFFu, w)) { ok = false; break; }   // warp-uniform (tcgen05.st below)
+        const uint8_t* idx_s = sW + it * Cfg::kWStride;
+        const uint16_t* lut = reinterpret_cast<const uint16_t*>(idx_s + Cfg::kIdxBytes);
+        uint8_t* a_s = sA + slot * Cfg::kABytes;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = t + 256 * j;
+          const int kc = (c >> 5) & 7, r = (c & 31) | ((c >> 8) << 5);
+          const uint2 iv = *reinterpret_cast<const uint2*>(idx_s + kc * 1024 + r * 8);
+          const uint16_t* L = lut + ((((r >> 6) << 2) + (kc >> 1)) << 8);
+          uint4 o;
+          o.x = L[iv.x & 255u] | (static_cast<uint32_t>(L[(iv.x >> 8) & 255u]) << 16);
+          o.y = L[(iv.x >> 16) & 255u] | (static_cast<uint32_t>(L[iv.x >> 24]) << 16);
+          o.z = L[iv.y & 255u] | (static_cast<uint32_t>(L[(iv.y >> 8) & 255u]) << 16);
+          o.w = L[(iv.y >> 16) & 255u] | (static_cast<uint32_t>(L[iv.y >> 24]) << 16);
+          *reinterpret_cast<uint4*>(a_s + r * 128 + ((kc ^ (r & 7)) << 4)) = o;
+        }
+        fence_proxy_async_smem();
+        if (warp < 6) {
+          if constexpr (SF == 0) {
+            tmem_st_scale_atoms<Cfg::kAtoms>(tmem + quad_lanes + sfa_col(it), idx_s + Cfg::kSfaOff, lane);
+          } else {
+            // lane i, column 4a + c: the 4 scales of row i + 32c in atom a (64 K = column QBlock
+            // a): PostScale's one QBlock byte, or PreScale+'s codebook entry of group a / 2
+            if (SF == 2 && it == 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(scbar, 0, 63)) && ok;
+            const uint8_t* tail = idx_s + Cfg::kSfaOff;
+            uint32_t v[16];
+#pragma unroll
+            for (int at = 0; at < 4; ++at)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int r = lane + 32 * c;
+                if constexpr (SF == 1) v[4 * at + c] = 0x01010101u * tail[(r >> 6) * 4 + at];
+                else v[4 * at + c] = *reinterpret_cast<const uint32_t*>(sScb + tail[r * 2 + (at >> 1)] * 8 + (at & 1) * 4);
+              }
+            tmem_st16(tmem + quad_lanes + sfa_col(it), v);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&decd[slot]);
+          if (warp < 6) mbar_arrive(&sfa_ok[it]);
+        }
+      }
+    } else if (warp < 6) {
+      // ---------------- the weight scales of every stage into TMEM as the blocks land
+      for (int it = 0; it < n_it && ok; ++it) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&wfull[it], 0, 56))) { ok = false; break; }
+        tmem_st_scale_atoms<Cfg::kAtoms>(tmem + quad_lanes + sfa_col(it), sW + it * Cfg::kWStride + Cfg::kSfaOff, lane);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfa_ok[it]);
+      }
+    }
+    if (warp < 6) {
+      // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+      const int q = warp & 3;
+      const int nl = q * 32 + lane;
+      const int n = n0 + nl;
+      const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const int et = threadIdx.x - 64;   // 0..127
+      if (n_it > 0) ok = bar_and(1, 128, ok && mbar_wait(accf, 0, 58) && mbar_wait(xready, 0, 59));
+      else ok = bar_and(1, 128, ok && mbar_wait(xready, 0, 59));
+      tc_fence_after();
+      float alpha = a.alpha;
+      if (!E8M0) alpha *= s_ts;
+      const uint32_t cnt = s_cnt;   // published before xready
+      const unsigned long long tag = dec_tag(cnt + 1u);
+      if (ok && a.splits == 1) {
+#pragma unroll 1
+        for (int c = 0; c < a.M; c += 8) {
+          uint32_t r[8];
+          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c + j < a.M && n < a.N) {
+              const float v = (n_it > 0 ? __uint_as_float(r[j]) : 0.f) * alpha;
+              const size_t o = static_cast<size_t>(c + j) * a.ldy + n;
+              a.y[o] = __float2bfloat16_rn(v);
+              if (a.y32 != nullptr) a.y32[o] = v;
+            }
+        }
+      } else if (ok) {
+        float* mine = a.partials + static_cast<size_t>(blockIdx.x) * BN * 128;
+#pragma unroll 1
+        for (int c = 0; c < a.M; c += 8) {
+          uint32_t r[8];
+          tmem_ld8(trow + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c + j < a.M) mine[(c + j) * 128 + nl] = n_it > 0 ? __uint_as_float(r[j]) : 0.f;
+        }
+        named_bar_sync(1, 128);   // the whole partial is written before the release
+        if (et == 0 && !withheld(blockIdx.x)) st_release_gpu_u64(&sy.pflags[blockIdx.x], tag | 1u);
+        bool pok = true;
+        if (et < a.splits) dec_wait_tag(&sy.pflags[tile * a.splits + et], tag, 60, pok);
+        ok = bar_and(1, 128, pok);
+        if (ok) {
+          // this split's share of the tile's outputs in groups of 4 consecutive rows: every
+          // split's partial loaded at once (16-byte loads through L2), then added in split order
+          const int E4 = a.M * 32;                     // float4 groups of the tile
+          const int q0 = static_cast<int>(static_cast<long>(E4) * z / a.splits);
+          const int q1 = static_cast<int>(static_cast<long>(E4) * (z + 1) / a.splits);
+          const float4* part0 = reinterpret_cast<const float4*>(a.partials) +
+                                static_cast<size_t>(tile) * a.splits * BN * 32;
+          for (int qq = q0 + et; qq < q1; qq += 128) {
+            float4 v[kDecMaxSplits];
+#pragma unroll
+            for (int r = 0; r < kDecMaxSplits; ++r)
+              if (r < a.splits) v[r] = __ldcg(part0 + static_cast<size_t>(r) * BN * 32 + qq);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < kDecMaxSplits; ++r)
+              if (r < a.splits) {
+                acc.x += v[r].x; acc.y += v[r].y; acc.z += v[r].z; acc.w += v[r].w;
+              }
+            const int m = qq >> 5, nn = n0 + (qq & 31) * 4;
+            const float o4[4] = {acc.x * alpha, acc.y * alpha, acc.z * alpha, acc.w * alpha};
+            const size_t o = static_cast<size_t>(m) * a.ldy + nn;
+            if (nn + 3 < a.N && (a.ldy & 3) == 0) {
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(o4[0], o4[1]);
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(o4[2], o4[3]);
+              uint2 pk;
+              pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+              pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+              *reinterpret_cast<uint2*>(a.y + o) = pk;
+              if (a.y32 != nullptr) *reinterpret_cast<float4*>(a.y32 + o) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (nn + j < a.N) {
+                  a.y[o + j] = __float2bfloat16_rn(o4[j]);
+                  if (a.y32 != nullptr) a.y32[o + j] = o4[j];
+                }
+            }
+          }
+        }
+      }
+    }
+  }
+  if (!ok) s_fail = 1;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+  // The next grid reads the counter only after this one has completed (griddepcontrol.wait).
+  if (threadIdx.x == 0) {
+    if (s_fail) atomicAdd(sy.counter, 2u);
+    else if (blockIdx.x == 0 && s_allseen) atomicAdd(sy.counter, 1u);
+  }
+}
+
+}  // namespace ql

@@ -70,9 +70,14 @@ struct Fp4GemmArgs {
   float* partials;          // split tiles: fp32 [tile - full_tiles][splits][BN][128]
   const uint8_t* xq;        // quantized activation codes [M, C/2] (read directly by decode launches)
   int* tickets;             // [split tiles] arrival counters, zero between launches
+  const uint8_t* scb;       // VQ PreScale+: scale codebook [256][8] E4M3 bytes
 };
 
-template <int BN, bool E8M0, bool VQ = false>
+// SF (VQ weights only): where the weight's E4M3 block scales come from -- 0 MXCode PreScale (the
+// stage's scale atoms are stored in its block), 1 PostScale (one scale per 64 x 64 QBlock: the
+// block ends with the stage's 8 QBlock bytes), 2 PreScale+ (the block ends with 2 scale indices
+// per row into a 256 x 8 scale codebook).  For 1 and 2 the decoders build the scale atoms.
+template <int BN, bool E8M0, bool VQ = false, int SF = 0>
 struct Fp4Cfg {
   // warps: 0 producer, 1 MMA, 2..5 epilogue; VQ adds decoders so that warps 2..9 decode
   static constexpr int kDecWarps = VQ ? 8 : 0;
@@ -88,9 +93,14 @@ struct Fp4Cfg {
   static constexpr int kLutBytes = VQ ? 8 * 512 : 0;    // VQ: 2 x 4 QBlock codebooks of 512 B
   // The weight block of one stage, as stored in HBM and copied by one bulk copy:
   // FP4: [codes 16 KB][SFA atoms]; VQ: [indices 8 KB, chunk-major][codebooks 4 KB][SFA atoms].
-  static constexpr int kWBytes = (VQ ? kIdxBytes + kLutBytes : kABytes) + kSfaBytes;
+  static_assert(SF == 0 || (VQ && !E8M0), "PostScale / PreScale+ scales: VQ E4M3-B16 weights");
+  static constexpr int kSfTail = SF == 0 ? kSfaBytes : SF == 1 ? 16 : 256;
+  static constexpr int kWBytes = (VQ ? kIdxBytes + kLutBytes : kABytes) + kSfTail;   // in HBM
+  static constexpr int kWStride = (kWBytes + 1023) / 1024 * 1024;                     // in smem
   static constexpr int kSfaOff = VQ ? kIdxBytes + kLutBytes : kABytes;
-  static constexpr int kStageBytes = kWBytes + kBBytes + kSfbBytes + (VQ ? kABytes : 0);
+  static constexpr int kSfaBuild = SF != 0 ? kSfaBytes : 0;   // built scale atoms per stage
+  static constexpr int kScbBytes = SF == 2 ? 2048 : 0;        // PreScale+ scale codebook
+  static constexpr int kStageBytes = kWStride + kBBytes + kSfbBytes + (VQ ? kABytes : 0) + kSfaBuild;
   static constexpr int kBudget = 212 * 1024;
   static constexpr int kStagesRaw = kBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : (kStagesRaw < 2 ? 2 : kStagesRaw);
@@ -100,7 +110,7 @@ struct Fp4Cfg {
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                  : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
   static_assert(kColsNeeded <= 512, "TMEM budget");
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kScbBytes + 1024 /*align*/ + 512 /*barriers*/;
   static_assert(BN * 128 * 4 <= kStages * kStageBytes, "output staging must fit the ring");
 };
 
@@ -108,11 +118,11 @@ struct Fp4Cfg {
 // create time exactly as the stage buffer wants it, and arrives by one 1-D bulk copy.
 // VQ = true (MXCode PreScale weights): the blocks hold 8-bit indices; warps 2..5 decode each
 // stage's operand tile from the shared-memory codebooks.
-template <int BN, bool E8M0, bool VQ = false>
-__global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
+template <int BN, bool E8M0, bool VQ = false, int SF = 0>
+__global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
                     const __grid_constant__ CUtensorMap tm_y32, const Fp4GemmArgs a) {
-  using Cfg = Fp4Cfg<BN, E8M0, VQ>;
+  using Cfg = Fp4Cfg<BN, E8M0, VQ, SF>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   // 1 KB aligned by offsetting the shared array itself, so that every pointer derived from it
@@ -120,18 +130,21 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   // ring layout (every region 1 KB aligned): weight blocks, B tiles, SFB atoms, decoded A (VQ)
   uint8_t* sW = smem;
-  uint8_t* sB = sW + S * Cfg::kWBytes;
+  uint8_t* sB = sW + S * Cfg::kWStride;
   uint8_t* sSfb = sB + S * Cfg::kBBytes;
   uint8_t* sAdec = sSfb + S * Cfg::kSfbBytes;
-  auto sA = [&](int st) { return VQ ? sAdec + st * Cfg::kABytes : sW + st * Cfg::kWBytes; };
-  uint64_t* full = reinterpret_cast<uint64_t*>(sAdec + (VQ ? S * Cfg::kABytes : 0));
+  auto sA = [&](int st) { return VQ ? sAdec + st * Cfg::kABytes : sW + st * Cfg::kWStride; };
+  uint8_t* sSfaB = sAdec + (VQ ? S * Cfg::kABytes : 0);   // SF 1/2: the stages' built scale atoms
+  uint8_t* sScb = sSfaB + S * Cfg::kSfaBuild;              // SF 2: the scale codebook
+  uint64_t* full = reinterpret_cast<uint64_t*>(sScb + Cfg::kScbBytes);
   uint64_t* empty = full + S;
   uint64_t* decd = empty + S;   // VQ: operand tile decoded
   uint64_t* wfull = decd + S;   // VQ: indices + codebooks + SFA landed
   uint64_t* afull = wfull + S;  // decode: activation tile + SFB landed by cp.async (count 32)
   uint64_t* accf = afull + S;   // accumulator complete
   uint64_t* rbar = accf + 1;    // split-K: the splits' partials landed in the idle ring
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 1);
+  uint64_t* scbar = rbar + 1;   // SF 2: the scale codebook landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(scbar + 1);
   __shared__ int s_last;
   griddep_launch_dependents();
 
@@ -180,10 +193,10 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
     if constexpr (VQ) {
       mbar_arrive_expect_tx(&wfull[st], Cfg::kWBytes);
       if (!lsu_act) mbar_arrive_expect_tx(&full[st], act_bytes);
-      bulk_load(sW + st * Cfg::kWBytes, wblk, Cfg::kWBytes, &wfull[st]);
+      bulk_load(sW + st * Cfg::kWStride, wblk, Cfg::kWBytes, &wfull[st]);
     } else {
       mbar_arrive_expect_tx(&full[st], Cfg::kWBytes + act_bytes);
-      bulk_load(sW + st * Cfg::kWBytes, wblk, Cfg::kWBytes, &full[st]);
+      bulk_load(sW + st * Cfg::kWStride, wblk, Cfg::kWBytes, &full[st]);
     }
   };
   const int pre = min(n_it, S);   // the first ring fill needs no empty-slot wait
@@ -202,10 +215,15 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
     if (lane == 0) {
       mbar_init(accf, 1);
       mbar_init(rbar, 1);
+      mbar_init(scbar, 1);
     }
     fence_mbar_init();
     __syncwarp();
     if (lane == 0) {
+      if constexpr (SF == 2) {
+        mbar_arrive_expect_tx(scbar, Cfg::kScbBytes);
+        bulk_load(sScb, a.scb, Cfg::kScbBytes, scbar);
+      }
       for (int it = 0; it < pre; ++it) issue_weight(it);
       prefetch_tmap(&tm_x);
     }
@@ -295,7 +313,8 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
       const int nat = valid / Cfg::kAtomK;
       const uint32_t ta = tmem + sfa_col0 + st * Cfg::kSfaCols;
       const uint32_t tb = tmem + sfb_col0 + st * Cfg::kSfbCols;
-      const uint32_t sfa_s = smem_u32(sW + st * Cfg::kWBytes + Cfg::kSfaOff);
+      const uint32_t sfa_s = SF != 0 ? smem_u32(sSfaB + st * Cfg::kSfaBuild)
+                                     : smem_u32(sW + st * Cfg::kWStride + Cfg::kSfaOff);
       const uint32_t sfb_s = smem_u32(sSfb + st * Cfg::kSfbBytes);
       const uint32_t a_base = smem_u32(sA(st));
       const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
@@ -350,7 +369,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
         if (!mbar_wait(&wfull[st], ph, 5)) { ok = false; break; }
-        const uint8_t* idx_s = sW + st * Cfg::kWBytes;
+        const uint8_t* idx_s = sW + st * Cfg::kWStride;
         const uint16_t* lut = reinterpret_cast<const uint16_t*>(idx_s + Cfg::kIdxBytes);
         uint8_t* a_s = sA(st);
 #pragma unroll
@@ -365,6 +384,25 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ>::kThreads, 1)
           o.z = L[iv.y & 255u] | (static_cast<uint32_t>(L[(iv.y >> 8) & 255u]) << 16);
           o.w = L[(iv.y >> 16) & 255u] | (static_cast<uint32_t>(L[iv.y >> 24]) << 16);
           *reinterpret_cast<uint4*>(a_s + r * 128 + ((kc ^ (r & 7)) << 4)) = o;
+        }
+        if constexpr (SF != 0) {
+          // the stage's four scale atoms (row r at (r%32)*16 + ((r/32)%4)*4, 4 scale columns per
+          // atom): PostScale gives all 16-blocks of a QBlock its one byte, PreScale+ looks the
+          // row's two 8-scale groups up in the scale codebook
+          if (SF == 2 && it == 0 && !mbar_wait(scbar, 0, 7)) { ok = false; }
+          const uint8_t* tail = idx_s + Cfg::kSfaOff;
+          uint8_t* sfa = sSfaB + st * Cfg::kSfaBuild;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int wi = t + kDT * j;          // 512 words: atom wi / 128, row wi % 128
+            if (wi < 512) {
+              const int at = wi >> 7, r = wi & 127;
+              uint32_t word;
+              if constexpr (SF == 1) word = 0x01010101u * tail[(r >> 6) * 4 + at];
+              else word = *reinterpret_cast<const uint32_t*>(sScb + tail[r * 2 + (at >> 1)] * 8 + (at & 1) * 4);
+              *reinterpret_cast<uint32_t*>(sfa + at * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4) = word;
+            }
+          }
         }
         fence_proxy_async_smem();   // every writer orders its stores for the tensor core
         __syncwarp();

@@ -7,6 +7,7 @@
 // from its caller; this entry point instead uses one scratch array that lives in the library
 // itself (a file-scope __device__ array, so every GPU that loads the library holds it until the
 // process exits).  The caller still passes x, y and the optional fp32 y.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -24,25 +25,52 @@ constexpr size_t kFixedScratchBytes = size_t(8) << 20;  // 8 MiB per device
 __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
 
 // In host code `g_fixed_scratch` names a host-side stand-in, not device memory: its device
-// address must be looked up once per device with that device current.
+// address must be looked up with the device current.  The address is cached per device ordinal
+// together with the context it belongs to, and looked up again when the current context is a
+// different one (after cudaDeviceReset the module is loaded anew and the array may move).
 constexpr int kMaxDevices = 64;
+struct ScratchEntry {
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+ScratchEntry g_scratch[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
 
 ql_status scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ql_set_error(QL_ERR_CUDA, "cudaGetDevice failed");
   if (dev < 0 || dev >= kMaxDevices)
     return ql_set_error(QL_ERR_UNSUPPORTED, "device ordinal beyond the fixed-scratch table");
+  CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (get_ctx == nullptr) return ql_set_error(QL_ERR_CUDA, "cuCtxGetCurrent unavailable");
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  CUcontext ctx = nullptr;
+  get_ctx(&ctx);
+  ScratchEntry& e = g_scratch[dev];
+  if (e.addr == nullptr || ctx == nullptr || e.ctx != ctx) {
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_fixed_scratch);
-    if (e != cudaSuccess || p == nullptr)
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_fixed_scratch);   // makes a context current
+    if (err != cudaSuccess || p == nullptr)
       return ql_set_error(QL_ERR_CUDA, "cudaGetSymbolAddress of the fixed scratch array failed");
-    g_scratch_addr[dev] = p;
+    get_ctx(&ctx);
+    e.ctx = ctx;
+    e.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return QL_OK;
 }
 

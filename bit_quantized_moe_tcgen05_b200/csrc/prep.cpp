@@ -339,3 +339,145 @@ extern "C" ql_status qlinear_prepare_int4_bsr(const uint16_t* w_bf16, int64_t N,
   *nnzb_out = static_cast<int32_t>(keep);
   return QL_OK;
 }
+
+// MXCode PostScale (MXCode abstract: "quantizes learned codebooks to MXFP4"): each QBlock's
+// learned codebook (256 x 4 values) is quantized to E2M1 with one E4M3 scale for the whole
+// codebook, relative to an FP32 tensor scale over all codebooks, so that every 16-block of the
+// decoded weight in the QBlock carries that scale (an MX-native operand; no per-weight scales).
+// Each 4-vector of W takes the nearest decoded entry (exact values, squared distance in double,
+// ties to the lowest index).
+extern "C" ql_status qlinear_prepare_vq_postscale(const uint16_t* w_bf16, int64_t N, int64_t K,
+                                                  const float* centroids, int32_t qn, int32_t qk,
+                                                  float* ts_out, uint8_t* codebooks_out,
+                                                  uint8_t* qscales_out, uint8_t* idx_out) {
+  if (w_bf16 == nullptr || centroids == nullptr || ts_out == nullptr || codebooks_out == nullptr ||
+      qscales_out == nullptr || idx_out == nullptr)
+    return QL_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || qn != 64 || qk != 64 || N % qn != 0 || K % qk != 0)
+    return QL_ERR_UNSUPPORTED;
+  static const E4m3Table tab;
+  const int64_t QR = N / qn, QC = K / qk, nq = QR * QC;
+  float amax_t = 0.f;
+  for (int64_t i = 0; i < nq * 1024; ++i) amax_t = std::max(amax_t, std::fabs(centroids[i]));
+  const float ts = amax_t == 0.f ? 1.f : amax_t / 2688.0f;
+  *ts_out = ts;
+  std::vector<double> vals(static_cast<size_t>(nq) * 1024);   // decoded entry values
+  for (int64_t q = 0; q < nq; ++q) {
+    const float* c = centroids + q * 1024;
+    float am = 0.f;
+    for (int i = 0; i < 1024; ++i) am = std::max(am, std::fabs(c[i]));
+    const float t = am / 6.0f;
+    const float r = t / ts;
+    const uint8_t s = tab.encode(r);
+    qscales_out[q] = s;
+    const float S = tab.v[s] * ts;
+    const double scale = static_cast<double>(tab.v[s]) * static_cast<double>(ts);
+    uint8_t* cb = codebooks_out + q * 512;
+    for (int e = 0; e < 256; ++e) {
+      uint8_t code[4];
+      for (int i = 0; i < 4; ++i) {
+        const float x = c[e * 4 + i];
+        code[i] = S == 0.f ? static_cast<uint8_t>(std::signbit(x) ? 8 : 0) : e2m1_code(x / S);
+        vals[q * 1024 + e * 4 + i] = static_cast<double>(e2m1_value(code[i])) * scale;
+      }
+      cb[e * 2] = static_cast<uint8_t>((code[0] & 0xF) | (code[1] << 4));
+      cb[e * 2 + 1] = static_cast<uint8_t>((code[2] & 0xF) | (code[3] << 4));
+    }
+  }
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t n = 0; n < N; ++n) {
+    const int64_t qr = n / qn;
+    for (int64_t j = 0; j < K / 4; ++j) {
+      const double* v = vals.data() + (qr * QC + (j * 4) / qk) * 1024;
+      int best = 0;
+      double bestd = 0;
+      for (int e = 0; e < 256; ++e) {
+        double d = 0;
+        for (int i = 0; i < 4; ++i) {
+          const double diff = static_cast<double>(bf16_to_f32(w_bf16[n * K + j * 4 + i])) - v[e * 4 + i];
+          d += diff * diff;
+        }
+        if (e == 0 || d < bestd) { bestd = d; best = e; }
+      }
+      idx_out[n * (K / 4) + j] = static_cast<uint8_t>(best);
+    }
+  }
+  return QL_OK;
+}
+
+// MXCode PreScale+ (MXCode abstract: PreScale's scales "further compressed using VQ"; appendix
+// Table 4 caption: Ks = 256, ds = 8): the E4M3 block scales of PreScale, 8 consecutive along K,
+// are replaced by the nearest of 256 scale vectors of a per-tensor scale codebook (squared
+// distance of decoded scale values in double, ties to the lowest index); W is then normalised by
+// the compressed scales and assigned as in PreScale.  Outputs: ts, the compressed scale bytes
+// [N, K/16], the scale indices [N, K/128] and the weight indices [N, K/4].
+extern "C" ql_status qlinear_prepare_vq_prescale_plus(const uint16_t* w_bf16, int64_t N, int64_t K,
+                                                      const uint8_t* codebooks,
+                                                      const uint8_t* scale_codebook, int32_t qn,
+                                                      int32_t qk, float* ts_out,
+                                                      uint8_t* scales_out, uint8_t* sidx_out,
+                                                      uint8_t* idx_out) {
+  if (w_bf16 == nullptr || codebooks == nullptr || scale_codebook == nullptr || ts_out == nullptr ||
+      scales_out == nullptr || sidx_out == nullptr || idx_out == nullptr)
+    return QL_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || qn != 64 || qk != 64 || N % qn != 0 || K % qk != 0 || K % 128 != 0)
+    return QL_ERR_UNSUPPORTED;
+  static const E4m3Table tab;
+  float amax = 0.f;
+  for (int64_t i = 0; i < N * K; ++i) amax = std::max(amax, std::fabs(bf16_to_f32(w_bf16[i])));
+  const float ts = amax == 0.f ? 1.f : amax / 2688.0f;
+  *ts_out = ts;
+  const int64_t QC = K / qk, G16 = K / 16;
+  static const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t n = 0; n < N; ++n) {
+    std::vector<uint8_t> s0(G16);
+    for (int64_t b = 0; b < G16; ++b) {
+      float am = 0.f;
+      for (int i = 0; i < 16; ++i) am = std::max(am, std::fabs(bf16_to_f32(w_bf16[n * K + b * 16 + i])));
+      const float t = am / 6.0f;
+      s0[b] = tab.encode(t / ts);
+    }
+    for (int64_t g = 0; g < G16 / 8; ++g) {   // nearest scale vector
+      int best = 0;
+      double bestd = 0;
+      for (int e = 0; e < 256; ++e) {
+        double d = 0;
+        for (int i = 0; i < 8; ++i) {
+          const uint8_t cb = scale_codebook[e * 8 + i];
+          const double diff = static_cast<double>(tab.v[s0[g * 8 + i] & 0x7F]) -
+                              static_cast<double>(cb <= 126 ? tab.v[cb] : 0.f);
+          d += diff * diff;
+        }
+        if (e == 0 || d < bestd) { bestd = d; best = e; }
+      }
+      sidx_out[n * (G16 / 8) + g] = static_cast<uint8_t>(best);
+      for (int i = 0; i < 8; ++i) scales_out[n * G16 + g * 8 + i] = scale_codebook[best * 8 + i];
+    }
+    std::vector<float> v(K);
+    for (int64_t b = 0; b < G16; ++b) {
+      const uint8_t s = scales_out[n * G16 + b];
+      const float S = (s <= 126 ? tab.v[s] : 0.f) * ts;
+      for (int i = 0; i < 16; ++i)
+        v[b * 16 + i] = S == 0.f ? 0.f : bf16_to_f32(w_bf16[n * K + b * 16 + i]) / S;
+    }
+    const int64_t qr = n / qn;
+    for (int64_t j = 0; j < K / 4; ++j) {
+      const uint8_t* cb = codebooks + ((qr * QC + (j * 4) / qk) * 256) * 2;
+      int best = 0;
+      double bestd = 0;
+      for (int e = 0; e < 256; ++e) {
+        double d = 0;
+        for (int i = 0; i < 4; ++i) {
+          const uint8_t c = (cb[e * 2 + i / 2] >> (4 * (i & 1))) & 0xF;
+          const double cv = (c & 8) ? -mag[c & 7] : mag[c & 7];
+          const double diff = static_cast<double>(v[j * 4 + i]) - cv;
+          d += diff * diff;
+        }
+        if (e == 0 || d < bestd) { bestd = d; best = e; }
+      }
+      idx_out[n * (K / 4) + j] = static_cast<uint8_t>(best);
+    }
+  }
+  return QL_OK;
+}

@@ -16,6 +16,19 @@ __device__ int g_dev_error_site;
 
 enum : int { DEV_OK = 0, DEV_TIMEOUT = 5 };
 
+// Limit of the bounded waits (ns), and, for tests of the timeout path only, the index of a CTA
+// whose grid-wide publications (slots of the E4M3-B16 amax agreement, decode flags) are withheld
+// so that the waits on them run out (-1: none).  Set from the host by ql_debug_inject.
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+__device__ int g_debug_withhold_cta = -1;
+
+__device__ __forceinline__ unsigned long long wait_limit_ns() {
+  return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
+__device__ __forceinline__ bool withheld(int cta) {
+  return cta == *reinterpret_cast<volatile int*>(&g_debug_withhold_cta);
+}
+
 __device__ __forceinline__ void record_error(int code, int site) {
   if (atomicCAS(&g_dev_error, 0, code) == 0) g_dev_error_site = site;
 }
@@ -80,10 +93,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait: spins until the phase with the given parity completes, or until `limit_ns`
-// elapses, in which case the device error word is set and false is returned.
+// (0: the library's wait limit, 2 s unless a test lowered it) elapses, in which case the device
+// error word is set and false is returned.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site,
-                                          uint64_t limit_ns = 2000000000ull) {
+                                          uint64_t limit_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (limit_ns == 0) limit_ns = wait_limit_ns();
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -329,6 +344,42 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Store 16 consecutive 32-bit TMEM columns of this thread's lane (32x32b shape; the warp writes
+// the 32 lanes of its own lane quadrant).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// The scale atoms of one 256-K stage (kAtoms x 512 B in shared memory, the tcgen05.cp 32x128b
+// source layout) into TMEM columns [col, col + 4 * kAtoms) of this warp's lane quadrant, laid
+// out as tcgen05.cp .32x128b.warpx4 would put them: lane i of every quadrant, column 4a + c,
+// holds the 4 bytes at atom a, offset 16 i + 4 c.  Called by four warps (one per quadrant); the
+// caller waits for the stores (tcgen05.wait::st) before signalling the MMA issuer.
+template <int kAtoms>
+__device__ __forceinline__ void tmem_st_scale_atoms(uint32_t taddr_lane, const uint8_t* atoms,
+                                                    int lane) {
+  static_assert(kAtoms == 2 || kAtoms == 4, "2 or 4 scale atoms per stage");
+  uint32_t v[16];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (a < kAtoms) w = *reinterpret_cast<const uint4*>(atoms + a * 512 + lane * 16);
+    v[4 * a] = w.x; v[4 * a + 1] = w.y; v[4 * a + 2] = w.z; v[4 * a + 3] = w.w;
+  }
+  if constexpr (kAtoms == 4) {
+    tmem_st16(taddr_lane, v);
+  } else {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr_lane),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+  }
 }
 
 // ---------------------------------------------------------------- descriptors

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -17,6 +18,7 @@
 #include "ptx.cuh"
 #include "quant_act.cuh"
 #include "gemm_fp4.cuh"
+#include "decode_fp4.cuh"
 #include "moe.cuh"
 #include "int4_gemm.cuh"
 #include "peak.cuh"
@@ -124,15 +126,15 @@ int sm_count() {
 // The GEMM is launched with programmatic stream serialization: it may start while the kernel
 // before it on the stream (the activation quantizer) is still running, and streams (and, for VQ,
 // decodes) weights until its griddepcontrol.wait.
-template <int BN, bool E8M0, bool VQ>
+template <int BN, bool E8M0, bool VQ, int SF = 0>
 ql_status launch_fp4_bn(const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& ty32,
                         const ql::Fp4GemmArgs& a, dim3 grid, cudaStream_t s) {
-  using Cfg = ql::Fp4Cfg<BN, E8M0, VQ>;
+  using Cfg = ql::Fp4Cfg<BN, E8M0, VQ, SF>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    QL_CUDA(cudaFuncSetAttribute(ql::fp4_gemm_kernel<BN, E8M0, VQ>,
+    QL_CUDA(cudaFuncSetAttribute(ql::fp4_gemm_kernel<BN, E8M0, VQ, SF>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
     attr_done[dev] = true;
   }
@@ -146,22 +148,57 @@ ql_status launch_fp4_bn(const CUtensorMap& tx, const CUtensorMap& ty, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_gemm_kernel<BN, E8M0, VQ>, tx, ty, ty32, a));
+  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_gemm_kernel<BN, E8M0, VQ, SF>, tx, ty, ty32, a));
   return QL_OK;
 }
 
-template <bool E8M0, bool VQ>
+template <bool E8M0, bool VQ, int SF = 0>
 ql_status launch_fp4(int BN, const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& ty32,
                      const ql::Fp4GemmArgs& a, dim3 grid, cudaStream_t s) {
   switch (BN) {
-    case 16: return launch_fp4_bn<16, E8M0, VQ>(tx, ty, ty32, a, grid, s);
-    case 32: return launch_fp4_bn<32, E8M0, VQ>(tx, ty, ty32, a, grid, s);
-    case 64: return launch_fp4_bn<64, E8M0, VQ>(tx, ty, ty32, a, grid, s);
-    case 128: return launch_fp4_bn<128, E8M0, VQ>(tx, ty, ty32, a, grid, s);
-    case 160: return launch_fp4_bn<160, E8M0, VQ>(tx, ty, ty32, a, grid, s);
-    case 256: return launch_fp4_bn<256, E8M0, VQ>(tx, ty, ty32, a, grid, s);
+    case 16: return launch_fp4_bn<16, E8M0, VQ, SF>(tx, ty, ty32, a, grid, s);
+    case 32: return launch_fp4_bn<32, E8M0, VQ, SF>(tx, ty, ty32, a, grid, s);
+    case 64: return launch_fp4_bn<64, E8M0, VQ, SF>(tx, ty, ty32, a, grid, s);
+    case 128: return launch_fp4_bn<128, E8M0, VQ, SF>(tx, ty, ty32, a, grid, s);
+    case 160: return launch_fp4_bn<160, E8M0, VQ, SF>(tx, ty, ty32, a, grid, s);
+    case 256: return launch_fp4_bn<256, E8M0, VQ, SF>(tx, ty, ty32, a, grid, s);
   }
   return fail(QL_ERR_UNSUPPORTED, "no GEMM tile for BN=%d", BN);
+}
+
+template <int BN, bool E8M0, bool VQ, int SF = 0>
+ql_status launch_dec_bn(const ql::DecodeArgs& a, int grid, cudaStream_t s) {
+  using Cfg = ql::DecCfg<BN, E8M0, VQ, SF>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    QL_CUDA(cudaFuncSetAttribute(ql::fp4_decode_kernel<BN, E8M0, VQ, SF>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+    attr_done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_decode_kernel<BN, E8M0, VQ, SF>, a));
+  return QL_OK;
+}
+
+template <bool E8M0, bool VQ, int SF = 0>
+ql_status launch_dec(int BN, const ql::DecodeArgs& a, int grid, cudaStream_t s) {
+  switch (BN) {
+    case 16: return launch_dec_bn<16, E8M0, VQ, SF>(a, grid, s);
+    case 32: return launch_dec_bn<32, E8M0, VQ, SF>(a, grid, s);
+    case 64: return launch_dec_bn<64, E8M0, VQ, SF>(a, grid, s);
+  }
+  return fail(QL_ERR_UNSUPPORTED, "no decode tile for BN=%d", BN);
 }
 
 // Token-tile width: the smallest power of two >= M up to 128.  Past 128 tokens, 256-wide tiles,
@@ -189,7 +226,9 @@ struct ql_linear {
   int64_t N, K, C;
   int32_t k_tail;
   bool e8m0 = true;            // E8M0-B32 scales (else E4M3-B16 + tensor scales)
-  bool vq = false;             // MXCode PreScale VQ weight
+  bool vq = false;             // MXCode VQ weight
+  int sfmode = 0;              // VQ scales: 0 PreScale atoms, 1 PostScale per QBlock, 2 PreScale+
+  uint8_t* d_scb = nullptr;    // PreScale+: scale codebook [256][8] on the device
   uint8_t* d_codes = nullptr;  // weight blocks [N/128][stages][codes or indices + codebooks, scales]
   size_t weight_bytes = 0;
   float w_ts = 1.f;
@@ -211,8 +250,18 @@ struct FwdPlan {
   size_t sync_off;   // E4M3 grid quantizer: launch counter and per-CTA amax slots
   size_t codes_off, sf_off, scal_off, tick_off, part_off, total;
   int n_tickets;   // split-K tickets (zeroed by the quantizer, re-armed by the GEMM)
+  bool decode = false;   // fp4_decode_kernel: M <= 64, one CTA per (weight tile, K range)
+  bool fusable = false;  // ... and the forward may quantize x inside it (one launch)
+  size_t dsync_off = 0;  // its launch counter, slots and flags
+  size_t xt_off = 0, st_off = 0;   // fused: per-stage B tiles and activation scale sets
 };
 
+
+// Every plan starts with the E4M3-B16 grid quantizer's sync block and the decode kernel's: the
+// launch counters there must survive whatever other layers write into a shared workspace.
+size_t sync_prefix_bytes() {
+  return align_up(align_up(ql::kE4m3SyncBytes, 256) + ql::kDecSyncBytes, 256);
+}
 
 FwdPlan plan_forward_int4(const ql_linear* L, int64_t M) {
   FwdPlan p{};
@@ -227,7 +276,9 @@ FwdPlan plan_forward_int4(const ql_linear* L, int64_t M) {
   p.spp = static_cast<int>(cdiv(total, splits));
   p.splits = static_cast<int>(cdiv(total, p.spp));
   p.sfb_atoms = p.tiles_m * p.BN;                       // ldt of the transposed scales
-  size_t off = 0;
+  // the sync blocks of the FP4 layers stay reserved, so that layers of different formats can
+  // share one workspace without clobbering each other's launch counters
+  size_t off = sync_prefix_bytes();
   p.codes_off = off;                                    // int8 activation [M, K]
   off = align_up(off + static_cast<size_t>(M) * L->K, 256);
   p.sf_off = off;                                       // scales [K/128][ldt]
@@ -237,9 +288,72 @@ FwdPlan plan_forward_int4(const ql_linear* L, int64_t M) {
   return p;
 }
 
+// Most weight stages one decode CTA keeps resident, per token-tile width and weight format.
+template <bool E8M0, bool VQ, int SF = 0>
+int dec_max_stages(int BN) {
+  switch (BN) {
+    case 16: return ql::DecCfg<16, E8M0, VQ, SF>::kMaxStages;
+    case 32: return ql::DecCfg<32, E8M0, VQ, SF>::kMaxStages;
+    default: return ql::DecCfg<64, E8M0, VQ, SF>::kMaxStages;
+  }
+}
+int dec_max_stages(const ql_linear* L, int BN) {
+  if (L->vq && L->sfmode == 1) return dec_max_stages<false, true, 1>(BN);
+  if (L->vq && L->sfmode == 2) return dec_max_stages<false, true, 2>(BN);
+  if (L->vq) return dec_max_stages<false, true>(BN);
+  return L->e8m0 ? dec_max_stages<true, false>(BN) : dec_max_stages<false, false>(BN);
+}
+
+// Decode launches (M <= 64): the weight tiles split along K so that the grid covers the SMs once;
+// each CTA keeps all its stages resident.  Returns false when no such split exists.
+bool plan_decode(const ql_linear* L, int64_t M, FwdPlan& p) {
+  if (L->int4 || M > 64 || M < 1) return false;
+  p.tiles_n = static_cast<int>(cdiv(L->N, 128));
+  p.BN = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.tiles_m = 1;
+  const int sms = std::min(sm_count(), ql::kDecMaxGrid);
+  if (p.tiles_n > sms) return false;
+  const int total = L->n_stages_total;
+  int splits = std::max(1, std::min({sms / p.tiles_n, total, ql::kDecMaxSplits}));
+  p.spp = static_cast<int>(cdiv(total, splits));
+  p.splits = static_cast<int>(cdiv(total, p.spp));
+  if (p.spp > dec_max_stages(L, p.BN)) return false;   // (VQ: leaves room for one ring tile)
+  // fused quantization: split z's units (M rows x its 32-column groups) over the split's tiles
+  const int64_t upr_max = std::min<int64_t>(static_cast<int64_t>(p.spp) * 8, L->C / 32);
+  p.fusable = cdiv(M * upr_max, p.tiles_n) <= 128 * ql::kDecQUnits;
+  p.full_tiles = 0;
+  p.decode = true;
+  return true;
+}
+
 FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   if (L->int4) return plan_forward_int4(L, M);
   FwdPlan p{};
+  if (plan_decode(L, M, p)) {
+    const int atomK = L->e8m0 ? 128 : 64;
+    p.sfb_atoms = static_cast<int>(cdiv(L->C, atomK));
+    p.sf_rows = 128;
+    p.sync_off = 0;   // (the E4M3 grid quantizer of qlinear_quantize_input)
+    p.dsync_off = align_up(ql::kE4m3SyncBytes, 256);
+    size_t off = sync_prefix_bytes();
+    p.codes_off = off;
+    off = align_up(off + static_cast<size_t>(M) * (L->C / 2), 256);
+    p.sf_off = off;   // one 128-row group of scale atoms (the quantizers write up to 2)
+    off = align_up(off + static_cast<size_t>(2) * p.sfb_atoms * 512, 256);
+    p.scal_off = off;   // [0] amax bit pattern, [1] tensor scale (E4M3-B16)
+    p.tick_off = off + 2 * sizeof(float);
+    p.n_tickets = 0;
+    off = align_up(p.tick_off, 256);
+    p.xt_off = off;     // per K stage: B tile [BN][128 B], then (st) its scale atoms
+    off = align_up(off + static_cast<size_t>(L->n_stages_total) * p.BN * 128, 256);
+    p.st_off = off;
+    off = align_up(off + static_cast<size_t>(L->n_stages_total) * (L->e8m0 ? 2 : 4) * 512, 256);
+    p.part_off = off;
+    if (p.splits > 1)
+      off = align_up(off + static_cast<size_t>(p.tiles_n) * p.splits * p.BN * 128 * 4, 256);
+    p.total = off;
+    return p;
+  }
   p.tiles_n = static_cast<int>(cdiv(L->N, 128));
   p.BN = pick_bn(M, p.tiles_n);
   p.tiles_m = static_cast<int>(cdiv(std::max<int64_t>(M, 1), p.BN));
@@ -264,9 +378,9 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   // 128-row atom groups of the tiled activation scales: ceil(sf_rows / 128) per token tile
   const int64_t sf_groups = std::max<int64_t>(cdiv(std::max<int64_t>(M, 1), 256) * 2,
                                               static_cast<int64_t>(p.tiles_m) * cdiv(p.sf_rows, 128));
-  size_t off = 0;
-  p.sync_off = off;
-  off = align_up(off + ql::kE4m3SyncBytes, 256);
+  p.sync_off = 0;
+  p.dsync_off = align_up(ql::kE4m3SyncBytes, 256);
+  size_t off = sync_prefix_bytes();
   p.codes_off = off;
   off = align_up(off + static_cast<size_t>(M) * (L->C / 2), 256);
   p.sf_off = off;
@@ -294,6 +408,38 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
 // then the stage's weight scales as 512-byte atoms of 128 rows x 4 scale columns (row r at
 // (r%32)*16 + ((r/32)%4)*4, column j at j%4; the layout tcgen05.cp moves into TMEM).  Rows past N
 // and elements past a partial stage are zero.  Returns the block size.
+// VQ weights with MXCode PostScale (sfmode 1) or PreScale+ (sfmode 2) scales: the same indices
+// and codebooks, then instead of the scale atoms the stage's 8 QBlock scale bytes (2 row QBlocks
+// x 4 column QBlocks; 16 bytes with padding) or its 128 x 2 scale indices (row-major).
+size_t repack_vq_blocks(const uint8_t* idx, const uint8_t* scales, const uint8_t* lut, int64_t N,
+                        int64_t K, int sfmode, std::vector<uint8_t>& out) {
+  const int64_t stages = cdiv(K, 256), tiles = cdiv(N, 128);
+  const size_t tail = sfmode == 1 ? 16 : 256;
+  const size_t blk_bytes = 128 * 64 + 8 * 512 + tail;
+  out.assign(static_cast<size_t>(tiles) * stages * blk_bytes, 0);
+  for (int64_t t = 0; t < tiles; ++t)
+    for (int64_t i = 0; i < stages; ++i) {
+      const int64_t kw = i * 256;
+      uint8_t* blk = out.data() + (static_cast<size_t>(t) * stages + i) * blk_bytes;
+      for (int r = 0; r < 128; ++r) {
+        const int64_t n = t * 128 + r;
+        if (n >= N) break;
+        for (int b = 0; b < 64; ++b) blk[(b >> 3) * 1024 + r * 8 + (b & 7)] = idx[n * (K / 4) + kw / 4 + b];
+        if (sfmode == 2)
+          for (int g = 0; g < 2; ++g) blk[128 * 64 + 8 * 512 + r * 2 + g] = scales[n * (K / 128) + kw / 128 + g];
+      }
+      for (int g2 = 0; g2 < 2; ++g2)
+        for (int q = 0; q < 4; ++q) {
+          const int64_t qr = t * 2 + g2, qc = kw / 64 + q;
+          if (qr * 64 < N && qc * 64 < K) {
+            std::memcpy(blk + 128 * 64 + g2 * 2048 + q * 512, lut + (static_cast<size_t>(qr) * (K / 64) + qc) * 512, 512);
+            if (sfmode == 1) blk[128 * 64 + 8 * 512 + g2 * 4 + q] = scales[qr * (K / 64) + qc];
+          }
+        }
+    }
+  return blk_bytes;
+}
+
 size_t repack_weight_blocks(const uint8_t* src, const uint8_t* scales, const uint8_t* lut,
                             int64_t N, int64_t K, int64_t C, int64_t k_tail, bool vq, bool e8m0,
                             std::vector<uint8_t>& out) {
@@ -419,11 +565,11 @@ ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, u
 // Cluster size for the one-launch quantizer: 16 CTAs where the device can co-schedule such a
 // cluster, else the portable 8.
 int e4m3_cluster_size() {
-  static int size[64] = {};
+  static std::atomic<int> size[64] = {};   // 0 until probed; host threads may race to probe
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 64) return 8;
-  if (size[dev] == 0) {
+  if (dev < 0 || dev >= 64) return 8;
+  if (size[dev].load(std::memory_order_acquire) == 0) {
     int want = 8;
     if (cudaFuncSetAttribute(ql::quant_e4m3_b16_cluster_kernel,
                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
@@ -443,9 +589,9 @@ int e4m3_cluster_size() {
         want = 16;
     }
     cudaGetLastError();
-    size[dev] = want;
+    size[dev].store(want, std::memory_order_release);
   }
-  return size[dev];
+  return size[dev].load(std::memory_order_acquire);
 }
 
 // Tensors whose 16-element blocks fit the registers of one cluster (kE4m3RegBlocks per thread)
@@ -638,7 +784,9 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
     return create_int4_bsr(d, reinterpret_cast<cudaStream_t>(stream), out);
   const bool mx = d->wfmt == QL_W_MXFP4_E8M0_B32;
   const bool nv = d->wfmt == QL_W_NVFP4_E4M3_B16;
-  const bool vq = d->wfmt == QL_W_VQ_PRESCALE_E4M3_B16;
+  const int sfmode = d->wfmt == QL_W_VQ_POSTSCALE_E4M3_B16 ? 1
+                   : d->wfmt == QL_W_VQ_PRESCALE_PLUS_E4M3_B16 ? 2 : 0;
+  const bool vq = d->wfmt == QL_W_VQ_PRESCALE_E4M3_B16 || sfmode != 0;
   if (!mx && !nv && !vq)
     return fail(QL_ERR_UNSUPPORTED, "weight format %d not supported by qlinear_create",
                 int(d->wfmt));
@@ -657,6 +805,9 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
     return fail(QL_ERR_UNSUPPORTED, "VQ layer needs N%%128==0, K%%256==0, 64x64 QBlocks, no tail");
   if ((nv || vq) && !(d->w_tensor_scale > 0.f))
     return fail(QL_ERR_INVALID_ARG, "E4M3-B16 weights need a positive FP32 tensor scale");
+  if (sfmode == 2 && (d->scale_codebook == nullptr || d->scale_codebook_entries != 256 ||
+                      d->scale_group != 8))
+    return fail(QL_ERR_UNSUPPORTED, "PreScale+ needs a scale codebook of 256 entries of 8 scales");
   if (d->N > (1 << 24) || d->K > (1 << 24))
     return fail(QL_ERR_UNSUPPORTED, "N/K too large");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -668,16 +819,22 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
   L->C = d->K - d->k_tail;
   L->e8m0 = mx;
   L->vq = vq;
+  L->sfmode = sfmode;
   L->w_ts = mx ? 1.f : d->w_tensor_scale;
   L->n_base_stages = static_cast<int>(cdiv(L->C, 256));
   L->n_stages_total = L->n_base_stages + static_cast<int>(cdiv(L->k_tail, 256));
   std::vector<uint8_t> blocks;
-  const size_t blk = repack_weight_blocks(vq ? static_cast<const uint8_t*>(d->indices)
-                          : static_cast<const uint8_t*>(d->codes),
-                       static_cast<const uint8_t*>(d->scales),
-                       vq ? static_cast<const uint8_t*>(d->codebooks) : nullptr, d->N, d->K, L->C,
-                       L->k_tail, vq, mx, blocks);
-  const size_t want = vq ? ql::Fp4Cfg<16, false, true>::kWBytes
+  const size_t blk = sfmode != 0
+      ? repack_vq_blocks(static_cast<const uint8_t*>(d->indices), static_cast<const uint8_t*>(d->scales),
+                         static_cast<const uint8_t*>(d->codebooks), d->N, d->K, sfmode, blocks)
+      : repack_weight_blocks(vq ? static_cast<const uint8_t*>(d->indices)
+                                : static_cast<const uint8_t*>(d->codes),
+                             static_cast<const uint8_t*>(d->scales),
+                             vq ? static_cast<const uint8_t*>(d->codebooks) : nullptr, d->N, d->K,
+                             L->C, L->k_tail, vq, mx, blocks);
+  const size_t want = sfmode == 1 ? ql::Fp4Cfg<16, false, true, 1>::kWBytes
+                    : sfmode == 2 ? ql::Fp4Cfg<16, false, true, 2>::kWBytes
+                    : vq ? ql::Fp4Cfg<16, false, true>::kWBytes
                          : (mx ? ql::Fp4Cfg<16, true, false>::kWBytes : ql::Fp4Cfg<16, false, false>::kWBytes);
   if (blk != want) {
     delete L;
@@ -686,9 +843,16 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
   const size_t code_bytes = blocks.size();
   auto cleanup = [&](ql_status st) {
     if (L->d_codes) cudaFree(L->d_codes);
+    if (L->d_scb) cudaFree(L->d_scb);
     delete L;
     return st;
   };
+  if (sfmode == 2) {
+    if (cudaMalloc(&L->d_scb, 256 * 8) != cudaSuccess)
+      return cleanup(fail(QL_ERR_OOM, "cudaMalloc of the scale codebook failed"));
+    if (cudaMemcpyAsync(L->d_scb, d->scale_codebook, 256 * 8, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return cleanup(fail(QL_ERR_CUDA, "scale codebook upload failed"));
+  }
   if (cudaMalloc(&L->d_codes, code_bytes) != cudaSuccess)
     return cleanup(fail(QL_ERR_OOM, "cudaMalloc of %zu weight bytes failed", code_bytes));
   if (cudaMemcpyAsync(L->d_codes, blocks.data(), code_bytes, cudaMemcpyHostToDevice, s) !=
@@ -703,6 +867,7 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
 ql_status qlinear_destroy(ql_linear* L) {
   if (L == nullptr) return QL_OK;
   if (L->d_codes) cudaFree(L->d_codes);
+  if (L->d_scb) cudaFree(L->d_scb);
   if (L->d_stage_start) cudaFree(L->d_stage_start);
   if (L->d_stage_group) cudaFree(L->d_stage_group);
   delete L;
@@ -750,6 +915,43 @@ ql_status qlinear_quantize_input(const ql_linear* L, const void* x, int64_t M, v
                          reinterpret_cast<cudaStream_t>(stream), nullptr, p.sf_rows);
 }
 
+// The decode kernel: x != null quantizes x inside it (qlinear_forward), else the workspace holds
+// the quantized activations (qlinear_quantize_input, then qlinear_gemm).
+static ql_status launch_decode(const ql_linear* L, int64_t M, const FwdPlan& p, const void* x,
+                               void* y, float* y32, uint8_t* w8, ql_stream_t stream) {
+  ql::DecodeArgs a{};
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(L->N);
+  a.C = static_cast<int>(L->C);
+  a.k_tail = L->k_tail;
+  a.n_base_stages = L->n_base_stages;
+  a.n_stages_total = L->n_stages_total;
+  a.spp = p.spp;
+  a.splits = p.splits;
+  a.fuse = x != nullptr ? 1 : 0;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.xq = w8 + p.codes_off;
+  a.sfb = w8 + p.sf_off;
+  a.xt = w8 + p.xt_off;
+  a.st = w8 + p.st_off;
+  a.ts_x = reinterpret_cast<float*>(w8 + p.scal_off) + 1;
+  a.alpha = L->w_ts;
+  a.wt = L->d_codes;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.y32 = y32;
+  a.ldy = static_cast<int>(L->N);
+  a.partials = reinterpret_cast<float*>(w8 + p.part_off);
+  a.sync = w8 + p.dsync_off;
+  a.scb = L->d_scb;
+  const int grid = p.tiles_n * p.splits;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (L->vq && L->sfmode == 1) return launch_dec<false, true, 1>(p.BN, a, grid, cs);
+  if (L->vq && L->sfmode == 2) return launch_dec<false, true, 2>(p.BN, a, grid, cs);
+  if (L->vq) return launch_dec<false, true>(p.BN, a, grid, cs);
+  if (!L->e8m0) return launch_dec<false, false>(p.BN, a, grid, cs);
+  return launch_dec<true, false>(p.BN, a, grid, cs);
+}
+
 ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void* ws,
                        size_t ws_bytes, ql_stream_t stream) {
   if (L != nullptr && M == 0) return QL_OK;
@@ -787,6 +989,7 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
       default: return launch_int4_bn<128>(tx, ty, ty32, a, grid, cs);
     }
   }
+  if (p.decode) return launch_decode(L, M, p, nullptr, y, y32, w8, stream);
   CUtensorMap tm_x;
   st = make_tmap_u8(&tm_x, w8 + p.codes_off, L->C / 2, M, L->C / 2, 128, p.BN);
   if (st != QL_OK) return st;
@@ -822,6 +1025,9 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   if (st == QL_OK) st = make_tmap_out(&tm_y32, y32 ? static_cast<const void*>(y32) : y, y32 != nullptr,
                                       L->N, M, L->N, p.BN);
   if (st != QL_OK) return st;
+  a.scb = L->d_scb;
+  if (L->vq && L->sfmode == 1) return launch_fp4<false, true, 1>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
+  if (L->vq && L->sfmode == 2) return launch_fp4<false, true, 2>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
   if (L->vq) return launch_fp4<false, true>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
   if (!L->e8m0) return launch_fp4<false, false>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
   return launch_fp4<true, false>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
@@ -832,6 +1038,16 @@ ql_status qlinear_forward(const ql_linear* L, const void* x, int64_t M, void* y,
   if (L == nullptr || M < 0) return fail(QL_ERR_INVALID_ARG, "null layer or negative M");
   if (M == 0) return QL_OK;
   if (x == nullptr || y == nullptr) return fail(QL_ERR_INVALID_ARG, "null x/y");
+  {
+    FwdPlan p;
+    ql_status st = check_ws(L, M, ws, ws_bytes, &p);
+    if (st != QL_OK) return st;
+    if (p.decode && p.fusable) {   // one launch: the activations are quantized inside the GEMM
+      if ((reinterpret_cast<uintptr_t>(x) & 15) != 0)
+        return fail(QL_ERR_INVALID_ARG, "x must be 16-byte aligned");
+      return launch_decode(L, M, p, x, y, y32, static_cast<uint8_t*>(ws), stream);
+    }
+  }
   ql_status st = qlinear_quantize_input(L, x, M, ws, ws_bytes, stream);
   if (st != QL_OK) return st;
   return qlinear_gemm(L, M, y, y32, ws, ws_bytes, stream);
@@ -892,6 +1108,16 @@ ql_status ql_tensor_peak(int32_t kind, int32_t n, int32_t iters, int32_t ctas,
     case 3 * 1000 + 256: return launch_peak<3, 256>(ctas, iters, s, flops_per_launch);
     default: return fail(QL_ERR_UNSUPPORTED, "tensor peak kind %d with N %d", int(kind), int(n));
   }
+}
+
+ql_status ql_debug_inject(int32_t withhold_cta, uint64_t wait_limit_ns) {
+  if (withhold_cta < -1) return fail(QL_ERR_INVALID_ARG, "withhold_cta must be >= -1");
+  const unsigned long long lim = wait_limit_ns == 0 ? 2000000000ull : wait_limit_ns;
+  const int cta = withhold_cta;
+  QL_CUDA(cudaDeviceSynchronize());   // no launch in flight sees a half-changed setting
+  QL_CUDA(cudaMemcpyToSymbol(ql::g_wait_limit_ns, &lim, sizeof(lim)));
+  QL_CUDA(cudaMemcpyToSymbol(ql::g_debug_withhold_cta, &cta, sizeof(cta)));
+  return QL_OK;
 }
 
 ql_status ql_check(ql_stream_t stream) {

@@ -204,13 +204,11 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
   return e == 0 ? static_cast<float>(m) * 0x1p-9f : __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-// Quantize the 16-element block j of row m with tensor scale ts: codes [M, K/2] (row stride
-// ldc), scales plain [M, K/16] and/or tiled (atoms of 64 K).
-// The same from the block's 16 bf16 values already in registers (element 2i low half of w[i]).
-__device__ __forceinline__ void quant_e4m3_regs(
-    const uint32_t (&w)[8], int m, int j, float ts, uint8_t* __restrict__ codes, int ldc,
-    uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
-    int sf_atoms_per_row, int sf_tile_rows) {
+// E4M3-B16 coding of one 16-element block held as 8 bf16x2 words (element 2i in the low half
+// of w[i]) with tensor scale ts: its two packed code words (elements 0..7, 8..15) and its E4M3
+// scale byte; the callers store them where their layouts want them.
+__device__ __forceinline__ void quant_e4m3_code_block(const uint32_t (&w)[8], float ts,
+                                                      uint32_t (&packed)[2], uint32_t& sb_out) {
   uint32_t mx = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
@@ -229,7 +227,6 @@ __device__ __forceinline__ void quant_e4m3_regs(
   // to zero keeps code 0x8).
   const bool fast = S >= 0x1p-126f;
   const float inv = fast ? __frcp_rn(S) : 0.f;
-  uint32_t packed[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint32_t ww[4] = {w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]};
@@ -261,6 +258,18 @@ __device__ __forceinline__ void quant_e4m3_regs(
     }
     packed[h] = code | bf16x8_sign_nibbles(ww);
   }
+  sb_out = sb;
+}
+
+// Quantize the 16-element block j of row m with tensor scale ts: codes [M, K/2] (row stride
+// ldc), scales plain [M, K/16] and/or tiled (atoms of 64 K), from the block's 16 bf16 values
+// already in registers.
+__device__ __forceinline__ void quant_e4m3_regs(
+    const uint32_t (&w)[8], int m, int j, float ts, uint8_t* __restrict__ codes, int ldc,
+    uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
+    int sf_atoms_per_row, int sf_tile_rows) {
+  uint32_t packed[2], sb;
+  quant_e4m3_code_block(w, ts, packed, sb);
   *reinterpret_cast<uint2*>(codes + static_cast<size_t>(m) * ldc + j * 8) =
       make_uint2(packed[0], packed[1]);
   if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = static_cast<uint8_t>(sb);
@@ -380,7 +389,8 @@ __global__ void __launch_bounds__(kE4m3ClusterThreads) quant_e4m3_b16_cluster_ke
 // CTAs wait for the tagged result (one word, so the polling does not pile onto the slots' cache
 // lines).  No word needs clearing between launches; a stale word would have to repeat a 48-bit tag
 // to be taken for a fresh one.  Launched with programmatic stream serialization like the cluster
-// kernel.  On a timeout the error word is set and no codes are written.
+// kernel.  On a timeout the error word is set and no codes are written, and each CTA whose wait
+// expired advances the counter by two, so the next launch's tag matches no word left behind.
 constexpr int kE4m3GridThreads = 256;
 constexpr int kE4m3GridMaxCtas = 256;   // CTA 0 polls one slot per thread
 constexpr int kE4m3SyncBytes = 16 + 8 * kE4m3GridMaxCtas;
@@ -395,12 +405,12 @@ __device__ __forceinline__ unsigned long long wait_tagged_u64(const unsigned lon
                                                               unsigned long long tag, bool& ok) {
   unsigned long long s = ld_acquire_gpu_u64(p);
   if ((s & ~0xFFFFull) == tag) return s;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = globaltimer_ns(), limit = wait_limit_ns();
   while (true) {
     __nanosleep(64);
     s = ld_acquire_gpu_u64(p);
     if ((s & ~0xFFFFull) == tag) return s;
-    if (globaltimer_ns() - t0 > 2000000000ull) {
+    if (globaltimer_ns() - t0 > limit) {
       record_error(DEV_TIMEOUT, 30);
       ok = false;
       return 0;
@@ -450,7 +460,7 @@ __global__ void __launch_bounds__(kE4m3GridThreads) quant_e4m3_b16_grid_kernel(
   __syncthreads();   // also publishes s_count
   const uint32_t cnt = s_count;
   const unsigned long long tag = e4m3_grid_tag(cnt);
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && !withheld(blockIdx.x)) {
     uint32_t v = 0;
     for (int i = 0; i < kE4m3GridThreads / 32; ++i) v = max(v, red[i]);
     st_release_gpu_u64(&slots[blockIdx.x], tag | v);
@@ -471,7 +481,7 @@ __global__ void __launch_bounds__(kE4m3GridThreads) quant_e4m3_b16_grid_kernel(
       s_amax = v;
       if (ok) {
         st_release_gpu_u64(result, tag | v);
-        *sync = cnt;
+        atomicAdd(sync, 1u);   // every CTA has read the counter (its slot carries the tag)
       }
     }
   } else if (threadIdx.x == 0) {
@@ -481,7 +491,13 @@ __global__ void __launch_bounds__(kE4m3GridThreads) quant_e4m3_b16_grid_kernel(
   }
   __syncthreads();
   if (blockIdx.x != 0) ok = s_ok != 0;
-  if (!ok) return;
+  if (!ok) {
+    // A CTA whose wait expired moves the counter on by two: one that read it late (value v,
+    // after CTA 0 gave up) tagged its slot v + 1 and leaves the counter at v + 2 or more, so no
+    // word of this launch can match the next launch's tag; the workspace needs no clearing.
+    if (threadIdx.x == 0) atomicAdd(sync, 2u);
+    return;
+  }
   const uint32_t amax16 = s_amax;
   const float ts = tensor_scale_from_amax16(amax16);
   if (tid == 0) {

@@ -59,8 +59,15 @@ typedef enum {
                                     fp32 tensor scale */
   QL_W_CLUSTER4_ROW16_BF16 = 4,  /* CodeQuant-style: 4-bit indices [N,K/2] into 16 bf16
                                     centroids per output row */
-  QL_W_INT4_G128_BSR = 5         /* INT4 codes [N,K/2] + fp16 scale per (row,128-group), plus a
+  QL_W_INT4_G128_BSR = 5,        /* INT4 codes [N,K/2] + fp16 scale per (row,128-group), plus a
                                     block-sparse INT4 residual on 16x128 blocks (BSR) */
+  QL_W_VQ_POSTSCALE_E4M3_B16 = 6,    /* MXCode PostScale: uint8 indices [N,K/4] into per-QBlock
+                                        codebooks of 256 x 4 E2M1 codes, ONE E4M3 scale byte per
+                                        QBlock [N/64,K/64] (scales), fp32 tensor scale */
+  QL_W_VQ_PRESCALE_PLUS_E4M3_B16 = 7 /* MXCode PreScale+: indices and codebooks as PreScale; the
+                                        E4M3 block scales by VQ: uint8 scale indices [N,K/128]
+                                        (scales) into scale_codebook [256][8] E4M3 bytes; fp32
+                                        tensor scale */
 } ql_wformat;
 
 typedef enum {
@@ -88,6 +95,9 @@ typedef struct ql_weight_desc {
   const void* bsr_codes;      /* [nnzb][bsr_block_n][bsr_block_k/2] int4 */
   const void* bsr_scales;     /* [nnzb][bsr_block_n] fp16 */
   int32_t bsr_block_n, bsr_block_k, bsr_nnzb;
+  const uint8_t* scale_codebook;       /* VQ PreScale+: [scale_codebook_entries][scale_group] */
+  int32_t scale_codebook_entries;      /* 256 */
+  int32_t scale_group;                 /* 8 consecutive E4M3 block scales along K per index */
 } ql_weight_desc;
 
 typedef struct ql_linear ql_linear;
@@ -97,8 +107,10 @@ typedef struct ql_moe ql_moe;
 const char* ql_version(void);
 const char* ql_last_error(void);
 
-/* Create a linear layer: validates the descriptor, copies the weights to device memory owned
- * by the returned handle and repacks scales into the tiled layout the MMA consumes.
+/* Create a linear layer (MXCode Table 1 formats; PRQuant §4 "Offline residual augmentation" for
+ * the tail; MXCode abstract for VQ codebooks; MosaicQuant "Dense Base and Sparse Residuals"):
+ * validates the descriptor, copies the weights to device memory owned by the returned handle
+ * and repacks them, with their scales, into the tiled layout the MMA consumes.
  * Supported:
  *   QL_W_MXFP4_E8M0_B32        N % 16 == 0, K % 128 == 0, k_tail % 128 == 0, 0 <= k_tail < K;
  *                              activations quantized to MXFP4 (E8M0-B32).
@@ -107,6 +119,12 @@ const char* ql_last_error(void);
  *   QL_W_VQ_PRESCALE_E4M3_B16  N % 128 == 0, K % 256 == 0, 64 x 64 QBlocks, no tail; indices,
  *                              codebooks, E4M3 scales [N,K/16] and w_tensor_scale; the weight
  *                              operand is rebuilt from the codebooks inside the GEMM.
+ *   QL_W_VQ_POSTSCALE_E4M3_B16 as PreScale, with scales = one E4M3 byte per QBlock [N/64,K/64]
+ *                              (the decoder gives every 16-block of the QBlock that scale).
+ *   QL_W_VQ_PRESCALE_PLUS_E4M3_B16 as PreScale, with scales = scale indices [N,K/128] into
+ *                              scale_codebook [256][8] (block scale 8g+i of a row is
+ *                              scale_codebook[index g][i]); scale_codebook_entries = 256,
+ *                              scale_group = 8.
  *   QL_W_INT4_G128_BSR         N % 128 == 0, K % 128 == 0, no tail; codes [N,K/2] (INT4, two's
  *                              complement nibbles), fp16 scales [N,K/128], and a 16 x 128
  *                              block-sparse INT4 residual (bsr_*: rowptr [N/16+1], col = group,
@@ -117,19 +135,28 @@ const char* ql_last_error(void);
 ql_status qlinear_create(const ql_weight_desc* desc, ql_stream_t stream, ql_linear** out);
 ql_status qlinear_destroy(ql_linear* layer);
 
-/* Bytes of device workspace that qlinear_forward needs for M tokens. */
+/* Bytes of device workspace that qlinear_forward needs for M tokens: the quantized activation
+ * (codes and tiled scales; PRQuant §4 quantizes it once), the grid-wide agreement words and the
+ * split-K partial tiles.  Host-only; *bytes is host memory. */
 ql_status qlinear_workspace_bytes(const ql_linear* layer, int64_t M, size_t* bytes);
 
-/* y[M,N] = X[M, K-k_tail] (quantized online) times the layer's weight.  x_bf16, y_bf16 and
- * the workspace are device pointers; y_f32 (device, [M,N]) may be NULL.  ws must be 256-byte
- * aligned and at least qlinear_workspace_bytes(M) long; its contents on entry do not matter
- * (the E4M3-B16 grid quantizer agrees on the tensor amax through words of the workspace that
- * carry a per-launch tag, so they need no clearing; after a device timeout reported by
- * ql_check, discard the workspace).  Calls that share a workspace must be stream-ordered.
- * Rows of x are contiguous (row stride K - k_tail elements).  M may be 0 (no-op).
- * Kernels are launched with programmatic stream serialization and release the next such grid
- * at once: a following qlinear call on the stream may start streaming its weights while this
- * one finishes, and reads this call's results only after it has completed. */
+/* y[M,N] = X[M, K-k_tail] (quantized online) times the layer's weight: the quantized linear
+ * layer the pages share -- PRQuant §4 "Kernel design for efficient inference" (the activation
+ * quantized to MXFP4 once, its tail reused, one GEMM over C + k), MXCode abstract and Table 1
+ * (E4M3-B16 activations, MX-native operands rebuilt from the codebooks), MosaicQuant
+ * "ZipperEngine" (INT4 base and residual in one GEMM).  x_bf16, y_bf16 and the workspace are
+ * device pointers; y_f32 (device, [M,N]) may be NULL.  ws must be 256-byte aligned and at least
+ * qlinear_workspace_bytes(M) long; its contents on entry do not matter: the grid-wide agreements
+ * (the E4M3-B16 tensor amax, the split-K hand-off) go through workspace words that carry a
+ * per-launch tag derived from a launch counter kept there, so nothing needs clearing, and after
+ * a device timeout the counter has moved past every tag the failed launch left.  Calls that
+ * share a workspace must be stream-ordered.  Rows of x are contiguous (row stride K - k_tail
+ * elements).  M may be 0 (no-op).  For M <= 64 with FP4 or VQ weights the forward is ONE launch:
+ * the GEMM's own warps quantize x (each element once across the grid) before its MMAs need it,
+ * while the weights already stream.  Kernels are launched with programmatic stream serialization
+ * and release the next such grid at once: a following qlinear call on the stream may start
+ * streaming its weights while this one finishes, and reads this call's results only after it
+ * has completed. */
 ql_status qlinear_forward(const ql_linear* layer, const void* x_bf16, int64_t M, void* y_bf16,
                           float* y_f32, void* ws, size_t ws_bytes, ql_stream_t stream);
 
@@ -156,7 +183,9 @@ ql_status qlinear_gemm(const ql_linear* layer, int64_t M, void* y_bf16, float* y
  * it until the process exits); M whose qlinear_workspace_bytes exceeds 8 MiB is rejected with
  * QL_ERR_WORKSPACE.  Nothing is allocated: no cudaMalloc/cudaFree, no library allocator.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress with that
- * device current); make that first call before any stream capture.  All calls share the one
+ * device current) and caches it with the current context; a call that finds another context
+ * current (after cudaDeviceReset, say) looks it up again.  Make the first call on a device, and
+ * the first after a context change, before any stream capture.  All calls share the one
  * array, which keeps whatever the last call left in it (the parts that must start at zero are
  * cleared by each call): calls that may overlap on the GPU (different streams, or different host
  * threads) race on it and must be serialised by the caller.  x, y and y_f32 are device pointers
@@ -189,6 +218,17 @@ ql_status quantize_act(ql_aformat fmt, const void* x_bf16, int64_t M, int64_t K,
  * denominator of its roofline.  Asynchronous; nothing is read back. */
 ql_status ql_tensor_peak(int32_t kind, int32_t n, int32_t iters, int32_t ctas,
                          double* flops_per_launch, ql_stream_t stream);
+
+/* Test hook for the timeout path (no step of the method).  Sets the limit of every bounded wait
+ * in the library's kernels (wait_limit_ns; 0 restores the default 2 s) and names one CTA index
+ * (withhold_cta >= 0; -1: none) whose grid-wide publications are withheld: its slot in the
+ * E4M3-B16 amax agreement and its flags in the decode GEMM are never written, so the waits on
+ * them run out after the limit, the kernels record QL_ERR_TIMEOUT in the device error word and
+ * return, and ql_check reports it.  Nothing faults or hangs.  Synchronises the device; affects
+ * every later launch on it until called again with (-1, 0).  The workspaces stay usable
+ * afterwards: the launch counters of the grid-wide protocols move past every tag a failed
+ * launch left behind. */
+ql_status ql_debug_inject(int32_t withhold_cta, uint64_t wait_limit_ns);
 
 /* Synchronise `stream` and report (then clear) the device error word. */
 ql_status ql_check(ql_stream_t stream);
@@ -254,6 +294,34 @@ ql_status moe_grouped_forward(const ql_moe* moe, const void* x_bf16, int64_t T,
 ql_status qlinear_prepare_vq_prescale(const uint16_t* w_bf16, int64_t N, int64_t K,
                                       const uint8_t* codebooks, int32_t qn, int32_t qk,
                                       float* ts_out, uint8_t* scales_out, uint8_t* idx_out);
+
+/* MXCode PostScale preparation (MXCode abstract: PostScale "quantizes learned codebooks to
+ * MXFP4"; reading: one E4M3 scale per QBlock codebook, relative to an FP32 tensor scale over all
+ * codebooks, so the decoded weight is an MX-native E4M3-B16 operand with no per-weight scales).
+ * w_bf16 [N,K]; centroids = learned codebooks, float [N/64][K/64][256][4] (bf16 values).
+ * Outputs: ts = amax(all centroids)/2688 (1 if 0); per QBlock the E4M3 byte
+ * s = E4M3_RNE_satfinite((amax(codebook)/6)/ts) (qscales [N/64][K/64]) and the packed E2M1
+ * entries code = E2M1_RNE(c / (dec(s)*ts)) (codebooks [N/64][K/64][256][2], element 2i low);
+ * indices [N,K/4]: the entry whose decoded value e2m1 * dec(s) * ts is nearest (squared distance
+ * in double, ties to the lowest index) to W[n,4j:4j+4].  fp32 steps in that order; qn == qk == 64.
+ * Host, CPU. */
+ql_status qlinear_prepare_vq_postscale(const uint16_t* w_bf16, int64_t N, int64_t K,
+                                       const float* centroids, int32_t qn, int32_t qk,
+                                       float* ts_out, uint8_t* codebooks_out,
+                                       uint8_t* qscales_out, uint8_t* idx_out);
+
+/* MXCode PreScale+ preparation (MXCode abstract: PreScale's scales "further compressed using VQ";
+ * appendix Table 4 caption: Ks = 256, ds = 8).  The PreScale E4M3 block scales of W, 8
+ * consecutive along K, become the nearest of the 256 vectors of scale_codebook [256][8] (E4M3
+ * bytes; squared distance of decoded values in double, ties to the lowest index); W is then
+ * normalised by the compressed scales and assigned to its QBlock codebook as in PreScale.
+ * Outputs: ts, the compressed scale bytes [N,K/16], the scale indices [N,K/128] and the weight
+ * indices [N,K/4].  K % 128 == 0, qn == qk == 64.  Host, CPU. */
+ql_status qlinear_prepare_vq_prescale_plus(const uint16_t* w_bf16, int64_t N, int64_t K,
+                                           const uint8_t* codebooks, const uint8_t* scale_codebook,
+                                           int32_t qn, int32_t qk, float* ts_out,
+                                           uint8_t* scales_out, uint8_t* sidx_out,
+                                           uint8_t* idx_out);
 
 /* MosaicQuant-style INT4 dense + block-sparse residual preparation (MosaicQuant, "Dense Base and
  * Sparse Residuals" and "Activation-aware Delta-Hessian Block Selection"; formulas are readings).

@@ -17,7 +17,8 @@ import torch
 
 __all__ = [
     "rng", "to_bf16_bits", "bf16_bits_to_f64", "f32_to_bf16_bits", "pick_channels",
-    "activations_bf16", "student_t", "uniform_nibble_bytes", "uniform_bytes",
+    "activations_bf16", "student_t", "uniform_nibble_bytes", "uniform_bytes", "vq_raw_codebooks",
+    "scale_codebook",
 ]
 
 
@@ -119,6 +120,61 @@ def vq_codebooks(seed: int, w: np.ndarray, qn: int = 64, qk: int = 64, entries: 
         snap = np.abs(cent[..., None] - _E2M1_GRID).argmin(-1)
         out[c0:c0 + B] = _E2M1_CODE[snap]
     return out.reshape(QR, QC, entries, 4)
+
+
+def vq_raw_codebooks(seed: int, w: np.ndarray, qn: int = 64, qk: int = 64, entries: int = 256,
+                     iters: int = 4, chunk: int = 128) -> np.ndarray:
+    """Learned codebooks in value space (bf16 centroids), one per qn x qk QBlock, by seeded
+    k-means on the raw 4-vectors along K (data synthesis only; the method then quantizes them).
+    Returns float32 [N/qn, K/qk, entries, 4] holding bf16 values."""
+    g = rng(seed * 37 + 11)
+    N, K = w.shape
+    QR, QC = N // qn, K // qk
+    pts = np.asarray(w, np.float64).reshape(QR, qn, QC, qk // 4, 4).transpose(0, 2, 1, 3, 4)
+    pts = pts.reshape(QR * QC, -1, 4)
+    out = np.empty((QR * QC, entries, 4), dtype=np.float32)
+    P = pts.shape[1]
+    for c0 in range(0, QR * QC, chunk):
+        p = pts[c0:c0 + chunk].astype(np.float32)
+        B = p.shape[0]
+        init = np.stack([g.choice(P, entries, replace=False) for _ in range(B)])
+        cent = np.take_along_axis(p, init[:, :, None], axis=1)
+        for _ in range(iters):
+            d = (p * p).sum(-1)[:, :, None] - 2 * p @ cent.transpose(0, 2, 1) + \
+                (cent * cent).sum(-1)[:, None, :]
+            lab = d.argmin(-1)
+            flat = (lab + np.arange(B)[:, None] * entries).reshape(-1)
+            sums = np.zeros((B * entries, 4), np.float64)
+            np.add.at(sums, flat, p.reshape(-1, 4))
+            cnt = np.bincount(flat, minlength=B * entries).astype(np.float64)
+            newc = (sums / np.maximum(cnt, 1)[:, None]).reshape(B, entries, 4).astype(np.float32)
+            cent = np.where((cnt == 0).reshape(B, entries, 1), cent, newc)
+        out[c0:c0 + B] = cent
+    bits = to_bf16_bits(out)
+    return bf16_bits_to_f64(bits).astype(np.float32).reshape(QR, QC, entries, 4)
+
+
+def scale_codebook(seed: int, sb: np.ndarray, entries: int = 256, ds: int = 8,
+                   iters: int = 6) -> np.ndarray:
+    """A per-tensor codebook of `entries` scale vectors of length ds (E4M3 bytes) for groups of ds
+    consecutive block scales along K: seeded k-means on the scale bytes of the groups, rounded to
+    the nearest byte (data synthesis only).  sb: E4M3 scale bytes [N, K/16]."""
+    g = rng(seed * 41 + 3)
+    pts = np.asarray(sb, np.float64).reshape(-1, ds)
+    uniq = np.unique(pts, axis=0)
+    if len(uniq) <= entries:
+        out = np.zeros((entries, ds), np.uint8)
+        out[:len(uniq)] = uniq.astype(np.uint8)
+        return out
+    cent = uniq[g.choice(len(uniq), entries, replace=False)]
+    for _ in range(iters):
+        d = (pts * pts).sum(-1)[:, None] - 2 * pts @ cent.T + (cent * cent).sum(-1)[None, :]
+        lab = d.argmin(-1)
+        sums = np.zeros((entries, ds))
+        np.add.at(sums, lab, pts)
+        cnt = np.bincount(lab, minlength=entries).astype(np.float64)
+        cent = np.where(cnt[:, None] > 0, sums / np.maximum(cnt, 1)[:, None], cent)
+    return np.clip(np.rint(cent), 0, 126).astype(np.uint8)
 
 
 def zipf_router_logits(seed: int, T: int, E: int = 128, s: float = 1.1) -> np.ndarray:

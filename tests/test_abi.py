@@ -74,6 +74,39 @@ def test_vq_prescale_host_preparation_matches_oracle(N, K):
     assert np.array_equal(idx, ref["idx"])
 
 
+@pytest.mark.parametrize("N,K", [(64, 256), (128, 512)])
+def test_vq_postscale_host_preparation_matches_oracle(N, K):
+    import bit_quantized_moe_tcgen05_b200 as ql
+    from oracle import vq
+    wb = synth.to_bf16_bits(synth.student_t(19 + K, (N, K), 4.0) * 0.02)
+    w = synth.bf16_bits_to_f64(wb)
+    cent = synth.vq_raw_codebooks(19, w)
+    ts, cbp, qs, idx = ql.prepare_vq_postscale(wb, cent)
+    ref = vq.postscale_prepare(w, cent)
+    assert ts == ref["ts"]
+    assert np.array_equal(qs, ref["sbq"])
+    assert np.array_equal(cbp, vq.pack_codebooks(ref["codes"]))
+    assert np.array_equal(idx, ref["idx"])
+
+
+@pytest.mark.parametrize("N,K", [(64, 256), (128, 512)])
+def test_vq_prescale_plus_host_preparation_matches_oracle(N, K):
+    import bit_quantized_moe_tcgen05_b200 as ql
+    from oracle import vq
+    wb = synth.to_bf16_bits(synth.student_t(23 + K, (N, K), 4.0))
+    w = synth.bf16_bits_to_f64(wb)
+    cb = synth.vq_codebooks(23, w)
+    _, sb0 = vq.prescale(w)
+    scb = synth.scale_codebook(23, sb0, entries=256)
+    scb[:40] = synth.scale_codebook(24, sb0, entries=40)       # fewer distinct vectors than groups
+    ts, sb, sidx, idx = ql.prepare_vq_prescale_plus(wb, vq.pack_codebooks(cb), scb)
+    ref = vq.prescale_plus_prepare(w, cb, scb)
+    assert ts == ref["ts"]
+    assert np.array_equal(sidx, ref["sidx"])
+    assert np.array_equal(sb, ref["sb"])
+    assert np.array_equal(idx, ref["idx"])
+
+
 @pytest.mark.parametrize("N,K,T", [(64, 512, 32), (128, 1024, 16)])
 def test_int4_bsr_host_preparation_matches_oracle(N, K, T):
     import bit_quantized_moe_tcgen05_b200 as ql

@@ -177,8 +177,9 @@ def test_forward_is_deterministic_and_reentrant():
 
 @pytest.mark.parametrize("M", [1, 16, 64])
 def test_gemm_repeat_without_requantize(M):
-    """The GEMM run again on the same quantized input (its split-K tickets re-armed by the kernel
-    itself, not by the quantizer) reproduces the forward's output bit for bit."""
+    """The GEMM run again and again on one quantized input (qlinear_quantize_input once) reproduces
+    the forward's output bit for bit: the split-K hand-off needs nothing re-armed between launches,
+    and the one-launch forward (quantizer fused in) computes the same bits as the two calls."""
     ql = _ql()
     codes, sb = random_mx_weight(17, 2560, 2048)
     xb, _ = synth.activations_bf16(17, M, 2048, 0.01, 20.0)
@@ -186,6 +187,7 @@ def test_gemm_repeat_without_requantize(M):
     x = dev_bf16(xb)
     ws = torch.empty(lin.workspace_bytes(M), dtype=torch.uint8, device="cuda")
     ref = lin.forward(x, ws=ws).clone()
+    lin.quantize_input(x, ws)
     outs = []
     for _ in range(3):
         y = torch.empty_like(ref)

@@ -250,3 +250,50 @@ def test_e4m3_grid_quantizer_shared_workspace():
                 assert np.array_equal(first[i], y32h), f"layer {i} round {rnd} not repeatable"
     for lin in layers:
         lin.close()
+
+
+# ------------------------------------------------------------------ PostScale / PreScale+
+def _postscale_layer(prep, ql):
+    return ql.QLinear(None, prep["sbq"], wfmt=ql.QL_W_VQ_POSTSCALE_E4M3_B16,
+                      w_tensor_scale=float(prep["ts"]), indices=prep["idx"],
+                      codebooks=vq.pack_codebooks(prep["codes"]))
+
+
+@pytest.mark.parametrize("N,K,M", [(256, 512, 1), (256, 1024, 8), (128, 768, 64), (256, 512, 200),
+                                   (512, 2048, 300)])
+def test_vq_postscale_linear(N, K, M):
+    """MXCode PostScale weights (one E4M3 scale per 64 x 64 QBlock codebook, no per-weight
+    scales): decode launches build the scale factors in TMEM, prefill launches in shared memory."""
+    ql = _ql()
+    w = synth.bf16_bits_to_f64(synth.to_bf16_bits(synth.student_t(80 + K, (N, K), 4.0) * 0.02))
+    cent = synth.vq_raw_codebooks(80, w)
+    prep = vq.postscale_prepare(w, cent)
+    lin = _postscale_layer(prep, ql)
+    xb, _ = synth.activations_bf16(81, M, K, 0.01, 30.0)
+    y, y32 = _run(lin, xb)
+    lin.close()
+    ref, t = vq.postscale_forward(synth.bf16_bits_to_f64(xb), prep)
+    check_fp32(y32, ref, t, f"postscale N={N} K={K} M={M}")
+    check_bf16(y, ref, t, f"postscale N={N} K={K} M={M}")
+
+
+@pytest.mark.parametrize("N,K,M", [(256, 512, 1), (256, 1024, 8), (128, 768, 64), (256, 512, 200),
+                                   (512, 2048, 300)])
+def test_vq_prescale_plus_linear(N, K, M):
+    """MXCode PreScale+ weights (block scales replaced by 8-scale vectors of a 256-entry scale
+    codebook): the decoders look the scales up per row and per 128-column group."""
+    ql = _ql()
+    w = synth.bf16_bits_to_f64(synth.to_bf16_bits(synth.student_t(82 + K, (N, K), 4.0)))
+    cb = synth.vq_codebooks(82, w)
+    _, sb0 = vq.prescale(w)
+    scb = synth.scale_codebook(82, sb0)
+    prep = vq.prescale_plus_prepare(w, cb, scb)
+    lin = ql.QLinear(None, prep["sidx"], wfmt=ql.QL_W_VQ_PRESCALE_PLUS_E4M3_B16,
+                     w_tensor_scale=float(prep["ts"]), indices=prep["idx"],
+                     codebooks=vq.pack_codebooks(cb), scale_codebook=scb)
+    xb, _ = synth.activations_bf16(83, M, K, 0.01, 30.0)
+    y, y32 = _run(lin, xb)
+    lin.close()
+    ref, t = vq.forward(synth.bf16_bits_to_f64(xb), prep, cb)
+    check_fp32(y32, ref, t, f"prescale+ N={N} K={K} M={M}")
+    check_bf16(y, ref, t, f"prescale+ N={N} K={K} M={M}")

@@ -55,3 +55,45 @@ def test_fixed_scratch_rejects_m_beyond_its_size():
         lin.forward_fixed_scratch(x)
     assert e.value.status == 6 and "8 MiB" in str(e.value)
     lin.close()
+
+
+def test_fixed_scratch_layers_of_different_formats_take_turns():
+    """Three layers of different formats share the one fixed scratch array, call after call: a VQ
+    layer at 64 x 9728 (one-launch decode forward, whose grid-wide agreement keeps a launch
+    counter and tagged words in the scratch), an INT4 + block-sparse layer (whose activation
+    codes start right after those words) and an MXFP4 layer.  Every call must reproduce, bit for
+    bit, the same layer's forward on a private workspace."""
+    import bit_quantized_moe_tcgen05_b200 as ql
+    from oracle import int4bsr
+    g = np.random.default_rng(77)
+    N, K = 256, 9728
+    cb = g.integers(0, 16, (N // 64, K // 64, 256, 4), dtype=np.uint8)
+    vql = ql.QLinear(None, g.integers(0x28, 0x48, (N, K // 16), dtype=np.uint8),
+                     wfmt=ql.QL_W_VQ_PRESCALE_E4M3_B16, w_tensor_scale=0.0071,
+                     indices=g.integers(0, 256, (N, K // 4), dtype=np.uint8),
+                     codebooks=F.pack_nibbles(cb))
+    w4 = synth.bf16_bits_to_f64(synth.to_bf16_bits(synth.student_t(78, (256, 1024), 4.0)))
+    xc, _ = synth.activations_bf16(79, 64, 1024, 0.08, 30.0)
+    p4 = int4bsr.prepare(w4, synth.bf16_bits_to_f64(xc), density=0.1)
+    i4l = ql.QLinear(F.pack_nibbles(F.int4_encode(p4["q"])), p4["sw"].view(np.uint16),
+                     wfmt=ql.QL_W_INT4_G128_BSR,
+                     bsr=dict(rowptr=p4["rowptr"], col=p4["col"],
+                              rcodes=F.pack_nibbles(F.int4_encode(p4["rq"])),
+                              rscales=p4["rs"].view(np.uint16)))
+    codes, sb = _layer_inputs(80, 1024, 2048)
+    mxl = ql.QLinear(codes, sb)
+    cases = [(vql, 64, K), (i4l, 16, 1024), (mxl, 16, 2048)]
+    for rnd in range(3):
+        for i, (lin, M, KK) in enumerate(cases):
+            xb, _ = synth.activations_bf16(90 + 7 * rnd + i, M, KK, 0.01, 20.0)
+            x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+            ws = torch.empty(lin.workspace_bytes(M), dtype=torch.uint8, device="cuda")
+            ref32 = torch.empty((M, lin.N), dtype=torch.float32, device="cuda")
+            ref = lin.forward(x, out_f32=ref32, ws=ws).clone()
+            got32 = torch.empty((M, lin.N), dtype=torch.float32, device="cuda")
+            got = lin.forward_fixed_scratch(x, out_f32=got32)
+            ql.check()
+            assert torch.equal(got, ref), f"round {rnd} layer {i}: bf16 outputs differ"
+            assert torch.equal(got32, ref32), f"round {rnd} layer {i}: fp32 outputs differ"
+    for lin, _, _ in cases:
+        lin.close()
