@@ -14,7 +14,7 @@ import numpy as np
 
 __all__ = [
     "lib", "LIB_PATH", "QLError", "WeightDesc", "QLinear", "quantize_act", "prepare_prquant",
-    "check", "debug_inject", "QL_W_MXFP4_E8M0_B32", "QL_A_MXFP4_E8M0_B32", "EXPORTED_SYMBOLS",
+    "check", "debug_inject", "decode_fuse_mode", "QL_W_MXFP4_E8M0_B32", "QL_A_MXFP4_E8M0_B32", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlinear.so")
@@ -37,6 +37,7 @@ EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_workspace_layout", "moe_grouped_forward",
     "qlinear_prepare_int4_bsr", "ql_tensor_peak", "ql_debug_inject",
     "qlinear_prepare_vq_postscale", "qlinear_prepare_vq_prescale_plus",
+    "qlinear_prepare_prquant_ex", "quantize_act_hadamard", "ql_decode_fuse_mode",
 )
 
 
@@ -58,6 +59,7 @@ class WeightDesc(ctypes.Structure):
         ("bsr_block_n", ctypes.c_int32), ("bsr_block_k", ctypes.c_int32),
         ("bsr_nnzb", ctypes.c_int32), ("scale_codebook", ctypes.c_void_p),
         ("scale_codebook_entries", ctypes.c_int32), ("scale_group", ctypes.c_int32),
+        ("had_block", ctypes.c_int32),
     ]
 
 
@@ -86,6 +88,8 @@ def _load() -> ctypes.CDLL:
         "quantize_act": [ctypes.c_int, vp, i64, i64, vp, vp, vp, vp],
         "ql_check": [vp],
         "qlinear_prepare_prquant": [vp, i64, i64, i32, vp, vp, vp],
+        "qlinear_prepare_prquant_ex": [vp, i64, i64, i32, i32, vp, vp, vp],
+        "quantize_act_hadamard": [ctypes.c_int, i32, vp, i64, i64, vp, vp, vp],
         "qlinear_prepare_vq_prescale": [vp, i64, i64, vp, i32, i32, vp, vp, vp],
         "moe_create": [ctypes.POINTER(WeightDesc), ctypes.POINTER(WeightDesc), i32, i32, vp,
                        ctypes.POINTER(vp)],
@@ -98,6 +102,7 @@ def _load() -> ctypes.CDLL:
                                      i32, vp],
         "ql_tensor_peak": [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_double), vp],
         "ql_debug_inject": [i32, ctypes.c_uint64],
+        "ql_decode_fuse_mode": [i32],
         "qlinear_prepare_vq_postscale": [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp],
         "qlinear_prepare_vq_prescale_plus": [vp, i64, i64, vp, vp, i32, i32, vp, vp, vp, vp],
     }
@@ -138,9 +143,18 @@ def debug_inject(withhold_cta: int = -1, wait_limit_ns: int = 0) -> None:
     _ok(lib.ql_debug_inject(int(withhold_cta), int(wait_limit_ns)), "ql_debug_inject")
 
 
-def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None):
+def decode_fuse_mode(mode: int = -1) -> None:
+    """How the decode kernel is organised: 1 activations quantized cooperatively over the grid,
+    2 each CTA its own stages, 3 as 2 with each weight tile's K-splits in one cluster, -1 chosen
+    per launch (see ql_decode_fuse_mode).  Every mode matches the oracle; modes 1 and 2 give
+    identical bits, mode 3 may split K differently."""
+    _ok(lib.ql_decode_fuse_mode(int(mode)), "ql_decode_fuse_mode")
+
+
+def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None, had_block: int = 0):
     """Quantize bf16 activations [M, K] on the GPU.
-    MXFP4 E8M0-B32 -> (codes uint8 [M, K/2], E8M0 scales uint8 [M, K/32]);
+    MXFP4 E8M0-B32 -> (codes uint8 [M, K/2], E8M0 scales uint8 [M, K/32]), optionally after an
+    online block-32 Hadamard (had_block = 32);
     E4M3-B16 + tensor scale -> (codes, E4M3 scales uint8 [M, K/16], ts float32 [1])."""
     import torch
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
@@ -148,8 +162,12 @@ def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None):
     codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
     if fmt == QL_A_MXFP4_E8M0_B32:
         scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
-        _ok(lib.quantize_act(fmt, x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), None,
-                             _stream(stream)), "quantize_act")
+        if had_block:
+            _ok(lib.quantize_act_hadamard(fmt, had_block, x.data_ptr(), M, K, codes.data_ptr(),
+                                          scales.data_ptr(), _stream(stream)), "quantize_act_hadamard")
+        else:
+            _ok(lib.quantize_act(fmt, x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), None,
+                                 _stream(stream)), "quantize_act")
         return codes, scales
     if fmt == QL_A_INT4_TOK_G128:
         scales = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
@@ -177,7 +195,8 @@ class QLinear:
     def __init__(self, codes: np.ndarray | None, scales: np.ndarray, k_tail: int = 0,
                  wfmt: int = QL_W_MXFP4_E8M0_B32, w_tensor_scale: float = 1.0,
                  indices: np.ndarray | None = None, codebooks: np.ndarray | None = None,
-                 bsr: dict | None = None, scale_codebook: np.ndarray | None = None, stream=None):
+                 bsr: dict | None = None, scale_codebook: np.ndarray | None = None,
+                 had_block: int = 0, stream=None):
         """MXFP4: codes [N, K/2] + E8M0 scales [N, K/32] (+ k_tail).  NVFP4 (E4M3-B16): codes +
         E4M3 scales [N, K/16] + w_tensor_scale.  VQ PreScale: indices [N, K/4] + packed codebooks
         [N/64, K/64, 256, 2] + E4M3 scales [N, K/16] + w_tensor_scale (codes = None).
@@ -228,7 +247,7 @@ class QLinear:
                        scales=scales.ctypes.data, w_tensor_scale=float(w_tensor_scale),
                        indices=iptr, codebooks=cbptr, qblock_n=64, qblock_k=64,
                        scale_codebook=scb_ptr, scale_codebook_entries=256 if scb_ptr else 0,
-                       scale_group=8 if scb_ptr else 0)
+                       scale_group=8 if scb_ptr else 0, had_block=int(had_block))
         h = ctypes.c_void_p()
         _ok(lib.qlinear_create(ctypes.byref(d), _stream(stream), ctypes.byref(h)), "qlinear_create")
         self._h = h
@@ -302,16 +321,18 @@ class QLinear:
             pass
 
 
-def prepare_prquant(w_bf16_bits: np.ndarray, k: int):
-    """Offline PRQuant preparation on the host (library C++ code, not the oracle).
+def prepare_prquant(w_bf16_bits: np.ndarray, k: int, scale_search: bool = False):
+    """Offline PRQuant preparation on the host (library C++ code, not the oracle); scale_search
+    selects the E8M0-W block-scale search.
     Returns (perm int32 [C], codes uint8 [N, (C+k)/2], scales uint8 [N, (C+k)/32])."""
     w = np.ascontiguousarray(w_bf16_bits, dtype=np.uint16)
     N, C = w.shape
     perm = np.empty(C, np.int32)
     codes = np.empty((N, (C + k) // 2), np.uint8)
     scales = np.empty((N, (C + k) // 32), np.uint8)
-    _ok(lib.qlinear_prepare_prquant(w.ctypes.data, N, C, k, perm.ctypes.data, codes.ctypes.data,
-                                    scales.ctypes.data), "qlinear_prepare_prquant")
+    _ok(lib.qlinear_prepare_prquant_ex(w.ctypes.data, N, C, k, int(bool(scale_search)),
+                                       perm.ctypes.data, codes.ctypes.data, scales.ctypes.data),
+        "qlinear_prepare_prquant_ex")
     return perm, codes, scales
 
 
@@ -378,7 +399,10 @@ class MoE:
     gu_idx uint8 [E*2I, H] 4-bit indices (values 0..15), gu_cent bf16 bit patterns [E*2I, 16];
     dn_idx [E*H, I], dn_cent [E*H, 16]; per expert the gate rows come first, then the up rows."""
 
-    def __init__(self, gu_idx, gu_cent, dn_idx, dn_cent, E: int, top_k: int, stream=None):
+    def __init__(self, gu_idx, gu_cent, dn_idx, dn_cent, E: int, top_k: int, had_x: bool = False,
+                 had_h: bool = False, stream=None):
+        """had_x / had_h: x (before gate/up), resp. h (before down), passes the online block-32
+        Hadamard before its MXFP4 quantization; the expert weights given are the rotated ones."""
         gi, di = _pack4(gu_idx), _pack4(dn_idx)
         gc = np.ascontiguousarray(gu_cent, dtype=np.uint16)
         dc = np.ascontiguousarray(dn_cent, dtype=np.uint16)
@@ -386,9 +410,9 @@ class MoE:
         self.H = gu_idx.shape[1]
         self.I = dn_idx.shape[1]
         g = WeightDesc(wfmt=QL_W_CLUSTER4_ROW16_BF16, N=gu_idx.shape[0], K=self.H,
-                       codes=gi.ctypes.data, codebooks=gc.ctypes.data)
+                       codes=gi.ctypes.data, codebooks=gc.ctypes.data, had_block=32 if had_x else 0)
         d = WeightDesc(wfmt=QL_W_CLUSTER4_ROW16_BF16, N=dn_idx.shape[0], K=self.I,
-                       codes=di.ctypes.data, codebooks=dc.ctypes.data)
+                       codes=di.ctypes.data, codebooks=dc.ctypes.data, had_block=32 if had_h else 0)
         h = ctypes.c_void_p()
         _ok(lib.moe_create(ctypes.byref(g), ctypes.byref(d), E, top_k, _stream(stream),
                            ctypes.byref(h)), "moe_create")

@@ -58,6 +58,7 @@ namespace ql {
 constexpr int kDecMaxGrid = 256;           // CTAs of one decode launch (slots and flags)
 constexpr int kDecQUnits = 2;              // 32-element activation units per quantizer thread
 constexpr int kDecMaxSplits = 16;          // K-splits of one weight tile
+constexpr int kDecLocalBatch = 4;          // local quantization: units a thread loads at once
 constexpr int kDecSyncBytes = 16 + 3 * 8 * kDecMaxGrid;
 
 // Workspace sync block: [0] launch counter, [8] amax result, [16..) slots, qflags, pflags (64-bit
@@ -112,7 +113,9 @@ struct DecodeArgs {
   int n_stages_total;         // + ceil(k_tail / 256)
   int spp;                    // K stages per split
   int splits;                 // CTAs per weight tile (consecutive blockIdx)
-  int fuse;                   // 1: quantize x inside the kernel
+  int fuse;                   // 0: x quantized by qlinear_quantize_input (plain layout); 1: inside
+                              // the kernel, cooperatively (per-stage tiles in the workspace);
+                              // 2: inside the kernel, each CTA its own stages (small x)
   const __nv_bfloat16* x;     // fuse: bf16 activations [M, C]
   uint8_t* xq;                // fuse = 0: quantized activation codes [M, C/2] (workspace)
   uint8_t* sfb;               // fuse = 0: activation scale atoms, 128-row group 0, [C / atomK]
@@ -127,6 +130,12 @@ struct DecodeArgs {
   float* partials;            // splits > 1: [grid][BN][128] fp32 (rows < M written)
   uint8_t* sync;              // DecSync block
   const uint8_t* scb;         // VQ PreScale+: scale codebook [256][8] E4M3 bytes
+  int had;                    // fuse, E8M0: online Hadamard (block 32) before quantizing x
+  int amax_coop;              // fuse = 2, E4M3: the tensor amax combined over the CTAs (each
+                              // reads a share of x), else every CTA reads all of x
+  int cluster;                // the K-splits of a weight tile form one thread-block cluster: the
+                              // split-K partials and the E4M3 amax meet in distributed shared
+                              // memory, and the workspace sync block is not used
 };
 
 // SF (VQ only): the weight's scales as in Fp4Cfg -- 0 PreScale atoms in the block, 1 PostScale
@@ -194,6 +203,28 @@ __device__ __forceinline__ void dec_code_mx(const uint32_t (&w)[16], uint4& code
   byte = static_cast<uint32_t>(e + 127);
 }
 
+// Four outputs y[m, nn .. nn + 3] = alpha * acc (bf16, and fp32 when requested).
+__device__ __forceinline__ void dec_store4(const DecodeArgs& a, int m, int nn, float4 acc, float alpha) {
+  const float o4[4] = {acc.x * alpha, acc.y * alpha, acc.z * alpha, acc.w * alpha};
+  const size_t o = static_cast<size_t>(m) * a.ldy + nn;
+  if (nn + 3 < a.N && (a.ldy & 3) == 0) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(o4[0], o4[1]);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(o4[2], o4[3]);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(a.y + o) = pk;
+    if (a.y32 != nullptr) *reinterpret_cast<float4*>(a.y32 + o) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (nn + j < a.N) {
+        a.y[o + j] = __float2bfloat16_rn(o4[j]);
+        if (a.y32 != nullptr) a.y32[o + j] = o4[j];
+      }
+  }
+}
+
 template <int BN, bool E8M0, bool VQ, int SF = 0>
 __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
     fp4_decode_kernel(const DecodeArgs a) {
@@ -221,12 +252,15 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
   uint64_t* bfull = xready + 1;                // every B tile + SFB set in shared memory
   uint64_t* sfb_ok = bfull + 1;                // activation scales in TMEM (4 quantizer warps)
   uint64_t* scbar = sfb_ok + 1;                // SF 2: the scale codebook landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(scbar + 1);
+  uint64_t* camax = scbar + 1;                 // cluster: every split's amax share arrived
+  uint64_t* cpart = camax + 1;                 // cluster: every split's partial is in its smem
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cpart + 1);
   __shared__ uint32_t s_cnt;
   __shared__ uint32_t s_red[4];
   __shared__ float s_ts;
   __shared__ int s_allseen;
   __shared__ int s_fail;   // some bounded wait of this CTA expired
+  __shared__ uint32_t s_camax[kDecMaxSplits];   // cluster: the amax share of each split
   griddep_launch_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -265,6 +299,8 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
       mbar_init(bfull, a.fuse ? 1 : 32);
       mbar_init(sfb_ok, 4);
       mbar_init(scbar, 1);
+      mbar_init(camax, a.splits);
+      mbar_init(cpart, a.splits);
       s_fail = 0;
       s_allseen = 0;
     }
@@ -287,15 +323,18 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  if (a.cluster) cluster_sync_all();   // every CTA of the cluster has its barriers initialised
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int S = a.splits;
 
   bool ok = true;
   if (warp == 0) {
-    // ---------------- the B operand of every stage, once the activations are quantized
-    ok = __all_sync(0xFFFFFFFFu, mbar_wait(xready, 0, 50));
-    if (a.fuse) {
+    // ---------------- the B operand of every stage, once the activations are quantized (the
+    // local mode writes it into shared memory directly)
+    if (a.fuse != 2) ok = __all_sync(0xFFFFFFFFu, mbar_wait(xready, 0, 50));
+    if (a.fuse == 1) {
       // stage tiles and scale sets of this CTA's stages are contiguous in the workspace
       if (lane == 0) {
         const uint32_t bbytes = n_it * Cfg::kBBytes, sbytes = n_it * Cfg::kSfBytes;
@@ -308,7 +347,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
           mbar_arrive(bfull);
         }
       }
-    } else {
+    } else if (a.fuse == 0) {
       // plain layout (qlinear_quantize_input): each stage's B tile by 16-byte cp.async from all
       // 32 lanes into the swizzled layout (rows past M zero-filled), then its scale atoms
       for (int it = 0; it < n_it && ok; ++it) {
@@ -376,7 +415,202 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
     const int tq = threadIdx.x - Cfg::kQWarp0 * 32;   // 0..127
     const int G = gridDim.x;
     griddep_wait();   // x, the workspace and the counter follow the grids before this one
-    if (tq == 0) s_cnt = *reinterpret_cast<volatile uint32_t*>(sy.counter);
+    if (tq == 0) s_cnt = a.cluster ? 0u : *reinterpret_cast<volatile uint32_t*>(sy.counter);
+    if (a.fuse == 2) {
+      // ---- local: this CTA reads all of x for the E4M3 tensor amax (no agreement needed) and
+      // quantizes the activations of its own stages straight into their shared-memory B tiles
+      // The E4M3 tensor amax: all of x read by every CTA (small x); or, in a cluster, each split
+      // reads the x columns of its own stages (together the splits cover x) and the shares meet
+      // in distributed shared memory; or, without a cluster, each CTA reads a share of x,
+      // publishes it in its slot, and CTA 0 gathers the slots and publishes one word that the
+      // others poll.
+      const bool xchg = !E8M0 && a.amax_coop && a.cluster;
+      const bool gather = !E8M0 && a.amax_coop && !a.cluster;
+      float ts = 1.f;
+      uint32_t mx = 0;
+      if constexpr (!E8M0) {
+        if (xchg) {
+          const int units = n_it * a.M * 8;
+          for (int u0 = tq; u0 < units; u0 += 128 * 4) {
+            uint4 v[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int u = u0 + 128 * j;
+              int kw, kx, valid, it = 0, m = 0, kc = 0;
+              if (u < units) {
+                it = u / (a.M * 8);
+                const int rem = u - it * (a.M * 8);
+                m = rem >> 3;
+                kc = rem & 7;
+              }
+              stage_coords(s_begin + it, kw, kx, valid);
+              const bool in = u < units && kc * 32 < valid;
+              const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * a.C + kx + kc * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) v[j][i] = in ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                mx = __vmaxu2(mx, v[j][i].x & 0x7FFF7FFFu);
+                mx = __vmaxu2(mx, v[j][i].y & 0x7FFF7FFFu);
+                mx = __vmaxu2(mx, v[j][i].z & 0x7FFF7FFFu);
+                mx = __vmaxu2(mx, v[j][i].w & 0x7FFF7FFFu);
+              }
+          }
+        } else {
+          const long n16 = static_cast<long>(a.M) * a.C / 8;
+          const long e0 = gather ? n16 * blockIdx.x / G : 0, e1 = gather ? n16 * (blockIdx.x + 1) / G : n16;
+          const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+          for (long base = e0 + tq; base < e1; base += 128 * 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const long i = base + 128L * j;
+              v[j] = i < e1 ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              mx = __vmaxu2(mx, v[j].x & 0x7FFF7FFFu);
+              mx = __vmaxu2(mx, v[j].y & 0x7FFF7FFFu);
+              mx = __vmaxu2(mx, v[j].z & 0x7FFF7FFFu);
+              mx = __vmaxu2(mx, v[j].w & 0x7FFF7FFFu);
+            }
+          }
+        }
+      }
+      uint32_t m16 = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, o));
+      if (lane == 0) s_red[tq >> 5] = m16;
+      named_bar_sync(2, 128);   // s_cnt and s_red
+      const uint32_t cnt = s_cnt;
+      const unsigned long long tag = dec_tag(cnt + 1u);
+      uint32_t amax16 = max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3]));
+      if (!a.cluster && tq == 0 && !withheld(blockIdx.x))
+        st_release_gpu_u64(&sy.slots[blockIdx.x], tag | (gather ? amax16 : 0u));
+      bool qok = true;
+      if (gather && blockIdx.x == 0) {
+        uint32_t a16 = 0;
+        for (int c = tq; c < G; c += 128)
+          a16 = max(a16, static_cast<uint32_t>(dec_wait_tag(&sy.slots[c], tag, 54, qok) & 0xFFFFull));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a16 = max(a16, __shfl_xor_sync(0xFFFFFFFFu, a16, o));
+        named_bar_sync(2, 128);   // s_red was read above
+        if (lane == 0) s_red[tq >> 5] = a16;
+        qok = bar_and(2, 128, qok);
+        amax16 = max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3]));
+        if (tq == 0) {
+          s_allseen = qok ? 1 : 0;
+          if (qok && !withheld(0)) st_release_gpu_u64(sy.result, tag | amax16);
+        }
+      } else if (gather) {
+        named_bar_sync(2, 128);   // s_red was read above
+        if (tq == 0) s_red[0] = static_cast<uint32_t>(dec_wait_tag(sy.result, tag, 61, qok) & 0xFFFFull);
+        qok = bar_and(2, 128, qok);
+        amax16 = s_red[0];
+      } else if (xchg) {
+        // this split's share into slot z of every split's s_camax, then an arrival on its barrier
+        if (tq < S && !withheld(blockIdx.x)) {
+          st_shared_cluster_u32(map_shared_rank(smem_u32(&s_camax[z]), tq), amax16);
+          mbar_arrive_remote(map_shared_rank(smem_u32(camax), tq));
+        }
+        bool w = true;
+        if (tq == 0) w = mbar_wait_cluster(camax, 0, 64);
+        qok = bar_and(2, 128, w);
+        if (qok)
+          for (int r = 0; r < S; ++r) amax16 = max(amax16, s_camax[r]);
+      }
+      if constexpr (!E8M0) ts = tensor_scale_from_amax16(amax16);
+      // (stage, row, 32-element chunk) units, kDecLocalBatch per thread loaded at once so that
+      // their L2 latencies overlap
+      const int units = qok ? n_it * a.M * 8 : 0;
+      for (int u0 = tq; u0 < units; u0 += 128 * kDecLocalBatch) {
+        uint32_t w[kDecLocalBatch][16];
+        int dst[kDecLocalBatch];   // it * 4096 + m * 8 + kc, or -1
+#pragma unroll
+        for (int j = 0; j < kDecLocalBatch; ++j) {
+          const int u = u0 + 128 * j;
+          dst[j] = -1;
+          if (u < units) {
+            const int it = u / (a.M * 8), rem = u - it * (a.M * 8), m = rem >> 3, kc = rem & 7;
+            int kw, kx, valid;
+            stage_coords(s_begin + it, kw, kx, valid);
+            if (kc * 32 < valid) {
+              dst[j] = it * 4096 + m * 8 + kc;
+              const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * a.C + kx + kc * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint4 v = __ldg(src + i);
+                w[j][4 * i] = v.x; w[j][4 * i + 1] = v.y; w[j][4 * i + 2] = v.z; w[j][4 * i + 3] = v.w;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kDecLocalBatch; ++j) {
+          if (dst[j] < 0) continue;
+          const int it = dst[j] >> 12, m = (dst[j] >> 3) & 511, kc = dst[j] & 7;
+          uint4 codes;
+          uint32_t sbytes;
+          if constexpr (E8M0) {
+            if (a.had) {
+              float v[32];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                v[2 * i] = __uint_as_float(w[j][i] << 16);
+                v[2 * i + 1] = __uint_as_float(w[j][i] & 0xFFFF0000u);
+              }
+              fwht32(v);
+              code_mx_f32(v, codes, sbytes);
+            } else {
+              dec_code_mx(w[j], codes, sbytes);
+            }
+          } else {
+            uint32_t p0[2], p1[2], b0, b1;
+            const uint32_t w0[8] = {w[j][0], w[j][1], w[j][2], w[j][3], w[j][4], w[j][5], w[j][6], w[j][7]};
+            const uint32_t w1[8] = {w[j][8], w[j][9], w[j][10], w[j][11], w[j][12], w[j][13], w[j][14], w[j][15]};
+            quant_e4m3_code_block(w0, ts, p0, b0);
+            quant_e4m3_code_block(w1, ts, p1, b1);
+            codes = make_uint4(p0[0], p0[1], p1[0], p1[1]);
+            sbytes = b0 | (b1 << 8);
+          }
+          *reinterpret_cast<uint4*>(sB + it * Cfg::kBBytes + m * 128 + ((kc ^ (m & 7)) << 4)) = codes;
+          uint8_t* sft = sSfb + it * Cfg::kSfBytes + (m & 31) * 16 + ((m >> 5) & 3) * 4;
+          if constexpr (E8M0) {
+            sft[(kc >> 2) * 512 + (kc & 3)] = static_cast<uint8_t>(sbytes);
+          } else {
+            const int j0 = 2 * kc;
+            sft[(j0 >> 2) * 512 + (j0 & 3)] = static_cast<uint8_t>(sbytes);
+            sft[((j0 + 1) >> 2) * 512 + ((j0 + 1) & 3)] = static_cast<uint8_t>(sbytes >> 8);
+          }
+        }
+      }
+      if (!E8M0 && blockIdx.x == 0 && tq == 0 && a.ts_x != nullptr) *a.ts_x = ts;
+      fence_proxy_async_smem();   // the B tiles, for the tensor core
+      named_bar_sync(2, 128);     // every scale byte is in shared memory
+      for (int it = 0; it < n_it; ++it)
+        tmem_st_scale_atoms<Cfg::kAtoms>(tmem + quad_lanes + sfb_col(it), sSfb + it * Cfg::kSfBytes, lane);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sfb_ok);
+      if (tq == 0) {
+        s_ts = ts;
+        if (qok) mbar_arrive(xready);   // else the epilogue's bounded wait records the failure
+        else s_fail = 1;
+      }
+      if (!a.cluster && blockIdx.x == 0 && !gather) {   // every slot before CTA 0 advances the counter
+        bool sok = true;
+        for (int c = tq; c < static_cast<int>(gridDim.x) && sok; c += 128) dec_wait_tag(&sy.slots[c], tag, 54, sok);
+        sok = bar_and(2, 128, sok);
+        if (tq == 0) {
+          s_allseen = sok ? 1 : 0;
+          if (!sok) s_fail = 1;
+        }
+      }
+    } else {
     named_bar_sync(2, 128);
     const uint32_t cnt = s_cnt;
     const unsigned long long tag = dec_tag(cnt + 1u);
@@ -410,7 +644,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
     for (int o = 16; o > 0; o >>= 1) m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, o));
     if (lane == 0) s_red[tq >> 5] = m16;
     named_bar_sync(2, 128);
-    if (tq == 0 && !withheld(blockIdx.x))   // this CTA has read the counter; E4M3: its amax
+    if (!a.cluster && tq == 0 && !withheld(blockIdx.x))   // this CTA has read the counter; E4M3: its amax
       st_release_gpu_u64(&sy.slots[blockIdx.x], tag | max(max(s_red[0], s_red[1]), max(s_red[2], s_red[3])));
     bool qok = true;
     float ts = 1.f;
@@ -449,7 +683,18 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
             uint4 codes;
             uint32_t sbytes;   // E8M0: one byte; E4M3: two (blocks 2j, 2j + 1)
             if constexpr (E8M0) {
-              dec_code_mx(w[k], codes, sbytes);
+              if (a.had) {   // online Hadamard of the 32-element block, then its MX coding
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  v[2 * i] = __uint_as_float(w[k][i] << 16);
+                  v[2 * i + 1] = __uint_as_float(w[k][i] & 0xFFFF0000u);
+                }
+                fwht32(v);
+                code_mx_f32(v, codes, sbytes);
+              } else {
+                dec_code_mx(w[k], codes, sbytes);
+              }
             } else {
               uint32_t p0[2], p1[2], b0, b1;
               const uint32_t w0[8] = {w[k][0], w[k][1], w[k][2], w[k][3], w[k][4], w[k][5], w[k][6], w[k][7]};
@@ -516,7 +761,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(sfb_ok);
     if (!bok) s_fail = 1;
-    if (blockIdx.x == 0 && !amax_needed) {
+    if (!a.cluster && blockIdx.x == 0 && !amax_needed) {
       // CTA 0 advances the counter at its end: first every CTA's slot (each has read the counter)
       bool sok = true;
       for (int c = tq; c < G && sok; c += 128) dec_wait_tag(&sy.slots[c], tag, 54, sok);
@@ -526,6 +771,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
         if (!sok) s_fail = 1;
       }
     }
+    }   // cooperative / plain
   } else {
     if constexpr (VQ) {
       // ---------------- VQ decode (warps 2..9) into the ring of operand tiles: one warp
@@ -623,6 +869,47 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
               if (a.y32 != nullptr) a.y32[o] = v;
             }
         }
+      } else if (a.cluster) {
+        // the partial [M][128] into this CTA's shared memory (the operand tiles are dead once
+        // the accumulator is final), an arrival on every split's barrier, then this split's
+        // share of the tile's outputs added over the splits in split order from their shared
+        // memory (distributed shared memory loads)
+        float* part = reinterpret_cast<float*>(smem);
+        if (ok) {
+#pragma unroll 1
+          for (int c = 0; c < a.M; c += 8) {
+            uint32_t r[8];
+            tmem_ld8(trow + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (c + j < a.M) part[(c + j) * 128 + nl] = n_it > 0 ? __uint_as_float(r[j]) : 0.f;
+          }
+        }
+        named_bar_sync(1, 128);   // the whole partial is written before the releases
+        if (et < S && !withheld(blockIdx.x)) mbar_arrive_remote(map_shared_rank(smem_u32(cpart), et));
+        bool w = true;
+        if (et == 0) w = mbar_wait_cluster(cpart, 0, 65);
+        ok = bar_and(1, 128, ok && w);
+        if (ok) {
+          const int E4 = a.M * 32;
+          const int q0 = static_cast<int>(static_cast<long>(E4) * z / S);
+          const int q1 = static_cast<int>(static_cast<long>(E4) * (z + 1) / S);
+          for (int qq = q0 + et; qq < q1; qq += 128) {
+            const uint32_t la = smem_u32(part + (qq >> 5) * 128 + (qq & 31) * 4);
+            float4 v[kDecMaxSplits];
+#pragma unroll
+            for (int r = 0; r < kDecMaxSplits; ++r)
+              if (r < S) v[r] = ld_shared_cluster_f32x4(map_shared_rank(la, r));
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < kDecMaxSplits; ++r)
+              if (r < S) {
+                acc.x += v[r].x; acc.y += v[r].y; acc.z += v[r].z; acc.w += v[r].w;
+              }
+            dec_store4(a, qq >> 5, n0 + (qq & 31) * 4, acc, alpha);
+          }
+        }
       } else if (ok) {
         float* mine = a.partials + static_cast<size_t>(blockIdx.x) * BN * 128;
 #pragma unroll 1
@@ -658,25 +945,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
               if (r < a.splits) {
                 acc.x += v[r].x; acc.y += v[r].y; acc.z += v[r].z; acc.w += v[r].w;
               }
-            const int m = qq >> 5, nn = n0 + (qq & 31) * 4;
-            const float o4[4] = {acc.x * alpha, acc.y * alpha, acc.z * alpha, acc.w * alpha};
-            const size_t o = static_cast<size_t>(m) * a.ldy + nn;
-            if (nn + 3 < a.N && (a.ldy & 3) == 0) {
-              const __nv_bfloat162 lo = __floats2bfloat162_rn(o4[0], o4[1]);
-              const __nv_bfloat162 hi = __floats2bfloat162_rn(o4[2], o4[3]);
-              uint2 pk;
-              pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-              pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-              *reinterpret_cast<uint2*>(a.y + o) = pk;
-              if (a.y32 != nullptr) *reinterpret_cast<float4*>(a.y32 + o) = make_float4(o4[0], o4[1], o4[2], o4[3]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                if (nn + j < a.N) {
-                  a.y[o + j] = __float2bfloat16_rn(o4[j]);
-                  if (a.y32 != nullptr) a.y32[o + j] = o4[j];
-                }
-            }
+            dec_store4(a, qq >> 5, n0 + (qq & 31) * 4, acc, alpha);
           }
         }
       }
@@ -684,10 +953,11 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
   }
   if (!ok) s_fail = 1;
   tc_fence_before();
-  __syncthreads();
+  if (a.cluster) cluster_sync_all();   // no CTA leaves while the others read its shared memory
+  else __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, 512);
   // The next grid reads the counter only after this one has completed (griddepcontrol.wait).
-  if (threadIdx.x == 0) {
+  if (!a.cluster && threadIdx.x == 0) {
     if (s_fail) atomicAdd(sy.counter, 2u);
     else if (blockIdx.x == 0 && s_allseen) atomicAdd(sy.counter, 1u);
   }

@@ -13,7 +13,7 @@
 //   moe_scatter_kernel     one CTA per expert: offsets and the expert's routed entries
 //                          (f = t*k + s) in ascending (t, s) order -- deterministic
 //   quant_mx_e8m0_b32_kernel (quant_act.cuh) with a bf16 dequantized copy of x
-//   moe_gemm_kernel<GATEUP> gate/up: B rows gathered per entry by TMA tile::gather4; epilogue
+//   moe_gemm_kernel<GATEUP> gate/up: B rows gathered per entry by cp.async; epilogue
 //                          h = silu(g) * u, MXFP4 requantization of h per 32 features, and the
 //                          exact bf16 value of the quantized h for the down projection
 //   moe_gemm_kernel<DOWN>  down: B = the expert's contiguous h rows; epilogue writes
@@ -150,6 +150,7 @@ struct MoeGemmArgs {
   __nv_bfloat16* h_dq;            // [T*k, I] exact bf16 of the quantized h
   float* h32;                     // optional [T*k, I] fp32 h before quantization
   float* yslot;                   // [T*k, H] gate * y per entry (down)
+  int had;                        // gate/up: online Hadamard (block 32) of h before requantizing
   int H;
 };
 
@@ -178,16 +179,6 @@ struct MoeCfg {
   static_assert(kSmemBytes + 4200 <= 227 * 1024, "dynamic + static shared memory per block");
   static_assert(kGatherLag < kStages, "gathers must be signalled before their slot comes round");
 };
-
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int x, int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-      "r"(smem_u32(bar))
-      : "memory");
-}
 
 // Persistent grouped GEMM.  Work items (expert e, 128-row weight tile nt, BN-token tile mt) are
 // enumerated expert by expert, nt fastest; CTA c takes items c, c + gridDim.x, ...  Warp roles:
@@ -450,28 +441,23 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
             const float* gr = sStg + c * Cfg::kStgLd + 32 * blk;
             const float* ur = gr + 64;
             float hv[32];
-            uint32_t am = 0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const float g = gr[i];
               hv[i] = g / (1.0f + expf(-g)) * ur[i];
-              am = max(am, __float_as_uint(hv[i]) & 0x7FFFFFFFu);
             }
-            const int E8 = static_cast<int>(am >> 23);
-            const int ex = (E8 == 0) ? -127 : max(E8 - 129, -127);
-            const float inv = __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
-            uint32_t code[4];
+            if (a.h32 != nullptr) {   // h as computed, before any rotation (stage-wise checks)
+              const size_t p = static_cast<size_t>(I.p0 + h0 + c);
+              float4* d32 = reinterpret_cast<float4*>(a.h32 + p * a.I + I.nt * 64 + 32 * blk);
 #pragma unroll
-            for (int w4 = 0; w4 < 4; ++w4) {
-              float f[8];
-              uint32_t sgn = 0;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                f[i] = hv[8 * w4 + i] * inv;
-                sgn |= ((__float_as_uint(hv[8 * w4 + i]) >> 31) << (4 * i + 3));
-              }
-              code[w4] = e2m1x8(f) | sgn;
+              for (int i = 0; i < 8; ++i) d32[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
             }
+            if (a.had) fwht32(hv);   // online Hadamard of h before its requantization
+            uint4 c4;
+            uint32_t byte;
+            code_mx_f32(hv, c4, byte);
+            const uint32_t code[4] = {c4.x, c4.y, c4.z, c4.w};
+            const int ex = static_cast<int>(byte) - 127;
             const size_t p = static_cast<size_t>(I.p0 + h0 + c);
             const int jf0 = I.nt * 64 + 32 * blk;                  // first intermediate feature
             *reinterpret_cast<uint4*>(a.h_codes + p * (a.I / 2) + jf0 / 2) =
@@ -489,11 +475,6 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
             uint4* dst = reinterpret_cast<uint4*>(a.h_dq + p * a.I + jf0);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(dq[4 * i], dq[4 * i + 1], dq[4 * i + 2], dq[4 * i + 3]);
-            if (a.h32 != nullptr) {
-              float4* d32 = reinterpret_cast<float4*>(a.h32 + p * a.I + jf0);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) d32[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
-            }
           }
           asm volatile("bar.sync 2, 128;" ::: "memory");
         }

@@ -62,11 +62,55 @@ void quant_row_mx(const float* x, int64_t K, uint8_t* codes, uint8_t* sbytes) {
   }
 }
 
+// MXFP4 quantization of one row with the E8M0-W local block-scale search (PRQuant §5.3): per
+// 32-block the OCP exponent e0 and its neighbours e0 + 1, e0 - 1 (clamped to [-127, 127]) are
+// tried in that order with the same element rule; the block keeps the first with the smallest
+// sum of squared errors (double, summed in element order; a later one only if strictly better).
+void quant_row_mx_search(const float* x, int64_t K, uint8_t* codes, uint8_t* sbytes) {
+  for (int64_t b = 0; b < K / 32; ++b) {
+    float amax = 0.f;
+    for (int i = 0; i < 32; ++i) amax = std::max(amax, std::fabs(x[b * 32 + i]));
+    const int E = static_cast<int>((f32_bits(amax) >> 23) & 0xFF);
+    const int e0 = (E == 0) ? -127 : std::max(E - 129, -127);
+    int best_e = e0;
+    double best_err = 0;
+    uint8_t best[32], cand[32];
+    for (int t = 0; t < 3; ++t) {
+      const int e = std::min(127, std::max(-127, e0 + (t == 0 ? 0 : t == 1 ? 1 : -1)));
+      double err = 0;
+      for (int i = 0; i < 32; ++i) {
+        const double v = static_cast<double>(x[b * 32 + i]);
+        cand[i] = e2m1_code(static_cast<float>(std::ldexp(v, -e)));
+        const double d = v - static_cast<double>(e2m1_value(cand[i])) * std::ldexp(1.0, e);
+        err += d * d;
+      }
+      if (t == 0 || err < best_err) {
+        best_err = err;
+        best_e = e;
+        std::memcpy(best, cand, 32);
+      }
+    }
+    sbytes[b] = static_cast<uint8_t>(best_e + 127);
+    std::memcpy(codes + b * 32, best, 32);
+  }
+}
+
 }  // namespace
+
+extern "C" ql_status qlinear_prepare_prquant_ex(const uint16_t* w_bf16, int64_t N, int64_t C,
+                                                int32_t k, int32_t scale_search, int32_t* perm_out,
+                                                uint8_t* codes_out, uint8_t* scales_out);
 
 extern "C" ql_status qlinear_prepare_prquant(const uint16_t* w_bf16, int64_t N, int64_t C,
                                              int32_t k, int32_t* perm_out, uint8_t* codes_out,
                                              uint8_t* scales_out) {
+  return qlinear_prepare_prquant_ex(w_bf16, N, C, k, 0, perm_out, codes_out, scales_out);
+}
+
+extern "C" ql_status qlinear_prepare_prquant_ex(const uint16_t* w_bf16, int64_t N, int64_t C,
+                                                int32_t k, int32_t scale_search, int32_t* perm_out,
+                                                uint8_t* codes_out, uint8_t* scales_out) {
+  auto quant_row = scale_search ? quant_row_mx_search : quant_row_mx;
   if (w_bf16 == nullptr || perm_out == nullptr || codes_out == nullptr || scales_out == nullptr)
     return QL_ERR_INVALID_ARG;
   if (N <= 0 || C <= 0 || k <= 0 || k > C) return QL_ERR_INVALID_ARG;
@@ -79,7 +123,7 @@ extern "C" ql_status qlinear_prepare_prquant(const uint16_t* w_bf16, int64_t N, 
     std::vector<uint8_t> codes(C), sb(C / 32);
     for (int64_t n = 0; n < N; ++n) {
       for (int64_t c = 0; c < C; ++c) row[c] = bf16_to_f32(w_bf16[n * C + c]);
-      quant_row_mx(row.data(), C, codes.data(), sb.data());
+      quant_row(row.data(), C, codes.data(), sb.data());
       for (int64_t c = 0; c < C; ++c) {
         const double d = static_cast<double>(row[c]) -
                          static_cast<double>(e2m1_value(codes[c])) * std::ldexp(1.0, sb[c / 32] - 127);
@@ -104,12 +148,12 @@ extern "C" ql_status qlinear_prepare_prquant(const uint16_t* w_bf16, int64_t N, 
   std::vector<uint8_t> codes(Kp), sb(Kp / 32);
   for (int64_t n = 0; n < N; ++n) {
     for (int64_t j = 0; j < C; ++j) row[j] = bf16_to_f32(w_bf16[n * C + perm_out[j]]);
-    quant_row_mx(row.data(), C, codes.data(), sb.data());
+    quant_row(row.data(), C, codes.data(), sb.data());
     for (int32_t j = 0; j < k; ++j) {
       const int64_t c = C - k + j;
       res[j] = row[c] - e2m1_value(codes[c]) * std::ldexp(1.0f, sb[c / 32] - 127);  // exact
     }
-    quant_row_mx(res.data(), k, codes.data() + C, sb.data() + C / 32);
+    quant_row(res.data(), k, codes.data() + C, sb.data() + C / 32);
     for (int64_t j = 0; j < Kp / 2; ++j)
       codes_out[n * (Kp / 2) + j] =
           static_cast<uint8_t>((codes[2 * j] & 0xF) | ((codes[2 * j + 1] & 0xF) << 4));

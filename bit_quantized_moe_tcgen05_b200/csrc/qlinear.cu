@@ -166,27 +166,76 @@ ql_status launch_fp4(int BN, const CUtensorMap& tx, const CUtensorMap& ty, const
   return fail(QL_ERR_UNSUPPORTED, "no GEMM tile for BN=%d", BN);
 }
 
+// The decode kernel's launch attributes, set once per device (dynamic shared memory above 48 KB;
+// clusters of up to 16 CTAs).
+template <int BN, bool E8M0, bool VQ, int SF = 0>
+ql_status dec_set_attrs() {
+  using Cfg = ql::DecCfg<BN, E8M0, VQ, SF>;
+  static std::atomic<bool> attr_done[64] = {};
+  int dev = 0;
+  QL_CUDA(cudaGetDevice(&dev));
+  if (dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
+    QL_CUDA(cudaFuncSetAttribute(ql::fp4_decode_kernel<BN, E8M0, VQ, SF>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+    QL_CUDA(cudaFuncSetAttribute(ql::fp4_decode_kernel<BN, E8M0, VQ, SF>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    if (dev < 64) attr_done[dev].store(true, std::memory_order_release);
+  }
+  return QL_OK;
+}
+
+// How many clusters of S decode CTAs the device can hold at once (0 if none), cached per
+// (device, S).
+template <int BN, bool E8M0, bool VQ, int SF = 0>
+int dec_max_clusters_bn(int S) {
+  using Cfg = ql::DecCfg<BN, E8M0, VQ, SF>;
+  static std::atomic<int> cache[64][ql::kDecMaxSplits + 1];
+  static std::atomic<bool> known[64][ql::kDecMaxSplits + 1];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || S < 1 || S > ql::kDecMaxSplits) return 0;
+  if (dev < 64 && known[dev][S].load(std::memory_order_acquire)) return cache[dev][S].load();
+  int n = 0;
+  if (dec_set_attrs<BN, E8M0, VQ, SF>() == QL_OK) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, 1, 1);
+    cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, ql::fp4_decode_kernel<BN, E8M0, VQ, SF>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  if (dev < 64) {
+    cache[dev][S].store(n);
+    known[dev][S].store(true, std::memory_order_release);
+  }
+  return n;
+}
+
 template <int BN, bool E8M0, bool VQ, int SF = 0>
 ql_status launch_dec_bn(const ql::DecodeArgs& a, int grid, cudaStream_t s) {
   using Cfg = ql::DecCfg<BN, E8M0, VQ, SF>;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    QL_CUDA(cudaFuncSetAttribute(ql::fp4_decode_kernel<BN, E8M0, VQ, SF>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
-    attr_done[dev] = true;
-  }
+  ql_status st = dec_set_attrs<BN, E8M0, VQ, SF>();
+  if (st != QL_OK) return st;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = a.cluster ? a.splits : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.cluster ? 2 : 1;
   QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_decode_kernel<BN, E8M0, VQ, SF>, a));
   return QL_OK;
 }
@@ -199,6 +248,14 @@ ql_status launch_dec(int BN, const ql::DecodeArgs& a, int grid, cudaStream_t s) 
     case 64: return launch_dec_bn<64, E8M0, VQ, SF>(a, grid, s);
   }
   return fail(QL_ERR_UNSUPPORTED, "no decode tile for BN=%d", BN);
+}
+template <bool E8M0, bool VQ, int SF = 0>
+int dec_max_clusters(int BN, int S) {
+  switch (BN) {
+    case 16: return dec_max_clusters_bn<16, E8M0, VQ, SF>(S);
+    case 32: return dec_max_clusters_bn<32, E8M0, VQ, SF>(S);
+    default: return dec_max_clusters_bn<64, E8M0, VQ, SF>(S);
+  }
 }
 
 // Token-tile width: the smallest power of two >= M up to 128.  Past 128 tokens, 256-wide tiles,
@@ -228,6 +285,7 @@ struct ql_linear {
   bool e8m0 = true;            // E8M0-B32 scales (else E4M3-B16 + tensor scales)
   bool vq = false;             // MXCode VQ weight
   int sfmode = 0;              // VQ scales: 0 PreScale atoms, 1 PostScale per QBlock, 2 PreScale+
+  int had = 0;                 // online block-32 Hadamard of the activations (MXFP4 layers)
   uint8_t* d_scb = nullptr;    // PreScale+: scale codebook [256][8] on the device
   uint8_t* d_codes = nullptr;  // weight blocks [N/128][stages][codes or indices + codebooks, scales]
   size_t weight_bytes = 0;
@@ -252,6 +310,9 @@ struct FwdPlan {
   int n_tickets;   // split-K tickets (zeroed by the quantizer, re-armed by the GEMM)
   bool decode = false;   // fp4_decode_kernel: M <= 64, one CTA per (weight tile, K range)
   bool fusable = false;  // ... and the forward may quantize x inside it (one launch)
+  int fuse_mode = 1;     // 1: cooperatively over the grid; 2: each CTA its own stages
+  bool amax_coop = false;   // fuse_mode 2, E4M3: the tensor amax combined over the CTAs
+  bool cluster = false;     // the K-splits of a tile form a cluster (fuse_mode 2 or 0)
   size_t dsync_off = 0;  // its launch counter, slots and flags
   size_t xt_off = 0, st_off = 0;   // fused: per-stage B tiles and activation scale sets
 };
@@ -303,6 +364,18 @@ int dec_max_stages(const ql_linear* L, int BN) {
   if (L->vq) return dec_max_stages<false, true>(BN);
   return L->e8m0 ? dec_max_stages<true, false>(BN) : dec_max_stages<false, false>(BN);
 }
+int dec_max_clusters(const ql_linear* L, int BN, int S) {
+  if (L->vq && L->sfmode == 1) return dec_max_clusters<false, true, 1>(BN, S);
+  if (L->vq && L->sfmode == 2) return dec_max_clusters<false, true, 2>(BN, S);
+  if (L->vq) return dec_max_clusters<false, true>(BN, S);
+  return L->e8m0 ? dec_max_clusters<true, false>(BN, S) : dec_max_clusters<false, false>(BN, S);
+}
+
+// Decode-kernel activation quantization: -1 chooses per launch, 1 or 2 forces that mode where
+// the launch allows it (ql_decode_fuse_mode).
+std::atomic<int> g_decode_fuse_mode{-1};
+constexpr int kDecLocalUnits = 8;                // local mode: units per quantizer thread at most
+constexpr int64_t kDecLocalAmaxElems = 128 * 1024;   // x elements every CTA may read for the amax
 
 // Decode launches (M <= 64): the weight tiles split along K so that the grid covers the SMs once;
 // each CTA keeps all its stages resident.  Returns false when no such split exists.
@@ -314,13 +387,43 @@ bool plan_decode(const ql_linear* L, int64_t M, FwdPlan& p) {
   const int sms = std::min(sm_count(), ql::kDecMaxGrid);
   if (p.tiles_n > sms) return false;
   const int total = L->n_stages_total;
+  const int max_stages = dec_max_stages(L, p.BN);   // (VQ: leaves room for one ring tile)
   int splits = std::max(1, std::min({sms / p.tiles_n, total, ql::kDecMaxSplits}));
   p.spp = static_cast<int>(cdiv(total, splits));
   p.splits = static_cast<int>(cdiv(total, p.spp));
-  if (p.spp > dec_max_stages(L, p.BN)) return false;   // (VQ: leaves room for one ring tile)
-  // fused quantization: split z's units (M rows x its 32-column groups) over the split's tiles
+  if (p.spp > max_stages) return false;
+  // each CTA quantizing its own stages: (stage, row, 32-column) units per quantizer thread
+  auto local_ok = [&](int spp) { return cdiv(static_cast<int64_t>(spp) * M * 8, 128) <= kDecLocalUnits; };
+  const int forced = g_decode_fuse_mode.load();
+  // Preferred: the splits of a tile as one cluster (no grid-wide waits at all), with the largest
+  // split count whose clusters the device holds at once.
+  p.cluster = false;
+  if (forced == -1 || forced == 3) {
+    for (int sp = p.splits; sp >= 1; --sp) {
+      const int spp = static_cast<int>(cdiv(total, sp));
+      const int s2 = static_cast<int>(cdiv(total, spp));
+      if (spp > max_stages) break;
+      if (s2 != sp) continue;
+      if (dec_max_clusters(L, p.BN, s2) >= p.tiles_n) {
+        p.spp = spp;
+        p.splits = s2;
+        p.cluster = true;
+        break;
+      }
+    }
+  }
+  // fused quantization without a cluster: split z's units (M rows x its 32-column groups) over
+  // the split's tiles (cooperative), or each CTA its own stages (local)
   const int64_t upr_max = std::min<int64_t>(static_cast<int64_t>(p.spp) * 8, L->C / 32);
-  p.fusable = cdiv(M * upr_max, p.tiles_n) <= 128 * ql::kDecQUnits;
+  const bool coop_ok = cdiv(M * upr_max, p.tiles_n) <= 128 * ql::kDecQUnits;
+  if (p.cluster) p.fuse_mode = local_ok(p.spp) ? 2 : 0;
+  else if (forced == 3) p.fuse_mode = 0;
+  else if (forced == 1) p.fuse_mode = coop_ok ? 1 : 0;
+  else if (forced == 2) p.fuse_mode = local_ok(p.spp) ? 2 : 0;
+  else p.fuse_mode = local_ok(p.spp) ? 2 : (coop_ok ? 1 : 0);
+  p.fusable = p.fuse_mode != 0;
+  // E4M3: every CTA reads all of x for the tensor amax while x is small, else the grid gathers it
+  p.amax_coop = !L->e8m0 && M * L->C > kDecLocalAmaxElems;
   p.full_tiles = 0;
   p.decode = true;
   return true;
@@ -548,7 +651,8 @@ ql_status launch_quant_int4(const void* x, int64_t M, int64_t K, int8_t* q8, uin
 
 ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
                           uint8_t* st, int st_atoms, int* zero_words, int nzero,
-                          cudaStream_t s, __nv_bfloat16* deq = nullptr, int st_rows = 128) {
+                          cudaStream_t s, __nv_bfloat16* deq = nullptr, int st_rows = 128,
+                          int had = 0) {
   const long total = static_cast<long>(M) * (K / 32);
   const long threads = std::max<long>(total, nzero);
   if (threads == 0) return QL_OK;
@@ -557,7 +661,7 @@ ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, u
   ql::quant_mx_e8m0_b32_kernel<<<static_cast<unsigned>(grid), block, 0, s>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K),
       static_cast<int>(K), codes, static_cast<int>(K / 2), sp, static_cast<int>(K / 32), st,
-      st_atoms, st_rows, zero_words, nzero, deq);
+      st_atoms, st_rows, zero_words, nzero, deq, had);
   QL_CUDA(cudaGetLastError());
   return QL_OK;
 }
@@ -808,6 +912,8 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
   if (sfmode == 2 && (d->scale_codebook == nullptr || d->scale_codebook_entries != 256 ||
                       d->scale_group != 8))
     return fail(QL_ERR_UNSUPPORTED, "PreScale+ needs a scale codebook of 256 entries of 8 scales");
+  if (d->had_block != 0 && (d->had_block != 32 || !mx))
+    return fail(QL_ERR_UNSUPPORTED, "online Hadamard: block 32 with MXFP4 (E8M0-B32) layers only");
   if (d->N > (1 << 24) || d->K > (1 << 24))
     return fail(QL_ERR_UNSUPPORTED, "N/K too large");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -820,6 +926,7 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
   L->e8m0 = mx;
   L->vq = vq;
   L->sfmode = sfmode;
+  L->had = d->had_block == 32 ? 1 : 0;
   L->w_ts = mx ? 1.f : d->w_tensor_scale;
   L->n_base_stages = static_cast<int>(cdiv(L->C, 256));
   L->n_stages_total = L->n_base_stages + static_cast<int>(cdiv(L->k_tail, 256));
@@ -912,7 +1019,7 @@ ql_status qlinear_quantize_input(const ql_linear* L, const void* x, int64_t M, v
   }
   return launch_quant_mx(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
                          reinterpret_cast<int*>(w8 + p.tick_off), p.n_tickets,
-                         reinterpret_cast<cudaStream_t>(stream), nullptr, p.sf_rows);
+                         reinterpret_cast<cudaStream_t>(stream), nullptr, p.sf_rows, L->had);
 }
 
 // The decode kernel: x != null quantizes x inside it (qlinear_forward), else the workspace holds
@@ -928,7 +1035,9 @@ static ql_status launch_decode(const ql_linear* L, int64_t M, const FwdPlan& p, 
   a.n_stages_total = L->n_stages_total;
   a.spp = p.spp;
   a.splits = p.splits;
-  a.fuse = x != nullptr ? 1 : 0;
+  a.fuse = x != nullptr ? p.fuse_mode : 0;
+  a.amax_coop = p.amax_coop ? 1 : 0;
+  a.cluster = p.cluster ? 1 : 0;
   a.x = static_cast<const __nv_bfloat16*>(x);
   a.xq = w8 + p.codes_off;
   a.sfb = w8 + p.sf_off;
@@ -943,6 +1052,7 @@ static ql_status launch_decode(const ql_linear* L, int64_t M, const FwdPlan& p, 
   a.partials = reinterpret_cast<float*>(w8 + p.part_off);
   a.sync = w8 + p.dsync_off;
   a.scb = L->d_scb;
+  a.had = L->had;
   const int grid = p.tiles_n * p.splits;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (L->vq && L->sfmode == 1) return launch_dec<false, true, 1>(p.BN, a, grid, cs);
@@ -1120,6 +1230,27 @@ ql_status ql_debug_inject(int32_t withhold_cta, uint64_t wait_limit_ns) {
   return QL_OK;
 }
 
+ql_status ql_decode_fuse_mode(int32_t mode) {
+  if (mode != -1 && (mode < 1 || mode > 3)) return fail(QL_ERR_INVALID_ARG, "mode must be -1, 1, 2 or 3");
+  g_decode_fuse_mode.store(mode);
+  return QL_OK;
+}
+
+ql_status quantize_act_hadamard(ql_aformat fmt, int32_t had_block, const void* x, int64_t M,
+                                int64_t K, void* codes, void* scales, ql_stream_t stream) {
+  if (M < 0 || K < 0) return fail(QL_ERR_INVALID_ARG, "negative size");
+  if (fmt != QL_A_MXFP4_E8M0_B32 || had_block != 32)
+    return fail(QL_ERR_UNSUPPORTED, "online Hadamard: block 32 before MXFP4 (E8M0-B32) only");
+  if (K % 32 != 0) return fail(QL_ERR_UNSUPPORTED, "MXFP4 needs K %% 32 == 0");
+  if (M == 0 || K == 0) return QL_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return fail(QL_ERR_INVALID_ARG, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(x) & 15) != 0 || (reinterpret_cast<uintptr_t>(codes) & 15) != 0)
+    return fail(QL_ERR_INVALID_ARG, "x and codes must be 16-byte aligned");
+  return launch_quant_mx(x, M, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                         nullptr, 0, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), nullptr,
+                         128, 1);
+}
+
 ql_status ql_check(ql_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   QL_CUDA(cudaStreamSynchronize(s));
@@ -1144,6 +1275,7 @@ struct ql_moe {
   __nv_bfloat16* d_cent_d = nullptr;  // [E*H][16]
   CUtensorMap tm_idx_gu, tm_idx_d;
   bool capture_h32 = false;
+  int had_x = 0, had_h = 0;           // online block-32 Hadamard of x (gate/up) and of h (down)
 };
 
 namespace {
@@ -1221,9 +1353,13 @@ ql_status moe_create(const ql_weight_desc* gu, const ql_weight_desc* dn, int32_t
     return fail(QL_ERR_INVALID_ARG, "gate/up must be [E*2I, H] and down [E*H, I]");
   if (I % 64 != 0 || H % 128 != 0 || H % 64 != 0 || I < 64)
     return fail(QL_ERR_UNSUPPORTED, "MoE needs I %% 64 == 0 and H %% 128 == 0");
+  if ((gu->had_block != 0 && gu->had_block != 32) || (dn->had_block != 0 && dn->had_block != 32))
+    return fail(QL_ERR_UNSUPPORTED, "online Hadamard: block 32 only");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   auto* m = new ql_moe();
   m->E = E; m->k = top_k; m->H = static_cast<int>(H); m->I = static_cast<int>(I);
+  m->had_x = gu->had_block == 32 ? 1 : 0;
+  m->had_h = dn->had_block == 32 ? 1 : 0;
   // gate/up rows in kernel order: per expert, per 128-row tile: 64 gate rows then the 64 up
   // rows with the same intermediate index, so SwiGLU pairs sit in one accumulator tile.
   const size_t rgu = static_cast<size_t>(E) * two_i;
@@ -1321,7 +1457,7 @@ ql_status moe_grouped_forward(const ql_moe* m, const void* x, int64_t T, const f
   QL_CUDA(cudaGetLastError());
   __nv_bfloat16* x_dq = reinterpret_cast<__nv_bfloat16*>(w8 + p.x_dq);
   ql_status st = launch_quant_mx(x, T, m->H, w8 + p.x_codes, w8 + p.x_scales, nullptr, 0, nullptr,
-                                 0, s, x_dq);
+                                 0, s, x_dq, 128, m->had_x);
   if (st != QL_OK) return st;
   CUtensorMap tm_x, tm_h;
   __nv_bfloat16* h_dq = reinterpret_cast<__nv_bfloat16*>(w8 + p.h_dq);
@@ -1334,6 +1470,7 @@ ql_status moe_grouped_forward(const ql_moe* m, const void* x, int64_t T, const f
   a.h_codes = w8 + p.h_codes; a.h_scales = w8 + p.h_scales; a.h_dq = h_dq;
   a.h32 = m->capture_h32 ? reinterpret_cast<float*>(w8 + p.h32) : nullptr;
   a.yslot = reinterpret_cast<float*>(w8 + p.yslot);
+  a.had = m->had_h;
   const int max_mtiles = m->E + (total + kMoeBN - 1) / kMoeBN;   // >= sum_e ceil(count_e / BN)
   a.rows_per_expert = 2 * m->I; a.kdim = m->H; a.n_tiles = 2 * m->I / 128; a.cent = m->d_cent_gu;
   st = launch_moe_gemm<kMoeBN, true>(m->tm_idx_gu, tm_x, a, a.n_tiles * max_mtiles, s);

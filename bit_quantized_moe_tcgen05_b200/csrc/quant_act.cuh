@@ -17,15 +17,6 @@
 
 namespace ql {
 
-// Round an (exactly scaled) fp32 value to the nearest E2M1 code, ties to the even code,
-// saturating at 6; the sign bit follows the input's sign bit.
-__device__ __forceinline__ uint32_t e2m1_rne(float v) {
-  const float a = fabsf(v);
-  uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
-               (a >= 3.5f) + (a > 5.0f);
-  return c | ((__float_as_uint(v) >> 28) & 8u);
-}
-
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -65,17 +56,6 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&f)[8]) {
   return out;
 }
 
-// Two E2M1 codes (lo -> low nibble, hi -> high nibble), RNE, satfinite; no sign fix-up.
-__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b0;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.u32.u8 %0, b0;\n\t}"
-      : "=r"(out)
-      : "f"(lo), "f"(hi));
-  return out;
-}
-
 // Value of an E2M1 code (bit 3 = sign).
 __device__ __forceinline__ float e2m1_code_value(uint32_t c) {
   const uint32_t m = c & 7u;
@@ -94,6 +74,52 @@ __device__ __forceinline__ uint32_t bf16x8_sign_nibbles(const uint32_t (&w)[4]) 
   return s;
 }
 
+// Online block Hadamard (CodeQuant's "had" variants: online Hadamard transforms during
+// quantization; block 32, the MX block): the 32 values of one block, in fp32, through the
+// Walsh-Hadamard butterfly in the order h = 1, 2, 4, 8, 16, each step (a, b) -> (a + b, a - b) a
+// plain fp32 addition or subtraction, so the result is x . H_32 (Sylvester order, unnormalised;
+// the weight carries H_32 / 32).
+__device__ __forceinline__ void fwht32(float (&v)[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < 32; i += 2 * h)
+#pragma unroll
+      for (int j = i; j < i + h; ++j) {
+        const float a = v[j], b = v[j + h];
+        v[j] = __fadd_rn(a, b);
+        v[j + h] = __fsub_rn(a, b);
+      }
+}
+
+// MX E8M0-B32 coding of 32 fp32 values (each exactly scalable by a power of two): the E8M0 byte
+// (e = floor(log2 amax) - 2 from the fp32 exponent, clamped to [-127, 127]; 0 for a zero or
+// subnormal amax) and 16 bytes of codes, element 2i in the low nibble, sign bits from the inputs.
+__device__ __forceinline__ void code_mx_f32(const float (&v)[32], uint4& codes, uint32_t& byte) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+  const int e = (E == 0) ? -127 : max(E - 129, -127);
+  // 2^-e as two exact power-of-two factors (2^-e alone overflows fp32 for e = -127)
+  const float inv1 = __uint_as_float(static_cast<uint32_t>(127 - (e >> 1)) << 23);
+  const float inv2 = __uint_as_float(static_cast<uint32_t>(127 - (e - (e >> 1))) << 23);
+  uint32_t packed[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float f[8];
+    uint32_t sgn = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[i] = __fmul_rn(__fmul_rn(v[8 * q + i], inv1), inv2);
+      sgn |= ((__float_as_uint(v[8 * q + i]) >> 31) << 3) << (4 * i);
+    }
+    packed[q] = e2m1x8(f) | sgn;
+  }
+  codes = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  byte = static_cast<uint32_t>(e + 127);
+}
+
 // One thread per 32-element block (4 x 16-byte loads in flight, one 16-byte code store).
 // x: bf16 [M, K] with row stride ldx (elements).  codes: [M, K/2] bytes (row stride ldc),
 // low nibble = even k.  Scales go to the plain [M, K/32] layout and/or the tiled layout.
@@ -103,7 +129,7 @@ __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, uint8_t* __restrict__ codes,
     int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
     int sf_atoms_per_row, int sf_tile_rows, int* __restrict__ zero_words, int nzero,
-    __nv_bfloat16* __restrict__ deq_out = nullptr) {
+    __nv_bfloat16* __restrict__ deq_out = nullptr, int had = 0) {
   griddep_launch_dependents();   // a GEMM launched behind this grid may start streaming weights
   const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (zero_words != nullptr && gtid < nzero) zero_words[gtid] = 0;
@@ -118,26 +144,42 @@ __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
     const uint4 v = __ldg(src + i);
     w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
   }
-  // amax over 32 bf16 magnitudes as 16-bit unsigned integers (order-preserving for finite values)
-  uint32_t mx = 0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
-  const uint32_t amax16 = max(mx & 0xFFFFu, mx >> 16);
-  // floor(log2 amax) from the bf16 exponent field; zero or subnormal amax clamps to e = -127.
-  const int E = static_cast<int>(amax16 >> 7);
-  const int e = (E == 0) ? -127 : max(E - 129, -127);
-  const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, normal
   uint32_t packed[4];
+  int e;
+  if (had) {
+    float v[32];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    float f[8];
-    const uint32_t ww[4] = {w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __uint_as_float(ww[i] << 16) * inv;
-      f[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u) * inv;
+    for (int i = 0; i < 16; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
-    packed[q] = e2m1x8(f) | bf16x8_sign_nibbles(ww);
+    fwht32(v);
+    uint4 c4;
+    uint32_t byte;
+    code_mx_f32(v, c4, byte);
+    packed[0] = c4.x; packed[1] = c4.y; packed[2] = c4.z; packed[3] = c4.w;
+    e = static_cast<int>(byte) - 127;
+  } else {
+    // amax over 32 bf16 magnitudes as 16-bit unsigned integers (order-preserving for finite values)
+    uint32_t mx = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
+    const uint32_t amax16 = max(mx & 0xFFFFu, mx >> 16);
+    // floor(log2 amax) from the bf16 exponent field; zero or subnormal amax clamps to e = -127.
+    const int E = static_cast<int>(amax16 >> 7);
+    e = (E == 0) ? -127 : max(E - 129, -127);
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, normal
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float f[8];
+      const uint32_t ww[4] = {w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(ww[i] << 16) * inv;
+        f[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u) * inv;
+      }
+      packed[q] = e2m1x8(f) | bf16x8_sign_nibbles(ww);
+    }
   }
   *reinterpret_cast<uint4*>(codes + static_cast<size_t>(m) * ldc + j * 16) =
       make_uint4(packed[0], packed[1], packed[2], packed[3]);

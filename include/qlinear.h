@@ -98,6 +98,10 @@ typedef struct ql_weight_desc {
   const uint8_t* scale_codebook;       /* VQ PreScale+: [scale_codebook_entries][scale_group] */
   int32_t scale_codebook_entries;      /* 256 */
   int32_t scale_group;                 /* 8 consecutive E4M3 block scales along K per index */
+  int32_t had_block;   /* 0, or 32: the layer's activation (MXFP4 layers; MoE: x for gate/up,
+                          h for down) passes an online block-32 Hadamard before quantization
+                          (CodeQuant's "had" variants), and the weight is given rotated,
+                          W . blockdiag(H_32) / 32; see quantize_act_hadamard */
 } ql_weight_desc;
 
 typedef struct ql_linear ql_linear;
@@ -230,6 +234,33 @@ ql_status ql_tensor_peak(int32_t kind, int32_t n, int32_t iters, int32_t ctas,
  * launch left behind. */
 ql_status ql_debug_inject(int32_t withhold_cta, uint64_t wait_limit_ns);
 
+/* How qlinear_forward's decode kernel (M <= 64, FP4 and VQ layers) is organised:
+ * 1 = the CTAs share the activation units out, exchange the E4M3 tensor amax and the finished
+ * stage tiles through the workspace; 2 = every CTA quantizes the activations of its own K stages
+ * straight into shared memory (the E4M3 amax read from all of x while x is small, else gathered
+ * over the grid through the workspace); 3 = the K-splits of each weight tile are launched as one
+ * thread-block cluster: the split-K partials (and the E4M3 amax shares) meet in distributed
+ * shared memory and no CTA waits on another outside its cluster; each CTA quantizes x for its
+ * own stages as in 2 while that is little work (M * stages small), else the separate quantizer
+ * runs first.  -1 (the default) = 3 where the device holds every cluster at once, else 2 or 1,
+ * chosen per launch from M, the split and the width.  A forced mode that a launch cannot take
+ * falls back to the separate quantizer launch.  Quantized codes are identical in every mode;
+ * outputs are identical between modes with the same K split (1 and 2), while mode 3 may split K
+ * into fewer parts (its clusters must fit the device at once), which reorders the fp32 split-K
+ * sum.  Process-wide; for tests and tuning.  QL_ERR_INVALID_ARG for other values. */
+ql_status ql_decode_fuse_mode(int32_t mode);
+
+/* MXFP4 activation quantization with an online block Hadamard in front (CodeQuant, accuracy
+ * tables: the "had" variants enable online Hadamard transforms during quantization; the size and
+ * algorithm are readings): each 32-element block of x (bf16, device) becomes x . H_32 (Sylvester,
+ * unnormalised) computed in fp32 by the Walsh-Hadamard butterfly h = 1, 2, 4, 8, 16, each step
+ * (a, b) -> (a + b, a - b) one IEEE fp32 operation; the result is quantized by the
+ * QL_A_MXFP4_E8M0_B32 rule of quantize_act.  fmt must be QL_A_MXFP4_E8M0_B32 and had_block 32;
+ * K % 32 == 0; codes [M,K/2], E8M0 scales [M,K/32] (device).  The matching weight is
+ * W . blockdiag(H_32) / 32, so the layer's product is unchanged. */
+ql_status quantize_act_hadamard(ql_aformat fmt, int32_t had_block, const void* x_bf16, int64_t M,
+                                int64_t K, void* codes, void* scales, ql_stream_t stream);
+
 /* Synchronise `stream` and report (then clear) the device error word. */
 ql_status ql_check(ql_stream_t stream);
 
@@ -243,6 +274,15 @@ ql_status ql_check(ql_stream_t stream);
  * Requires C % 128 == 0, k % 128 == 0, 0 < k <= C. */
 ql_status qlinear_prepare_prquant(const uint16_t* w_bf16, int64_t N, int64_t C, int32_t k,
                                   int32_t* perm_out, uint8_t* codes_out, uint8_t* scales_out);
+/* The same with scale_search = 1: every weight block (the per-column error pass, W~ and R) takes
+ * the E8M0-W local block-scale search of PRQuant §5.3 ("PRQuant (E8M0-W)"): per 32-block the
+ * OCP exponent e0 and its neighbours e0 + 1 and e0 - 1 (clamped to [-127,127]) are tried in that
+ * order with the same element rule, and the block keeps the first with the smallest sum of
+ * squared errors (double, element order; a later candidate only if strictly better).
+ * scale_search = 0 is qlinear_prepare_prquant. */
+ql_status qlinear_prepare_prquant_ex(const uint16_t* w_bf16, int64_t N, int64_t C, int32_t k,
+                                     int32_t scale_search, int32_t* perm_out, uint8_t* codes_out,
+                                     uint8_t* scales_out);
 
 /* ---- MoE grouped FFN (CodeQuant-style cluster-codebook experts) ----------------------------
  * CodeQuant abstract and Figure 4 (table in SM shared memory); gated FFN of PRQuant's Eq. (1).

@@ -17,6 +17,7 @@ import numpy as np
 
 from . import formats as F
 from . import gemm as G
+from . import hadamard as Hd
 from . import mx
 
 
@@ -91,17 +92,25 @@ def down_combine(hq: np.ndarray, r: dict, Wd: list, T: int, k: int) -> tuple[np.
 
 
 def forward(xd: np.ndarray, logits: np.ndarray, Wgu: list, Wd: list, k: int,
-            h_given: np.ndarray | None = None) -> dict:
+            h_given: np.ndarray | None = None, had_x: bool = False, had_h: bool = False) -> dict:
     """The whole routed FFN.  xd: bf16 activations as float64 [T, H].  Wgu[e]: [2I, H] float64,
     Wd[e]: [H, I] float64.  h_given (optional): the intermediate h (expert-sorted order) to
-    requantize instead of the oracle's own, for stage-wise comparison."""
+    requantize instead of the oracle's own, for stage-wise comparison; it must then be float32
+    values when had_h is set.  had_x / had_h: x, resp. h, passes the online block-32 Hadamard
+    (hadamard.rotate_activation_f32) before its MXFP4 quantization; the weights given are then
+    the rotated ones."""
     T = xd.shape[0]
     I = Wd[0].shape[1]
-    xc, xs = mx.quantize_e8m0_b32(xd)
+    xsrc = Hd.rotate_activation_f32(xd.astype(np.float32)).astype(np.float64) if had_x else xd
+    xc, xs = mx.quantize_e8m0_b32(xsrc)
     xq = mx.dequant_e8m0_b32(xc, xs)
     r = route(logits, k)
     g, u, h, tg, tu = gate_up(xq, r, Wgu, I, k)
     hsrc = h if h_given is None else h_given
+    if had_h:
+        h32 = hsrc.astype(np.float32)
+        assert h_given is None or np.array_equal(h32.astype(np.float64), hsrc), "h_given: float32 values"
+        hsrc = Hd.rotate_activation_f32(h32).astype(np.float64)
     hc, hs = mx.quantize_e8m0_b32(hsrc)
     hq = mx.dequant_e8m0_b32(hc, hs)
     out, tout = down_combine(hq, r, Wd, T, k)

@@ -42,6 +42,41 @@ def quantize_e8m0_b32(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     return codes, (e + 127).astype(np.uint8)
 
 
+def quantize_e8m0_b32_searched(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP4 with a local search of the E8M0 block scale (PRQuant §5.3, "PRQuant (E8M0-W)": a
+    weight-side local block-scale search).  Reading: per 32-block the candidates are the OCP
+    exponent e0 = floor(log2 amax) - 2 and its neighbours e0 + 1 and e0 - 1 (clamped to
+    [-127, 127]); each is applied with the same element rule (RNE to E2M1, saturating at 6) and
+    the block keeps the one with the smallest sum of squared errors (float64, summed over the 32
+    elements in order), trying e0, then e0 + 1, then e0 - 1, a later one only if strictly
+    better.  Same outputs as quantize_e8m0_b32."""
+    x = np.asarray(x, dtype=np.float64)
+    R, K = x.shape
+    assert K % 32 == 0
+    blocks = x.reshape(R, K // 32, 32)
+    e0 = mx_shared_exponent(np.abs(blocks).max(axis=-1))
+    best_e = e0.copy()
+    best_codes = F.e2m1_encode(blocks * np.ldexp(1.0, -e0)[..., None])
+    best_err = _block_sq_err(blocks, best_codes, e0)
+    for de in (1, -1):
+        e = np.clip(e0 + de, -127, 127)
+        codes = F.e2m1_encode(blocks * np.ldexp(1.0, -e)[..., None])
+        err = _block_sq_err(blocks, codes, e)
+        better = err < best_err
+        best_e = np.where(better, e, best_e)
+        best_codes = np.where(better[..., None], codes, best_codes)
+        best_err = np.where(better, err, best_err)
+    return best_codes.reshape(R, K).astype(np.uint8), (best_e + 127).astype(np.uint8)
+
+
+def _block_sq_err(blocks: np.ndarray, codes: np.ndarray, e: np.ndarray) -> np.ndarray:
+    d = blocks - F.e2m1_decode(codes) * np.ldexp(1.0, e)[..., None]
+    acc = np.zeros(blocks.shape[:-1])
+    for i in range(blocks.shape[-1]):                   # summed in element order
+        acc += d[..., i] * d[..., i]
+    return acc
+
+
 def dequant_e8m0_b32(codes: np.ndarray, sbytes: np.ndarray) -> np.ndarray:
     R, K = codes.shape
     v = F.e2m1_decode(codes).reshape(R, K // 32, 32)

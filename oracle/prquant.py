@@ -19,10 +19,14 @@ from . import gemm as G
 from . import mx
 
 
-def column_errors(w: np.ndarray) -> np.ndarray:
+def _qw(search: bool):
+    return mx.quantize_e8m0_b32_searched if search else mx.quantize_e8m0_b32
+
+
+def column_errors(w: np.ndarray, search: bool = False) -> np.ndarray:
     """Per input channel: sum over output rows of (w - deq Q(w))^2, float64, accumulated in row
     order n = 0, 1, ... (a fixed order, so the top-k choice is reproducible to the last bit)."""
-    codes, sb = mx.quantize_e8m0_b32(w)
+    codes, sb = _qw(search)(w)
     d = w - mx.dequant_e8m0_b32(codes, sb)
     acc = np.zeros(w.shape[1])
     for n in range(w.shape[0]):
@@ -44,20 +48,22 @@ def permutation(C: int, tail: np.ndarray) -> np.ndarray:
     return np.concatenate([np.nonzero(~mask)[0], np.asarray(tail, dtype=np.int64)])
 
 
-def prepare(w: np.ndarray, k: int) -> dict:
-    """Offline preparation.  w float64 [N, C] (bf16 values), k % 32 == 0.
+def prepare(w: np.ndarray, k: int, search: bool = False) -> dict:
+    """Offline preparation.  w float64 [N, C] (bf16 values), k % 32 == 0.  search = True quantizes
+    every weight block with the E8M0-W block-scale search (§5.3) instead of the OCP rule.
 
     Returns perm [C], the augmented weight codes [N, C+k] (nibbles) and E8M0 bytes
     [N, (C+k)/32], and the residual R_W [N, k] for inspection.
     """
     N, C = w.shape
     assert C % 32 == 0 and k % 32 == 0 and 0 < k <= C
-    tail = select_tail(column_errors(w), k)
+    q = _qw(search)
+    tail = select_tail(column_errors(w, search), k)
     perm = permutation(C, tail)
     wp = w[:, perm]
-    q_codes, q_sb = mx.quantize_e8m0_b32(wp)
+    q_codes, q_sb = q(wp)
     r = wp[:, C - k:] - mx.dequant_e8m0_b32(q_codes[:, C - k:], q_sb[:, (C - k) // 32:])
-    r_codes, r_sb = mx.quantize_e8m0_b32(r)
+    r_codes, r_sb = q(r)
     return dict(perm=perm, tail=tail,
                 w_codes=np.concatenate([q_codes, r_codes], axis=1),
                 w_sb=np.concatenate([q_sb, r_sb], axis=1),

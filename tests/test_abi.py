@@ -48,13 +48,14 @@ def test_bad_arguments_rejected_without_device():
     assert ql.lib.quantize_act(1, None, 0, 32, None, None, None, None) == 0        # empty is a no-op
 
 
-@pytest.mark.parametrize("N,C,k", [(32, 512, 128), (64, 1024, 256)])
-def test_prquant_host_preparation_matches_oracle(N, C, k):
+@pytest.mark.parametrize("N,C,k,search", [(32, 512, 128, False), (64, 1024, 256, False),
+                                          (32, 512, 128, True), (64, 1024, 256, True)])
+def test_prquant_host_preparation_matches_oracle(N, C, k, search):
     import bit_quantized_moe_tcgen05_b200 as ql
     from oracle import formats as F, prquant
     wb = synth.to_bf16_bits(synth.student_t(11 + N, (N, C), 3.0))
-    perm, codes, scales = ql.prepare_prquant(wb, k)
-    ref = prquant.prepare(synth.bf16_bits_to_f64(wb), k)
+    perm, codes, scales = ql.prepare_prquant(wb, k, scale_search=search)
+    ref = prquant.prepare(synth.bf16_bits_to_f64(wb), k, search=search)
     assert np.array_equal(perm, ref["perm"])
     assert np.array_equal(codes, F.pack_nibbles(ref["w_codes"]))
     assert np.array_equal(scales, ref["w_sb"])

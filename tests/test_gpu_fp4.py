@@ -130,11 +130,13 @@ def test_fp4_gemm_bruteforce_tiny():
     check_fp32(y32, G.naive_gemm(xq, wq), G.abs_scale(xq, wq), "tiny")
 
 
-@pytest.mark.parametrize("N,C,k,M", [(256, 512, 128, 8), (256, 640, 256, 100), (128, 384, 128, 300),
-                                     (384, 1024, 384, 1)])
-def test_prquant_tail_gemm_small(N, C, k, M):
+@pytest.mark.parametrize("N,C,k,M,search", [(256, 512, 128, 8, False), (256, 640, 256, 100, False),
+                                            (128, 384, 128, 300, False), (384, 1024, 384, 1, False),
+                                            (256, 1024, 256, 16, True), (256, 1024, 128, 300, True)])
+def test_prquant_tail_gemm_small(N, C, k, M, search):
+    """PRQuant augmented GEMM, with the OCP block scales or the E8M0-W block-scale search (§5.3)."""
     w = synth.bf16_bits_to_f64(synth.to_bf16_bits(synth.student_t(21 + C, (N, C), 3.0)))
-    prep = prquant.prepare(w, k)
+    prep = prquant.prepare(w, k, search=search)
     xb, _ = synth.activations_bf16(21, M, C, 0.005 * 8, 50.0)
     xpb = np.ascontiguousarray(xb[:, prep["perm"]])
     check_linear(F.pack_nibbles(prep["w_codes"]), prep["w_sb"], k, xpb, f"tail N={N} C={C} k={k} M={M}")

@@ -62,11 +62,12 @@ def run_case(seed, E, H, I, T, k, logits=None):
     return got, xb, logits, Wgu, Wd
 
 
-def check_all(got, xb, logits, Wgu, Wd, k):
+def check_all(got, xb, logits, Wgu, Wd, k, had_x=False, had_h=False):
     T, H = got["y"].shape
     I = Wd[0].shape[1]
     xd = F.bf16_decode(xb)
-    ref = moe.forward(xd, logits, Wgu, Wd, k, h_given=got["h32"].astype(np.float64))
+    ref = moe.forward(xd, logits, Wgu, Wd, k, h_given=got["h32"].astype(np.float64), had_x=had_x,
+                      had_h=had_h)
     r = ref["route"]
     # routing: exact
     assert np.array_equal(got["ids"], r["ids"])

@@ -1,8 +1,9 @@
 """The device-timeout path, made to happen without any fault: a test hook withholds one CTA's
-grid-wide publications (the E4M3-B16 amax slot, the decode flags) and lowers the wait limit to
-2 ms, so that the bounded waits on them run out.  The kernels record QL_ERR_TIMEOUT and return;
-ql_check reports it; after the hook is lifted the same workspace gives the same bits as a fresh
-one (the launch counters moved past every tag the failed launch left behind)."""
+publications to other CTAs (the E4M3-B16 amax slot, the decode flags, its arrivals on cluster
+peers' barriers) and lowers the wait limit to 2 ms, so that the bounded waits on them run out.
+The kernels record QL_ERR_TIMEOUT and return; ql_check reports it; after the hook is lifted the
+same workspace gives the same bits as a fresh one (the launch counters moved past every tag the
+failed launch left behind)."""
 import numpy as np
 import pytest
 import torch
@@ -42,21 +43,29 @@ def _expect_timeout(fn):
     ql.check()                                     # the error word was cleared
 
 
-def test_decode_forward_timeout_then_recovers():
-    """One-launch decode forward (E4M3-B16 activations quantized inside the GEMM): CTA 1's amax
-    slot and flags are withheld, every other CTA's wait runs out."""
+@pytest.mark.parametrize("mode", [1, 2, 3])
+def test_decode_forward_timeout_then_recovers(mode):
+    """One-launch decode forward (E4M3-B16 activations quantized inside the GEMM), in each of the
+    decode kernel's organisations: CTA 1 withholds what it publishes to the others (mode 1: its
+    amax slot and its quantized and split-K flags in the workspace; mode 2: its slot and split-K
+    flag; mode 3: its arrivals on its cluster peers' split-K barriers), and the waits on them run
+    out."""
     ql = _ql()
     lin = _nvfp4_layer(512, 2048, 61)
     M = 8
     x = _x(M, 2048, 62)
-    ws = torch.empty(lin.workspace_bytes(M), dtype=torch.uint8, device="cuda")
-    y = torch.empty((M, 512), dtype=torch.bfloat16, device="cuda")
-    _expect_timeout(lambda: lin.forward(x, out=y, ws=ws))
-    for _ in range(2):                             # the same workspace, twice, after the failure
-        got = lin.forward(x, ws=ws).clone()
-        fresh = lin.forward(x, ws=torch.zeros_like(ws)).clone()
-        ql.check()
-        assert torch.equal(got, fresh)
+    try:
+        ql.decode_fuse_mode(mode)
+        ws = torch.empty(lin.workspace_bytes(M), dtype=torch.uint8, device="cuda")
+        y = torch.empty((M, 512), dtype=torch.bfloat16, device="cuda")
+        _expect_timeout(lambda: lin.forward(x, out=y, ws=ws))
+        for _ in range(2):                         # the same workspace, twice, after the failure
+            got = lin.forward(x, ws=ws).clone()
+            fresh = lin.forward(x, ws=torch.zeros_like(ws)).clone()
+            ql.check()
+            assert torch.equal(got, fresh)
+    finally:
+        ql.decode_fuse_mode(-1)
     lin.close()
 
 
