@@ -13,7 +13,8 @@
 //   moe_scatter_kernel     one CTA per expert: offsets and the expert's routed entries
 //                          (f = t*k + s) in ascending (t, s) order -- deterministic
 //   quant_mx_e8m0_b32_kernel (quant_act.cuh) with a bf16 dequantized copy of x
-//   moe_gemm_kernel<GATEUP> gate/up: B rows gathered per entry by cp.async; epilogue
+//   moe_gather_kernel      the bf16 row of x for every routed entry, in expert-sorted order
+//   moe_gemm_kernel<GATEUP> gate/up: B = the expert's contiguous gathered rows; epilogue
 //                          h = silu(g) * u, MXFP4 requantization of h per 32 features, and the
 //                          exact bf16 value of the quantized h for the down projection
 //   moe_gemm_kernel<DOWN>  down: B = the expert's contiguous h rows; epilogue writes
@@ -132,6 +133,22 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restric
   if (out32 != nullptr) *reinterpret_cast<float4*>(out32 + t * H + n) = acc;
 }
 
+// xs[p, :] = x_dq[entries[p] / k, :] for every routed entry p (expert-sorted order), so that each
+// expert's activation rows are contiguous and the gate/up GEMM reads them as plain TMA tiles.
+// One thread per 16 bytes.
+__global__ void __launch_bounds__(256) moe_gather_kernel(const __nv_bfloat16* __restrict__ x_dq,
+                                                         const int* __restrict__ entries, int P,
+                                                         int H, int k,
+                                                         __nv_bfloat16* __restrict__ xs) {
+  const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int per_row = H / 8;
+  if (i >= static_cast<long>(P) * per_row) return;
+  const int p = static_cast<int>(i / per_row), c = static_cast<int>(i - static_cast<long>(p) * per_row);
+  const int t = __ldg(entries + p) / k;
+  reinterpret_cast<uint4*>(xs + static_cast<size_t>(p) * H)[c] =
+      __ldg(reinterpret_cast<const uint4*>(x_dq + static_cast<size_t>(t) * H) + c);
+}
+
 // ------------------------------------------------------------------------------ grouped GEMM
 struct MoeGemmArgs {
   int E, k;
@@ -142,7 +159,7 @@ struct MoeGemmArgs {
   const int* offsets;             // [E+1]
   const int* entries;             // [T*k] routed entries, expert-sorted
   const __nv_bfloat16* cent;      // [E*rows_per_expert][16] centroids (kernel row order)
-  const __nv_bfloat16* x_dq;      // [T, H] exact bf16 of the quantized x (gate/up B rows)
+
   const float* gates;             // [T*k] gate weights by entry (down)
   int I;                          // intermediate width
   uint8_t* h_codes;               // [T*k, I/2] MXFP4 codes of h, sorted order (gate/up)
@@ -153,12 +170,6 @@ struct MoeGemmArgs {
   int had;                        // gate/up: online Hadamard (block 32) of h before requantizing
   int H;
 };
-
-// Stages of token-row gathers the gate/up producer keeps in flight before signalling one.  A
-// stage's slot can only be refilled after it was signalled and consumed, so the consumers can
-// run at most kStages - kGatherLag stages ahead of the gathers: the lag trades latency hiding
-// for consumer slack.
-constexpr int kGatherLag = 2;
 
 template <int BN>
 struct MoeCfg {
@@ -175,15 +186,14 @@ struct MoeCfg {
   static constexpr int kDecWarps = 8;
   static constexpr int kThreads = (2 + kDecWarps + 4) * 32;
   static constexpr int kSmemBytes =
-      kStages * kStageBytes + 2 * kCentBytes + kStgBytes + 2 * BN * 4 + 1024 + 512;
+      kStages * kStageBytes + 2 * kCentBytes + kStgBytes + 1024 + 512;
   static_assert(kSmemBytes + 4200 <= 227 * 1024, "dynamic + static shared memory per block");
-  static_assert(kGatherLag < kStages, "gathers must be signalled before their slot comes round");
 };
 
 // Persistent grouped GEMM.  Work items (expert e, 128-row weight tile nt, BN-token tile mt) are
 // enumerated expert by expert, nt fastest; CTA c takes items c, c + gridDim.x, ...  Warp roles:
-// 0 producer (TMA: index tile, B rows -- gathered token rows for gate/up, contiguous h rows for
-// down -- and the item's 128 centroid rows), 1 TMEM allocator + MMA issuer (kind::f16, N = the
+// 0 producer (TMA: index tile, B rows -- the expert's contiguous gathered x rows for gate/up, its
+// h rows for down -- and the item's 128 centroid rows), 1 TMEM allocator + MMA issuer (kind::f16, N = the
 // item's token count rounded up to 16), 2..9 decode (4-bit indices -> bf16 operand tile),
 // 10..13 epilogue.  Two TMEM accumulators alternate between items, so the epilogue of one item
 // overlaps the main loop of the next.  GATEUP: the weight rows of a tile are 64 gate rows then
@@ -203,8 +213,7 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
   uint8_t* sIdx = sB + S * Cfg::kBBytes;
   __nv_bfloat16* sCent = reinterpret_cast<__nv_bfloat16*>(sIdx + S * Cfg::kIdxBytes);    // [2][128][16]
   float* sStg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sCent) + 2 * Cfg::kCentBytes);
-  int* sRow = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(sStg) + Cfg::kStgBytes);  // [2][BN]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sRow + 2 * BN);   // B rows (and indices) landed
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sStg) + Cfg::kStgBytes);   // B rows landed
   uint64_t* ifull = full + S;                                       // index tile landed
   uint64_t* empty = ifull + S;
   uint64_t* decd = empty + S;
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], GATEUP ? 32 : 1);   // gate/up: one arrival per producer lane
+      mbar_init(&full[s], 1);
       mbar_init(&ifull[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&decd[s], Cfg::kDecWarps * 32);
@@ -281,19 +290,8 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       const Item I = item_of(id);
       const int b = j & 1;
       const int row0 = I.e * a.rows_per_expert + I.nt * 128;
-      const int nrow = min(BN, (I.cnt + 15) & ~15);
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&cempty[b], ((j >> 1) & 1) ^ 1, 11));
       if (!ok) break;
-      int* rows = sRow + b * BN;
-      int fv[BN / 32];
-#pragma unroll
-      for (int u = 0; u < BN / 32; ++u) {   // all loads in flight, then the stores
-        const int c = lane + 32 * u;
-        fv[u] = a.entries[I.p0 + (c < I.cnt ? c : 0)];
-      }
-#pragma unroll
-      for (int u = 0; u < BN / 32; ++u) rows[lane + 32 * u] = GATEUP ? fv[u] / a.k : fv[u];
-      __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(&cfull[b], Cfg::kCentBytes);
         bulk_load(sCent + b * 128 * 16, a.cent + static_cast<size_t>(row0) * 16, Cfg::kCentBytes, &cfull[b]);
@@ -306,36 +304,10 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(&ifull[st], Cfg::kIdxBytes);
           tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_idx, &ifull[st], i * 32, row0);
-          if constexpr (!GATEUP) {
-            mbar_arrive_expect_tx(&full[st], Cfg::kBBytes);
-            tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, I.p0);
-          }
-        }
-        if constexpr (GATEUP) {
-          // Gather the item's token rows (64 bf16 of each, in the 128-byte-swizzled K-major
-          // layout) with 16-byte cp.async from all lanes; a stage is signalled kGatherLag stages
-          // later, once its copies have landed, so that several stages are in flight.
-          const uint32_t bdst = smem_u32(sB + st * Cfg::kBBytes);
-          for (int c = lane; c < nrow * 8; c += 32) {
-            const int r = c >> 3, kc = c & 7;
-            cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4),
-                       a.x_dq + static_cast<size_t>(rows[r]) * a.kdim + i * 64 + kc * 8, 16u);
-          }
-          cp_async_commit();
-          if (it >= kGatherLag) {
-            cp_async_wait_pending(kGatherLag);
-            fence_proxy_async_smem();
-            mbar_arrive(&full[(it - kGatherLag) % S]);
-          }
+          mbar_arrive_expect_tx(&full[st], Cfg::kBBytes);
+          tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, I.p0);
         }
         __syncwarp();
-      }
-    }
-    if constexpr (GATEUP) {   // signal the stages still in flight
-      for (int k = max(0, it - kGatherLag); k < it; ++k) {
-        cp_async_wait_pending(it - 1 - k);
-        fence_proxy_async_smem();
-        mbar_arrive(&full[k % S]);
       }
     }
   } else if (warp == 1) {

@@ -376,6 +376,7 @@ int dec_max_clusters(const ql_linear* L, int BN, int S) {
 std::atomic<int> g_decode_fuse_mode{-1};
 constexpr int kDecLocalUnits = 8;                // local mode: units per quantizer thread at most
 constexpr int64_t kDecLocalAmaxElems = 128 * 1024;   // x elements every CTA may read for the amax
+constexpr int64_t kDecClusterAmaxElems = 16 * 1024;  // ... when a cluster exchange is the other way
 
 // Decode launches (M <= 64): the weight tiles split along K so that the grid covers the SMs once;
 // each CTA keeps all its stages resident.  Returns false when no such split exists.
@@ -423,7 +424,7 @@ bool plan_decode(const ql_linear* L, int64_t M, FwdPlan& p) {
   else p.fuse_mode = local_ok(p.spp) ? 2 : (coop_ok ? 1 : 0);
   p.fusable = p.fuse_mode != 0;
   // E4M3: every CTA reads all of x for the tensor amax while x is small, else the grid gathers it
-  p.amax_coop = !L->e8m0 && M * L->C > kDecLocalAmaxElems;
+  p.amax_coop = !L->e8m0 && M * L->C > (p.cluster ? kDecClusterAmaxElems : kDecLocalAmaxElems);
   p.full_tiles = 0;
   p.decode = true;
   return true;
@@ -1283,8 +1284,8 @@ namespace {
 constexpr int kMoeBN = 128;
 
 struct MoePlan {
-  size_t counts, offsets, entries, ids, gates, x_codes, x_scales, x_dq, h_codes, h_scales, h_dq,
-      h32, yslot, total;
+  size_t counts, offsets, entries, ids, gates, x_codes, x_scales, x_dq, xs, h_codes, h_scales,
+      h_dq, h32, yslot, total;
 };
 
 MoePlan plan_moe(const ql_moe* m, int64_t T) {
@@ -1304,6 +1305,7 @@ MoePlan plan_moe(const ql_moe* m, int64_t T) {
   p.x_codes = take(static_cast<size_t>(T) * m->H / 2);
   p.x_scales = take(static_cast<size_t>(T) * m->H / 32);
   p.x_dq = take(static_cast<size_t>(T) * m->H * 2);
+  p.xs = take(P * m->H * 2);   // x rows per routed entry, expert-sorted
   p.h_codes = take(P * m->I / 2);
   p.h_scales = take(P * m->I / 32);
   p.h_dq = take(P * m->I * 2);
@@ -1459,14 +1461,21 @@ ql_status moe_grouped_forward(const ql_moe* m, const void* x, int64_t T, const f
   ql_status st = launch_quant_mx(x, T, m->H, w8 + p.x_codes, w8 + p.x_scales, nullptr, 0, nullptr,
                                  0, s, x_dq, 128, m->had_x);
   if (st != QL_OK) return st;
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(w8 + p.xs);
+  {
+    const long n16 = static_cast<long>(total) * (m->H / 8);
+    ql::moe_gather_kernel<<<static_cast<unsigned>((n16 + 255) / 256), 256, 0, s>>>(
+        x_dq, entries, total, m->H, m->k, xs);
+    QL_CUDA(cudaGetLastError());
+  }
   CUtensorMap tm_x, tm_h;
   __nv_bfloat16* h_dq = reinterpret_cast<__nv_bfloat16*>(w8 + p.h_dq);
-  st = make_tmap_bf16(&tm_x, x_dq, m->H, T, 1);
+  st = make_tmap_bf16(&tm_x, xs, m->H, total, kMoeBN);
   if (st == QL_OK) st = make_tmap_bf16(&tm_h, h_dq, m->I, total, kMoeBN);
   if (st != QL_OK) return st;
   ql::MoeGemmArgs a{};
   a.E = m->E; a.k = m->k; a.counts = counts; a.offsets = offsets; a.entries = entries;
-  a.gates = gates; a.I = m->I; a.H = m->H; a.x_dq = x_dq;
+  a.gates = gates; a.I = m->I; a.H = m->H;
   a.h_codes = w8 + p.h_codes; a.h_scales = w8 + p.h_scales; a.h_dq = h_dq;
   a.h32 = m->capture_h32 ? reinterpret_cast<float*>(w8 + p.h32) : nullptr;
   a.yslot = reinterpret_cast<float*>(w8 + p.yslot);

@@ -305,7 +305,9 @@ ql_status moe_workspace_bytes(const ql_moe* moe, int64_t T, size_t* bytes);
  * ascending f inside an expert), ids int[T,k], gates float[T,k], x_codes [T,H/2], x_scales
  * [T,H/32] (MXFP4 of x), x_dq bf16 [T,H] (its exact values), h_codes [T*k,I/2], h_scales
  * [T*k,I/32] (MXFP4 of h, rows in entry order), h_dq bf16 [T*k,I], h32 float [T*k,I] (only when
- * captured), yslot float [T*k,H] (gate-weighted expert outputs by entry f). */
+ * captured), yslot float [T*k,H] (gate-weighted expert outputs by entry f).  The workspace also
+ * holds buffers that are not listed (the bf16 x row of every routed entry, expert-sorted, that
+ * the gate/up GEMM reads as contiguous tiles). */
 typedef struct ql_moe_ws_layout {
   size_t counts, offsets, entries, ids, gates, x_codes, x_scales, x_dq, h_codes, h_scales, h_dq,
       h32, yslot, total;
