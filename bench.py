@@ -42,7 +42,7 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the timed GEMM
 # kernel, from an ncu --set full capture of that kernel (the VQ layer's M = 64 launch; the PRQuant
 # M = 2048 launch).  Set an entry to None whenever its kernel changes until it is captured again.
-NCU_TRAFFIC_PER_LAUNCH = {"vq": 11.33e6, "prquant_m2048": 24.58e6}
+NCU_TRAFFIC_PER_LAUNCH = {"vq": None, "prquant_m2048": None}   # to be re-captured for the current kernels
 
 
 def measured_peaks() -> dict:
@@ -306,6 +306,30 @@ def _elapsed(fn, reps: int, stream) -> float:
     return a.elapsed_time(b)
 
 
+def count_kernel_launches(fn) -> int | None:
+    """Kernel launches that fn issues: fn is captured into a CUDA graph and its kernel nodes
+    counted (None where the graph cannot be inspected)."""
+    import torch
+    try:
+        from cuda.bindings import runtime as cudart
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g):
+            fn()
+        err, _, n = cudart.cudaGraphGetNodes(g.raw_cuda_graph(), 0)
+        if err != cudart.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = cudart.cudaGraphGetNodes(g.raw_cuda_graph(), n)
+        kernels = 0
+        for nd in nodes:
+            e2, t = cudart.cudaGraphNodeGetType(nd)
+            if e2 == cudart.cudaError_t.cudaSuccess and t == cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kernels += 1
+        del g
+        return kernels
+    except Exception:
+        return None
+
+
 def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes: int = 0):
     """Device time per step (ms) of w's forwards (every M of w["Ms"] per step), replayed from a
     CUDA graph over R rotating weight copies with R * weight bytes > L2 (or with an explicit L2
@@ -370,6 +394,7 @@ def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes:
             for _ in range(warmup):
                 g.replay()
     ql.check()
+    kernels_per_step = count_kernel_launches(lambda: [fwd(layer, M) for M in Ms for layer in layers[:1]])
 
     def timed(graph, pgraph):
         if flush_buf is None:
@@ -387,7 +412,7 @@ def run_case(w, steps: int, warmup: int, device, e2e: bool = False, flush_bytes:
         return tot / steps
 
     out = dict(R=R, step_ms=timed(g_all, p_all), quant_ms=timed(g_q, p_q),
-               gemm_ms=timed(g_g, p_g), steps=steps)
+               gemm_ms=timed(g_g, p_g), steps=steps, kernels_per_step=kernels_per_step)
     ql.check()
     if e2e:
         xh = {M: torch.from_numpy(w["xs"][M].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -585,16 +610,18 @@ def main():
     fp4_peak = tp["fp4_mxf4_block32"]["burst"]
     int8_peak = tp["int8"]["burst"]
     nl = len(head["Ms"])
-    # the dominant kernel: for decode sizes the one-launch forward (the GEMM with the activation
-    # quantizer fused in), timed by the graph of forwards; else the GEMM alone
-    one_launch = decode
+    # the dominant kernel: the GEMM launch of each forward (it streams the weight), timed alone
+    # by the graph of GEMM calls on a quantized workspace: at M = 1 the decode kernel, above it
+    # (E4M3-B16 activations) the general split-K GEMM, as the forward's plan chooses
     if decode:
-        alg = sum(forward_bytes_of(head, M) for M in head["Ms"]) / nl
-        ach = alg / (res["step_ms"] / nl * 1e-3) / 1e9
+        alg = sum(gemm_bytes_of(head, M) for M in head["Ms"]) / nl
+        ach = alg / (res["gemm_ms"] / nl * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
                     "frac": ach / peaks["hbm"], "traffic": NCU_TRAFFIC_PER_LAUNCH.get(args.workload),
-                    "kernel": "fp4_decode_kernel (E4M3-B16 quantizer fused, VQ decode, block16 MMA)"
-                    if head["kind"] == "vq" else "fp4_decode_kernel (mxf4)",
+                    "kernel": ("GEMM launch per forward, averaged over M = " +
+                               ", ".join(map(str, head["Ms"])) +
+                               ": fp4_decode_kernel at M = 1, fp4_gemm_kernel (split-K) above; "
+                               "VQ decode in shared memory, block16 MMA"),
                     "algorithmic_bytes_per_launch": alg,
                     "peak_source": f"{peaks['src']} HBM copy bandwidth (MEASURED_PEAKS.json)"}
     else:
@@ -660,8 +687,7 @@ def main():
     if rank != 0:
         return
 
-    def kernels_per_fwd(M):   # library kernels one forward launches
-        return 1 if one_launch else 2
+    kps = res.get("kernels_per_step")   # counted in a captured graph of one step's forwards
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": res["steps"],
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -671,7 +697,7 @@ def main():
         "data": "synthetic", "config": config, "roofline": roofline,
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
-        "gpu_launches": sum(kernels_per_fwd(M) for M in head["Ms"]) * res["steps"],
+        "gpu_launches": kps * res["steps"] if kps is not None else None,
         "clocks": clk.summary(),
         "kernel_us_per_step": {"forward": res["step_ms"] * 1e3,
                                "split_api_quantize": res["quant_ms"] * 1e3,

@@ -19,7 +19,7 @@
 // tensor scale needs the amax of the whole tensor: each CTA publishes the amax of its units in a
 // slot, CTA 0 gathers the slots and publishes the maximum in one word, which the others poll.
 // With fuse = 0 the workspace already holds the quantized activations in the plain layout
-// (qlinear_quantize_input) and the producer warp copies each stage's B tile by cp.async.
+// (qlinear_quantize_input) and the producer warp copies each stage's B tile with one TMA tile.
 //
 // Issuing tcgen05 instructions costs the issuing thread tens of cycles each, so the MMA issuer
 // issues MMAs only: the scale factors reach TMEM through tcgen05.st from the warps that hold them
@@ -117,7 +117,8 @@ struct DecodeArgs {
                               // the kernel, cooperatively (per-stage tiles in the workspace);
                               // 2: inside the kernel, each CTA its own stages (small x)
   const __nv_bfloat16* x;     // fuse: bf16 activations [M, C]
-  uint8_t* xq;                // fuse = 0: quantized activation codes [M, C/2] (workspace)
+  uint8_t* xq;                // fuse = 0: quantized activation codes [M, C/2] (workspace; read
+                              // through the kernel's tensor map, box 128 B x BN rows)
   uint8_t* sfb;               // fuse = 0: activation scale atoms, 128-row group 0, [C / atomK]
   uint8_t* xt;                // fuse = 1: per K stage the B tile [BN][128 B], 128-byte swizzle
   uint8_t* st;                // fuse = 1: per K stage its activation scale atoms
@@ -227,7 +228,7 @@ __device__ __forceinline__ void dec_store4(const DecodeArgs& a, int m, int nn, f
 
 template <int BN, bool E8M0, bool VQ, int SF = 0>
 __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
-    fp4_decode_kernel(const DecodeArgs a) {
+    fp4_decode_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeArgs a) {
   using Cfg = DecCfg<BN, E8M0, VQ, SF>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
     if (lane == 0) {
       mbar_init(accf, 1);
       mbar_init(xready, 1);
-      mbar_init(bfull, a.fuse ? 1 : 32);
+      mbar_init(bfull, 1);
       mbar_init(sfb_ok, 4);
       mbar_init(scbar, 1);
       mbar_init(camax, a.splits);
@@ -348,27 +349,31 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
         }
       }
     } else if (a.fuse == 0) {
-      // plain layout (qlinear_quantize_input): each stage's B tile by 16-byte cp.async from all
-      // 32 lanes into the swizzled layout (rows past M zero-filled), then its scale atoms
-      for (int it = 0; it < n_it && ok; ++it) {
-        int kw, kx, valid;
-        stage_coords(s_begin + it, kw, kx, valid);
-        const int nat = valid / Cfg::kAtomK;
-        const uint32_t bdst = smem_u32(sB + it * Cfg::kBBytes);
-        for (int c = lane; c < BN * 8; c += 32) {
-          const int r = c >> 3, kc = c & 7;
-          const bool in = r < a.M && kc * 32 < valid;
-          const uint8_t* src = a.xq + static_cast<size_t>(in ? r : 0) * (a.C / 2) + (kx >> 1) + (in ? kc * 16 : 0);
-          cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4), src, in ? 16u : 0u);
+      // plain layout (qlinear_quantize_input): each stage's B tile by one TMA tile (128-byte
+      // swizzle; rows past M and columns past C read as zeros), then its scale atoms by one bulk
+      // copy, all on one barrier
+      if (lane == 0) {
+        uint32_t bytes = 0;
+        for (int it = 0; it < n_it; ++it) {
+          int kw, kx, valid;
+          stage_coords(s_begin + it, kw, kx, valid);
+          bytes += Cfg::kBBytes + (valid / Cfg::kAtomK) * 512;
         }
-        const uint8_t* sfsrc = a.sfb + static_cast<size_t>(kx / Cfg::kAtomK) * 512;
-        const uint32_t sfdst = smem_u32(sSfb + it * Cfg::kSfBytes);
-        for (int c = lane; c < nat * 32; c += 32) cp_async16(sfdst + c * 16, sfsrc + c * 16, 16u);
+        if (ok && n_it > 0) {
+          mbar_arrive_expect_tx(bfull, bytes);
+          for (int it = 0; it < n_it; ++it) {
+            int kw, kx, valid;
+            stage_coords(s_begin + it, kw, kx, valid);
+            tma_load_2d(sB + it * Cfg::kBBytes, &tm_x, bfull, kx >> 1, 0);
+            const int nat = valid / Cfg::kAtomK;
+            if (nat > 0)
+              bulk_load(sSfb + it * Cfg::kSfBytes, a.sfb + static_cast<size_t>(kx / Cfg::kAtomK) * 512,
+                        nat * 512, bfull);
+          }
+        } else {
+          mbar_arrive(bfull);
+        }
       }
-      cp_async_commit();
-      cp_async_wait_pending(0);
-      fence_proxy_async_smem();
-      mbar_arrive(bfull);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer: MMAs only (the scale factors are placed by other warps)
@@ -376,8 +381,9 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
     ok = __all_sync(0xFFFFFFFFu, mbar_wait(sfb_ok, 0, 52));
     for (int it = 0; it < n_it && ok; ++it) {
       const int slot = VQ ? it % R : 0;
-      bool w = mbar_wait(&sfa_ok[it], 0, 51);
-      if constexpr (VQ) w = w && mbar_wait(&decd[slot], (it / R) & 1, 53);
+      // VQ: the decoder warps that place the weight scales arrive on decd only after their
+      // tcgen05.st completed, so one wait covers both
+      const bool w = VQ ? mbar_wait(&decd[slot], (it / R) & 1, 53) : mbar_wait(&sfa_ok[it], 0, 51);
       ok = __all_sync(0xFFFFFFFFu, w);
       if (!ok) break;
       tc_fence_after();

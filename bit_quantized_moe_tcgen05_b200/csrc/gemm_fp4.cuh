@@ -14,7 +14,8 @@
 //
 // Warp roles (192 threads; 320 for VQ weights): warp 0 = TMA producer, warp 1 = TMEM allocator +
 // MMA issuer (one lane issues), warps 2..5 = epilogue; with VQ weights warps 2..9 first rebuild
-// each stage's operand tile from the codebooks.  A STAGES-deep ring of
+// each stage's operand tile from the codebooks.  Without VQ, where TMEM holds two accumulators,
+// warp 2 issues the MMAs of every other stage into the second one (the epilogue adds the two).  A STAGES-deep ring of
 // shared-memory stages, each 256 K-elements deep, is guarded by full/empty mbarriers; MMA
 // completion is signalled by tcgen05.commit.  Every wait is bounded (see ptx.cuh).
 //
@@ -106,7 +107,12 @@ struct Fp4Cfg {
   static constexpr int kStages = kStagesRaw > 12 ? 12 : (kStagesRaw < 2 ? 2 : kStagesRaw);
   static constexpr int kSfaCols = kAtoms * 4;          // TMEM columns per stage
   static constexpr int kSfbCols = kAtoms * 4 * kG;
-  static constexpr int kColsNeeded = BN + kStages * (kSfaCols + kSfbCols);
+  // Without VQ decoders, the first epilogue warp (idle during the main loop) issues the MMAs of
+  // every other stage into a second accumulator where TMEM holds two: issuing a block-scaled MMA
+  // and its scale copies costs the issuing thread more than the tensor core needs to run it.
+  static constexpr int kIssuers = (!VQ && 2 * BN + kStages * (kSfaCols + kSfbCols) <= 512) ? 2 : 1;
+  static constexpr int kColsNeeded = kIssuers * BN + kStages * (kSfaCols + kSfbCols);
+  static constexpr int kProducers = VQ ? 1 : 2;   // without VQ, warp 3 also produces
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                  : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
   static_assert(kColsNeeded <= 512, "TMEM budget");
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
       mbar_init(&afull[s], 32);
     }
     if (lane == 0) {
-      mbar_init(accf, 1);
+      mbar_init(accf, Cfg::kIssuers);
       mbar_init(rbar, 1);
       mbar_init(scbar, 1);
     }
@@ -236,69 +242,15 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t sfa_col0 = BN, sfb_col0 = BN + S * Cfg::kSfaCols;
+  const uint32_t sfa_col0 = Cfg::kIssuers * BN, sfb_col0 = Cfg::kIssuers * BN + S * Cfg::kSfaCols;
 
   bool ok = true;
-  if (warp == 0) {
-    // ---------------- producer: the whole warp runs the loop; one elected lane issues copies.
-    // Activation part (written by the quantizer grid): B codes and SFB, by the bulk-copy engine.
-    auto issue_act = [&](int it) {
-      const int i = s_begin + it, st = it % S;
-      int kw, kx, valid;
-      stage_coords(i, kw, kx, valid);
-      const int nat = valid / Cfg::kAtomK;
-      tma_load_2d(sB + st * Cfg::kBBytes, &tm_x, &full[st], kx >> 1, m0);
-#pragma unroll
-      for (int g = 0; g < Cfg::kG; ++g)
-        bulk_load(sSfb + st * Cfg::kSfbBytes + g * Cfg::kAtoms * 512,
-                  a.sfb + (static_cast<size_t>(sf_group0 + g) * a.sfb_atoms + kx / Cfg::kAtomK) * 512,
-                  nat * 512, &full[st]);
-    };
-    griddep_wait();
-    if (lsu_act) {
-      // Every stage's activation tile (BN rows x 128 B, stored with the 128-byte swizzle) and its
-      // scale atoms, 16 bytes per cp.async from all 32 lanes; rows past M are zero-filled.
-      for (int it = 0; it < n_it; ++it) {
-        int kw, kx, valid;
-        stage_coords(s_begin + it, kw, kx, valid);
-        const int nat = valid / Cfg::kAtomK;
-        const uint32_t bdst = smem_u32(sB + it * Cfg::kBBytes);
-        for (int c = lane; c < BN * 8; c += 32) {
-          const int r = c >> 3, kc = c & 7;
-          const bool in = m0 + r < a.M;
-          const uint8_t* src = a.xq + static_cast<size_t>(in ? m0 + r : 0) * (a.C / 2) + (kx >> 1) + kc * 16;
-          cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4), src, in ? 16u : 0u);
-        }
-        const uint8_t* sfsrc = a.sfb + (static_cast<size_t>(sf_group0) * a.sfb_atoms + kx / Cfg::kAtomK) * 512;
-        const uint32_t sfdst = smem_u32(sSfb + it * Cfg::kSfbBytes);
-        for (int c = lane; c < nat * 32; c += 32) cp_async16(sfdst + c * 16, sfsrc + c * 16, 16u);
-        cp_async_commit();
-      }
-      for (int it = 0; it < n_it; ++it) {   // stage it complete -> visible to the tensor core
-        cp_async_wait_pending(n_it - 1 - it);
-        fence_proxy_async_smem();
-        mbar_arrive(&afull[it]);
-      }
-    } else {
-      if (elect_one())
-        for (int it = 0; it < pre; ++it) issue_act(it);
-      __syncwarp();
-      for (int it = pre; it < n_it && ok; ++it) {
-        const int st = it % S;
-        const uint32_t ph = (it / S) & 1;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 1));
-        if (!ok) break;
-        if (elect_one()) {
-          issue_weight(it);
-          issue_act(it);
-        }
-        __syncwarp();
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer: converged warp, one lane issues the tcgen05 instructions
+  // ---------------- MMA issuer j (converged warp, one lane issues the tcgen05 instructions):
+  // stages j, j + kIssuers, ... into accumulator j
+  auto mma_issue = [&](int j) {
     const uint32_t idesc0 = idesc_fp4_block(BN, E8M0);
-    for (int it = 0; it < n_it && ok; ++it) {
+    const uint32_t dacc = tmem + j * BN;
+    for (int it = j; it < n_it && ok; it += Cfg::kIssuers) {
       const int i = s_begin + it, st = it % S;
       const uint32_t ph = (it / S) & 1;
       bool w = true;
@@ -340,11 +292,11 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
             const uint32_t idd = idesc0 | (byte << 29) | (byte << 4);
             const uint32_t sa = (ta + at * 4) | (byte << 30);
             const uint32_t sb = (tb + at * 4 * Cfg::kG) | (byte << 30);
-            const uint32_t acc = (it == 0 && kk == 0) ? 0u : 1u;
+            const uint32_t acc = (it == j && kk == 0) ? 0u : 1u;
             if (E8M0)
-              mma_mxf4_block32(tmem, ad, bd, idd, sa, sb, acc);
+              mma_mxf4_block32(dacc, ad, bd, idd, sa, sb, acc);
             else
-              mma_nvf4_block16(tmem, ad, bd, idd, sa, sb, acc);
+              mma_nvf4_block16(dacc, ad, bd, idd, sa, sb, acc);
           }
         }
         tc_commit(&empty[st]);
@@ -353,6 +305,72 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
     }
     if (lane == 0) tc_commit(accf);
     __syncwarp();
+  };
+  // ---------------- producer: the whole warp runs the loop; one elected lane issues copies.
+  // Activation part (written by the quantizer grid): B codes and SFB, by the bulk-copy engine.
+  auto issue_act = [&](int it) {
+    const int i = s_begin + it, st = it % S;
+    int kw, kx, valid;
+    stage_coords(i, kw, kx, valid);
+    const int nat = valid / Cfg::kAtomK;
+    tma_load_2d(sB + st * Cfg::kBBytes, &tm_x, &full[st], kx >> 1, m0);
+#pragma unroll
+    for (int g = 0; g < Cfg::kG; ++g)
+      bulk_load(sSfb + st * Cfg::kSfbBytes + g * Cfg::kAtoms * 512,
+                a.sfb + (static_cast<size_t>(sf_group0 + g) * a.sfb_atoms + kx / Cfg::kAtomK) * 512,
+                nat * 512, &full[st]);
+  };
+  // Steady state of the ring from stage `pre` on: producer j takes the stages of parity j (two
+  // producers without VQ: a stage's empty-slot wait and its copies cost the issuing thread
+  // about as long as the tensor core needs for the stage).
+  auto produce = [&](int j) {
+    for (int it = pre; it < n_it && ok; ++it) {
+      if (Cfg::kProducers == 2 && (it & 1) != j) continue;
+      const int st = it % S;
+      const uint32_t ph = (it / S) & 1;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 1));
+      if (!ok) break;
+      if (elect_one()) {
+        issue_weight(it);
+        issue_act(it);
+      }
+      __syncwarp();
+    }
+  };
+  if (warp == 0) {
+    griddep_wait();
+    if (lsu_act) {
+      // Every stage's activation tile (BN rows x 128 B, stored with the 128-byte swizzle) and its
+      // scale atoms, 16 bytes per cp.async from all 32 lanes; rows past M are zero-filled.
+      for (int it = 0; it < n_it; ++it) {
+        int kw, kx, valid;
+        stage_coords(s_begin + it, kw, kx, valid);
+        const int nat = valid / Cfg::kAtomK;
+        const uint32_t bdst = smem_u32(sB + it * Cfg::kBBytes);
+        for (int c = lane; c < BN * 8; c += 32) {
+          const int r = c >> 3, kc = c & 7;
+          const bool in = m0 + r < a.M;
+          const uint8_t* src = a.xq + static_cast<size_t>(in ? m0 + r : 0) * (a.C / 2) + (kx >> 1) + kc * 16;
+          cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4), src, in ? 16u : 0u);
+        }
+        const uint8_t* sfsrc = a.sfb + (static_cast<size_t>(sf_group0) * a.sfb_atoms + kx / Cfg::kAtomK) * 512;
+        const uint32_t sfdst = smem_u32(sSfb + it * Cfg::kSfbBytes);
+        for (int c = lane; c < nat * 32; c += 32) cp_async16(sfdst + c * 16, sfsrc + c * 16, 16u);
+        cp_async_commit();
+      }
+      for (int it = 0; it < n_it; ++it) {   // stage it complete -> visible to the tensor core
+        cp_async_wait_pending(n_it - 1 - it);
+        fence_proxy_async_smem();
+        mbar_arrive(&afull[it]);
+      }
+    } else {
+      if (elect_one())
+        for (int it = 0; it < pre; ++it) issue_act(it);
+      __syncwarp();
+      produce(0);
+    }
+  } else if (warp == 1) {
+    mma_issue(0);
   } else {
     if constexpr (VQ) {
       // ---------------- VQ decode (warps 2..9): for each stage rebuild the 128 x 256 E2M1 operand
@@ -409,6 +427,11 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
         if (lane == 0) mbar_arrive(&decd[st]);
       }
     }
+    if (Cfg::kIssuers == 2 && warp == 2) mma_issue(1);
+    if (Cfg::kProducers == 2 && warp == 3 && !lsu_act) {
+      griddep_wait();   // the activations of this grid's quantizer
+      produce(1);
+    }
     if (warp < 6) {   // (extra VQ decoders, warps 6..9, take no part in the epilogue)
       // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
       const int q = warp & 3;
@@ -416,6 +439,20 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
       const int n = n0 + nl;
       const int mcount = min(BN, a.M - m0);
       const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      // 8 accumulator columns from c: the second issuer's accumulator added when it ran a stage
+      const bool two = Cfg::kIssuers == 2 && n_it > 1;
+      auto ld_acc = [&](int c, uint32_t (&r)[8]) {
+        tmem_ld8(trow + c, r);
+        if (two) {
+          uint32_t r2[8];
+          tmem_ld8(trow + BN + c, r2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) r[jj] = __float_as_uint(__uint_as_float(r[jj]) + __uint_as_float(r2[jj]));
+        } else {
+          tmem_ld_wait();
+        }
+      };
       griddep_wait();   // alpha_dev, the workspace and y belong to / follow earlier grids
       float alpha = a.alpha;
       if (a.alpha_dev != nullptr) alpha *= *a.alpha_dev;
@@ -430,8 +467,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < BN; c += 8) {
           uint32_t r[8];
-          tmem_ld8(trow + c, r);
-          tmem_ld_wait();
+          ld_acc(c, r);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             ybuf[(c + j) * 128 + nl] = __float2bfloat16_rn((n_it > 0 ? __uint_as_float(r[j]) : 0.f) * alpha);
@@ -448,8 +484,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < BN; c += 8) {
             uint32_t r[8];
-            tmem_ld8(trow + c, r);
-            tmem_ld_wait();
+            ld_acc(c, r);
 #pragma unroll
             for (int j = 0; j < 8; ++j) y32buf[(c + j) * 128 + nl] = (n_it > 0 ? __uint_as_float(r[j]) : 0.f) * alpha;
           }
@@ -470,8 +505,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < mcount; c += 8) {
           uint32_t r[8];
-          tmem_ld8(trow + c, r);
-          tmem_ld_wait();
+          ld_acc(c, r);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             if (c + j < mcount) mine[(c + j) * 128 + nl] = n_it > 0 ? __uint_as_float(r[j]) : 0.f;

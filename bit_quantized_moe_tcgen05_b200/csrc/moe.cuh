@@ -34,9 +34,12 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__
                                                        int E, int k, int* __restrict__ ids,
                                                        float* __restrict__ gates,
                                                        int* __restrict__ counts) {
+  __shared__ int s_hist[256];   // this CTA's routed count per expert (one global add per expert)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
+  if (warp < T) {
   float v[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -70,43 +73,82 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__
     for (int s = 0; s < k; ++s) {
       ids[static_cast<size_t>(warp) * k + s] = sid[s];
       gates[static_cast<size_t>(warp) * k + s] = ex[s] / sum;
-      atomicAdd(&counts[sid[s]], 1);
+      atomicAdd(&s_hist[sid[s]], 1);
     }
   }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (s_hist[e] != 0) atomicAdd(&counts[e], s_hist[e]);
 }
 
-// One CTA (256 threads) per expert e: offsets[e] = sum of counts[<e]; the entries f with
+// One CTA (1024 threads) per expert e: offsets[e] = sum of counts[<e]; the entries f with
 // ids[f] == e are written, ascending, to entries[offsets[e] ...].  CTA 0 also writes offsets[E].
-__global__ void __launch_bounds__(256) moe_scatter_kernel(const int* __restrict__ ids, int total,
-                                                          int E, const int* __restrict__ counts,
-                                                          int* __restrict__ offsets,
-                                                          int* __restrict__ entries) {
+// Each thread tests 16 consecutive entries per pass (a bit mask), a block-wide exclusive scan of
+// the hit counts gives every hit its place.
+constexpr int kScatterThreads = 1024;
+__global__ void __launch_bounds__(kScatterThreads) moe_scatter_kernel(
+    const int* __restrict__ ids, int total, int E, const int* __restrict__ counts,
+    int* __restrict__ offsets, int* __restrict__ entries) {
   const int e = blockIdx.x;
-  __shared__ int s_base, s_warp[8];
-  if (threadIdx.x == 0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_base, s_pass, s_warp[32];
+  if (warp == 0) {
     int b = 0;
-    for (int i = 0; i < e; ++i) b += counts[i];
-    s_base = b;
-    offsets[e] = b;
-    if (e == 0) offsets[E] = total;
+    for (int i = lane; i < e; i += 32) b += counts[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
+    if (lane == 0) {
+      s_base = b;
+      offsets[e] = b;
+      if (e == 0) offsets[E] = total;
+    }
   }
   __syncthreads();
   int pos = s_base;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int f0 = 0; f0 < total; f0 += blockDim.x) {
-    const int f = f0 + threadIdx.x;
-    const bool hit = f < total && ids[f] == e;
-    const unsigned m = __ballot_sync(0xFFFFFFFFu, hit);
-    if (lane == 0) s_warp[warp] = __popc(m);
-    __syncthreads();
-    int before = 0, all = 0;
-    for (int w = 0; w < 8; ++w) {
-      if (w < warp) before += s_warp[w];
-      all += s_warp[w];
+  for (int c0 = 0; c0 < total; c0 += kScatterThreads * 16) {
+    const int f0 = c0 + threadIdx.x * 16;
+    uint32_t mask = 0;
+    if (f0 + 16 <= total && (total & 3) == 0) {
+      const int4* src = reinterpret_cast<const int4*>(ids + f0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int4 v = __ldg(src + q);
+        mask |= (v.x == e ? 1u : 0u) << (4 * q) | (v.y == e ? 1u : 0u) << (4 * q + 1) |
+                (v.z == e ? 1u : 0u) << (4 * q + 2) | (v.w == e ? 1u : 0u) << (4 * q + 3);
+      }
+    } else {
+      for (int j = 0; j < 16; ++j)
+        if (f0 + j < total && __ldg(ids + f0 + j) == e) mask |= 1u << j;
     }
-    if (hit) entries[pos + before + __popc(m & ((1u << lane) - 1u))] = f;
-    pos += all;
+    const int cnt = __popc(mask);
+    int incl = cnt;   // inclusive scan over the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) s_warp[warp] = incl;
     __syncthreads();
+    if (warp == 0) {
+      int w = s_warp[lane], wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+        if (lane >= o) wi += u;
+      }
+      s_warp[lane] = wi - w;   // exclusive prefix of the warps
+      if (lane == 31) s_pass = wi;   // hits of this pass
+    }
+    __syncthreads();
+    int at = pos + s_warp[warp] + incl - cnt;
+    while (mask != 0) {
+      const int j = __ffs(mask) - 1;
+      entries[at++] = f0 + j;
+      mask &= mask - 1;
+    }
+    pos += s_pass;
+    __syncthreads();   // s_warp and s_pass are rewritten by the next pass
   }
 }
 
@@ -177,9 +219,9 @@ struct MoeCfg {
   static constexpr int kBBytes = BN * 128;        // BN rows x 64 bf16
   static constexpr int kIdxBytes = 128 * 32;      // 128 rows x 64 4-bit indices
   static constexpr int kStageBytes = kABytes + kBBytes + kIdxBytes;
-  static constexpr int kStages = 5;
+  static constexpr int kStages = BN > 128 ? 3 : 5;
   static constexpr int kCentBytes = 128 * 16 * 2;
-  static constexpr int kHalf = BN / 2;            // tokens per epilogue pass
+  static constexpr int kHalf = 64;                // tokens per epilogue pass
   static constexpr int kStgLd = 129;              // padded row of the transposed staging tile
   static constexpr int kStgBytes = kHalf * kStgLd * 4;
   static constexpr int kTmemCols = 2 * BN;        // two accumulators (ping-pong across items)
@@ -187,7 +229,7 @@ struct MoeCfg {
   static constexpr int kThreads = (2 + kDecWarps + 4) * 32;
   static constexpr int kSmemBytes =
       kStages * kStageBytes + 2 * kCentBytes + kStgBytes + 1024 + 512;
-  static_assert(kSmemBytes + 4200 <= 227 * 1024, "dynamic + static shared memory per block");
+  static_assert(kSmemBytes + 5200 <= 227 * 1024, "dynamic + static shared memory per block");
 };
 
 // Persistent grouped GEMM.  Work items (expert e, 128-row weight tile nt, BN-token tile mt) are
@@ -239,7 +281,7 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&ifull[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&decd[s], Cfg::kDecWarps * 32);
+      mbar_init(&decd[s], Cfg::kDecWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&cfull[b], 1);
@@ -301,11 +343,11 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
         const uint32_t ph = (it / S) & 1;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[st], ph ^ 1, 12));
         if (!ok) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&ifull[st], Cfg::kIdxBytes);
-          tma_load_2d(sIdx + st * Cfg::kIdxBytes, &tm_idx, &ifull[st], i * 32, row0);
-          mbar_arrive_expect_tx(&full[st], Cfg::kBBytes);
-          tma_load_2d(sB + st * Cfg::kBBytes, &tm_b, &full[st], i * 64, I.p0);
+        if (lane < 2) {   // both copies in one instruction stream: lane 0 the indices, lane 1 B
+          uint64_t* bar = lane == 0 ? &ifull[st] : &full[st];
+          mbar_arrive_expect_tx(bar, lane == 0 ? Cfg::kIdxBytes : Cfg::kBBytes);
+          tma_load_2d(lane == 0 ? static_cast<void*>(sIdx + st * Cfg::kIdxBytes) : static_cast<void*>(sB + st * Cfg::kBBytes),
+                      lane == 0 ? &tm_idx : &tm_b, bar, lane == 0 ? i * 32 : i * 64, lane == 0 ? row0 : I.p0);
         }
         __syncwarp();
       }
@@ -325,7 +367,8 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       for (int i = 0; i < nstages && ok; ++i, ++it) {
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[st], ph, 13) && mbar_wait(&decd[st], ph, 14));
+        // decd: the stage's A tile is decoded and (each decoder warp waited for it) its B tile landed
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&decd[st], ph, 14));
         if (!ok) break;
         tc_fence_after();
         const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
@@ -371,7 +414,12 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
           *reinterpret_cast<uint4*>(a_s + r * 128 + ((kc ^ (r & 7)) << 4)) = o;
         }
         fence_proxy_async_smem();
-        mbar_arrive(&decd[st]);
+        __syncwarp();
+        if (lane == 0) {
+          if (!mbar_wait(&full[st], ph, 13)) ok = false;
+          mbar_arrive(&decd[st]);
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
       }
       if (ok) mbar_arrive(&cempty[b]);
     }
@@ -453,10 +501,10 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       } else {
         // down: y_e[token, n] * gate, scattered to the token's slot row (coalesced along n).
         // The item's routed entries and gates are fetched once, in parallel, into shared memory.
-        if (et < I.cnt) {
-          const int f = a.entries[I.p0 + et];
-          s_f[et] = f;
-          s_g[et] = a.gates[f];
+        for (int c = et; c < I.cnt; c += 128) {
+          const int f = a.entries[I.p0 + c];
+          s_f[c] = f;
+          s_g[c] = a.gates[f];
         }
         named_bar_sync(2, 128);
         const int n = I.nt * 128 + row;

@@ -218,7 +218,7 @@ int dec_max_clusters_bn(int S) {
 }
 
 template <int BN, bool E8M0, bool VQ, int SF = 0>
-ql_status launch_dec_bn(const ql::DecodeArgs& a, int grid, cudaStream_t s) {
+ql_status launch_dec_bn(const CUtensorMap& tm_x, const ql::DecodeArgs& a, int grid, cudaStream_t s) {
   using Cfg = ql::DecCfg<BN, E8M0, VQ, SF>;
   ql_status st = dec_set_attrs<BN, E8M0, VQ, SF>();
   if (st != QL_OK) return st;
@@ -236,16 +236,16 @@ ql_status launch_dec_bn(const ql::DecodeArgs& a, int grid, cudaStream_t s) {
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.cluster ? 2 : 1;
-  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_decode_kernel<BN, E8M0, VQ, SF>, a));
+  QL_CUDA(cudaLaunchKernelEx(&cfg, ql::fp4_decode_kernel<BN, E8M0, VQ, SF>, tm_x, a));
   return QL_OK;
 }
 
 template <bool E8M0, bool VQ, int SF = 0>
-ql_status launch_dec(int BN, const ql::DecodeArgs& a, int grid, cudaStream_t s) {
+ql_status launch_dec(int BN, const CUtensorMap& tm_x, const ql::DecodeArgs& a, int grid, cudaStream_t s) {
   switch (BN) {
-    case 16: return launch_dec_bn<16, E8M0, VQ, SF>(a, grid, s);
-    case 32: return launch_dec_bn<32, E8M0, VQ, SF>(a, grid, s);
-    case 64: return launch_dec_bn<64, E8M0, VQ, SF>(a, grid, s);
+    case 16: return launch_dec_bn<16, E8M0, VQ, SF>(tm_x, a, grid, s);
+    case 32: return launch_dec_bn<32, E8M0, VQ, SF>(tm_x, a, grid, s);
+    case 64: return launch_dec_bn<64, E8M0, VQ, SF>(tm_x, a, grid, s);
   }
   return fail(QL_ERR_UNSUPPORTED, "no decode tile for BN=%d", BN);
 }
@@ -378,6 +378,20 @@ constexpr int kDecLocalUnits = 8;                // local mode: units per quanti
 constexpr int64_t kDecLocalAmaxElems = 128 * 1024;   // x elements every CTA may read for the amax
 constexpr int64_t kDecClusterAmaxElems = 16 * 1024;  // ... when a cluster exchange is the other way
 
+// Whether a forward of M tokens runs the decode kernel (when it also plans): forced by
+// ql_decode_fuse_mode, else by what measured faster on the B200 in chains of CUDA-graph replayed
+// layers of 2560 x 9728.  With E4M3-B16 activations (VQ and NVFP4 layers) the separate grid
+// quantizer and the general GEMM won from M = 8 up (VQ: 15.5 against 20.4 us at M = 8, 22.0
+// against 22.5 at M = 64) and tied at M = 1 (14.2 / 14.1); with MXFP4 activations the decode
+// kernel won at M = 1 (9.5 against 10.0) and from M = 64 (14.5 against 16.3) and lost in between.
+bool use_decode_kernel(const ql_linear* L, int64_t M) {
+  const int forced = g_decode_fuse_mode.load();
+  if (forced == 0) return false;
+  if (forced > 0) return true;
+  if (M == 1) return true;
+  return L->e8m0 && !L->vq && M > 32;
+}
+
 // Decode launches (M <= 64): the weight tiles split along K so that the grid covers the SMs once;
 // each CTA keeps all its stages resident.  Returns false when no such split exists.
 bool plan_decode(const ql_linear* L, int64_t M, FwdPlan& p) {
@@ -433,7 +447,7 @@ bool plan_decode(const ql_linear* L, int64_t M, FwdPlan& p) {
 FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   if (L->int4) return plan_forward_int4(L, M);
   FwdPlan p{};
-  if (plan_decode(L, M, p)) {
+  if (use_decode_kernel(L, M) && plan_decode(L, M, p)) {
     const int atomK = L->e8m0 ? 128 : 64;
     p.sfb_atoms = static_cast<int>(cdiv(L->C, atomK));
     p.sf_rows = 128;
@@ -1056,11 +1070,17 @@ static ql_status launch_decode(const ql_linear* L, int64_t M, const FwdPlan& p, 
   a.had = L->had;
   const int grid = p.tiles_n * p.splits;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (L->vq && L->sfmode == 1) return launch_dec<false, true, 1>(p.BN, a, grid, cs);
-  if (L->vq && L->sfmode == 2) return launch_dec<false, true, 2>(p.BN, a, grid, cs);
-  if (L->vq) return launch_dec<false, true>(p.BN, a, grid, cs);
-  if (!L->e8m0) return launch_dec<false, false>(p.BN, a, grid, cs);
-  return launch_dec<true, false>(p.BN, a, grid, cs);
+  CUtensorMap tm_x;   // the plain-layout activation codes (read only when x is quantized already)
+  std::memset(&tm_x, 0, sizeof(tm_x));
+  if (x == nullptr) {
+    ql_status st = make_tmap_u8(&tm_x, w8 + p.codes_off, L->C / 2, M, L->C / 2, 128, p.BN);
+    if (st != QL_OK) return st;
+  }
+  if (L->vq && L->sfmode == 1) return launch_dec<false, true, 1>(p.BN, tm_x, a, grid, cs);
+  if (L->vq && L->sfmode == 2) return launch_dec<false, true, 2>(p.BN, tm_x, a, grid, cs);
+  if (L->vq) return launch_dec<false, true>(p.BN, tm_x, a, grid, cs);
+  if (!L->e8m0) return launch_dec<false, false>(p.BN, tm_x, a, grid, cs);
+  return launch_dec<true, false>(p.BN, tm_x, a, grid, cs);
 }
 
 ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void* ws,
@@ -1232,7 +1252,7 @@ ql_status ql_debug_inject(int32_t withhold_cta, uint64_t wait_limit_ns) {
 }
 
 ql_status ql_decode_fuse_mode(int32_t mode) {
-  if (mode != -1 && (mode < 1 || mode > 3)) return fail(QL_ERR_INVALID_ARG, "mode must be -1, 1, 2 or 3");
+  if (mode < -1 || mode > 3) return fail(QL_ERR_INVALID_ARG, "mode must be -1, 0, 1, 2 or 3");
   g_decode_fuse_mode.store(mode);
   return QL_OK;
 }
@@ -1281,7 +1301,7 @@ struct ql_moe {
 
 namespace {
 
-constexpr int kMoeBN = 128;
+constexpr int kMoeBN = 256;   // tokens per work item (N of the MMA; two accumulators fill TMEM)
 
 struct MoePlan {
   size_t counts, offsets, entries, ids, gates, x_codes, x_scales, x_dq, xs, h_codes, h_scales,
@@ -1455,7 +1475,7 @@ ql_status moe_grouped_forward(const ql_moe* m, const void* x, int64_t T, const f
   ql::moe_topk_kernel<<<static_cast<unsigned>((T * 32 + 255) / 256), 256, 0, s>>>(
       logits, static_cast<int>(T), m->E, m->k, ids, gates, counts);
   QL_CUDA(cudaGetLastError());
-  ql::moe_scatter_kernel<<<m->E, 256, 0, s>>>(ids, total, m->E, counts, offsets, entries);
+  ql::moe_scatter_kernel<<<m->E, ql::kScatterThreads, 0, s>>>(ids, total, m->E, counts, offsets, entries);
   QL_CUDA(cudaGetLastError());
   __nv_bfloat16* x_dq = reinterpret_cast<__nv_bfloat16*>(w8 + p.x_dq);
   ql_status st = launch_quant_mx(x, T, m->H, w8 + p.x_codes, w8 + p.x_scales, nullptr, 0, nullptr,

@@ -235,6 +235,7 @@ ql_status ql_tensor_peak(int32_t kind, int32_t n, int32_t iters, int32_t ctas,
 ql_status ql_debug_inject(int32_t withhold_cta, uint64_t wait_limit_ns);
 
 /* How qlinear_forward's decode kernel (M <= 64, FP4 and VQ layers) is organised:
+ * 0 = no decode kernel: the separate quantizer, then the general split-K GEMM;
  * 1 = the CTAs share the activation units out, exchange the E4M3 tensor amax and the finished
  * stage tiles through the workspace; 2 = every CTA quantizes the activations of its own K stages
  * straight into shared memory (the E4M3 amax read from all of x while x is small, else gathered
@@ -242,8 +243,9 @@ ql_status ql_debug_inject(int32_t withhold_cta, uint64_t wait_limit_ns);
  * thread-block cluster: the split-K partials (and the E4M3 amax shares) meet in distributed
  * shared memory and no CTA waits on another outside its cluster; each CTA quantizes x for its
  * own stages as in 2 while that is little work (M * stages small), else the separate quantizer
- * runs first.  -1 (the default) = 3 where the device holds every cluster at once, else 2 or 1,
- * chosen per launch from M, the split and the width.  A forced mode that a launch cannot take
+ * runs first.  -1 (the default) = the decode kernel for M = 1, and for MXFP4 layers above 32
+ * tokens, else 0 (what measured faster on the B200); where it runs, 3 if the device holds every
+ * cluster at once, else 2 or 1, chosen from M, the split and the width.  A forced mode that a launch cannot take
  * falls back to the separate quantizer launch.  Quantized codes are identical in every mode;
  * outputs are identical between modes with the same K split (1 and 2), while mode 3 may split K
  * into fewer parts (its clusters must fit the device at once), which reorders the fp32 split-K

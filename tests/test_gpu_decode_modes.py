@@ -17,7 +17,7 @@ from tests._parity import check_bf16, check_fp32
 
 pytestmark = pytest.mark.gpu
 
-MODES = (-1, 1, 2, 3)
+MODES = (-1, 0, 1, 2, 3)
 
 
 def _ql():
@@ -132,7 +132,7 @@ def test_vq_decode_modes(M):
 
 def test_bad_mode_rejected():
     ql = _ql()
-    for bad in (0, 4, -2):
+    for bad in (4, -2):
         with pytest.raises(ql.QLError):
             ql.decode_fuse_mode(bad)
 
