@@ -38,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "qlinear_prepare_int4_bsr", "ql_tensor_peak", "ql_debug_inject",
     "qlinear_prepare_vq_postscale", "qlinear_prepare_vq_prescale_plus",
     "qlinear_prepare_prquant_ex", "quantize_act_hadamard", "ql_decode_fuse_mode",
+    "quantize_act_augmented",
 )
 
 
@@ -59,7 +60,7 @@ class WeightDesc(ctypes.Structure):
         ("bsr_block_n", ctypes.c_int32), ("bsr_block_k", ctypes.c_int32),
         ("bsr_nnzb", ctypes.c_int32), ("scale_codebook", ctypes.c_void_p),
         ("scale_codebook_entries", ctypes.c_int32), ("scale_group", ctypes.c_int32),
-        ("had_block", ctypes.c_int32),
+        ("had_block", ctypes.c_int32), ("tail_copy", ctypes.c_int32),
     ]
 
 
@@ -90,6 +91,7 @@ def _load() -> ctypes.CDLL:
         "qlinear_prepare_prquant": [vp, i64, i64, i32, vp, vp, vp],
         "qlinear_prepare_prquant_ex": [vp, i64, i64, i32, i32, vp, vp, vp],
         "quantize_act_hadamard": [ctypes.c_int, i32, vp, i64, i64, vp, vp, vp],
+        "quantize_act_augmented": [ctypes.c_int, vp, i64, i64, i32, vp, vp, vp],
         "qlinear_prepare_vq_prescale": [vp, i64, i64, vp, i32, i32, vp, vp, vp],
         "moe_create": [ctypes.POINTER(WeightDesc), ctypes.POINTER(WeightDesc), i32, i32, vp,
                        ctypes.POINTER(vp)],
@@ -151,14 +153,23 @@ def decode_fuse_mode(mode: int = -1) -> None:
     _ok(lib.ql_decode_fuse_mode(int(mode)), "ql_decode_fuse_mode")
 
 
-def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None, had_block: int = 0):
+def quantize_act(x, fmt: int = QL_A_MXFP4_E8M0_B32, stream=None, had_block: int = 0,
+                 k_tail: int = 0):
     """Quantize bf16 activations [M, K] on the GPU.
     MXFP4 E8M0-B32 -> (codes uint8 [M, K/2], E8M0 scales uint8 [M, K/32]), optionally after an
-    online block-32 Hadamard (had_block = 32);
+    online block-32 Hadamard (had_block = 32), or (k_tail > 0) the PRQuant augmented activation
+    (codes [M, (K + k_tail)/2], scales [M, (K + k_tail)/32]: the last k_tail channels appended);
     E4M3-B16 + tensor scale -> (codes, E4M3 scales uint8 [M, K/16], ts float32 [1])."""
     import torch
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
     M, K = x.shape
+    if k_tail:
+        assert fmt == QL_A_MXFP4_E8M0_B32 and not had_block
+        codes = torch.empty((M, (K + k_tail) // 2), dtype=torch.uint8, device=x.device)
+        scales = torch.empty((M, (K + k_tail) // 32), dtype=torch.uint8, device=x.device)
+        _ok(lib.quantize_act_augmented(fmt, x.data_ptr(), M, K, int(k_tail), codes.data_ptr(),
+                                       scales.data_ptr(), _stream(stream)), "quantize_act_augmented")
+        return codes, scales
     codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
     if fmt == QL_A_MXFP4_E8M0_B32:
         scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
@@ -196,7 +207,7 @@ class QLinear:
                  wfmt: int = QL_W_MXFP4_E8M0_B32, w_tensor_scale: float = 1.0,
                  indices: np.ndarray | None = None, codebooks: np.ndarray | None = None,
                  bsr: dict | None = None, scale_codebook: np.ndarray | None = None,
-                 had_block: int = 0, stream=None):
+                 had_block: int = 0, tail_copy: bool = False, stream=None):
         """MXFP4: codes [N, K/2] + E8M0 scales [N, K/32] (+ k_tail).  NVFP4 (E4M3-B16): codes +
         E4M3 scales [N, K/16] + w_tensor_scale.  VQ PreScale: indices [N, K/4] + packed codebooks
         [N/64, K/64, 256, 2] + E4M3 scales [N, K/16] + w_tensor_scale (codes = None).
@@ -247,7 +258,8 @@ class QLinear:
                        scales=scales.ctypes.data, w_tensor_scale=float(w_tensor_scale),
                        indices=iptr, codebooks=cbptr, qblock_n=64, qblock_k=64,
                        scale_codebook=scb_ptr, scale_codebook_entries=256 if scb_ptr else 0,
-                       scale_group=8 if scb_ptr else 0, had_block=int(had_block))
+                       scale_group=8 if scb_ptr else 0, had_block=int(had_block),
+                       tail_copy=1 if tail_copy else 0)
         h = ctypes.c_void_p()
         _ok(lib.qlinear_create(ctypes.byref(d), _stream(stream), ctypes.byref(h)), "qlinear_create")
         self._h = h

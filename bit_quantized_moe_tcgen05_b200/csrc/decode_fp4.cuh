@@ -134,6 +134,8 @@ struct DecodeArgs {
   int had;                    // fuse, E8M0: online Hadamard (block 32) before quantizing x
   int amax_coop;              // fuse = 2, E4M3: the tensor amax combined over the CTAs (each
                               // reads a share of x), else every CTA reads all of x
+  int act_aug;                // fuse = 0: the plain layout is augmented ([M, C + k_tail], the
+                              // tail copied behind): tail stages read coordinate C + j
   int cluster;                // the K-splits of a weight tile form one thread-block cluster: the
                               // split-K partials and the E4M3 amax meet in distributed shared
                               // memory, and the workspace sync block is not used
@@ -364,6 +366,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
           for (int it = 0; it < n_it; ++it) {
             int kw, kx, valid;
             stage_coords(s_begin + it, kw, kx, valid);
+            if (a.act_aug) kx = kw;
             tma_load_2d(sB + it * Cfg::kBBytes, &tm_x, bfull, kx >> 1, 0);
             const int nat = valid / Cfg::kAtomK;
             if (nat > 0)

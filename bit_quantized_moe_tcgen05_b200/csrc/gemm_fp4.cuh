@@ -72,6 +72,9 @@ struct Fp4GemmArgs {
   const uint8_t* xq;        // quantized activation codes [M, C/2] (read directly by decode launches)
   int* tickets;             // [split tiles] arrival counters, zero between launches
   const uint8_t* scb;       // VQ PreScale+: scale codebook [256][8] E4M3 bytes
+  int act_aug;              // the quantized activation is already augmented ([M, C + k_tail]:
+                            // the tail copied behind, PRQuant's offline copy): tail stages read
+                            // activation coordinate C + j, like the weight
 };
 
 // SF (VQ weights only): where the weight's E4M3 block scales come from -- 0 MXCode PreScale (the
@@ -312,6 +315,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
     const int i = s_begin + it, st = it % S;
     int kw, kx, valid;
     stage_coords(i, kw, kx, valid);
+    if (a.act_aug) kx = kw;
     const int nat = valid / Cfg::kAtomK;
     tma_load_2d(sB + st * Cfg::kBBytes, &tm_x, &full[st], kx >> 1, m0);
 #pragma unroll
@@ -342,15 +346,17 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
     if (lsu_act) {
       // Every stage's activation tile (BN rows x 128 B, stored with the 128-byte swizzle) and its
       // scale atoms, 16 bytes per cp.async from all 32 lanes; rows past M are zero-filled.
+      const int xw2 = (a.act_aug ? a.C + a.k_tail : a.C) / 2;   // bytes per activation row
       for (int it = 0; it < n_it; ++it) {
         int kw, kx, valid;
         stage_coords(s_begin + it, kw, kx, valid);
+        if (a.act_aug) kx = kw;
         const int nat = valid / Cfg::kAtomK;
         const uint32_t bdst = smem_u32(sB + it * Cfg::kBBytes);
         for (int c = lane; c < BN * 8; c += 32) {
           const int r = c >> 3, kc = c & 7;
           const bool in = m0 + r < a.M;
-          const uint8_t* src = a.xq + static_cast<size_t>(in ? m0 + r : 0) * (a.C / 2) + (kx >> 1) + kc * 16;
+          const uint8_t* src = a.xq + static_cast<size_t>(in ? m0 + r : 0) * xw2 + (kx >> 1) + kc * 16;
           cp_async16(bdst + r * 128 + ((kc ^ (r & 7)) << 4), src, in ? 16u : 0u);
         }
         const uint8_t* sfsrc = a.sfb + (static_cast<size_t>(sf_group0) * a.sfb_atoms + kx / Cfg::kAtomK) * 512;

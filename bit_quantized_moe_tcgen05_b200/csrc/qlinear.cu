@@ -286,6 +286,7 @@ struct ql_linear {
   bool vq = false;             // MXCode VQ weight
   int sfmode = 0;              // VQ scales: 0 PreScale atoms, 1 PostScale per QBlock, 2 PreScale+
   int had = 0;                 // online block-32 Hadamard of the activations (MXFP4 layers)
+  bool tail_copy = false;      // the quantized activation in the workspace is [Z~, Z~_tail]
   uint8_t* d_scb = nullptr;    // PreScale+: scale codebook [256][8] on the device
   uint8_t* d_codes = nullptr;  // weight blocks [N/128][stages][codes or indices + codebooks, scales]
   size_t weight_bytes = 0;
@@ -299,6 +300,9 @@ struct ql_linear {
 };
 
 namespace {
+
+// Channels of the quantized activation in the workspace: C, or C + k_tail with the tail copied.
+int64_t act_width(const ql_linear* L) { return L->tail_copy ? L->C + L->k_tail : L->C; }
 
 struct FwdPlan {
   int BN, splits, spp, tiles_n, tiles_m;
@@ -449,13 +453,13 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   FwdPlan p{};
   if (use_decode_kernel(L, M) && plan_decode(L, M, p)) {
     const int atomK = L->e8m0 ? 128 : 64;
-    p.sfb_atoms = static_cast<int>(cdiv(L->C, atomK));
+    p.sfb_atoms = static_cast<int>(cdiv(act_width(L), atomK));
     p.sf_rows = 128;
     p.sync_off = 0;   // (the E4M3 grid quantizer of qlinear_quantize_input)
     p.dsync_off = align_up(ql::kE4m3SyncBytes, 256);
     size_t off = sync_prefix_bytes();
     p.codes_off = off;
-    off = align_up(off + static_cast<size_t>(M) * (L->C / 2), 256);
+    off = align_up(off + static_cast<size_t>(M) * (act_width(L) / 2), 256);
     p.sf_off = off;   // one 128-row group of scale atoms (the quantizers write up to 2)
     off = align_up(off + static_cast<size_t>(2) * p.sfb_atoms * 512, 256);
     p.scal_off = off;   // [0] amax bit pattern, [1] tensor scale (E4M3-B16)
@@ -491,7 +495,7 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   p.spp = static_cast<int>(cdiv(total, splits));
   p.splits = static_cast<int>(cdiv(total, p.spp));
   const int atomK = L->e8m0 ? 128 : 64;  // K elements covered by one 512-byte scale atom
-  p.sfb_atoms = static_cast<int>(cdiv(L->C, atomK));
+  p.sfb_atoms = static_cast<int>(cdiv(act_width(L), atomK));
   p.sf_rows = std::max(p.BN, 128);
   // 128-row atom groups of the tiled activation scales: ceil(sf_rows / 128) per token tile
   const int64_t sf_groups = std::max<int64_t>(cdiv(std::max<int64_t>(M, 1), 256) * 2,
@@ -500,7 +504,7 @@ FwdPlan plan_forward(const ql_linear* L, int64_t M) {
   p.dsync_off = align_up(ql::kE4m3SyncBytes, 256);
   size_t off = sync_prefix_bytes();
   p.codes_off = off;
-  off = align_up(off + static_cast<size_t>(M) * (L->C / 2), 256);
+  off = align_up(off + static_cast<size_t>(M) * (act_width(L) / 2), 256);
   p.sf_off = off;
   off = align_up(off + static_cast<size_t>(sf_groups) * p.sfb_atoms * 512, 256);
   // [0] amax bit pattern and [1] tensor scale of E4M3-B16 activations, then the split-K tickets
@@ -664,19 +668,23 @@ ql_status launch_quant_int4(const void* x, int64_t M, int64_t K, int8_t* q8, uin
   return QL_OK;
 }
 
+// k_tail > 0: the outputs are the augmented activation [Z~, Z~_tail] of K + k_tail channels
+// (the codes and scales of the last k_tail channels written a second time behind the others).
 ql_status launch_quant_mx(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sp,
                           uint8_t* st, int st_atoms, int* zero_words, int nzero,
                           cudaStream_t s, __nv_bfloat16* deq = nullptr, int st_rows = 128,
-                          int had = 0) {
+                          int had = 0, int64_t k_tail = 0) {
   const long total = static_cast<long>(M) * (K / 32);
   const long threads = std::max<long>(total, nzero);
   if (threads == 0) return QL_OK;
   const int block = 256;
   const long grid = (threads + block - 1) / block;
+  const int64_t W = K + k_tail;   // output channels
   ql::quant_mx_e8m0_b32_kernel<<<static_cast<unsigned>(grid), block, 0, s>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<int>(M), static_cast<int>(K),
-      static_cast<int>(K), codes, static_cast<int>(K / 2), sp, static_cast<int>(K / 32), st,
-      st_atoms, st_rows, zero_words, nzero, deq, had);
+      static_cast<int>(K), codes, static_cast<int>(W / 2), sp, static_cast<int>(W / 32), st,
+      st_atoms, st_rows, zero_words, nzero, deq, had,
+      k_tail > 0 ? static_cast<int>(K - k_tail) : -1, static_cast<int>(K));
   QL_CUDA(cudaGetLastError());
   return QL_OK;
 }
@@ -929,6 +937,8 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
     return fail(QL_ERR_UNSUPPORTED, "PreScale+ needs a scale codebook of 256 entries of 8 scales");
   if (d->had_block != 0 && (d->had_block != 32 || !mx))
     return fail(QL_ERR_UNSUPPORTED, "online Hadamard: block 32 with MXFP4 (E8M0-B32) layers only");
+  if (d->tail_copy != 0 && (d->tail_copy != 1 || !mx || d->k_tail == 0))
+    return fail(QL_ERR_INVALID_ARG, "tail_copy = 1 needs an MXFP4 layer with k_tail > 0");
   if (d->N > (1 << 24) || d->K > (1 << 24))
     return fail(QL_ERR_UNSUPPORTED, "N/K too large");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -942,6 +952,7 @@ ql_status qlinear_create(const ql_weight_desc* d, ql_stream_t stream, ql_linear*
   L->vq = vq;
   L->sfmode = sfmode;
   L->had = d->had_block == 32 ? 1 : 0;
+  L->tail_copy = d->tail_copy == 1;
   L->w_ts = mx ? 1.f : d->w_tensor_scale;
   L->n_base_stages = static_cast<int>(cdiv(L->C, 256));
   L->n_stages_total = L->n_base_stages + static_cast<int>(cdiv(L->k_tail, 256));
@@ -1034,7 +1045,8 @@ ql_status qlinear_quantize_input(const ql_linear* L, const void* x, int64_t M, v
   }
   return launch_quant_mx(x, M, L->C, w8 + p.codes_off, nullptr, w8 + p.sf_off, p.sfb_atoms,
                          reinterpret_cast<int*>(w8 + p.tick_off), p.n_tickets,
-                         reinterpret_cast<cudaStream_t>(stream), nullptr, p.sf_rows, L->had);
+                         reinterpret_cast<cudaStream_t>(stream), nullptr, p.sf_rows, L->had,
+                         L->tail_copy ? L->k_tail : 0);
 }
 
 // The decode kernel: x != null quantizes x inside it (qlinear_forward), else the workspace holds
@@ -1053,6 +1065,7 @@ static ql_status launch_decode(const ql_linear* L, int64_t M, const FwdPlan& p, 
   a.fuse = x != nullptr ? p.fuse_mode : 0;
   a.amax_coop = p.amax_coop ? 1 : 0;
   a.cluster = p.cluster ? 1 : 0;
+  a.act_aug = L->tail_copy ? 1 : 0;
   a.x = static_cast<const __nv_bfloat16*>(x);
   a.xq = w8 + p.codes_off;
   a.sfb = w8 + p.sf_off;
@@ -1073,7 +1086,7 @@ static ql_status launch_decode(const ql_linear* L, int64_t M, const FwdPlan& p, 
   CUtensorMap tm_x;   // the plain-layout activation codes (read only when x is quantized already)
   std::memset(&tm_x, 0, sizeof(tm_x));
   if (x == nullptr) {
-    ql_status st = make_tmap_u8(&tm_x, w8 + p.codes_off, L->C / 2, M, L->C / 2, 128, p.BN);
+    ql_status st = make_tmap_u8(&tm_x, w8 + p.codes_off, act_width(L) / 2, M, act_width(L) / 2, 128, p.BN);
     if (st != QL_OK) return st;
   }
   if (L->vq && L->sfmode == 1) return launch_dec<false, true, 1>(p.BN, tm_x, a, grid, cs);
@@ -1122,7 +1135,7 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
   }
   if (p.decode) return launch_decode(L, M, p, nullptr, y, y32, w8, stream);
   CUtensorMap tm_x;
-  st = make_tmap_u8(&tm_x, w8 + p.codes_off, L->C / 2, M, L->C / 2, 128, p.BN);
+  st = make_tmap_u8(&tm_x, w8 + p.codes_off, act_width(L) / 2, M, act_width(L) / 2, 128, p.BN);
   if (st != QL_OK) return st;
   ql::Fp4GemmArgs a{};
   a.M = static_cast<int>(M);
@@ -1157,6 +1170,7 @@ ql_status qlinear_gemm(const ql_linear* L, int64_t M, void* y, float* y32, void*
                                       L->N, M, L->N, p.BN);
   if (st != QL_OK) return st;
   a.scb = L->d_scb;
+  a.act_aug = L->tail_copy ? 1 : 0;
   if (L->vq && L->sfmode == 1) return launch_fp4<false, true, 1>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
   if (L->vq && L->sfmode == 2) return launch_fp4<false, true, 2>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
   if (L->vq) return launch_fp4<false, true>(p.BN, tm_x, tm_y, tm_y32, a, grid, cs);
@@ -1255,6 +1269,22 @@ ql_status ql_decode_fuse_mode(int32_t mode) {
   if (mode < -1 || mode > 3) return fail(QL_ERR_INVALID_ARG, "mode must be -1, 0, 1, 2 or 3");
   g_decode_fuse_mode.store(mode);
   return QL_OK;
+}
+
+ql_status quantize_act_augmented(ql_aformat fmt, const void* x, int64_t M, int64_t C,
+                                 int32_t k_tail, void* codes, void* scales, ql_stream_t stream) {
+  if (M < 0 || C < 0 || k_tail < 0) return fail(QL_ERR_INVALID_ARG, "negative size");
+  if (fmt != QL_A_MXFP4_E8M0_B32)
+    return fail(QL_ERR_UNSUPPORTED, "the augmented activation is MXFP4 (E8M0-B32) only");
+  if (C % 32 != 0 || k_tail % 32 != 0 || k_tail > C)
+    return fail(QL_ERR_UNSUPPORTED, "needs C %% 32 == 0, k_tail %% 32 == 0, k_tail <= C");
+  if (M == 0 || C == 0) return QL_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return fail(QL_ERR_INVALID_ARG, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(x) & 15) != 0 || (reinterpret_cast<uintptr_t>(codes) & 15) != 0)
+    return fail(QL_ERR_INVALID_ARG, "x and codes must be 16-byte aligned");
+  return launch_quant_mx(x, M, C, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                         nullptr, 0, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), nullptr,
+                         128, 0, k_tail);
 }
 
 ql_status quantize_act_hadamard(ql_aformat fmt, int32_t had_block, const void* x, int64_t M,

@@ -3,8 +3,10 @@
 //  * quant_mx_e8m0_b32_kernel -- OCP-MX / MXFP4: per 32 elements along K a shared exponent
 //    e = floor(log2 amax) - 2 (clamped to [-127,127], stored as the E8M0 byte e+127), elements
 //    x * 2^-e rounded to nearest-even E2M1 and saturated at +-6.  PRQuant, §4 "Kernel design for
-//    efficient inference" quantizes the reordered activation to MXFP4 once; the tail copy that
-//    page appends is realised by the GEMM reading the same quantized tail twice.
+//    efficient inference" quantizes the reordered activation to MXFP4 once and appends the
+//    quantized tail: either the GEMM reads the same quantized tail twice (online), or this
+//    kernel writes the tail blocks a second time behind the others (offline copy, "Activation
+//    tail construction").
 //  * quant_e4m3_b16 kernels -- E4M3-B16-FP4 with an FP32 tensor scale (MXCode, Table 1).
 //  * quant_int4_g128_kernel -- symmetric INT4 per (token, 128-group), fp32 scale amax/7
 //    (MosaicQuant W4A4 INT4 path).
@@ -129,7 +131,8 @@ __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
     const __nv_bfloat16* __restrict__ x, int M, int K, int ldx, uint8_t* __restrict__ codes,
     int ldc, uint8_t* __restrict__ scales_plain, int lds, uint8_t* __restrict__ scales_tiled,
     int sf_atoms_per_row, int sf_tile_rows, int* __restrict__ zero_words, int nzero,
-    __nv_bfloat16* __restrict__ deq_out = nullptr, int had = 0) {
+    __nv_bfloat16* __restrict__ deq_out = nullptr, int had = 0, int tail_from = -1,
+    int tail_to = 0) {
   griddep_launch_dependents();   // a GEMM launched behind this grid may start streaming weights
   const long gtid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (zero_words != nullptr && gtid < nzero) zero_words[gtid] = 0;
@@ -181,11 +184,17 @@ __global__ void __launch_bounds__(256) quant_mx_e8m0_b32_kernel(
       packed[q] = e2m1x8(f) | bf16x8_sign_nibbles(ww);
     }
   }
-  *reinterpret_cast<uint4*>(codes + static_cast<size_t>(m) * ldc + j * 16) =
-      make_uint4(packed[0], packed[1], packed[2], packed[3]);
   const uint8_t b = static_cast<uint8_t>(e + 127);
-  if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + j] = b;
-  if (scales_tiled != nullptr) scales_tiled[sf_tiled_offset(m, j, sf_atoms_per_row, sf_tile_rows)] = b;
+  // PRQuant offline copy: blocks of the last channels [tail_from, K) are written a second time
+  // at [tail_to, ...), so that the codes hold the augmented activation [Z~, Z~_tail]
+  const int ncopy = (tail_from >= 0 && j * 32 >= tail_from) ? 2 : 1;
+  for (int cpy = 0; cpy < ncopy; ++cpy) {
+    const int jd = cpy == 0 ? j : (tail_to + j * 32 - tail_from) >> 5;
+    *reinterpret_cast<uint4*>(codes + static_cast<size_t>(m) * ldc + jd * 16) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    if (scales_plain != nullptr) scales_plain[static_cast<size_t>(m) * lds + jd] = b;
+    if (scales_tiled != nullptr) scales_tiled[sf_tiled_offset(m, jd, sf_atoms_per_row, sf_tile_rows)] = b;
+  }
   if (deq_out != nullptr) {
     uint32_t o[16];
 #pragma unroll

@@ -102,6 +102,12 @@ typedef struct ql_weight_desc {
                           h for down) passes an online block-32 Hadamard before quantization
                           (CodeQuant's "had" variants), and the weight is given rotated,
                           W . blockdiag(H_32) / 32; see quantize_act_hadamard */
+  int32_t tail_copy;   /* MXFP4 layers with k_tail > 0: 0 = the GEMM reads the activation's last
+                          k_tail channels a second time for the tail stages (PRQuant "online"
+                          tail); 1 = the activation quantizer writes the augmented activation
+                          [Z~, Z~_tail] (C + k_tail channels, the tail copied behind, PRQuant §4
+                          "Activation tail construction", offline copy) and the GEMM reads it
+                          straight through.  Same results. */
 } ql_weight_desc;
 
 typedef struct ql_linear ql_linear;
@@ -262,6 +268,15 @@ ql_status ql_decode_fuse_mode(int32_t mode);
  * W . blockdiag(H_32) / 32, so the layer's product is unchanged. */
 ql_status quantize_act_hadamard(ql_aformat fmt, int32_t had_block, const void* x_bf16, int64_t M,
                                 int64_t K, void* codes, void* scales, ql_stream_t stream);
+
+/* MXFP4 activation quantization of a PRQuant-reordered activation with its tail appended
+ * (PRQuant §4 "Activation tail construction" and "Kernel design for efficient inference": the
+ * activation is quantized once and the quantized tail block is appended): x bf16 [M, C] (device);
+ * codes [M, (C + k_tail)/2] and E8M0 scales [M, (C + k_tail)/32] (device) hold Q(x) followed by a
+ * copy of the codes and scales of its last k_tail channels.  fmt must be QL_A_MXFP4_E8M0_B32;
+ * C % 32 == 0, k_tail % 32 == 0, 0 <= k_tail <= C (k_tail = 0 is quantize_act). */
+ql_status quantize_act_augmented(ql_aformat fmt, const void* x_bf16, int64_t M, int64_t C,
+                                 int32_t k_tail, void* codes, void* scales, ql_stream_t stream);
 
 /* Synchronise `stream` and report (then clear) the device error word. */
 ql_status ql_check(ql_stream_t stream);

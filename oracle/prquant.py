@@ -71,8 +71,10 @@ def prepare(w: np.ndarray, k: int, search: bool = False) -> dict:
 
 
 def quantize_activation_augmented(xp: np.ndarray, k: int) -> tuple[np.ndarray, np.ndarray]:
-    """Online copy: quantize the permuted activation once, then append its quantized tail
-    (codes and block scales).  Returns codes [M, C+k], bytes [M, (C+k)/32]."""
+    """The augmented activation Q([X~, X~_tail]): quantize the permuted activation once, then
+    append its quantized tail (codes and block scales) -- what both of PRQuant's tail
+    constructions hand the GEMM (the online one by reading the tail twice, the offline one by
+    writing the copy).  Returns codes [M, C+k], bytes [M, (C+k)/32]."""
     M, C = xp.shape
     codes, sb = mx.quantize_e8m0_b32(xp)
     return (np.concatenate([codes, codes[:, C - k:]], axis=1),

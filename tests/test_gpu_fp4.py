@@ -209,3 +209,57 @@ def test_fp4_gemm_prefill_shapes(N, K, M):
     codes, sb = random_mx_weight(23, N, K)
     xb, _ = synth.activations_bf16(23, M, K, 0.01, 20.0)
     check_linear(codes, sb, 0, xb, f"prefill N={N} K={K} M={M}")
+
+
+@pytest.mark.parametrize("M,C,k", [(1, 1024, 128), (37, 640, 64), (300, 9728, 128), (5, 96, 32)])
+def test_quant_augmented_bitexact(M, C, k):
+    """quantize_act with k_tail (PRQuant's offline tail copy): Q(x) followed by a copy of the codes
+    and scales of its last k channels, against the oracle's augmented activation."""
+    ql = _ql()
+    xb, _ = synth.activations_bf16(170 + M, M, C, 0.005, 50.0)
+    codes, sb = ql.quantize_act(dev_bf16(xb), k_tail=k)
+    ql.check()
+    rc, rs = prquant.quantize_activation_augmented(synth.bf16_bits_to_f64(xb), k)
+    assert np.array_equal(sb.cpu().numpy(), rs)
+    assert np.array_equal(codes.cpu().numpy(), F.pack_nibbles(rc))
+
+
+@pytest.mark.parametrize("M", [1, 16, 64, 300])
+def test_prquant_offline_tail_copy_layer(M):
+    """A PRQuant layer whose quantizer writes the augmented activation (tail_copy) computes the
+    same bits as the online layer (the GEMM reading the tail twice), in the one-launch forward and
+    through quantize_input + gemm, in every decode organisation, and matches the oracle."""
+    ql = _ql()
+    N, C, k = 512, 2048, 256
+    w = synth.bf16_bits_to_f64(synth.to_bf16_bits(synth.student_t(180, (N, C), 3.0)))
+    prep = prquant.prepare(w, k)
+    codes = F.pack_nibbles(prep["w_codes"])
+    online = ql.QLinear(codes, prep["w_sb"], k_tail=k)
+    offline = ql.QLinear(codes, prep["w_sb"], k_tail=k, tail_copy=True)
+    xb, _ = synth.activations_bf16(181 + M, M, C, 0.005, 50.0)
+    x = dev_bf16(np.ascontiguousarray(xb[:, prep["perm"]]))
+    xq = mx.dequant_e8m0_b32(*prquant.quantize_activation_augmented(synth.bf16_bits_to_f64(
+        np.ascontiguousarray(xb[:, prep["perm"]])), k))
+    wq = mx.dequant_e8m0_b32(prep["w_codes"], prep["w_sb"])
+    ref, t = G.gemm_ref(xq, wq), G.abs_scale(xq, wq)
+    try:
+        for mode in ((-1, 0, 1, 2, 3) if M <= 64 else (-1,)):
+            ql.decode_fuse_mode(mode)
+            outs = []
+            for lin in (online, offline):
+                y32 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+                lin(x, out_f32=y32)
+                ws = torch.empty(lin.workspace_bytes(M), dtype=torch.uint8, device="cuda")
+                lin.quantize_input(x, ws)
+                y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+                y2_32 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+                lin.gemm(M, y, ws, out_f32=y2_32)
+                ql.check()
+                outs += [y32.cpu().numpy(), y2_32.cpu().numpy()]
+            check_fp32(outs[0], ref, t, f"online M={M} mode {mode}")
+            for o in outs[1:]:
+                assert np.array_equal(o, outs[0]), f"M={M} mode {mode}: offline / two-call differ"
+    finally:
+        ql.decode_fuse_mode(-1)
+    online.close()
+    offline.close()
