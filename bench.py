@@ -42,7 +42,9 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the timed GEMM
 # kernel, from an ncu --set full capture of that kernel (the VQ layer's M = 64 launch; the PRQuant
 # M = 2048 launch).  Set an entry to None whenever its kernel changes until it is captured again.
-NCU_TRAFFIC_PER_LAUNCH = {"vq": None, "prquant_m2048": None}   # to be re-captured for the current kernels
+# dram read + write bytes per launch from one ncu capture of the current kernels (profiles/):
+# the headline's GEMM launches averaged over M = 1, 8, 64, and the PRQuant M = 2048 GEMM
+NCU_TRAFFIC_PER_LAUNCH = {"vq": (11.014e6 + 11.059e6 + 11.333e6) / 3, "prquant_m2048": 24.59e6}
 
 
 def measured_peaks() -> dict:
