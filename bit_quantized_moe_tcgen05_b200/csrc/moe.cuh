@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&ifull[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&decd[s], Cfg::kDecWarps);
+      mbar_init(&decd[s], Cfg::kDecWarps / 2);   // one decoder group per stage
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&cfull[b], 1);
@@ -386,18 +386,23 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       }
     }
   } else if (warp < 2 + Cfg::kDecWarps) {
-    // ---------------- decode: 4-bit indices -> bf16 operand tile through the row centroids
-    const int t = threadIdx.x - 64;
-    constexpr int kDT = Cfg::kDecWarps * 32;
+    // ---------------- decode: 4-bit indices -> bf16 operand tile through the row centroids.
+    // Two groups of decoder warps take alternate stages: a stage's barrier waits and arrivals
+    // cost a group about as long as its decode, so the groups overlap one another's.
+    constexpr int kDT = Cfg::kDecWarps * 16;                  // threads per group
+    const int grp = (warp - 2) / (Cfg::kDecWarps / 2);
+    const int t = threadIdx.x - 64 - grp * kDT;
     int it = 0;
     for (int id = blockIdx.x, j = 0; id < n_items && ok; id += gridDim.x, ++j) {
       const int b = j & 1;
-      if (!mbar_wait(&cfull[b], (j >> 1) & 1, 15)) { ok = false; break; }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&cfull[b], (j >> 1) & 1, 15))) { ok = false; break; }
       const uint16_t* cent = reinterpret_cast<const uint16_t*>(sCent + b * 128 * 16);
       for (int i = 0; i < nstages && ok; ++i, ++it) {
+        if ((it & 1) != grp) continue;
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait(&ifull[st], ph, 16)) { ok = false; break; }   // indices only: runs ahead of B
+        // indices only: runs ahead of B (warp-uniform: the warp leaves the loop together)
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ifull[st], ph, 16))) { ok = false; break; }
         const uint8_t* idx_s = sIdx + st * Cfg::kIdxBytes;
         uint8_t* a_s = sA + st * Cfg::kABytes;
 #pragma unroll

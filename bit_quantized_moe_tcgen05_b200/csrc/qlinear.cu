@@ -1331,7 +1331,7 @@ struct ql_moe {
 
 namespace {
 
-constexpr int kMoeBN = 256;   // tokens per work item (N of the MMA; two accumulators fill TMEM)
+constexpr int kMoeBN = 128;   // tokens per work item (N of the MMA; 256 measured slower)
 
 struct MoePlan {
   size_t counts, offsets, entries, ids, gates, x_codes, x_scales, x_dq, xs, h_codes, h_scales,
