@@ -271,19 +271,29 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
         const float rs = reinterpret_cast<const float*>(sRaw(st) + 128 * 64)[row];
         const float2 rs2 = make_float2(rs, rs);
         const float* sx = sSx(st) + col0;
+        // the accumulator loads of up to 32 columns in flight at once, then one wait (a wait per
+        // 8 columns serialised the TMEM latency eight times per stage)
+        constexpr int kBatch = Cfg::kCols < 32 ? Cfg::kCols : 32;
 #pragma unroll
-        for (int c = 0; c < Cfg::kCols; c += 8) {
-          uint32_t r[8];
-          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN + col0 + c, r);
-          const float4 s0 = *reinterpret_cast<const float4*>(sx + c);
-          const float4 s1 = *reinterpret_cast<const float4*>(sx + c + 4);
+        for (int c0 = 0; c0 < Cfg::kCols; c0 += kBatch) {
+          uint32_t r[kBatch];
+#pragma unroll
+          for (int c = 0; c < kBatch; c += 8)
+            tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN + col0 + c0 + c,
+                     *reinterpret_cast<uint32_t(*)[8]>(r + c));
           tmem_ld_wait();
-          const float2 w0 = f2_mul(rs2, make_float2(s0.x, s0.y)), w1 = f2_mul(rs2, make_float2(s0.z, s0.w));
-          const float2 w2 = f2_mul(rs2, make_float2(s1.x, s1.y)), w3 = f2_mul(rs2, make_float2(s1.z, s1.w));
-          acc[c / 2 + 0] = f2_fma(small_ints_to_float2(r[0], r[1]), w0, acc[c / 2 + 0]);
-          acc[c / 2 + 1] = f2_fma(small_ints_to_float2(r[2], r[3]), w1, acc[c / 2 + 1]);
-          acc[c / 2 + 2] = f2_fma(small_ints_to_float2(r[4], r[5]), w2, acc[c / 2 + 2]);
-          acc[c / 2 + 3] = f2_fma(small_ints_to_float2(r[6], r[7]), w3, acc[c / 2 + 3]);
+#pragma unroll
+          for (int c = 0; c < kBatch; c += 8) {
+            const float4 s0 = *reinterpret_cast<const float4*>(sx + c0 + c);
+            const float4 s1 = *reinterpret_cast<const float4*>(sx + c0 + c + 4);
+            const float2 w0 = f2_mul(rs2, make_float2(s0.x, s0.y)), w1 = f2_mul(rs2, make_float2(s0.z, s0.w));
+            const float2 w2 = f2_mul(rs2, make_float2(s1.x, s1.y)), w3 = f2_mul(rs2, make_float2(s1.z, s1.w));
+            const int ca = (c0 + c) / 2;
+            acc[ca + 0] = f2_fma(small_ints_to_float2(r[c + 0], r[c + 1]), w0, acc[ca + 0]);
+            acc[ca + 1] = f2_fma(small_ints_to_float2(r[c + 2], r[c + 3]), w1, acc[ca + 1]);
+            acc[ca + 2] = f2_fma(small_ints_to_float2(r[c + 4], r[c + 5]), w2, acc[ca + 2]);
+            acc[ca + 3] = f2_fma(small_ints_to_float2(r[c + 6], r[c + 7]), w3, acc[ca + 3]);
+          }
         }
       }
       tc_fence_before();
