@@ -40,7 +40,8 @@
 // publishes its flag; every CTA of the tile waits for the tile's flags and reduces 1/S of the
 // tile's outputs, adding the splits' partials in split order (deterministic), and writes y.
 //
-// Warp roles: 0 producer (weight bulk copies, then the B tiles), 1 TMEM allocator + MMA issuer,
+// Warp roles: 0 producer (weight bulk copies, then the B tiles; then the MMA issuer of the odd
+// stages into a second accumulator), 1 TMEM allocator + MMA issuer of the even stages,
 // VQ: 2..9 decoders (the operand tile of each stage rebuilt from the codebooks into a ring of up
 // to eight shared-memory tiles, as many as the memory left by the resident stages holds; warps
 // 2..5 also move the stage's weight scales to TMEM), 2..5 epilogue (without VQ they move the
@@ -166,7 +167,7 @@ struct DecCfg {
   static constexpr int kData = kSmemBytes - 2048 - kScbBytes;   // minus slack, barriers, codebook
   static constexpr int kMaxRing = 8;                 // VQ: decoded operand tiles in flight
   static constexpr int kSfCols = kAtoms * 4;         // TMEM columns of one scale set
-  static constexpr int kMaxStagesTmem = (512 - BN) / (2 * kSfCols);
+  static constexpr int kMaxStagesTmem = (512 - 2 * BN) / (2 * kSfCols);   // two accumulators
   static constexpr int kMaxStagesSmem = (kData - (VQ ? kABytes : 0)) / kPerStage;
   static constexpr int kMaxStagesRaw = kMaxStagesSmem < kMaxStagesTmem ? kMaxStagesSmem : kMaxStagesTmem;
   static constexpr int kMaxStages = kMaxStagesRaw > 16 ? 16 : kMaxStagesRaw;
@@ -283,9 +284,10 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
       valid = min(256, a.k_tail - j);
     }
   };
-  // TMEM columns: accumulator [0, BN), then per stage the weight's and the activation's scales
-  auto sfa_col = [&](int it) { return static_cast<uint32_t>(BN + it * 2 * Cfg::kSfCols); };
-  auto sfb_col = [&](int it) { return static_cast<uint32_t>(BN + it * 2 * Cfg::kSfCols + Cfg::kSfCols); };
+  // TMEM columns: accumulators [0, BN) (even stages) and [BN, 2 BN) (odd stages), then per stage
+  // the weight's and the activation's scales
+  auto sfa_col = [&](int it) { return static_cast<uint32_t>(2 * BN + it * 2 * Cfg::kSfCols); };
+  auto sfb_col = [&](int it) { return static_cast<uint32_t>(2 * BN + it * 2 * Cfg::kSfCols + Cfg::kSfCols); };
 
   if (warp == 0) {
     for (int s = lane; s < Cfg::kMaxStages; s += 32) {
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
       mbar_init(&aempty[lane], 1);
     }
     if (lane == 0) {
-      mbar_init(accf, 1);
+      mbar_init(accf, 2);   // one commit per MMA issuer
       mbar_init(xready, 1);
       mbar_init(bfull, 1);
       mbar_init(sfb_ok, 4);
@@ -333,6 +335,50 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
   const int S = a.splits;
 
   bool ok = true;
+  // ---------------- MMA issuer j (MMAs only: the scale factors are placed by other warps): the
+  // stages of parity j into accumulator j.  Warp 1 and, once its copies are issued, warp 0.
+  auto mma_issue = [&](int j) {
+    const uint32_t idesc0 = idesc_fp4_block(BN, E8M0);
+    const uint32_t dacc = tmem + j * BN;
+    ok = __all_sync(0xFFFFFFFFu, mbar_wait(sfb_ok, 0, 52)) && ok;
+    for (int it = j; it < n_it && ok; it += 2) {
+      const int slot = VQ ? it % R : 0;
+      // VQ: the decoder warps that place the weight scales arrive on decd only after their
+      // tcgen05.st completed, so one wait covers both
+      const bool w = VQ ? mbar_wait(&decd[slot], (it / R) & 1, 53) : mbar_wait(&sfa_ok[it], 0, 51);
+      ok = __all_sync(0xFFFFFFFFu, w);
+      if (!ok) break;
+      tc_fence_after();
+      int kw, kx, valid;
+      stage_coords(s_begin + it, kw, kx, valid);
+      const uint32_t ta = tmem + sfa_col(it), tb = tmem + sfb_col(it);
+      const uint32_t a_base = VQ ? smem_u32(sA + slot * Cfg::kABytes) : smem_u32(sW + it * Cfg::kWStride);
+      const uint32_t b_base = smem_u32(sB + it * Cfg::kBBytes);
+      const int nk = valid / 64;
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          if (kk < nk) {
+            const int at = (kk * 64) / Cfg::kAtomK;
+            const uint32_t byte = E8M0 ? static_cast<uint32_t>((kk & 1) * 2) : 0u;
+            const uint64_t ad = make_sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bd = make_sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128);
+            const uint32_t idd = idesc0 | (byte << 29) | (byte << 4);
+            const uint32_t sa = (ta + at * 4) | (byte << 30);
+            const uint32_t sb = (tb + at * 4) | (byte << 30);
+            const uint32_t acc = (it == j && kk == 0) ? 0u : 1u;
+            if (E8M0)
+              mma_mxf4_block32(dacc, ad, bd, idd, sa, sb, acc);
+            else
+              mma_nvf4_block16(dacc, ad, bd, idd, sa, sb, acc);
+          }
+        if (VQ && it + R < n_it) tc_commit(&aempty[slot]);   // the slot may be rewritten once these complete
+      }
+      __syncwarp();
+    }
+    if (lane == 0) tc_commit(accf);
+    __syncwarp();
+  };
   if (warp == 0) {
     // ---------------- the B operand of every stage, once the activations are quantized (the
     // local mode writes it into shared memory directly)
@@ -378,47 +424,9 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
         }
       }
     }
+    mma_issue(1);
   } else if (warp == 1) {
-    // ---------------- MMA issuer: MMAs only (the scale factors are placed by other warps)
-    const uint32_t idesc0 = idesc_fp4_block(BN, E8M0);
-    ok = __all_sync(0xFFFFFFFFu, mbar_wait(sfb_ok, 0, 52));
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int slot = VQ ? it % R : 0;
-      // VQ: the decoder warps that place the weight scales arrive on decd only after their
-      // tcgen05.st completed, so one wait covers both
-      const bool w = VQ ? mbar_wait(&decd[slot], (it / R) & 1, 53) : mbar_wait(&sfa_ok[it], 0, 51);
-      ok = __all_sync(0xFFFFFFFFu, w);
-      if (!ok) break;
-      tc_fence_after();
-      int kw, kx, valid;
-      stage_coords(s_begin + it, kw, kx, valid);
-      const uint32_t ta = tmem + sfa_col(it), tb = tmem + sfb_col(it);
-      const uint32_t a_base = VQ ? smem_u32(sA + slot * Cfg::kABytes) : smem_u32(sW + it * Cfg::kWStride);
-      const uint32_t b_base = smem_u32(sB + it * Cfg::kBBytes);
-      const int nk = valid / 64;
-      if (lane == 0) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          if (kk < nk) {
-            const int at = (kk * 64) / Cfg::kAtomK;
-            const uint32_t byte = E8M0 ? static_cast<uint32_t>((kk & 1) * 2) : 0u;
-            const uint64_t ad = make_sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128);
-            const uint64_t bd = make_sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128);
-            const uint32_t idd = idesc0 | (byte << 29) | (byte << 4);
-            const uint32_t sa = (ta + at * 4) | (byte << 30);
-            const uint32_t sb = (tb + at * 4) | (byte << 30);
-            const uint32_t acc = (it == 0 && kk == 0) ? 0u : 1u;
-            if (E8M0)
-              mma_mxf4_block32(tmem, ad, bd, idd, sa, sb, acc);
-            else
-              mma_nvf4_block16(tmem, ad, bd, idd, sa, sb, acc);
-          }
-        if (VQ && it + R < n_it) tc_commit(&aempty[slot]);   // the slot may be rewritten once these complete
-      }
-      __syncwarp();
-    }
-    if (lane == 0) tc_commit(accf);
-    __syncwarp();
+    mma_issue(0);
   } else if (warp >= Cfg::kQWarp0) {
     // ---------------- quantizer warps
     const int tq = threadIdx.x - Cfg::kQWarp0 * 32;   // 0..127
@@ -856,6 +864,19 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
       const int n = n0 + nl;
       const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
       const int et = threadIdx.x - 64;   // 0..127
+      // 8 accumulator columns from c: the odd stages' accumulator added when there were any
+      auto ld_acc = [&](int c, uint32_t (&r)[8]) {
+        tmem_ld8(trow + c, r);
+        if (n_it > 1) {
+          uint32_t r2[8];
+          tmem_ld8(trow + BN + c, r2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) r[jj] = __float_as_uint(__uint_as_float(r[jj]) + __uint_as_float(r2[jj]));
+        } else {
+          tmem_ld_wait();
+        }
+      };
       if (n_it > 0) ok = bar_and(1, 128, ok && mbar_wait(accf, 0, 58) && mbar_wait(xready, 0, 59));
       else ok = bar_and(1, 128, ok && mbar_wait(xready, 0, 59));
       tc_fence_after();
@@ -867,8 +888,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < a.M; c += 8) {
           uint32_t r[8];
-          tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
-          tmem_ld_wait();
+          ld_acc(c, r);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             if (c + j < a.M && n < a.N) {
@@ -888,8 +908,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < a.M; c += 8) {
             uint32_t r[8];
-            tmem_ld8(trow + c, r);
-            tmem_ld_wait();
+            ld_acc(c, r);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               if (c + j < a.M) part[(c + j) * 128 + nl] = n_it > 0 ? __uint_as_float(r[j]) : 0.f;
@@ -924,8 +943,7 @@ __global__ void __launch_bounds__(DecCfg<BN, E8M0, VQ, SF>::kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < a.M; c += 8) {
           uint32_t r[8];
-          tmem_ld8(trow + c, r);
-          tmem_ld_wait();
+          ld_acc(c, r);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             if (c + j < a.M) mine[(c + j) * 128 + nl] = n_it > 0 ? __uint_as_float(r[j]) : 0.f;

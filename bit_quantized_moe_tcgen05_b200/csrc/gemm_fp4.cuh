@@ -12,10 +12,11 @@
 // channels are read a second time for the tail stages (activation coordinate C - k + j while
 // the weight coordinate is C + j).  No tail copy is materialised.
 //
-// Warp roles (192 threads; 320 for VQ weights): warp 0 = TMA producer, warp 1 = TMEM allocator +
+// Warp roles (192 threads; 352 for VQ weights): warp 0 = TMA producer, warp 1 = TMEM allocator +
 // MMA issuer (one lane issues), warps 2..5 = epilogue; with VQ weights warps 2..9 first rebuild
-// each stage's operand tile from the codebooks.  Without VQ, where TMEM holds two accumulators,
-// warp 2 issues the MMAs of every other stage into the second one (the epilogue adds the two).  A STAGES-deep ring of
+// each stage's operand tile from the codebooks.  Where TMEM holds two accumulators, a second warp
+// (warp 2, or warp 10 with VQ) issues the MMAs of every other stage into the second one (the
+// epilogue adds the two).  A STAGES-deep ring of
 // shared-memory stages, each 256 K-elements deep, is guarded by full/empty mbarriers; MMA
 // completion is signalled by tcgen05.commit.  Every wait is bounded (see ptx.cuh).
 //
@@ -85,7 +86,7 @@ template <int BN, bool E8M0, bool VQ = false, int SF = 0>
 struct Fp4Cfg {
   // warps: 0 producer, 1 MMA, 2..5 epilogue; VQ adds decoders so that warps 2..9 decode
   static constexpr int kDecWarps = VQ ? 8 : 0;
-  static constexpr int kThreads = VQ ? 320 : 192;
+  static constexpr int kThreads = VQ ? 352 : 192;   // VQ: warp 10 is the second MMA issuer
   static constexpr int kAtomK = E8M0 ? 128 : 64;      // K elements covered by one SF atom
   static constexpr int kAtoms = 256 / kAtomK;         // SF atoms per stage per 128 rows
   static constexpr int kG = (BN + 127) / 128;          // 128-row groups of the B operand
@@ -110,10 +111,12 @@ struct Fp4Cfg {
   static constexpr int kStages = kStagesRaw > 12 ? 12 : (kStagesRaw < 2 ? 2 : kStagesRaw);
   static constexpr int kSfaCols = kAtoms * 4;          // TMEM columns per stage
   static constexpr int kSfbCols = kAtoms * 4 * kG;
-  // Without VQ decoders, the first epilogue warp (idle during the main loop) issues the MMAs of
-  // every other stage into a second accumulator where TMEM holds two: issuing a block-scaled MMA
-  // and its scale copies costs the issuing thread more than the tensor core needs to run it.
-  static constexpr int kIssuers = (!VQ && 2 * BN + kStages * (kSfaCols + kSfbCols) <= 512) ? 2 : 1;
+  // Where TMEM holds two accumulators a second warp (without VQ the first epilogue warp, idle
+  // during the main loop; with VQ an extra warp) issues the MMAs of every other stage into the
+  // second one: issuing a block-scaled MMA and its scale copies costs the issuing thread more
+  // than the tensor core needs to run it.
+  static constexpr int kIssuers = (2 * BN + kStages * (kSfaCols + kSfbCols) <= 512) ? 2 : 1;
+  static constexpr int kIssuer2Warp = VQ ? 10 : 2;
   static constexpr int kColsNeeded = kIssuers * BN + kStages * (kSfaCols + kSfbCols);
   static constexpr int kProducers = VQ ? 1 : 2;   // without VQ, warp 3 also produces
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
@@ -377,6 +380,8 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
     }
   } else if (warp == 1) {
     mma_issue(0);
+  } else if (VQ && warp == Cfg::kIssuer2Warp) {
+    if (Cfg::kIssuers == 2) mma_issue(1);
   } else {
     if constexpr (VQ) {
       // ---------------- VQ decode (warps 2..9): for each stage rebuild the 128 x 256 E2M1 operand
@@ -433,7 +438,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)
         if (lane == 0) mbar_arrive(&decd[st]);
       }
     }
-    if (Cfg::kIssuers == 2 && warp == 2) mma_issue(1);
+    if (!VQ && Cfg::kIssuers == 2 && warp == Cfg::kIssuer2Warp) mma_issue(1);
     if (Cfg::kProducers == 2 && warp == 3 && !lsu_act) {
       griddep_wait();   // the activations of this grid's quantizer
       produce(1);

@@ -161,12 +161,13 @@ ql_status qlinear_workspace_bytes(const ql_linear* layer, int64_t M, size_t* byt
  * per-launch tag derived from a launch counter kept there, so nothing needs clearing, and after
  * a device timeout the counter has moved past every tag the failed launch left.  Calls that
  * share a workspace must be stream-ordered.  Rows of x are contiguous (row stride K - k_tail
- * elements).  M may be 0 (no-op).  For M <= 64 with FP4 or VQ weights the forward is ONE launch:
- * the GEMM's own warps quantize x (each element once across the grid) before its MMAs need it,
- * while the weights already stream.  Kernels are launched with programmatic stream serialization
- * and release the next such grid at once: a following qlinear call on the stream may start
- * streaming its weights while this one finishes, and reads this call's results only after it
- * has completed. */
+ * elements, with or without tail_copy).  M may be 0 (no-op).  Where the decode kernel runs
+ * (ql_decode_fuse_mode; by default M = 1, and MXFP4 layers from 33 to 64 tokens) the forward is
+ * ONE launch whose own warps quantize x before its MMAs need it, while the weights already
+ * stream; otherwise it is the activation quantizer followed by the split-K or prefill GEMM.
+ * Kernels are launched with programmatic stream serialization and release the next such grid at
+ * once: a following qlinear call on the stream may start streaming its weights while this one
+ * finishes, and reads this call's results only after it has completed. */
 ql_status qlinear_forward(const ql_linear* layer, const void* x_bf16, int64_t M, void* y_bf16,
                           float* y_f32, void* ws, size_t ws_bytes, ql_stream_t stream);
 
