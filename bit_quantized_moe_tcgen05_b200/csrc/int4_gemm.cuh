@@ -89,17 +89,12 @@ struct Int4Cfg {
   static constexpr int kABytes = 128 * 128;        // int8 tile, 128 rows x 128 B
   static constexpr int kBBytes = BN * 128;
   static constexpr int kSxBytes = BN * 4 < 16 ? 16 : BN * 4;
-  // Two rings: the copied stages [B tile][raw weight block][sx] (kept until the fold has read the
-  // stage's scales), and a shorter ring of decoded int8 A tiles (free once the MMAs read them), so
-  // that more copied stages are in flight than a ring of whole stages would hold.
-  static constexpr int kAStages = 3;
-  static constexpr int kStageBytes = ((kBBytes + kRawBytes + kSxBytes) + 1023) / 1024 * 1024;
-  static constexpr int kStagesRaw = (200 * 1024 - kAStages * kABytes) / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 10 ? 10 : kStagesRaw;
+  static constexpr int kStageBytes = ((kRawBytes + kABytes + kBBytes + kSxBytes) + 1023) / 1024 * 1024;
+  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
-  static constexpr int kRingBytes = kAStages * kABytes + kStages * kStageBytes;
-  static constexpr int kSmemBytes = kRingBytes + 1024 + 512;
-  static_assert(BN * 128 * 4 <= kRingBytes, "output staging must fit the rings");
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 512;
+  static_assert(BN * 128 * 4 <= kStages * kStageBytes, "output staging must fit the ring");
   static_assert(kCols % 8 == 0, "fold columns come in tcgen05.ld groups of 8");
 };
 
@@ -150,21 +145,17 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
   // 1 KB aligned by offsetting the shared array itself, so that every pointer derived from it
   // stays a shared-space pointer (plain ld/st.shared, not generic accesses)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  // [A ring: kAStages int8 tiles of 16 KB][copied stages: B tile, raw weight block, sx]
-  // (A tiles and B tiles 1024-aligned)
-  constexpr int SA = Cfg::kAStages;
-  uint8_t* ring = smem + SA * Cfg::kABytes;
-  auto sA = [&](int sa) { return smem + sa * Cfg::kABytes; };
-  auto sB = [&](int st) { return ring + st * Cfg::kStageBytes; };
-  auto sRaw = [&](int st) { return ring + st * Cfg::kStageBytes + Cfg::kBBytes; };
+  // stage st: [A int8 tile 16 KB][B tile][raw weight block][sx]  (A and B 1024-aligned)
+  auto sA = [&](int st) { return smem + st * Cfg::kStageBytes; };
+  auto sB = [&](int st) { return smem + st * Cfg::kStageBytes + Cfg::kABytes; };
+  auto sRaw = [&](int st) { return smem + st * Cfg::kStageBytes + Cfg::kABytes + Cfg::kBBytes; };
   auto sSx = [&](int st) {
-    return reinterpret_cast<float*>(ring + st * Cfg::kStageBytes + Cfg::kBBytes + Cfg::kRawBytes);
+    return reinterpret_cast<float*>(smem + st * Cfg::kStageBytes + Cfg::kABytes + Cfg::kBBytes + Cfg::kRawBytes);
   };
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes);
-  uint64_t* empty = full + S;     // copied stage free: MMAs done and the fold read its scales
-  uint64_t* decd = empty + S;     // [SA] A tile decoded
-  uint64_t* aempty = decd + SA;   // [SA] A tile read by the MMAs
-  uint64_t* accf = aempty + SA;   // [2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* decd = empty + S;
+  uint64_t* accf = decd + S;      // [2]
   uint64_t* acce = accf + 2;      // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
 
@@ -184,10 +175,7 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 2);     // MMA commit + fold release
-    }
-    for (int s = 0; s < SA; ++s) {
       mbar_init(&decd[s], Cfg::kDecWarps * 32);
-      mbar_init(&aempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accf[b], 1);
@@ -230,19 +218,15 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
       for (int j = 0; j < nst && ok; ++j) {
         const int st = j % S, b = j & 1;
         const uint32_t ph = (j / S) & 1;
-        const int sa = j % SA;
-        // decd implies full: the decoders waited for the copied stage before decoding
-        if (!mbar_wait(&decd[sa], (j / SA) & 1, 23) ||
+        if (!mbar_wait(&full[st], ph, 22) || !mbar_wait(&decd[st], ph, 23) ||
             !mbar_wait(&acce[b], ((j >> 1) & 1) ^ 1, 24)) { ok = false; break; }
-        (void)ph;
         tc_fence_after();
-        const uint32_t ab = smem_u32(sA(sa)), bb = smem_u32(sB(st));
+        const uint32_t ab = smem_u32(sA(st)), bb = smem_u32(sB(st));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_i8(tmem + b * BN, make_sdesc(ab + kk * 32, 16, 1024, kLayoutSW128),
                  make_sdesc(bb + kk * 32, 16, 1024, kLayoutSW128), idesc, kk > 0 ? 1u : 0u);
         tc_commit(&empty[st]);
-        tc_commit(&aempty[sa]);
         tc_commit(&accf[b]);
       }
     }
@@ -252,11 +236,9 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
     for (int j = 0; j < nst && ok; ++j) {
       const int st = j % S;
       const uint32_t ph = (j / S) & 1;
-      const int sa = j % SA;
-      if (!mbar_wait(&full[st], ph, 25) ||
-          (j >= SA && !mbar_wait(&aempty[sa], ((j / SA) - 1) & 1, 28))) { ok = false; break; }
+      if (!mbar_wait(&full[st], ph, 25)) { ok = false; break; }
       const uint8_t* raw = sRaw(st);
-      uint8_t* at = sA(sa);
+      uint8_t* at = sA(st);
 #pragma unroll 4
       for (int i = 0; i < 8; ++i) {
         const int c = t + 128 * i;                 // 16-byte output chunk: row r, chunk kc
@@ -274,7 +256,7 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
         *reinterpret_cast<uint4*>(at + r * 128 + ((kc ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       fence_proxy_async_smem();
-      mbar_arrive(&decd[sa]);
+      mbar_arrive(&decd[st]);
     }
   } else {
     // ---------------- fold: acc += I * (s_w * s_x) per 128-input group, on packed fp32 pairs.
