@@ -129,9 +129,18 @@ __device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
 }
 // Exact float of an int32 x with |x| < 2^22: in [2^23, 2^24) the float grid is the integers, so
 // the bit pattern of 1.5 * 2^23 plus x is the float 1.5 * 2^23 + x; the subtraction is exact.
+// (Starting the TMEM accumulators at that bit pattern, re-written by the fold after each read,
+// would save the integer adds; the extra TMEM stores measured far slower.)
 __device__ __forceinline__ float2 small_ints_to_float2(uint32_t x0, uint32_t x1) {
   return f2_add(make_float2(__uint_as_float(x0 + 0x4B400000u), __uint_as_float(x1 + 0x4B400000u)),
                 make_float2(-12582912.0f, -12582912.0f));
+}
+// Sign-extend the eight 4-bit two's-complement fields of w to bytes: lo gets the low nibble of each
+// byte, hi the high nibble. A field with bit 3 set gains 0xF0 (8 * 30 = 240 stays inside its byte).
+__device__ __forceinline__ void int4x8_to_int8(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  lo = (w & 0x0F0F0F0Fu) | ((w & 0x08080808u) * 30u);
+  const uint32_t w4 = w >> 4;
+  hi = (w4 & 0x0F0F0F0Fu) | ((w4 & 0x08080808u) * 30u);
 }
 
 template <int BN>
@@ -192,6 +201,7 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t tfold = tmem + (static_cast<uint32_t>(q * 32) << 16) + col0;   // a fold thread's lane and columns
 
   bool ok = true;
   float2 acc[Cfg::kCols / 2];
@@ -247,9 +257,8 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
         uint32_t o[4];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint32_t w = h ? pw.y : pw.x;
-          const uint32_t lo = __vsub4((w & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
-          const uint32_t hi = __vsub4(((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+          uint32_t lo, hi;
+          int4x8_to_int8(h ? pw.y : pw.x, lo, hi);
           o[2 * h] = __byte_perm(lo, hi, 0x5140);
           o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
         }
@@ -279,8 +288,7 @@ __global__ void __launch_bounds__(Int4Cfg<BN>::kThreads, 1)
           uint32_t r[kBatch];
 #pragma unroll
           for (int c = 0; c < kBatch; c += 8)
-            tmem_ld8(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN + col0 + c0 + c,
-                     *reinterpret_cast<uint32_t(*)[8]>(r + c));
+            tmem_ld8(tfold + b * BN + c0 + c, *reinterpret_cast<uint32_t(*)[8]>(r + c));
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < kBatch; c += 8) {

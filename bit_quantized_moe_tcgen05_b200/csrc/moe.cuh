@@ -225,7 +225,8 @@ struct MoeCfg {
   static constexpr int kStgLd = 129;              // padded row of the transposed staging tile
   static constexpr int kStgBytes = kHalf * kStgLd * 4;
   static constexpr int kTmemCols = 2 * BN;        // two accumulators (ping-pong across items)
-  static constexpr int kDecWarps = 8;
+  static constexpr int kDecGroups = 3;            // decoder groups, each on every third stage
+  static constexpr int kDecWarps = 4 * kDecGroups;
   static constexpr int kThreads = (2 + kDecWarps + 4) * 32;
   static constexpr int kSmemBytes =
       kStages * kStageBytes + 2 * kCentBytes + kStgBytes + 1024 + 512;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&ifull[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&decd[s], Cfg::kDecWarps / 2);   // one decoder group per stage
+      mbar_init(&decd[s], 4);   // one decoder group (4 warps) per stage
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&cfull[b], 1);
@@ -387,10 +388,11 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
     }
   } else if (warp < 2 + Cfg::kDecWarps) {
     // ---------------- decode: 4-bit indices -> bf16 operand tile through the row centroids.
-    // Two groups of decoder warps take alternate stages: a stage's barrier waits and arrivals
-    // cost a group about as long as its decode, so the groups overlap one another's.
-    constexpr int kDT = Cfg::kDecWarps * 16;                  // threads per group
-    const int grp = (warp - 2) / (Cfg::kDecWarps / 2);
+    // kDecGroups groups of four decoder warps take the stages round-robin: a stage's barrier
+    // waits, index loads and table lookups cost a group more than the MMAs need, so the groups
+    // overlap one another's.
+    constexpr int kDT = 128;                                  // threads per group
+    const int grp = (warp - 2) / 4;
     const int t = threadIdx.x - 64 - grp * kDT;
     int it = 0;
     for (int id = blockIdx.x, j = 0; id < n_items && ok; id += gridDim.x, ++j) {
@@ -398,7 +400,7 @@ __global__ void __launch_bounds__(MoeCfg<BN>::kThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&cfull[b], (j >> 1) & 1, 15))) { ok = false; break; }
       const uint16_t* cent = reinterpret_cast<const uint16_t*>(sCent + b * 128 * 16);
       for (int i = 0; i < nstages && ok; ++i, ++it) {
-        if ((it & 1) != grp) continue;
+        if (it % Cfg::kDecGroups != grp) continue;
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
         // indices only: runs ahead of B (warp-uniform: the warp leaves the loop together)
