@@ -39,12 +39,11 @@ NOMINAL_FP4_OVER_BF16 = 4.0      # 9 PFLOP/s dense FP4 / 2.25 PFLOP/s dense bf16
 L2_BYTES = 126 * 1024 * 1024
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the timed GEMM
-# kernel, from an ncu --set full capture of that kernel (the VQ layer's M = 64 launch; the PRQuant
-# M = 2048 launch).  Set an entry to None whenever its kernel changes until it is captured again.
-# dram read + write bytes per launch from one ncu capture of the current kernels (profiles/):
-# the headline's GEMM launches averaged over M = 1, 8, 64, and the PRQuant M = 2048 GEMM
-NCU_TRAFFIC_PER_LAUNCH = {"vq": (11.014e6 + 11.059e6 + 11.333e6) / 3, "prquant_m2048": 24.59e6}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the timed GEMM kernel,
+# from ncu captures under profiles/: the headline's GEMM launches averaged over M = 1, 8, 64. An
+# entry is None while its kernel has changed since its capture: the PRQuant M = 2048 GEMM's
+# unsplit epilogue was changed after its capture (24.59 MB per launch then).
+NCU_TRAFFIC_PER_LAUNCH = {"vq": (11.014e6 + 11.059e6 + 11.333e6) / 3, "prquant_m2048": None}
 
 
 def measured_peaks() -> dict:
