@@ -16,7 +16,7 @@
 // MMA issuer (one lane issues), warps 2..5 = epilogue; with VQ weights warps 2..9 first rebuild
 // each stage's operand tile from the codebooks.  Where TMEM holds two accumulators, a second warp
 // (warp 2, or warp 10 with VQ) issues the MMAs of every other stage into the second one (the
-// epilogue adds the two).  A STAGES-deep ring of
+// epilogue adds the two); without VQ, warp 3 produces every other stage.  A STAGES-deep ring of
 // shared-memory stages, each 256 K-elements deep, is guarded by full/empty mbarriers; MMA
 // completion is signalled by tcgen05.commit.  Every wait is bounded (see ptx.cuh).
 //
@@ -128,7 +128,7 @@ struct Fp4Cfg {
 
 // The weight operand of each (128-row tile, K stage) is one contiguous block in HBM, laid out at
 // create time exactly as the stage buffer wants it, and arrives by one 1-D bulk copy.
-// VQ = true (MXCode PreScale weights): the blocks hold 8-bit indices; warps 2..5 decode each
+// VQ = true (MXCode PreScale weights): the blocks hold 8-bit indices; warps 2..9 decode each
 // stage's operand tile from the shared-memory codebooks.
 template <int BN, bool E8M0, bool VQ = false, int SF = 0>
 __global__ void __launch_bounds__(Fp4Cfg<BN, E8M0, VQ, SF>::kThreads, 1)

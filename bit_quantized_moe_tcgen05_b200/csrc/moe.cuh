@@ -237,8 +237,8 @@ struct MoeCfg {
 // enumerated expert by expert, nt fastest; CTA c takes items c, c + gridDim.x, ...  Warp roles:
 // 0 producer (TMA: index tile, B rows -- the expert's contiguous gathered x rows for gate/up, its
 // h rows for down -- and the item's 128 centroid rows), 1 TMEM allocator + MMA issuer (kind::f16, N = the
-// item's token count rounded up to 16), 2..9 decode (4-bit indices -> bf16 operand tile),
-// 10..13 epilogue.  Two TMEM accumulators alternate between items, so the epilogue of one item
+// item's token count rounded up to 16), 2 .. 1 + kDecWarps decode (4-bit indices -> bf16 operand
+// tile; groups of four warps take the stages round-robin), the last four warps the epilogue.  Two TMEM accumulators alternate between items, so the epilogue of one item
 // overlaps the main loop of the next.  GATEUP: the weight rows of a tile are 64 gate rows then
 // the 64 matching up rows (repacked at create time), so the SwiGLU pairs meet inside one tile.
 template <int BN, bool GATEUP>
