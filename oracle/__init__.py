@@ -12,8 +12,11 @@ Modules
 formats   E2M1 / E8M0 / E4M3 / UE5M3 / INT4 codecs (MXCode, Table 1; OCP MX formats).
 mx        Activation/weight quantizers: E8M0-B32, E4M3-B16 + FP32 tensor scale, INT4 g128.
 gemm      Block-scaled W4A4 GEMM reference and the per-element tolerance scale.
-prquant   PRQuant offline column selection, permutation, tail residual, augmented GEMM.
-vq        MXCode PreScale VQ: E4M3-B16 scales, per-QBlock FP4 codebooks, index assignment.
+prquant   PRQuant offline column selection (optionally with the E8M0-W block-scale search),
+          permutation, tail residual, the augmented activation and GEMM.
+vq        MXCode VQ: PreScale E4M3-B16 scales, per-QBlock FP4 codebooks, index assignment;
+          PostScale (one scale per codebook) and PreScale+ (scale indices into a scale codebook).
+hadamard  Block-32 Walsh-Hadamard of the activations ahead of the MXFP4 quantizer (CodeQuant had).
 moe       Top-k routing and the grouped SwiGLU expert FFN with cluster-codebook weights.
 int4bsr   MosaicQuant-style INT4 dense base + block-sparse INT4 residual.
 
