@@ -40,10 +40,10 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the timed GEMM kernel,
-# from ncu captures under profiles/: the headline's GEMM launches averaged over M = 1, 8, 64. An
-# entry is None while its kernel has changed since its capture: the PRQuant M = 2048 GEMM's
-# unsplit epilogue was changed after its capture (24.59 MB per launch then).
-NCU_TRAFFIC_PER_LAUNCH = {"vq": (11.014e6 + 11.059e6 + 11.333e6) / 3, "prquant_m2048": None}
+# from ncu captures under profiles/: the headline's GEMM launches averaged over M = 1, 8, 64 (the
+# current kernels). An entry is None while its kernel has changed since its capture: the PRQuant
+# M = 2048 GEMM's unsplit epilogue was changed after its capture (24.59 MB per launch then).
+NCU_TRAFFIC_PER_LAUNCH = {"vq": (11.0144e6 + 11.0659e6 + 11.3400e6) / 3, "prquant_m2048": None}
 
 
 def measured_peaks() -> dict:
