@@ -385,8 +385,8 @@ constexpr int64_t kDecClusterAmaxElems = 16 * 1024;  // ... when a cluster excha
 // Whether a forward of M tokens runs the decode kernel (when it also plans): forced by
 // ql_decode_fuse_mode, else by what measured faster on the B200 in chains of CUDA-graph replayed
 // layers of 2560 x 9728.  With E4M3-B16 activations (VQ and NVFP4 layers) the separate grid
-// quantizer and the general GEMM won from M = 8 up (VQ: 15.5 against 20.4 us at M = 8, 22.0
-// against 22.5 at M = 64) and tied at M = 1 (14.2 / 14.1); with MXFP4 activations the decode
+// quantizer and the general GEMM won from M = 8 up (VQ: 13.9 against 18.6 us at M = 8, 21.3
+// against 22.5 at M = 64) and tied at M = 1 (12.6 / 12.5); with MXFP4 activations the decode
 // kernel won at M = 1 (9.5 against 10.0) and from M = 64 (14.5 against 16.3) and lost in between.
 bool use_decode_kernel(const ql_linear* L, int64_t M) {
   const int forced = g_decode_fuse_mode.load();

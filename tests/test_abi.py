@@ -123,3 +123,20 @@ def test_int4_bsr_host_preparation_matches_oracle(N, K, T):
     assert np.array_equal(got["rcodes"].reshape(len(ref["sel"]), 16, 64),
                           F.pack_nibbles(F.int4_encode(ref["rq"])))
     assert np.array_equal(got["rscales"], ref["rs"].view(np.uint16))
+
+
+def test_decode_mode_and_augmented_quantizer_checks_without_device():
+    """Host-side checks of two entry points: the decode organisation switch accepts -1..3 only,
+    and the augmented (offline tail copy) quantizer refuses bad formats and shapes before any
+    launch; an empty tensor is a no-op."""
+    import bit_quantized_moe_tcgen05_b200 as ql
+    for bad in (-2, 4, 100):
+        assert ql.lib.ql_decode_fuse_mode(bad) == 1
+    for good in (0, 1, 2, 3, -1):
+        assert ql.lib.ql_decode_fuse_mode(good) == 0   # ends on -1, the measured choice
+    assert ql.lib.quantize_act_augmented(1, None, -1, 64, 32, None, None, None) == 1    # negative M
+    assert ql.lib.quantize_act_augmented(2, None, 4, 64, 32, None, None, None) == 2     # not MXFP4
+    assert ql.lib.quantize_act_augmented(1, None, 4, 64, 16, None, None, None) == 2     # k_tail % 32
+    assert ql.lib.quantize_act_augmented(1, None, 4, 64, 96, None, None, None) == 2     # k_tail > C
+    assert ql.lib.quantize_act_augmented(1, None, 4, 64, 32, None, None, None) == 1     # null pointers
+    assert ql.lib.quantize_act_augmented(1, None, 0, 64, 32, None, None, None) == 0     # empty
