@@ -140,3 +140,26 @@ def test_decode_mode_and_augmented_quantizer_checks_without_device():
     assert ql.lib.quantize_act_augmented(1, None, 4, 64, 96, None, None, None) == 2     # k_tail > C
     assert ql.lib.quantize_act_augmented(1, None, 4, 64, 32, None, None, None) == 1     # null pointers
     assert ql.lib.quantize_act_augmented(1, None, 0, 64, 32, None, None, None) == 0     # empty
+
+
+def test_moe_arguments_rejected_without_device():
+    """moe_create and the MoE workspace / forward calls check their arguments on the host, before
+    any device allocation or launch."""
+    import bit_quantized_moe_tcgen05_b200 as ql
+    h = ctypes.c_void_p()
+    codes = np.zeros((256, 64), np.uint8)
+    cb = np.zeros((256, 16), np.uint16)
+    good = dict(wfmt=4, N=256, K=128, codes=codes.ctypes.data, codebooks=cb.ctypes.data)
+    gu, dn = ql.WeightDesc(**good), ql.WeightDesc(**good)
+    assert ql.lib.moe_create(None, ctypes.byref(dn), 2, 1, None, ctypes.byref(h)) == 1
+    bad_fmt = ql.WeightDesc(**dict(good, wfmt=1))
+    assert ql.lib.moe_create(ctypes.byref(bad_fmt), ctypes.byref(dn), 2, 1, None, ctypes.byref(h)) == 2
+    for E, k in ((0, 1), (300, 8), (8, 0), (8, 17), (4, 8)):          # 0 < k <= 16, k <= E <= 256
+        assert ql.lib.moe_create(ctypes.byref(gu), ctypes.byref(dn), E, k, None, ctypes.byref(h)) == 2
+    no_cb = ql.WeightDesc(**dict(good, codebooks=None))
+    assert ql.lib.moe_create(ctypes.byref(no_cb), ctypes.byref(dn), 2, 1, None, ctypes.byref(h)) == 1
+    uneven = ql.WeightDesc(**dict(good, N=250))
+    assert ql.lib.moe_create(ctypes.byref(uneven), ctypes.byref(dn), 4, 1, None, ctypes.byref(h)) == 1
+    nbytes = ctypes.c_size_t()
+    assert ql.lib.moe_workspace_bytes(None, 16, ctypes.byref(nbytes)) == 1
+    assert ql.lib.moe_grouped_forward(None, None, 16, None, None, None, None, None, None, 0, None) == 1
