@@ -163,3 +163,26 @@ def test_moe_arguments_rejected_without_device():
     nbytes = ctypes.c_size_t()
     assert ql.lib.moe_workspace_bytes(None, 16, ctypes.byref(nbytes)) == 1
     assert ql.lib.moe_grouped_forward(None, None, 16, None, None, None, None, None, None, 0, None) == 1
+
+
+def test_offline_preparation_rejects_bad_arguments():
+    """The host preparation entries refuse null buffers and unsupported shapes (CPU only)."""
+    import bit_quantized_moe_tcgen05_b200 as ql
+    w = np.zeros((128, 256), np.uint16)
+    perm = np.zeros(256, np.int32)
+    codes = np.zeros((128, 256), np.uint8)
+    sc = np.zeros((128, 16), np.uint8)
+    P = lambda a: a.ctypes.data
+    f = ql.lib.qlinear_prepare_prquant_ex
+    assert f(None, 128, 256, 128, 0, P(perm), P(codes), P(sc)) == 1          # null weight
+    assert f(P(w), 128, 256, 0, 0, P(perm), P(codes), P(sc)) == 1            # k = 0
+    assert f(P(w), 128, 256, 384, 0, P(perm), P(codes), P(sc)) == 1          # k > C
+    assert f(P(w), 128, 256, 64, 0, P(perm), P(codes), P(sc)) == 2           # k % 128
+    assert f(P(w), 128, 200, 128, 0, P(perm), P(codes), P(sc)) == 2          # C % 128
+    ts = np.zeros(1, np.float32)
+    cbk = np.zeros(4096, np.uint8)
+    idx = np.zeros((128, 64), np.uint8)
+    g = ql.lib.qlinear_prepare_vq_prescale
+    assert g(P(w), 128, 256, None, 64, 64, P(ts), P(sc), P(idx)) == 1          # null codebooks
+    assert g(P(w), 128, 256, P(cbk), 32, 64, P(ts), P(sc), P(idx)) == 2        # QBlock not 64 x 64
+    assert g(P(w), 100, 256, P(cbk), 64, 64, P(ts), P(sc), P(idx)) == 2        # N % 64
